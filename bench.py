@@ -1,0 +1,344 @@
+#!/usr/bin/env python3
+"""Decode-step benchmark: sparse-attention decode tokens/s at 128K context, batch 8.
+
+One step = one ls_decode_step over a batch of 8 requests at 131,072 tokens each:
+fp8 indexer over every cached token (64 heads x 128), per-request top-2048, MLA
+attention (128 heads, 576-wide latent KV, bf16) over the selected rows, all inputs
+resident in HBM.  Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun): every rank runs its own batch of 8 requests (requests are
+independent; no collective on the data path); the time is the max over ranks.
+--impl reference times the CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn decode tokens/s at 128K ctx, batch 8; indexer+attn HBM GB/s vs peak"
+UNIT = "tokens/s"
+BATCH, CTX, TOPK = 8, 131072, 2048
+H_I, D_I = 64, 128
+INDEX_BYTES_PER_TOKEN = D_I + 4 + 4      # e4m3 key row + fp32 key scale read, fp32 score written
+ATTN_ROW_BYTES = 576 * 2
+WORKLOAD = "mla_decode_b8_ctx131072_top2048"
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "index_score_tc_mla_decode_b8_ctx131072.md")
+CONFIG = {"workload": WORKLOAD, "batch": BATCH, "ctx": CTX, "topk": TOPK, "indexer": "64x128 e4m3",
+          "attention": "MLA 128 heads x 576 (V 512) bf16", "page": 64,
+          "l2": "flushed between timed steps (256 MB write)"}
+
+
+def rank_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)),
+            int(os.environ.get("LOCAL_RANK", 0)))
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def profile_traffic():
+    """Per-launch DRAM bytes of the indexer kernel from the committed ncu summary, valid
+    only while the kernel source is unchanged since the capture."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None
+    text = open(PROFILE_SUMMARY).read()
+    m = re.search(r"dram_bytes_per_full_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
+    if not m or not h:
+        return None
+    src = os.path.join(ROOT, "sparse_attention_decode_ls_b200", "csrc", "index_score.cuh")
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != h.group(1):
+        return None
+    return float(m.group(1))
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting",
+               0x1: "gpu_idle"}
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def _oracle_cores():
+    try:
+        from threadpoolctl import threadpool_info
+        return int(max([i.get("num_threads", 1) for i in threadpool_info()] + [1]))
+    except Exception:  # noqa: BLE001
+        return 1
+
+
+def oracle_request_runner(ctx, k, seed=1002):
+    """Inputs of one request of the workload (context `ctx`, top-`k`) and a callable that
+    runs the CPU oracle's decode step on it."""
+    import oracle.ls_oracle as O
+    from sparse_attention_decode_ls_b200 import synthetic as syn
+    inp = syn.indexer_fp8([ctx], seed=seed)
+    q, kv = syn.mla_attention(1, inp.key_pool.shape[0], seed=seed + 1000)
+    qb = q.view(torch.int16).numpy().view(np.uint16)
+    kvb = kv.view(torch.int16).numpy().view(np.uint16)
+    wb = inp.w.view(torch.int16).numpy().view(np.uint16)
+
+    def run():
+        O.decode_step(q8=inp.q.numpy(), q_scale=inp.q_scale.numpy(), w_bits=wb, key_pool=inp.key_pool.numpy(),
+                      key_scale_pool=inp.key_scale.numpy(), page_table=inp.page_table.numpy(), lens=[ctx], k=k,
+                      q_attn_bits=qb, kv_pool_bits=kvb, scale=syn.softmax_scale(576), dv=512)
+    return run
+
+
+def cpu_oracle_sample(seconds_budget=15.0):
+    """The CPU oracle on whole requests of the workload (indexer over 131,072 tokens,
+    top-2048, MLA attention), as many as fit the budget (at least one)."""
+    run = oracle_request_runner(CTX, TOPK)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        run()
+        done += 1
+        el = time.perf_counter() - t0
+        if el * (done + 1) / done > seconds_budget:
+            break
+    return {"value": done / el, "unit": UNIT, "cores": _oracle_cores(), "kind": "oracle",
+            "sample": f"{done} whole request(s) of {WORKLOAD} (one decode token each), float64 numpy, "
+                      f"{el:.1f} s"}
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle as it stands.  Each step runs it on one request whose
+    context (and selection) is a fixed fraction f of the workload's, sized so the whole
+    run stays within LS_REF_BUDGET_S seconds; a step counts as f decode tokens."""
+    rank, world, _ = rank_env()
+    if rank != 0:
+        return 0
+    budget = float(os.environ.get("LS_REF_BUDGET_S", "150"))
+    full = oracle_request_runner(CTX, TOPK)
+    t0 = time.perf_counter()
+    full()
+    t_full = time.perf_counter() - t0
+    n = args.warmup + args.steps
+    f = min(1.0, budget / max(n * t_full, 1e-9))
+    ctx_f = max(64 * 64, int(round(f * CTX / 64)) * 64)
+    f = ctx_f / CTX
+    k_f = max(1, int(round(TOPK * f)))
+    run = full if ctx_f == CTX else oracle_request_runner(ctx_f, k_f)
+    times = []
+    for i in range(n):
+        t0 = time.perf_counter()
+        run()
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    value = len(times) * f / sum(times)
+    sample = (f"each step: 1 request at context {ctx_f} with top-{k_f} ({f:.4f} of a {WORKLOAD} request) on the "
+              f"CPU oracle (float64 numpy); one full request took {t_full:.2f} s")
+    out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": 1e3 * BATCH / value, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": CONFIG,
+           "impl": "reference",
+           "cpu_baseline": {"value": value, "unit": UNIT, "cores": _oracle_cores(), "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_ours(args):
+    rank, world, local = rank_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    from sparse_attention_decode_ls_b200 import binding as B
+    from sparse_attention_decode_ls_b200 import workload as W
+
+    wl = W.mla_decode(batch=BATCH, ctx=CTX, k=TOPK, seed=1002 + 7919 * rank, device="cuda")
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    K, Wm = args.steps, args.warmup
+
+    def new_events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in evs:
+            e.record(stream)
+        return evs
+
+    for _ in range(Wm):
+        flush.zero_()
+        wl.step()
+    torch.cuda.synchronize()
+    B.ls_check_device_status()
+    stage_ev = [new_events(6) for _ in range(K)]
+    step_ev = [new_events(2) for _ in range(K)]
+    arrs = [B.event_array(s) for s in stage_ev]
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(K):
+            flush.zero_()
+            step_ev[i][0].record(stream)
+            wl.step(events=arrs[i])
+            step_ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    status = B.ls_check_device_status()
+    step_ms = [s[0].elapsed_time(s[1]) for s in step_ev]
+    idx_ms = [s[0].elapsed_time(s[1]) for s in stage_ev]
+    topk_ms = [s[1].elapsed_time(s[4]) for s in stage_ev]
+    attn_ms = [s[4].elapsed_time(s[5]) for s in stage_ev]
+    total_ms = sum(step_ms)
+    if dist:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    value = world * BATCH / (ms_per_step / 1e3)
+
+    # ---- end to end through the C ABI with host buffers: per-step inputs (queries,
+    # head weights, scales, lengths, page tables) go host->device, outputs come back
+    t = wl.tensors
+    h2d_names = ["i_q", "i_q_scale", "i_w", "i_lens", "i_page_table", "a_q"]
+    host_in = {n: torch.empty_like(t[n], device="cpu").pin_memory() for n in h2d_names}
+    for n in h2d_names:
+        host_in[n].copy_(t[n])
+    host_o = torch.empty_like(t["o"], device="cpu").pin_memory()
+    host_lse = torch.empty_like(t["lse"], device="cpu").pin_memory()
+    h2d_bytes = sum(host_in[n].numel() * host_in[n].element_size() for n in h2d_names)
+    d2h_bytes = host_o.numel() * host_o.element_size() + host_lse.numel() * host_lse.element_size()
+    e2e_ev = [new_events(2) for _ in range(K)]
+    for i in range(Wm + K):
+        flush.zero_()
+        if i >= Wm:
+            e2e_ev[i - Wm][0].record(stream)
+        for n in h2d_names:
+            t[n].copy_(host_in[n], non_blocking=True)
+        wl.step()
+        host_o.copy_(t["o"], non_blocking=True)
+        host_lse.copy_(t["lse"], non_blocking=True)
+        if i >= Wm:
+            e2e_ev[i - Wm][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(s[0].elapsed_time(s[1]) for s in e2e_ev)
+    if dist:
+        tt = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e_value = world * BATCH / (e2e_ms / K / 1e3)
+
+    peak, peak_kind = measured_peaks()
+    idx_bytes = BATCH * CTX * INDEX_BYTES_PER_TOKEN
+    idx_mean_ms = statistics.mean(idx_ms)
+    achieved = idx_bytes / (idx_mean_ms / 1e3) / 1e9
+    attn_bytes = BATCH * TOPK * ATTN_ROW_BYTES + BATCH * 128 * (576 + 512) * 2
+    combined = (idx_bytes + attn_bytes) / ((idx_mean_ms + statistics.mean(attn_ms)) / 1e3) / 1e9
+    traffic = profile_traffic()
+    out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": Wm,
+           "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "e4m3+bf16 (f32 accumulate)", "data": "synthetic",
+           "config": dict(CONFIG, parallelism=f"requests sharded, {BATCH} per GPU" if world > 1 else "1 GPU"),
+           "roofline": {"bound": "hbm", "kernel": "index_score_tc", "achieved": achieved, "peak": peak,
+                        "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
+                        "algorithmic_bytes_per_launch": idx_bytes,
+                        "indexer_ms": idx_mean_ms, "topk_ms": statistics.mean(topk_ms),
+                        "attn_ms": statistics.mean(attn_ms),
+                        "indexer_plus_attn_GBps": combined, "indexer_plus_attn_frac": combined / peak},
+           "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d_bytes,
+                   "d2h_bytes_per_step": d2h_bytes},
+           "clocks": clk.summary(), "gpu_launches": K * wl.kernels_per_step, "device_status": status}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_oracle_sample(seconds_budget=args.cpu_seconds)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

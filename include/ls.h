@@ -1,0 +1,374 @@
+/*
+ * ls.h -- C ABI of the sparse-attention decode library (sm_100a, NVIDIA B200).
+ *
+ * One decode step of a DSA-style sparse-attention layer, split into the calls a
+ * serving loop makes:
+ *
+ *   ls_index_score        indexer score of every cached token          (a1)
+ *   ls_topk_select        per-request top-k of those scores            (a2)
+ *   ls_block_bound_prune  coarse-to-fine indexer: block bounds, prune,  (a3)
+ *                         exact re-score of survivors, top-k
+ *   ls_hotbuf_resolve     hit/miss of the selection against the HBM    (a4)
+ *                         hot buffer, miss compaction, slot replacement
+ *   ls_gather_misses      copy missed KV rows from pinned host memory  (a5)
+ *   ls_sparse_attn_decode attention over the selected rows only        (a6)
+ *   ls_decode_step        a1 (or a3) -> a2 -> [a4 -> a5] -> a6         (a7)
+ *
+ * Sources.  "LeanSparse: Memory-Efficient Serving for Native Sparse-Attention LLMs"
+ * (abstract): sparse attention limits the history each query reads; indexer keys
+ * and KV are separate caches reused across steps; coarse-to-fine indexing searches
+ * compact representations and retrieves original indexer keys only to refine
+ * candidates.  "XM-Sparse: Pushing the Throughput Frontier of Sparse Attention with
+ * Netpreme X-Mem" (section on the hot buffer): HBM keeps a per-request hot KV buffer
+ * (4,096 tokens) and the indexer-key cache; after each step's selection (2,048 KV)
+ * only selected-but-missed KV is fetched from the full history; (section on the KV
+ * lifecycle) decode fetches only selected-but-missed KV.  The DSA abstract on the
+ * "Related papers: SparseServe" page: attention is restricted to a top-k subset of
+ * the cached entries.  The pages print no formulas; the definitions each call
+ * implements are stated at the call.
+ *
+ * Conventions for every call.
+ *   - All arrays are caller-owned.  Pointers are CUDA device pointers unless a
+ *     field says otherwise.  The library never allocates memory, never frees it,
+ *     and never synchronises the stream inside a compute call.
+ *   - Calls are asynchronous: they validate their arguments on the host, enqueue
+ *     kernels on `stream` and return.  LS_OK means "enqueued".
+ *   - Argument errors are reported before anything is launched
+ *     (LS_ERR_INVALID_ARG / LS_ERR_UNSUPPORTED); a launch failure gives LS_ERR_CUDA.
+ *     ls_get_error_string() then describes the last error of the calling thread.
+ *   - Values that only the device knows (lengths, counts, page ids) are checked in
+ *     the kernels: an out-of-range value is skipped, never dereferenced, and a bit
+ *     is set in the device status word, which ls_check_device_status() reads.
+ *   - Integers are int32 unless named int64; "bf16" and "e4m3" arrays hold the raw
+ *     bit patterns (uint16 / uint8).  Row-major layouts throughout.
+ *   - Pages hold 64 tokens; coarse-to-fine blocks are those same 64-token pages.
+ */
+#ifndef LS_H_
+#define LS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object types as cudaStream_t / cudaEvent_t (and CUstream / CUevent). */
+typedef struct CUstream_st* ls_stream_t;
+typedef struct CUevent_st* ls_event_t;
+
+typedef enum ls_status {
+  LS_OK = 0,
+  LS_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, workspace too small */
+  LS_ERR_UNSUPPORTED = 2,   /* dtype / shape combination that is not built */
+  LS_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+  LS_ERR_DEVICE_STATUS = 4  /* a kernel flagged a problem (see ls_check_device_status) */
+} ls_status;
+
+typedef enum ls_dtype {
+  LS_F32 = 0,
+  LS_BF16 = 1,
+  LS_E4M3 = 2               /* OCP FP8 E4M3 (bias 7, max 448, no inf) */
+} ls_dtype;
+
+/* Device status bits (ls_check_device_status). */
+#define LS_DEV_BOUNDS   0x1u  /* an index or length was out of range and was skipped */
+#define LS_DEV_TIMEOUT  0x2u  /* a bounded wait inside a kernel gave up */
+#define LS_DEV_CAPACITY 0x4u  /* more misses than unpinned hot-buffer slots */
+
+#define LS_PAGE 64            /* tokens per page and per coarse-to-fine block */
+
+/* ------------------------------------------------------------------------------
+ * a1. Indexer score.
+ *
+ *   score[b][s] = key_scale[s] * sum_h (w[b][h] * q_scale[b][h]) * ReLU(q8[b][h] . k8[s])
+ *
+ * for every cached position s < lens[b] of request b.  Because the scales are
+ * positive this equals sum_h w_h * ReLU(q_h . k_s) on the dequantised operands
+ * q_h = q_scale_h * e4m3(q8_h), k_s = key_scale_s * e4m3(k8_s) -- the DSA
+ * lightning-indexer form; the pages name the indexer keys and scores (LeanSparse,
+ * abstract) but print no formula.  Position s of request b lives in physical page
+ * page_table[b][s / 64] at row s % 64 of key_pool.
+ *
+ * Built combinations:
+ *   key_dtype LS_E4M3: heads == 64, dim == 128, w_dtype LS_BF16 or LS_F32; q is
+ *     e4m3 [B,64,128] with q_scale [B,64]; key_pool e4m3 [num_pages,64,128] with
+ *     key_scale [num_pages,64].  tcgen05 fp8 MMA path.
+ *   key_dtype LS_F32: 1 <= heads <= 64, 1 <= dim <= 128, dim % 4 == 0; q, w,
+ *     key_pool f32; q_scale and key_scale must be NULL.  CUDA-core path.
+ * scores[b][s] is written for s < lens[b] only; other entries are left untouched.
+ * key_pool and the q rows must be 16-byte aligned.
+ * --------------------------------------------------------------------------- */
+typedef struct ls_index_score_args {
+  int32_t batch;              /* B >= 1 */
+  int32_t heads;              /* indexer heads H */
+  int32_t dim;                /* indexer head dim D */
+  int32_t max_pages;          /* row stride of page_table */
+  int32_t max_len;            /* row stride of scores; lens[b] <= min(max_len, 64*max_pages) */
+  int32_t key_dtype;          /* ls_dtype: LS_E4M3 or LS_F32 */
+  int32_t w_dtype;            /* ls_dtype: LS_BF16 or LS_F32 */
+  int32_t variant;            /* 0: fastest built kernel; 1: CUDA-core kernel (any key_dtype) */
+  int64_t num_pages;          /* pages in key_pool (page ids must be < num_pages) */
+  const void* q;              /* [B,H,D] */
+  const float* q_scale;       /* [B,H] (e4m3 only) */
+  const void* w;              /* [B,H] head weights */
+  const void* key_pool;       /* [num_pages,64,D] */
+  const float* key_scale;     /* [num_pages,64] (e4m3 only) */
+  const int32_t* page_table;  /* [B,max_pages] */
+  const int32_t* lens;        /* [B] */
+  float* scores;              /* [B,max_len] out */
+} ls_index_score_args;
+
+ls_status ls_index_score(const ls_index_score_args* args, ls_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * a2. Top-k selection.
+ *
+ * For each request, the k positions with the largest score (ties: lower position
+ * first), written to idx[b][0..k) in ascending position order.  If lens[b] < k the
+ * first lens[b] entries are 0..lens[b]-1 and the rest are -1.  sel_score (optional)
+ * receives the score of each selected position (0 for padding).  Comparison is on
+ * IEEE order with -0 == +0; NaN scores are not supported.  The DSA top-k subset
+ * ("Related papers: SparseServe" page, DSA abstract); 2,048 per step in
+ * XM-Sparse's hot-buffer section.
+ * Limits: 1 <= k <= 4096; scores rows 16-byte aligned (max_len % 4 == 0).
+ * --------------------------------------------------------------------------- */
+typedef struct ls_topk_args {
+  int32_t batch;
+  int32_t k;
+  int32_t max_len;            /* row stride of scores */
+  const float* scores;        /* [B,max_len] */
+  const int32_t* lens;        /* [B] */
+  int32_t* idx;               /* [B,k] out */
+  float* sel_score;           /* [B,k] out, may be NULL */
+} ls_topk_args;
+
+ls_status ls_topk_select(const ls_topk_args* args, ls_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * Block summaries (non-timed helper, run when pages are appended).
+ *
+ * For each request and 64-token block j: kmax/kmin per dim over the block's valid
+ * tokens of k = key_scale * e4m3(k8), stored as e4m3 codes times a float32 block
+ * scale bs_j (about amax_j/448, raised by one float32 step when 448*bs_j < amax_j;
+ * 1 for an all-zero block), the max rounded up and the min rounded down in exact
+ * arithmetic, so the stored box contains every key.  Layout: summaries[b][j] =
+ * [kmax codes (D bytes) | kmin codes (D bytes)], block_scale[b][j].
+ * LeanSparse (abstract): "coarse-to-fine indexing searches compact representations".
+ * Requires key_dtype LS_E4M3, dim 128.
+ * --------------------------------------------------------------------------- */
+ls_status ls_build_block_summaries(const ls_index_score_args* keys, uint8_t* summaries,
+                                   float* block_scale, int32_t max_blocks, ls_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * a3. Coarse-to-fine indexer (LeanSparse, abstract: decode can find promising
+ * candidates before comparing their original indexer scores; original indexer
+ * keys are read only for candidate refinement).  Exact: idx equals what
+ * ls_index_score + ls_topk_select return on the same inputs.
+ *
+ *  1. UB[b][j] = bs_j * sum_h w'_h * ReLU(hi_hj) for w'_h >= 0, w'_h * ReLU(lo_hj)
+ *     for w'_h < 0, with w'_h = w_h * q_scale_h and hi/lo = sum_d max/min(q8_hd *
+ *     kmax_jd, q8_hd * kmin_jd) -- an upper bound on every score in block j
+ *     (for w >= 0: sum_h w_h ReLU(sum_d max(q_hd Kmax_jd, q_hd Kmin_jd))).
+ *  2. tau0 = the k-th largest exact score over the ceil(k/64)+1 blocks with the
+ *     largest UB (never above the true k-th score).
+ *  3. survivors = blocks with UB >= tau0 - eps_j, eps_j = eps_rel * M_j, where
+ *     M_j = 448 * bs_j * sum_h |w'_h| * sum_d |e4m3(q8_hd)| bounds |score| in the
+ *     block; the margin absorbs float32 rounding so no true top-k block is lost.
+ *  4. exact scores of the survivors' tokens, then top-k over them.
+ * summaries/block_scale as built by ls_build_block_summaries.  Requires the e4m3
+ * indexer (heads 64, dim 128).  idx/sel_score as in ls_topk_select.  survivors
+ * receives each request's surviving block ids (ascending), n_survivors the count.
+ * Needs a workspace of ls_block_bound_prune_workspace_size() bytes (256-aligned).
+ * --------------------------------------------------------------------------- */
+typedef struct ls_block_bound_prune_args {
+  ls_index_score_args index;  /* a1 inputs; index.scores is ignored */
+  int32_t k;
+  int32_t max_blocks;         /* row stride of summaries/block_scale/survivors;
+                                 >= ceil(lens[b]/64) */
+  float eps_rel;              /* <= 0 selects the default 2^-10 */
+  const uint8_t* summaries;   /* [B,max_blocks,2*128] e4m3 */
+  const float* block_scale;   /* [B,max_blocks] */
+  int32_t* idx;               /* [B,k] out */
+  float* sel_score;           /* [B,k] out, may be NULL */
+  int32_t* survivors;         /* [B,max_blocks] out */
+  int32_t* n_survivors;       /* [B] out */
+  float* ub;                  /* [B,max_blocks] out, may be NULL */
+} ls_block_bound_prune_args;
+
+size_t ls_block_bound_prune_workspace_size(const ls_block_bound_prune_args* args);
+ls_status ls_block_bound_prune(const ls_block_bound_prune_args* args, void* workspace,
+                               size_t workspace_bytes, ls_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * a4. Hot-buffer resolve (XM-Sparse, hot-buffer section: a per-request HBM hot
+ * buffer; after each step's selection only the selected KV that misses it is
+ * fetched).  The pages state no replacement policy; this call implements:
+ *   - selection j (sel[b][j] >= 0) hits when slot_of_pos[b][p] >= 0; its slot is
+ *     pinned for this step;
+ *   - misses are listed in selection order (ascending position) in miss_pos;
+ *   - victims are the unpinned slots, empty slots (pos_of_slot == -1) first in slot
+ *     order, then occupied slots by (recent_score ascending, slot ascending); the
+ *     i-th miss takes the i-th victim (miss_slot[i]); the victim's old position
+ *     leaves the buffer (slot_of_pos = -1) and the miss moves in;
+ *   - sel_slot[b][j] = the slot that holds selection j after the step (-1 padding);
+ *   - recent_score of every selected slot becomes sel_score[b][j].
+ * pos_of_slot / slot_of_pos must be mutually inverse on entry and are on exit.
+ * k <= n_slots <= 4096 guarantees enough unpinned slots; recent_score must not be
+ * NaN.  Only the maps change here: the KV rows move in ls_gather_misses.
+ * --------------------------------------------------------------------------- */
+typedef struct ls_hotbuf_args {
+  int32_t batch;
+  int32_t k;
+  int32_t n_slots;            /* hot-buffer slots per request (<= 4096) */
+  int32_t max_len;            /* row stride of slot_of_pos; positions < max_len */
+  const int32_t* sel;         /* [B,k] selected positions, ascending, -1 padded */
+  const float* sel_score;     /* [B,k] */
+  int32_t* pos_of_slot;       /* [B,n_slots] in/out (-1 = empty) */
+  float* recent_score;        /* [B,n_slots] in/out */
+  int32_t* slot_of_pos;       /* [B,max_len] in/out (-1 = not resident) */
+  int32_t* sel_slot;          /* [B,k] out */
+  int32_t* miss_pos;          /* [B,k] out, -1 padded */
+  int32_t* miss_slot;         /* [B,k] out, -1 padded */
+  int32_t* n_miss;            /* [B] out */
+} ls_hotbuf_args;
+
+ls_status ls_hotbuf_resolve(const ls_hotbuf_args* args, ls_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * a5. Miss gather (XM-Sparse: the full history sits outside HBM; decode fetches
+ * only selected-but-missed KV).  For i < n_miss[b]:
+ *   hbuf[b][miss_slot[b][i]] = host_kv[page_table[b][p/64]][p%64],  p = miss_pos[b][i]
+ * a byte copy of row_bytes per row, read by the SMs straight from pinned host
+ * memory in 16-byte vectors.  host_kv is a DEVICE-ACCESSIBLE address of page-locked
+ * host memory (the pointer returned by cudaHostAlloc / cudaHostGetDevicePointer;
+ * with unified addressing it equals the host pointer).  row_bytes % 16 == 0 and
+ * both bases 16-byte aligned.
+ * --------------------------------------------------------------------------- */
+typedef struct ls_gather_args {
+  int32_t batch;
+  int32_t k;                  /* row stride of miss_pos / miss_slot */
+  int32_t n_slots;
+  int32_t max_pages;
+  int64_t row_bytes;
+  int64_t num_pages;          /* pages in host_kv */
+  const void* host_kv;        /* [num_pages,64,row_bytes] pinned host (device-accessible) */
+  const int32_t* page_table;  /* [B,max_pages] */
+  const int32_t* miss_pos;    /* [B,k] */
+  const int32_t* miss_slot;   /* [B,k] */
+  const int32_t* n_miss;      /* [B] */
+  void* hbuf;                 /* [B,n_slots,row_bytes] */
+} ls_gather_args;
+
+ls_status ls_gather_misses(const ls_gather_args* args, ls_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * a6. Sparse attention decode over the selected rows (LeanSparse, abstract:
+ * sparse attention limits the history read by each query).  Per request b and
+ * head h, over the selected rows j (sel[b][j] >= 0):
+ *   s_j = softmax_scale * q[b][h] . K_j[0:dk];  o[b][h] = sum_j softmax(s)_j V_j[0:dv];
+ *   lse[b][h] = log sum_j exp(s_j)   (natural log; -inf and o = 0 if nothing selected)
+ * Row address: LS_ROWS_PAGED: row = page_table[b][p/64]*64 + p%64 for position p;
+ *              LS_ROWS_SLOTS: row = b*n_slots + slot.
+ * K_j = k_rows + row*row_stride, V_j = v_rows + row*row_stride (elements).
+ * Built: LS_BF16 MLA-absorbed (heads 128, dk 576, dv 512, one latent KV head, V =
+ * the first 512 dims: pass v_rows == k_rows), tcgen05 bf16 MMA path, o bf16;
+ *        LS_F32 (heads <= 64, dk, dv <= 128, multiples of 4), CUDA-core path, o f32.
+ * Needs a workspace of ls_sparse_attn_workspace_size() bytes (256-aligned).
+ * --------------------------------------------------------------------------- */
+#define LS_ROWS_PAGED 0
+#define LS_ROWS_SLOTS 1
+
+typedef struct ls_sparse_attn_args {
+  int32_t batch;
+  int32_t heads;
+  int32_t dk;
+  int32_t dv;
+  int32_t k;                  /* row stride of sel */
+  int32_t dtype;              /* ls_dtype: LS_BF16 or LS_F32 */
+  int32_t variant;            /* 0: fastest built kernel; 1: CUDA-core kernel (any dtype) */
+  float softmax_scale;
+  int32_t addressing;         /* LS_ROWS_PAGED or LS_ROWS_SLOTS */
+  int32_t max_pages;          /* PAGED: row stride of page_table */
+  int32_t n_slots;            /* SLOTS: slots per request */
+  int64_t row_stride;         /* elements between consecutive rows (>= dk, % 8 == 0) */
+  int64_t num_rows;           /* rows addressable from k_rows / v_rows */
+  const void* q;              /* [B,heads,dk] */
+  const void* k_rows;
+  const void* v_rows;
+  const int32_t* page_table;  /* PAGED: [B,max_pages] */
+  const int32_t* sel;         /* [B,k] positions (PAGED) or slots (SLOTS); -1 skipped */
+  void* o;                    /* [B,heads,dv] out */
+  float* lse;                 /* [B,heads] out */
+} ls_sparse_attn_args;
+
+size_t ls_sparse_attn_workspace_size(const ls_sparse_attn_args* args);
+ls_status ls_sparse_attn_decode(const ls_sparse_attn_args* args, void* workspace,
+                                size_t workspace_bytes, ls_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * a7. One decode step: indexer (or coarse-to-fine indexer) -> top-k -> [hot-buffer
+ * resolve -> miss gather] -> sparse attention, all on `stream`, with no allocation
+ * (the caller provides the workspace) and no host synchronisation.
+ *
+ * index:   a1 inputs; index.scores may be NULL (then the scores live in workspace).
+ * c2f:     use_c2f != 0 selects a3 (summaries required).
+ * attn:    a6 inputs; attn.sel / attn.addressing / attn.k are set by the step:
+ *          without the hot buffer rows come from attn.k_rows through
+ *          index.page_table (paged KV pool in HBM); with it (use_hotbuf != 0) rows
+ *          come from the hot buffer `hbuf` through the resolved slots.
+ * hot buffer: state arrays as in a4, host history as in a5 (uses index.page_table).
+ * idx / sel_score: optional outputs of the selection.
+ * events: optional; when non-NULL, events[i] is recorded on `stream` before stage
+ *   i (0 indexer, 1 top-k, 2 resolve, 3 gather, 4 attention) and events[5] after
+ *   the last stage, so a caller can time each stage.
+ * --------------------------------------------------------------------------- */
+typedef struct ls_decode_step_args {
+  ls_index_score_args index;
+  int32_t k;
+  int32_t use_c2f;
+  int32_t max_blocks;
+  float eps_rel;
+  const uint8_t* summaries;
+  const float* block_scale;
+  int32_t* survivors;         /* c2f: [B,max_blocks] out, may be NULL (workspace) */
+  int32_t* n_survivors;       /* c2f: [B] out, may be NULL (workspace) */
+  ls_sparse_attn_args attn;
+  int32_t use_hotbuf;
+  int32_t n_slots;
+  int32_t* pos_of_slot;
+  float* recent_score;
+  int32_t* slot_of_pos;       /* [B,index.max_len] */
+  const void* host_kv;        /* device-accessible pinned host history [num_pages,64,row_bytes] */
+  int64_t host_num_pages;
+  void* hbuf;                 /* [B,n_slots,row_bytes] */
+  int32_t* n_miss;            /* [B] out, may be NULL (workspace) */
+  int32_t* idx;               /* [B,k] out, may be NULL (workspace) */
+  float* sel_score;           /* [B,k] out, may be NULL (workspace) */
+  ls_event_t* events;         /* NULL or 6 events */
+} ls_decode_step_args;
+
+size_t ls_decode_step_workspace_size(const ls_decode_step_args* args);
+ls_status ls_decode_step(const ls_decode_step_args* args, void* workspace,
+                         size_t workspace_bytes, ls_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * Diagnostics.
+ * --------------------------------------------------------------------------- */
+/* Message of the calling thread's last error (empty string if none). */
+const char* ls_get_error_string(void);
+
+/* Synchronises `stream`, returns the device status bits raised since the last
+ * check in *flags (may be NULL) and clears them.  LS_OK when no bit was set,
+ * LS_ERR_DEVICE_STATUS otherwise.  The status word is per device and shared by all
+ * streams. */
+ls_status ls_check_device_status(ls_stream_t stream, uint32_t* flags);
+
+/* Library version string. */
+const char* ls_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LS_H_ */

@@ -1,0 +1,714 @@
+// Host side of the C ABI declared in include/ls.h: argument validation, launch
+// configuration, TMA descriptors, workspace carving and the decode-step orchestration.
+// The kernels are in the .cuh files included below (one translation unit, so the
+// device status word is a single symbol).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "attn.cuh"
+#include "c2f.cuh"
+#include "common.cuh"
+#include "hotbuf.cuh"
+#include "index_score.cuh"
+#include "topk.cuh"
+
+#define LS_VERSION_STRING "sparse_attention_decode_ls_b200 0.1 (sm_100a)"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+ls_status fail(ls_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+ls_status ok() {
+  g_last_error.clear();
+  return LS_OK;
+}
+
+ls_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(LS_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return LS_OK;
+}
+
+#define LS_REQUIRE(cond, ...)                                   \
+  do {                                                          \
+    if (!(cond)) return fail(LS_ERR_INVALID_ARG, __VA_ARGS__);  \
+  } while (0)
+#define LS_TRY(expr)                   \
+  do {                                 \
+    ls_status _s = (expr);             \
+    if (_s != LS_OK) return _s;        \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// ---- per-device cached properties -------------------------------------------------
+int device_sms() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) dev = 0;
+  int v = cache[dev].load();
+  if (v <= 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cache[dev].store(v);
+  }
+  return v;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device.
+template <typename K>
+cudaError_t allow_smem(K kernel, int bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load() & bit) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit);
+  return e;
+}
+
+// ---- TMA descriptor ----------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2D byte tensor [rows][inner] with row stride `stride` bytes; boxes of 128 bytes x 64
+// rows, 128-byte swizzle.
+ls_status make_tmap_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t stride) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {stride};
+  cuuint32_t box[2] = {128, 64};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return LS_OK;
+}
+
+// ---- indexer launches ----------------------------------------------------------------
+ls_status validate_index(const ls_index_score_args* a, bool need_scores) {
+  LS_REQUIRE(a, "args is NULL");
+  LS_REQUIRE(a->batch >= 1, "batch must be >= 1");
+  LS_REQUIRE(a->max_pages >= 1 && a->max_len >= 1, "max_pages and max_len must be >= 1");
+  LS_REQUIRE(a->num_pages >= 1, "num_pages must be >= 1");
+  LS_REQUIRE(a->q && a->w && a->key_pool && a->page_table && a->lens, "a required pointer is NULL");
+  LS_REQUIRE(!need_scores || a->scores, "scores is NULL");
+  LS_REQUIRE(a->w_dtype == LS_BF16 || a->w_dtype == LS_F32, "w_dtype must be LS_BF16 or LS_F32");
+  LS_REQUIRE(a->variant == 0 || a->variant == 1, "variant must be 0 or 1");
+  if (a->key_dtype == LS_E4M3) {
+    if (a->heads != 64 || a->dim != 128)
+      return fail(LS_ERR_UNSUPPORTED, "e4m3 indexer is built for 64 heads x 128 dims (got %d x %d)", a->heads,
+                  a->dim);
+    LS_REQUIRE(a->q_scale && a->key_scale, "q_scale and key_scale are required for e4m3 keys");
+    LS_REQUIRE(aligned16(a->q) && aligned16(a->key_pool), "q and key_pool must be 16-byte aligned");
+  } else if (a->key_dtype == LS_F32) {
+    if (a->heads < 1 || a->heads > 64 || a->dim < 1 || a->dim > 128 || (a->dim & 3))
+      return fail(LS_ERR_UNSUPPORTED, "f32 indexer: heads in [1,64], dim in [4,128] multiple of 4");
+    LS_REQUIRE(!a->q_scale && !a->key_scale, "q_scale/key_scale must be NULL for f32 keys");
+  } else {
+    return fail(LS_ERR_UNSUPPORTED, "key_dtype must be LS_E4M3 or LS_F32");
+  }
+  return LS_OK;
+}
+
+std::atomic<uint64_t> g_smem_idx_simt_f32{0}, g_smem_idx_simt_e4m3{0}, g_smem_idx_tc{0}, g_smem_bound_tc{0};
+
+ls_status launch_index_simt(const ls_index_score_args* a, cudaStream_t st) {
+  ls::IdxSimtParams p{};
+  p.B = a->batch; p.H = a->heads; p.D = a->dim; p.max_pages = a->max_pages; p.max_len = a->max_len;
+  p.num_pages = a->num_pages; p.q = a->q; p.qs = a->q_scale; p.w = a->w; p.w_bf16 = a->w_dtype == LS_BF16;
+  p.keys = a->key_pool; p.ks = a->key_scale; p.page_table = a->page_table; p.lens = a->lens; p.out = a->scores;
+  const int smem = (p.H * p.D + 64 * (p.D + 1) + p.H + 256) * 4;
+  const int smem_max = (64 * 128 + 64 * 129 + 64 + 256) * 4;
+  const int gx = std::min(a->max_pages, (a->max_len + 63) / 64);
+  dim3 grid(gx, a->batch);
+  if (a->key_dtype == LS_E4M3) {
+    if (allow_smem(ls::index_score_simt<true>, smem_max, g_smem_idx_simt_e4m3) != cudaSuccess)
+      return check_launch("index_score_simt attribute");
+    ls::index_score_simt<true><<<grid, 256, smem, st>>>(p);
+  } else {
+    if (allow_smem(ls::index_score_simt<false>, smem_max, g_smem_idx_simt_f32) != cudaSuccess)
+      return check_launch("index_score_simt attribute");
+    ls::index_score_simt<false><<<grid, 256, smem, st>>>(p);
+  }
+  return check_launch("index_score_simt");
+}
+
+// tcgen05 tile engine over keys (mode 0) or block summaries (mode 1).
+ls_status launch_index_tc(const ls_index_score_args* a, int mode, const int* unit_list, const int* unit_count,
+                          int list_stride, float* out, long long out_stride, const uint8_t* summ,
+                          const float* bscale, int max_blocks, float* out_plain, float eps_rel, cudaStream_t st) {
+  ls::IdxTcParams p{};
+  p.mode = mode; p.B = a->batch; p.max_pages = a->max_pages; p.max_len = a->max_len; p.max_blocks = max_blocks;
+  p.num_pages = a->num_pages; p.q8 = (const uint8_t*)a->q; p.qs = a->q_scale; p.w = a->w;
+  p.w_bf16 = a->w_dtype == LS_BF16; p.page_table = a->page_table; p.lens = a->lens;
+  p.unit_list = unit_list; p.unit_count = unit_count; p.list_stride = list_stride;
+  p.out = out; p.out_stride = out_stride; p.out_plain = out_plain; p.eps_rel = eps_rel;
+  CUtensorMap tmap;
+  const int sms = device_sms();
+  long long max_units;
+  if (mode == 0) {
+    p.row_scale = a->key_scale;
+    LS_TRY(make_tmap_u8(&tmap, a->key_pool, 128, (uint64_t)a->num_pages * 64, 128));
+    max_units = unit_list ? list_stride : (a->max_len + 63) / 64;
+  } else {
+    p.row_scale = bscale;
+    LS_TRY(make_tmap_u8(&tmap, summ, 256, (uint64_t)a->batch * max_blocks, 256));
+    max_units = (max_blocks + 63) / 64;
+  }
+  const long long max_tiles = (max_units + 1) / 2;
+  const int per_sm = (mode == 0) ? 2 : 1;
+  long long c = std::max<long long>(1, (long long)per_sm * sms / a->batch);
+  c = std::min<long long>(c, std::max<long long>(1, max_tiles));
+  p.ctas_per_req = (int)c;
+  dim3 grid((unsigned)c, a->batch);
+  if (mode == 0) {
+    using C = ls::IdxTc<1, 64>;
+    if (allow_smem(ls::index_score_tc<1, 64>, C::kSmem, g_smem_idx_tc) != cudaSuccess)
+      return check_launch("index_score_tc attribute");
+    ls::index_score_tc<1, 64><<<grid, C::kThreads, C::kSmem, st>>>(p, tmap);
+  } else {
+    using C = ls::IdxTc<2, 128>;
+    if (allow_smem(ls::index_score_tc<2, 128>, C::kSmem, g_smem_bound_tc) != cudaSuccess)
+      return check_launch("block_bound_tc attribute");
+    ls::index_score_tc<2, 128><<<grid, C::kThreads, C::kSmem, st>>>(p, tmap);
+  }
+  return check_launch(mode == 0 ? "index_score_tc" : "block_bound_tc");
+}
+
+// ---- top-k launch -------------------------------------------------------------------
+std::atomic<uint64_t> g_smem_topk{0};
+constexpr int kTopkCluster = 8;
+
+ls_status launch_topk(int B, int k, const float* scores, int stride, const int* lens, int len_mul, int len_div,
+                      int len_limit, const int* unit_list, int list_stride, int* idx, float* sel, float* thr,
+                      cudaStream_t st) {
+  ls::TopkParams p{};
+  p.B = B; p.k = k; p.stride = stride; p.scores = scores; p.lens = lens; p.len_mul = len_mul;
+  p.len_div = len_div; p.len_limit = len_limit; p.unit_list = unit_list; p.list_stride = list_stride;
+  p.idx = idx; p.sel = sel; p.thr = thr;
+  const int lc = (((len_limit + kTopkCluster - 1) / kTopkCluster) + 3) & ~3;
+  p.cache_keys = lc <= ls::kTopkCacheKeys ? lc : 0;
+  const int smem = p.cache_keys * 4;
+  if (allow_smem(ls::topk_cluster<kTopkCluster>, ls::kTopkCacheKeys * 4, g_smem_topk) != cudaSuccess)
+    return check_launch("topk attribute");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(B * kTopkCluster);
+  cfg.blockDim = dim3(ls::kTopkThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kTopkCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, ls::topk_cluster<kTopkCluster>, p);
+  if (e != cudaSuccess) return fail(LS_ERR_CUDA, "topk_cluster: %s", cudaGetErrorString(e));
+  return check_launch("topk_cluster");
+}
+
+// ---- attention ------------------------------------------------------------------------
+int attn_nsplit(const ls_sparse_attn_args* a) {
+  if (a->dtype != LS_BF16 || a->variant != 0) return 1;
+  const int tiles = (a->k + ls::mla::N - 1) / ls::mla::N;
+  int ns = device_sms() / (2 * a->batch);
+  ns = std::max(1, std::min(ns, (tiles + 1) / 2));
+  return ns;
+}
+
+size_t attn_ws_bytes(const ls_sparse_attn_args* a) {
+  const int ns = attn_nsplit(a);
+  if (ns <= 1) return 0;
+  return align256((size_t)a->batch * ns * a->heads * a->dv * 4) + align256((size_t)a->batch * ns * a->heads * 8);
+}
+
+ls_status validate_attn(const ls_sparse_attn_args* a, bool need_sel) {
+  LS_REQUIRE(a, "args is NULL");
+  LS_REQUIRE(a->batch >= 1 && a->k >= 1 && a->k <= 4096, "batch >= 1 and 1 <= k <= 4096 required");
+  LS_REQUIRE(a->q && a->k_rows && a->v_rows && a->o && a->lse, "a required pointer is NULL");
+  LS_REQUIRE(!need_sel || a->sel, "sel is NULL");
+  LS_REQUIRE(a->addressing == LS_ROWS_PAGED || a->addressing == LS_ROWS_SLOTS, "bad addressing mode");
+  LS_REQUIRE(a->addressing != LS_ROWS_PAGED || (a->page_table && a->max_pages >= 1),
+             "paged addressing needs page_table and max_pages");
+  LS_REQUIRE(a->addressing != LS_ROWS_SLOTS || a->n_slots >= 1, "slot addressing needs n_slots");
+  LS_REQUIRE(a->num_rows >= 1, "num_rows must be >= 1");
+  LS_REQUIRE(a->variant == 0 || a->variant == 1, "variant must be 0 or 1");
+  LS_REQUIRE(std::isfinite(a->softmax_scale), "softmax_scale must be finite");
+  if (a->dtype == LS_BF16) {
+    if (a->variant == 0 && (a->heads != 128 || a->dk != 576 || a->dv != 512))
+      return fail(LS_ERR_UNSUPPORTED, "bf16 tensor-core attention is built for 128 heads, dk 576, dv 512");
+    if (a->variant == 0) {
+      LS_REQUIRE(a->k_rows == a->v_rows, "MLA attention reads V from the latent rows (v_rows == k_rows)");
+      LS_REQUIRE(a->row_stride >= 576 && (a->row_stride % 8) == 0, "row_stride must be >= 576 and % 8 == 0");
+      LS_REQUIRE(aligned16(a->k_rows) && aligned16(a->q), "k_rows and q must be 16-byte aligned");
+    }
+  } else if (a->dtype != LS_F32) {
+    return fail(LS_ERR_UNSUPPORTED, "attention dtype must be LS_BF16 or LS_F32");
+  }
+  if (a->variant == 1 || a->dtype == LS_F32) {
+    LS_REQUIRE(a->heads >= 1 && a->dk >= 1 && a->dv >= 1 && a->dk <= 1024 && a->dv <= 1024,
+               "CUDA-core attention: heads >= 1, 1 <= dk, dv <= 1024");
+    LS_REQUIRE(a->row_stride >= std::max(a->dk, a->dv), "row_stride must cover dk and dv");
+  }
+  return LS_OK;
+}
+
+std::atomic<uint64_t> g_smem_attn_tc{0}, g_smem_attn_simt_f{0}, g_smem_attn_simt_b{0};
+
+ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressing, const int* page_table,
+                      int max_pages, int n_slots, const void* rows, long long num_rows, void* ws, size_t ws_bytes,
+                      cudaStream_t st) {
+  ls::AttnParams p{};
+  p.B = a->batch; p.H = a->heads; p.dk = a->dk; p.dv = a->dv; p.k = a->k; p.scale = a->softmax_scale;
+  p.addressing = addressing; p.max_pages = max_pages; p.n_slots = n_slots; p.row_stride = a->row_stride;
+  p.num_rows = num_rows; p.q = a->q; p.krows = rows ? rows : a->k_rows; p.vrows = rows ? rows : a->v_rows;
+  p.page_table = page_table; p.sel = sel; p.o = a->o; p.lse = a->lse;
+  if (a->dtype == LS_BF16 && a->variant == 0) {
+    const int ns = attn_nsplit(a);
+    p.nsplit = ns;
+    if (ns > 1) {
+      const size_t need = attn_ws_bytes(a);
+      LS_REQUIRE(ws && ws_bytes >= need, "attention workspace too small (%zu < %zu bytes)", ws_bytes, need);
+      LS_REQUIRE(((uintptr_t)ws & 255) == 0, "workspace must be 256-byte aligned");
+      p.part_o = (float*)ws;
+      p.part_ml = (float*)((char*)ws + align256((size_t)a->batch * ns * a->heads * a->dv * 4));
+    }
+    if (allow_smem(ls::attn_mla_tc, ls::mla::kSmem, g_smem_attn_tc) != cudaSuccess)
+      return check_launch("attn_mla_tc attribute");
+    ls::attn_mla_tc<<<dim3(2 * ns, a->batch), ls::mla::kThreads, ls::mla::kSmem, st>>>(p);
+    LS_TRY(check_launch("attn_mla_tc"));
+    if (ns > 1) {
+      ls::attn_combine<<<(a->batch * ls::mla::H + 3) / 4, 128, 0, st>>>(p);
+      LS_TRY(check_launch("attn_combine"));
+    }
+    return LS_OK;
+  }
+  const int smem = (((a->dk + 1) & ~1) + ((a->k + 1) & ~1)) * 4 + a->k * 8;
+  LS_REQUIRE(smem <= 200 * 1024, "CUDA-core attention: dk + 3k too large for shared memory");
+  dim3 grid(a->heads, a->batch);
+  if (a->dtype == LS_BF16) {
+    if (allow_smem(ls::attn_simt<true>, 200 * 1024, g_smem_attn_simt_b) != cudaSuccess)
+      return check_launch("attn_simt attribute");
+    ls::attn_simt<true><<<grid, 256, smem, st>>>(p);
+  } else {
+    if (allow_smem(ls::attn_simt<false>, 200 * 1024, g_smem_attn_simt_f) != cudaSuccess)
+      return check_launch("attn_simt attribute");
+    ls::attn_simt<false><<<grid, 256, smem, st>>>(p);
+  }
+  return check_launch("attn_simt");
+}
+
+// ---- hot buffer -------------------------------------------------------------------------
+std::atomic<uint64_t> g_smem_hb{0};
+
+ls_status validate_hotbuf(const ls_hotbuf_args* a) {
+  LS_REQUIRE(a, "args is NULL");
+  LS_REQUIRE(a->batch >= 1 && a->k >= 1, "batch and k must be >= 1");
+  LS_REQUIRE(a->n_slots >= 1 && a->n_slots <= ls::kHbMaxSlots, "n_slots must be in [1, 4096]");
+  LS_REQUIRE(a->k <= a->n_slots, "k must not exceed n_slots (every selection needs a slot)");
+  LS_REQUIRE(a->max_len >= 1, "max_len must be >= 1");
+  LS_REQUIRE(a->sel && a->sel_score && a->pos_of_slot && a->recent_score && a->slot_of_pos && a->sel_slot &&
+                 a->miss_pos && a->miss_slot && a->n_miss,
+             "a required pointer is NULL");
+  return LS_OK;
+}
+
+ls_status launch_hotbuf(const ls_hotbuf_args* a, cudaStream_t st) {
+  ls::HotbufParams p{};
+  p.B = a->batch; p.k = a->k; p.n_slots = a->n_slots; p.max_len = a->max_len; p.sel = a->sel;
+  p.sel_score = a->sel_score; p.pos_of_slot = a->pos_of_slot; p.recent = a->recent_score;
+  p.slot_of_pos = a->slot_of_pos; p.sel_slot = a->sel_slot; p.miss_pos = a->miss_pos; p.miss_slot = a->miss_slot;
+  p.n_miss = a->n_miss;
+  int pow2 = 1;
+  while (pow2 < a->n_slots) pow2 <<= 1;
+  const int smem = pow2 * 8;
+  if (allow_smem(ls::hotbuf_resolve_kernel, ls::kHbMaxSlots * 8, g_smem_hb) != cudaSuccess)
+    return check_launch("hotbuf attribute");
+  ls::hotbuf_resolve_kernel<<<a->batch, ls::kHbThreads, smem, st>>>(p);
+  return check_launch("hotbuf_resolve");
+}
+
+ls_status validate_gather(const ls_gather_args* a) {
+  LS_REQUIRE(a, "args is NULL");
+  LS_REQUIRE(a->batch >= 1 && a->k >= 1 && a->n_slots >= 1 && a->max_pages >= 1 && a->num_pages >= 1,
+             "batch, k, n_slots, max_pages, num_pages must be >= 1");
+  LS_REQUIRE(a->row_bytes >= 16 && (a->row_bytes % 16) == 0, "row_bytes must be a positive multiple of 16");
+  LS_REQUIRE(a->host_kv && a->page_table && a->miss_pos && a->miss_slot && a->n_miss && a->hbuf,
+             "a required pointer is NULL");
+  LS_REQUIRE(aligned16(a->host_kv) && aligned16(a->hbuf), "host_kv and hbuf must be 16-byte aligned");
+  return LS_OK;
+}
+
+ls_status launch_gather(const ls_gather_args* a, cudaStream_t st) {
+  ls::GatherParams p{};
+  p.B = a->batch; p.k = a->k; p.n_slots = a->n_slots; p.max_pages = a->max_pages; p.row_bytes = a->row_bytes;
+  p.num_pages = a->num_pages; p.host = (const char*)a->host_kv; p.page_table = a->page_table;
+  p.miss_pos = a->miss_pos; p.miss_slot = a->miss_slot; p.n_miss = a->n_miss; p.hbuf = (char*)a->hbuf;
+  const int rows_per_cta = 8 * 4;
+  int g = (a->k + rows_per_cta - 1) / rows_per_cta;
+  g = std::max(1, std::min(g, (8 * device_sms()) / a->batch + 1));
+  ls::gather_misses_kernel<<<dim3(g, a->batch), 256, 0, st>>>(p);
+  return check_launch("gather_misses");
+}
+
+// ---- coarse-to-fine ---------------------------------------------------------------------
+struct C2fLayout {
+  int nb0, ub_stride;
+  size_t off_ub, off_blk, off_cnt1, off_clen1, off_tau, off_clen2, off_nsurv, off_surv, off_c1, off_c2, total;
+};
+
+C2fLayout c2f_layout(const ls_block_bound_prune_args* a) {
+  C2fLayout l{};
+  const int B = a->index.batch;
+  l.nb0 = std::min(a->max_blocks, (a->k + 63) / 64 + 1);
+  l.ub_stride = (a->max_blocks + 3) & ~3;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t r = o; o += align256(bytes); return r; };
+  l.off_ub = take((size_t)B * l.ub_stride * 4);
+  l.off_blk = take((size_t)B * l.nb0 * 4);
+  l.off_cnt1 = take((size_t)B * 4);
+  l.off_clen1 = take((size_t)B * 4);
+  l.off_tau = take((size_t)B * 4);
+  l.off_clen2 = take((size_t)B * 4);
+  l.off_nsurv = take((size_t)B * 4);
+  l.off_surv = take((size_t)B * a->max_blocks * 4);
+  l.off_c1 = take((size_t)B * l.nb0 * 64 * 4);
+  l.off_c2 = take((size_t)B * a->max_blocks * 64 * 4);
+  l.total = o;
+  return l;
+}
+
+ls_status validate_c2f(const ls_block_bound_prune_args* a) {
+  LS_REQUIRE(a, "args is NULL");
+  LS_TRY(validate_index(&a->index, false));
+  if (a->index.key_dtype != LS_E4M3) return fail(LS_ERR_UNSUPPORTED, "coarse-to-fine needs e4m3 indexer keys");
+  LS_REQUIRE(a->k >= 1 && a->k <= 4096, "1 <= k <= 4096 required");
+  LS_REQUIRE(a->max_blocks >= 1, "max_blocks must be >= 1");
+  LS_REQUIRE((long long)a->max_blocks * 64 <= (1ll << 30), "max_blocks too large");
+  LS_REQUIRE(a->summaries && a->block_scale && a->idx, "summaries, block_scale and idx are required");
+  LS_REQUIRE(aligned16(a->summaries), "summaries must be 16-byte aligned");
+  return LS_OK;
+}
+
+ls_status run_c2f(const ls_block_bound_prune_args* a, void* ws, size_t ws_bytes, int* survivors, int* n_surv,
+                  ls_event_t ev_topk, cudaStream_t st) {
+  const C2fLayout l = c2f_layout(a);
+  LS_REQUIRE(ws && ws_bytes >= l.total, "coarse-to-fine workspace too small (%zu < %zu bytes)", ws_bytes, l.total);
+  LS_REQUIRE(((uintptr_t)ws & 255) == 0, "workspace must be 256-byte aligned");
+  char* w = (char*)ws;
+  float* ub = (float*)(w + l.off_ub);
+  int* blk = (int*)(w + l.off_blk);
+  int* cnt1 = (int*)(w + l.off_cnt1);
+  int* clen1 = (int*)(w + l.off_clen1);
+  float* tau = (float*)(w + l.off_tau);
+  int* clen2 = (int*)(w + l.off_clen2);
+  if (!n_surv) n_surv = (int*)(w + l.off_nsurv);
+  if (!survivors) survivors = (int*)(w + l.off_surv);
+  float* c1 = (float*)(w + l.off_c1);
+  float* c2 = (float*)(w + l.off_c2);
+  const ls_index_score_args* ix = &a->index;
+  const int B = ix->batch;
+  const float eps = a->eps_rel > 0.f ? a->eps_rel : 1.0f / 1024.0f;
+  // 1. block bounds (+ margin) over the summaries
+  LS_TRY(launch_index_tc(ix, 1, nullptr, nullptr, 0, ub, l.ub_stride, a->summaries, a->block_scale, a->max_blocks,
+                         a->ub, eps, st));
+  // 2. the blocks with the largest bounds
+  LS_TRY(launch_topk(B, l.nb0, ub, l.ub_stride, ix->lens, 1, 64, a->max_blocks, nullptr, 0, blk, nullptr, nullptr,
+                     st));
+  ls::c2f_phase1_kernel<<<(B + 127) / 128, 128, 0, st>>>(B, l.nb0, ix->lens, blk, cnt1, clen1);
+  LS_TRY(check_launch("c2f_phase1"));
+  // 3. their exact scores; tau0 = the k-th largest
+  LS_TRY(launch_index_tc(ix, 0, blk, cnt1, l.nb0, c1, (long long)l.nb0 * 64, nullptr, nullptr, 0, nullptr, 0.f,
+                         st));
+  LS_TRY(launch_topk(B, a->k, c1, l.nb0 * 64, clen1, 1, 1, l.nb0 * 64, nullptr, 0, nullptr, nullptr, tau, st));
+  // 4. survivors
+  ls::c2f_survivors_kernel<<<B, 1024, 0, st>>>(B, a->max_blocks, l.ub_stride, ix->lens, ub, tau, survivors, n_surv,
+                                               clen2);
+  LS_TRY(check_launch("c2f_survivors"));
+  // 5. exact scores of the survivors, then the top-k over them
+  LS_TRY(launch_index_tc(ix, 0, survivors, n_surv, a->max_blocks, c2, (long long)a->max_blocks * 64, nullptr,
+                         nullptr, 0, nullptr, 0.f, st));
+  if (ev_topk) cudaEventRecord((cudaEvent_t)ev_topk, st);
+  LS_TRY(launch_topk(B, a->k, c2, a->max_blocks * 64, clen2, 1, 1, a->max_blocks * 64, survivors, a->max_blocks,
+                     a->idx, a->sel_score, nullptr, st));
+  return LS_OK;
+}
+
+// ---- decode step workspace ------------------------------------------------------------
+struct StepLayout {
+  size_t off_scores, off_idx, off_sel, off_selslot, off_mpos, off_mslot, off_nmiss, off_attn, off_c2f, total;
+};
+
+ls_block_bound_prune_args step_c2f_args(const ls_decode_step_args* a, int* idx, float* sel) {
+  ls_block_bound_prune_args c{};
+  c.index = a->index;
+  c.k = a->k;
+  c.max_blocks = a->max_blocks;
+  c.eps_rel = a->eps_rel;
+  c.summaries = a->summaries;
+  c.block_scale = a->block_scale;
+  c.idx = idx;
+  c.sel_score = sel;
+  c.survivors = a->survivors;
+  c.n_survivors = a->n_survivors;
+  c.ub = nullptr;
+  return c;
+}
+
+ls_sparse_attn_args step_attn_args(const ls_decode_step_args* a) {
+  ls_sparse_attn_args t = a->attn;
+  t.batch = a->index.batch;
+  t.k = a->k;
+  return t;
+}
+
+StepLayout step_layout(const ls_decode_step_args* a) {
+  StepLayout l{};
+  const int B = a->index.batch, k = a->k;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t r = o; o += align256(bytes); return r; };
+  l.off_scores = take(a->use_c2f ? 0 : (size_t)B * a->index.max_len * 4);
+  l.off_idx = take((size_t)B * k * 4);
+  l.off_sel = take((size_t)B * k * 4);
+  l.off_selslot = take(a->use_hotbuf ? (size_t)B * k * 4 : 0);
+  l.off_mpos = take(a->use_hotbuf ? (size_t)B * k * 4 : 0);
+  l.off_mslot = take(a->use_hotbuf ? (size_t)B * k * 4 : 0);
+  l.off_nmiss = take(a->use_hotbuf ? (size_t)B * 4 : 0);
+  ls_sparse_attn_args t = step_attn_args(a);
+  l.off_attn = take(attn_ws_bytes(&t));
+  if (a->use_c2f) {
+    ls_block_bound_prune_args c = step_c2f_args(a, nullptr, nullptr);
+    l.off_c2f = take(c2f_layout(&c).total);
+  } else {
+    l.off_c2f = o;
+  }
+  l.total = o;
+  return l;
+}
+
+}  // namespace
+
+// =========================================================================================
+// C ABI
+// =========================================================================================
+extern "C" {
+
+const char* ls_version(void) { return LS_VERSION_STRING; }
+
+const char* ls_get_error_string(void) { return g_last_error.c_str(); }
+
+ls_status ls_check_device_status(ls_stream_t stream, uint32_t* flags) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return fail(LS_ERR_CUDA, "cudaStreamSynchronize: %s", cudaGetErrorString(e));
+  unsigned int v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, ls::g_status, sizeof(v));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(ls::g_status, &zero, sizeof(zero));
+  if (e != cudaSuccess) return fail(LS_ERR_CUDA, "device status: %s", cudaGetErrorString(e));
+  if (flags) *flags = v;
+  if (v) return fail(LS_ERR_DEVICE_STATUS, "device status bits 0x%x", v);
+  return ok();
+}
+
+ls_status ls_index_score(const ls_index_score_args* args, ls_stream_t stream) {
+  LS_TRY(validate_index(args, true));
+  cudaStream_t st = (cudaStream_t)stream;
+  if (args->key_dtype == LS_E4M3 && args->variant == 0) {
+    LS_TRY(launch_index_tc(args, 0, nullptr, nullptr, 0, args->scores, args->max_len, nullptr, nullptr, 0, nullptr,
+                           0.f, st));
+  } else {
+    LS_TRY(launch_index_simt(args, st));
+  }
+  return ok();
+}
+
+ls_status ls_topk_select(const ls_topk_args* a, ls_stream_t stream) {
+  LS_REQUIRE(a, "args is NULL");
+  LS_REQUIRE(a->batch >= 1 && a->k >= 1 && a->k <= 4096, "batch >= 1 and 1 <= k <= 4096 required");
+  LS_REQUIRE(a->max_len >= 1 && (a->max_len % 4) == 0, "max_len must be a positive multiple of 4");
+  LS_REQUIRE(a->scores && a->lens && a->idx, "scores, lens and idx are required");
+  LS_REQUIRE(aligned16(a->scores), "scores must be 16-byte aligned");
+  LS_TRY(launch_topk(a->batch, a->k, a->scores, a->max_len, a->lens, 1, 1, a->max_len, nullptr, 0, a->idx,
+                     a->sel_score, nullptr, (cudaStream_t)stream));
+  return ok();
+}
+
+ls_status ls_build_block_summaries(const ls_index_score_args* keys, uint8_t* summaries, float* block_scale,
+                                   int32_t max_blocks, ls_stream_t stream) {
+  LS_TRY(validate_index(keys, false));
+  if (keys->key_dtype != LS_E4M3) return fail(LS_ERR_UNSUPPORTED, "summaries need e4m3 keys");
+  LS_REQUIRE(summaries && block_scale && max_blocks >= 1, "summaries, block_scale, max_blocks required");
+  ls::SummParams p{};
+  p.B = keys->batch; p.max_pages = keys->max_pages; p.max_len = keys->max_len; p.max_blocks = max_blocks;
+  p.num_pages = keys->num_pages; p.keys = (const uint8_t*)keys->key_pool; p.ks = keys->key_scale;
+  p.page_table = keys->page_table; p.lens = keys->lens; p.summ = summaries; p.bscale = block_scale;
+  const int gx = std::min(max_blocks, std::min(keys->max_pages, (keys->max_len + 63) / 64));
+  ls::build_summaries_kernel<<<dim3(gx, keys->batch), 128, 0, (cudaStream_t)stream>>>(p);
+  LS_TRY(check_launch("build_summaries"));
+  return ok();
+}
+
+size_t ls_block_bound_prune_workspace_size(const ls_block_bound_prune_args* args) {
+  if (!args) return 0;
+  return c2f_layout(args).total;
+}
+
+ls_status ls_block_bound_prune(const ls_block_bound_prune_args* args, void* workspace, size_t workspace_bytes,
+                               ls_stream_t stream) {
+  LS_TRY(validate_c2f(args));
+  LS_TRY(run_c2f(args, workspace, workspace_bytes, args->survivors, args->n_survivors, nullptr,
+                 (cudaStream_t)stream));
+  return ok();
+}
+
+ls_status ls_hotbuf_resolve(const ls_hotbuf_args* args, ls_stream_t stream) {
+  LS_TRY(validate_hotbuf(args));
+  LS_TRY(launch_hotbuf(args, (cudaStream_t)stream));
+  return ok();
+}
+
+ls_status ls_gather_misses(const ls_gather_args* args, ls_stream_t stream) {
+  LS_TRY(validate_gather(args));
+  LS_TRY(launch_gather(args, (cudaStream_t)stream));
+  return ok();
+}
+
+size_t ls_sparse_attn_workspace_size(const ls_sparse_attn_args* args) {
+  if (!args) return 0;
+  return attn_ws_bytes(args);
+}
+
+ls_status ls_sparse_attn_decode(const ls_sparse_attn_args* a, void* workspace, size_t workspace_bytes,
+                                ls_stream_t stream) {
+  LS_TRY(validate_attn(a, true));
+  LS_TRY(launch_attn(a, a->sel, a->addressing, a->page_table, a->max_pages, a->n_slots, nullptr, a->num_rows,
+                     workspace, workspace_bytes, (cudaStream_t)stream));
+  return ok();
+}
+
+size_t ls_decode_step_workspace_size(const ls_decode_step_args* args) {
+  if (!args) return 0;
+  return step_layout(args).total;
+}
+
+ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t workspace_bytes,
+                         ls_stream_t stream) {
+  LS_REQUIRE(a, "args is NULL");
+  LS_REQUIRE(a->k >= 1 && a->k <= 4096, "1 <= k <= 4096 required");
+  cudaStream_t st = (cudaStream_t)stream;
+  const ls_index_score_args* ix = &a->index;
+  LS_TRY(validate_index(ix, false));
+  LS_REQUIRE(a->use_c2f || (ix->max_len % 4) == 0, "index.max_len must be a multiple of 4");
+  ls_sparse_attn_args at = step_attn_args(a);
+  LS_TRY(validate_attn(&at, false));
+  if (a->use_hotbuf) {
+    LS_REQUIRE(a->pos_of_slot && a->recent_score && a->slot_of_pos && a->host_kv && a->hbuf,
+               "hot-buffer state, host_kv and hbuf are required");
+    LS_REQUIRE(a->n_slots >= a->k && a->n_slots <= ls::kHbMaxSlots, "need k <= n_slots <= 4096");
+    LS_REQUIRE(a->host_num_pages >= 1, "host_num_pages must be >= 1");
+    LS_REQUIRE(aligned16(a->host_kv) && aligned16(a->hbuf), "host_kv and hbuf must be 16-byte aligned");
+  } else {
+    LS_REQUIRE(at.addressing == LS_ROWS_PAGED, "without the hot buffer attention reads the paged pool");
+  }
+  const StepLayout l = step_layout(a);
+  LS_REQUIRE(workspace_bytes >= l.total && (l.total == 0 || workspace), "decode-step workspace too small (%zu < %zu)",
+             workspace_bytes, l.total);
+  LS_REQUIRE(((uintptr_t)workspace & 255) == 0, "workspace must be 256-byte aligned");
+  char* w = (char*)workspace;
+  int* idx = a->idx ? a->idx : (int*)(w + l.off_idx);
+  float* sel = a->sel_score ? a->sel_score : (float*)(w + l.off_sel);
+  ls_event_t* ev = a->events;
+  auto rec = [&](int i) {
+    if (ev && ev[i]) cudaEventRecord((cudaEvent_t)ev[i], st);
+  };
+  // a1 (+a2) or a3
+  rec(0);
+  if (a->use_c2f) {
+    ls_block_bound_prune_args c = step_c2f_args(a, idx, sel);
+    LS_TRY(validate_c2f(&c));
+    LS_TRY(run_c2f(&c, w + l.off_c2f, l.total - l.off_c2f, a->survivors, a->n_survivors, ev ? ev[1] : nullptr, st));
+  } else {
+    float* scores = ix->scores ? ix->scores : (float*)(w + l.off_scores);
+    if (ix->key_dtype == LS_E4M3 && ix->variant == 0) {
+      LS_TRY(launch_index_tc(ix, 0, nullptr, nullptr, 0, scores, ix->max_len, nullptr, nullptr, 0, nullptr, 0.f, st));
+    } else {
+      ls_index_score_args tmp = *ix;
+      tmp.scores = scores;
+      LS_TRY(launch_index_simt(&tmp, st));
+    }
+    rec(1);
+    LS_TRY(launch_topk(ix->batch, a->k, scores, ix->max_len, ix->lens, 1, 1, ix->max_len, nullptr, 0, idx, sel,
+                       nullptr, st));
+  }
+  void* attn_ws = w + l.off_attn;
+  const size_t attn_ws_b = attn_ws_bytes(&at);
+  if (a->use_hotbuf) {
+    int* sel_slot = (int*)(w + l.off_selslot);
+    int* mpos = (int*)(w + l.off_mpos);
+    int* mslot = (int*)(w + l.off_mslot);
+    int* nmiss = a->n_miss ? a->n_miss : (int*)(w + l.off_nmiss);
+    rec(2);
+    ls_hotbuf_args h{};
+    h.batch = ix->batch; h.k = a->k; h.n_slots = a->n_slots; h.max_len = ix->max_len; h.sel = idx;
+    h.sel_score = sel; h.pos_of_slot = a->pos_of_slot; h.recent_score = a->recent_score;
+    h.slot_of_pos = a->slot_of_pos; h.sel_slot = sel_slot; h.miss_pos = mpos; h.miss_slot = mslot; h.n_miss = nmiss;
+    LS_TRY(launch_hotbuf(&h, st));
+    rec(3);
+    ls_gather_args g{};
+    g.batch = ix->batch; g.k = a->k; g.n_slots = a->n_slots; g.max_pages = ix->max_pages;
+    g.row_bytes = at.row_stride * (at.dtype == LS_BF16 ? 2 : 4); g.num_pages = a->host_num_pages;
+    g.host_kv = a->host_kv; g.page_table = ix->page_table; g.miss_pos = mpos; g.miss_slot = mslot;
+    g.n_miss = nmiss; g.hbuf = a->hbuf;
+    LS_TRY(launch_gather(&g, st));
+    rec(4);
+    LS_TRY(launch_attn(&at, sel_slot, LS_ROWS_SLOTS, nullptr, 0, a->n_slots, a->hbuf,
+                       (long long)ix->batch * a->n_slots, attn_ws, attn_ws_b, st));
+  } else {
+    rec(2);
+    rec(3);
+    rec(4);
+    const int* pt = at.page_table ? at.page_table : ix->page_table;
+    const int mp = at.page_table ? at.max_pages : ix->max_pages;
+    LS_TRY(launch_attn(&at, idx, LS_ROWS_PAGED, pt, mp, 0, nullptr, at.num_rows, attn_ws, attn_ws_b, st));
+  }
+  rec(5);
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,469 @@
+// a6. Sparse attention over the selected rows only (LeanSparse, abstract: sparse
+// attention limits the history read by each query).
+//
+//   s_j = scale * q_h . K_j,  o_h = sum_j softmax(s)_j V_j,  lse_h = log sum_j exp(s_j)
+//
+// * attn_mla_tc: MLA-absorbed decode, 128 query heads against one 576-wide latent KV
+//   head whose first 512 dims are V, bf16, on tcgen05 tensor cores.
+//     - Heads are the MMA M dimension (128); a tile of 32 selected rows is N.
+//     - S = Q K^T (K = 576) and O += P V are tcgen05.mma kind::f16 with f32 TMEM
+//       accumulators.  O for all 512 V dims would fill the whole 512-column TMEM,
+//       so each CTA owns one 256-wide half of V (the pair recomputes S) and keeps
+//       O_half (256 columns) + a double-buffered S (2 x 32 columns) in TMEM.
+//     - Rows are gathered through the page table or the hot-buffer slots by
+//       cp.async 16-byte copies straight into 128-byte-swizzled panels; the same
+//       panels serve as the K-major B operand of S and the MN-major B operand of PV.
+//     - Online softmax in the exp2 domain with lazy rescaling (O is only rescaled
+//       when the running max grows by more than 2^8).
+//     - Split-KV across CTAs (enough CTAs to fill the GPU at small batch), merged
+//       by attn_combine with the log-sum-exp rule.
+// * attn_simt: CUDA-core kernel for fp32 (and a bf16 cross-check variant).
+#pragma once
+#include "common.cuh"
+
+namespace ls {
+
+struct AttnParams {
+  int B, H, dk, dv, k;
+  float scale;       // softmax scale (natural-log domain)
+  int addressing;    // LS_ROWS_PAGED / LS_ROWS_SLOTS
+  int max_pages, n_slots;
+  long long row_stride, num_rows;
+  const void* q;
+  const void* krows;
+  const void* vrows;
+  const int* page_table;
+  const int* sel;
+  void* o;
+  float* lse;
+  int nsplit;
+  float* part_o;     // [B,nsplit,H,dv] unnormalised partial outputs
+  float* part_ml;    // [B,nsplit,H,2] running max (log2 domain) and sum
+};
+
+// Row index of selection value sv of request b, or -1 (padding or out of range).
+__device__ __forceinline__ long long attn_row(const AttnParams& p, int b, int sv) {
+  if (sv < 0) return -1;
+  long long row;
+  if (p.addressing == LS_ROWS_PAGED) {
+    const int lp = sv >> 6;
+    if (lp >= p.max_pages) { flag(LS_DEV_BOUNDS); return -1; }
+    const int page = p.page_table[(size_t)b * p.max_pages + lp];
+    if (page < 0) { flag(LS_DEV_BOUNDS); return -1; }
+    row = (long long)page * 64 + (sv & 63);
+  } else {
+    if (sv >= p.n_slots) { flag(LS_DEV_BOUNDS); return -1; }
+    row = (long long)b * p.n_slots + sv;
+  }
+  if (row >= p.num_rows) { flag(LS_DEV_BOUNDS); return -1; }
+  return row;
+}
+
+// =====================================================================================
+// CUDA-core kernel: one (request, head) per CTA.
+// =====================================================================================
+template <bool BF16>
+__global__ void __launch_bounds__(256) attn_simt(const AttnParams p) {
+  extern __shared__ __align__(16) float sm_a[];
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, warp = warp_id(), lane = lane_id();
+  float* qs = sm_a;                       // [dk]
+  float* s = qs + ((p.dk + 1) & ~1);      // [k]
+  long long* rows = (long long*)(s + ((p.k + 1) & ~1));  // [k], 8-byte aligned
+  __shared__ float red[32];
+  using T = typename std::conditional<BF16, __nv_bfloat16, float>::type;
+  const T* q = (const T*)p.q + ((size_t)b * p.H + h) * p.dk;
+  for (int d = tid; d < p.dk; d += 256) qs[d] = (float)q[d];
+  for (int j = tid; j < p.k; j += 256) rows[j] = attn_row(p, b, p.sel[(size_t)b * p.k + j]);
+  __syncthreads();
+  const T* K = (const T*)p.krows;
+  const T* V = (const T*)p.vrows;
+  for (int j = warp; j < p.k; j += 8) {
+    const long long r = rows[j];
+    float acc = 0.f;
+    if (r >= 0) {
+      const T* kr = K + r * p.row_stride;
+      for (int d = lane; d < p.dk; d += 32) acc = fmaf(qs[d], (float)kr[d], acc);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) s[j] = r >= 0 ? acc * p.scale : -INFINITY;
+  }
+  __syncthreads();
+  float mx = -INFINITY;
+  for (int j = tid; j < p.k; j += 256) mx = fmaxf(mx, s[j]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  mx = red[0];
+  for (int w = 1; w < 8; ++w) mx = fmaxf(mx, red[w]);
+  __syncthreads();
+  float sum = 0.f;
+  for (int j = tid; j < p.k; j += 256) {
+    const float e = rows[j] >= 0 ? expf(s[j] - mx) : 0.f;
+    s[j] = e;
+    sum += e;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) red[warp] = sum;
+  __syncthreads();
+  float l = 0.f;
+  for (int w = 0; w < 8; ++w) l += red[w];
+  T* o = (T*)p.o + ((size_t)b * p.H + h) * p.dv;
+  for (int d = tid; d < p.dv; d += 256) {
+    float acc = 0.f;
+    for (int j = 0; j < p.k; ++j) {
+      const long long r = rows[j];
+      if (r >= 0) acc = fmaf(s[j], (float)V[r * p.row_stride + d], acc);
+    }
+    o[d] = (T)(l > 0.f ? acc / l : 0.f);
+  }
+  if (tid == 0) p.lse[(size_t)b * p.H + h] = l > 0.f ? mx + logf(l) : -INFINITY;
+}
+
+// =====================================================================================
+// tcgen05 MLA kernel
+// =====================================================================================
+namespace mla {
+constexpr int H = 128, DK = 576, DV = 512, DVH = 256, N = 32;
+constexpr int kPanels = DK / 64;                       // 9 panels of 64 bf16 (128 bytes)
+constexpr int kQBytes = kPanels * H * 128;             // 147456
+constexpr int kKvPanel = N * 128;                      // 4096
+constexpr int kKvBytes = kPanels * kKvPanel;           // 36864
+constexpr int kOffKv = kQBytes;
+constexpr int kOffP = kOffKv + 2 * kKvBytes;           // 221184
+constexpr int kPBytes = H * N * 2;                     // 8192
+constexpr int kOffBar = kOffP + kPBytes;               // 229376
+constexpr int kNumBars = 2 + 2 + 2 + 1 + 1 + 1;        // kv_full[2] kv_empty[2] s_full[2] p_full p_free o_done
+constexpr int kOffTmem = kOffBar + kNumBars * 8;
+constexpr int kSmem = 1024 + kOffTmem + 16;
+constexpr int kThreads = 256;
+constexpr int kLoaders = 96;                           // warps 0, 1, 3
+constexpr int kChunksPerRow = DK * 2 / 16;             // 72
+constexpr uint32_t kIdescS = make_idesc(1 /*bf16*/, 128, N, false, false);
+constexpr uint32_t kIdescO = make_idesc(1 /*bf16*/, 128, DVH, false, true);
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+}  // namespace mla
+
+__global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
+  using namespace mla;
+  extern __shared__ uint8_t sm_raw_a[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)sm_raw_a + 1023) & ~(uintptr_t)1023);
+  uint64_t* bars = (uint64_t*)(sm + kOffBar);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = bars + 2;
+  uint64_t* s_full = bars + 4;
+  uint64_t* p_full = bars + 6;
+  uint64_t* p_free = bars + 7;
+  uint64_t* o_done = bars + 8;
+  uint32_t* tmem_slot = (uint32_t*)(sm + kOffTmem);
+  __shared__ long long s_rowoff[2][N];  // byte offset of each row of a stage, -1 if absent
+  __shared__ int s_abort;
+  __shared__ int s_loader_go;
+
+  const int b = blockIdx.y;
+  const int half = blockIdx.x & 1;
+  const int split = blockIdx.x >> 1;
+  const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
+  const int T_all = (p.k + N - 1) / N;
+  const int t0 = (int)(((long long)T_all * split) / p.nsplit);
+  const int t1 = (int)(((long long)T_all * (split + 1)) / p.nsplit);
+  const int my_tiles = t1 - t0;
+  const uint32_t sbase = smem_u32(sm);
+  const char* kv_base = (const char*)p.krows;
+
+  // ---- Q (128 heads x 576) into nine 128-byte-swizzled K-major panels
+  {
+    const char* q = (const char*)p.q + (size_t)b * H * DK * 2;
+    for (int e = tid; e < H * kChunksPerRow; e += kThreads) {
+      const int h = e / kChunksPerRow, c = e - h * kChunksPerRow;
+      const int pn = c >> 3, j = c & 7;
+      cp_async_16(sbase + pn * (H * 128) + h * 128 + ((j ^ (h & 7)) << 4), q + (size_t)h * DK * 2 + c * 16);
+    }
+    cp_async_commit();
+  }
+  if (tid == 0) {
+    mbar_init(&kv_full[0], kLoaders);
+    mbar_init(&kv_full[1], kLoaders);
+    mbar_init(&kv_empty[0], 1);
+    mbar_init(&kv_empty[1], 1);
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
+    mbar_init(p_full, 128);
+    mbar_init(p_free, 1);
+    mbar_init(o_done, 1);
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) tmem_alloc(tmem_slot, 512);
+  cp_async_wait<0>();
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tm_o = tmem;          // columns [0, 256): O half
+  const uint32_t tm_s = tmem + 256;    // columns [256, 320): S double buffer
+
+  if (warp == 0 || warp == 1 || warp == 3) {
+    // ================= loaders: gather the tile's rows =================
+    const int lt = (warp == 3) ? 64 + lane : warp * 32 + lane;
+    for (int i = 0; i < my_tiles; ++i) {
+      const int st = i & 1;
+      // one thread decides whether to go on, so the named barrier stays uniform
+      if (lt == 0) {
+        bool go = (i < 2) || mbar_wait(&kv_empty[st], ((i >> 1) - 1) & 1);
+        if (*(volatile int*)&s_abort) go = false;
+        if (!go) s_abort = 1;
+        s_loader_go = go ? 1 : 0;
+      }
+      const int j0 = (t0 + i) * N;
+      if (lt < N) {
+        const int j = j0 + lt;
+        long long off = -1;
+        if (j < p.k) {
+          const long long r = attn_row(p, b, p.sel[(size_t)b * p.k + j]);
+          if (r >= 0) off = r * p.row_stride * 2;
+        }
+        s_rowoff[st][lt] = off;
+      }
+      asm volatile("bar.sync 1, 96;" ::: "memory");
+      if (!s_loader_go) break;
+      const uint32_t dst0 = sbase + kOffKv + st * kKvBytes;
+      for (int e = lt; e < N * kChunksPerRow; e += kLoaders) {
+        const int r = e / kChunksPerRow, c = e - r * kChunksPerRow;
+        const int pn = c >> 3, jj = c & 7;
+        const uint32_t dst = dst0 + pn * kKvPanel + r * 128 + ((jj ^ (r & 7)) << 4);
+        const long long off = s_rowoff[st][r];
+        if (off >= 0) {
+          cp_async_16(dst, kv_base + off + c * 16);
+        } else {
+          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0) : "memory");
+        }
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
+      mbar_arrive(&kv_full[st]);
+      asm volatile("bar.sync 1, 96;" ::: "memory");  // s_rowoff / s_loader_go reusable
+    }
+  } else if (warp == 2) {
+    // ================= MMA issuer =================
+    if (lane == 0 && my_tiles > 0) {
+      const uint32_t q_addr = sbase;
+      const uint32_t p_addr = sbase + kOffP;
+      auto issue_s = [&](int i) -> bool {
+        const int st = i & 1;
+        if (!mbar_wait(&kv_full[st], (i >> 1) & 1)) return false;
+        tc_fence_after();
+        const uint32_t kv = sbase + kOffKv + st * kKvBytes;
+#pragma unroll 1
+        for (int pn = 0; pn < kPanels; ++pn) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = make_sdesc(q_addr + pn * (H * 128) + kk * 32, 16, 1024, kSwizzle128);
+            const uint64_t bd = make_sdesc(kv + pn * kKvPanel + kk * 32, 16, 1024, kSwizzle128);
+            mma_bf16(tm_s + st * N, ad, bd, kIdescS, (pn | kk) != 0);
+          }
+        }
+        tc_commit(&s_full[st]);
+        return true;
+      };
+      bool ok = issue_s(0);
+      if (ok && my_tiles > 1) ok = issue_s(1);
+      for (int i = 0; ok && i < my_tiles; ++i) {
+        const int st = i & 1;
+        if (!mbar_wait(p_full, i & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t v = sbase + kOffKv + st * kKvBytes + half * 4 * kKvPanel;
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint64_t ad = make_sdesc(p_addr + kk * 2 * 2048, 2048, 128, kSwizzleNone);
+          const uint64_t bd = make_sdesc(v + kk * 16 * 128, kKvPanel, 1024, kSwizzle128);
+          mma_bf16(tm_o, ad, bd, kIdescO, (i > 0 || kk > 0));
+        }
+        tc_commit(&kv_empty[st]);
+        tc_commit(p_free);
+        if (i + 2 < my_tiles) ok = issue_s(i + 2);
+      }
+      if (!ok) s_abort = 1;
+      tc_commit(o_done);
+    }
+  } else {
+    // ================= softmax: warps 4..7, thread = head =================
+    const int wq = warp & 3;
+    const int h = wq * 32 + lane;
+    const float sl2 = p.scale * kLog2e;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int i = 0; i < my_tiles; ++i) {
+      const int st = i & 1;
+      const int j0 = (t0 + i) * N;
+      uint32_t vmask = 0;
+#pragma unroll 4
+      for (int r = 0; r < N; ++r) {
+        const int j = j0 + r;
+        if (j < p.k && attn_row(p, b, p.sel[(size_t)b * p.k + j]) >= 0) vmask |= 1u << r;
+      }
+      if (!mbar_wait(&s_full[st], (i >> 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      float s[N];
+      tmem_ld32(tm_s + lane_off + st * N, s);
+      tmem_wait_ld();
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < N; ++r)
+        if (vmask >> r & 1u) tmax = fmaxf(tmax, s[r]);
+      const float mt = tmax * sl2;
+      float factor = 1.f;
+      bool rescale = false;
+      if (mt > m_run + 8.f) {  // also true for the first tile with data
+        if (m_run != -INFINITY) {
+          factor = exp2f(m_run - mt);
+          rescale = true;
+        }
+        m_run = mt;
+      }
+      float pr[N];
+      float psum = 0.f;
+#pragma unroll
+      for (int r = 0; r < N; ++r) {
+        pr[r] = (vmask >> r & 1u) ? exp2f(fmaf(s[r], sl2, -m_run)) : 0.f;
+        psum += pr[r];
+      }
+      if (i >= 1 && !mbar_wait(p_free, (i - 1) & 1)) { ok = false; break; }
+      if (rescale) {
+        tc_fence_after();
+#pragma unroll 1
+        for (int c0 = 0; c0 < DVH; c0 += 32) {
+          float v[32];
+          tmem_ld32(tm_o + lane_off + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) v[c] *= factor;
+          tmem_st32(tm_o + lane_off + c0, v);
+        }
+        tmem_wait_st();
+      }
+      l_run = l_run * factor + psum;
+      uint8_t* pbuf = sm + kOffP;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          __nv_bfloat162 two = __floats2bfloat162_rn(pr[c * 8 + 2 * e], pr[c * 8 + 2 * e + 1]);
+          w[e] = *(uint32_t*)&two;
+        }
+        *(uint4*)(pbuf + h * 16 + c * 2048) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(p_full);
+    }
+    // ---- epilogue
+    if (ok && my_tiles > 0 && mbar_wait(o_done, 0)) {
+      tc_fence_after();
+      const bool single = p.nsplit == 1;
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      for (int c0 = 0; c0 < DVH; c0 += 32) {
+        float v[32];
+        tmem_ld32(tm_o + lane_off + c0, v);
+        tmem_wait_ld();
+        if (single) {
+          __nv_bfloat16* o = (__nv_bfloat16*)p.o + ((size_t)b * H + h) * DV + half * DVH + c0;
+#pragma unroll
+          for (int c = 0; c < 32; c += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 two = __floats2bfloat162_rn(v[c + 2 * e] * inv, v[c + 2 * e + 1] * inv);
+              w[e] = *(uint32_t*)&two;
+            }
+            *(uint4*)(o + c) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        } else {
+          float* o = p.part_o + (((size_t)b * p.nsplit + split) * H + h) * DV + half * DVH + c0;
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            *(float4*)(o + c) = make_float4(l_run > 0.f ? v[c] : 0.f, l_run > 0.f ? v[c + 1] : 0.f,
+                                            l_run > 0.f ? v[c + 2] : 0.f, l_run > 0.f ? v[c + 3] : 0.f);
+        }
+      }
+      if (half == 0) {
+        if (single) {
+          p.lse[(size_t)b * H + h] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+        } else {
+          float* ml = p.part_ml + (((size_t)b * p.nsplit + split) * H + h) * 2;
+          ml[0] = l_run > 0.f ? m_run : -INFINITY;
+          ml[1] = l_run;
+        }
+      }
+    } else if (my_tiles == 0 && p.nsplit > 1) {
+      float* o = p.part_o + (((size_t)b * p.nsplit + split) * H + h) * DV + half * DVH;
+      for (int c = 0; c < DVH; ++c) o[c] = 0.f;
+      if (half == 0) {
+        float* ml = p.part_ml + (((size_t)b * p.nsplit + split) * H + h) * 2;
+        ml[0] = -INFINITY;
+        ml[1] = 0.f;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Merge split-KV partials: o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
+// One warp per (request, head); each lane owns 16 of the 512 output dims.
+__global__ void __launch_bounds__(128) attn_combine(const AttnParams p) {
+  using namespace mla;
+  const int gw = blockIdx.x * 4 + warp_id();
+  const int lane = lane_id();
+  if (gw >= p.B * H) return;
+  const int b = gw / H, h = gw - b * H;
+  float M = -INFINITY;
+  for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, p.part_ml[(((size_t)b * p.nsplit + s) * H + h) * 2]);
+  float acc[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+  float Lsum = 0.f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < p.nsplit; ++s) {
+      const float* ml = p.part_ml + (((size_t)b * p.nsplit + s) * H + h) * 2;
+      if (ml[1] <= 0.f) continue;
+      const float wgt = exp2f(ml[0] - M);
+      Lsum += wgt * ml[1];
+      const float* po = p.part_o + (((size_t)b * p.nsplit + s) * H + h) * DV + lane * 16;
+#pragma unroll
+      for (int e = 0; e < 16; e += 4) {
+        const float4 v = *(const float4*)(po + e);
+        acc[e] += wgt * v.x;
+        acc[e + 1] += wgt * v.y;
+        acc[e + 2] += wgt * v.z;
+        acc[e + 3] += wgt * v.w;
+      }
+    }
+  }
+  const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+  __nv_bfloat16* o = (__nv_bfloat16*)p.o + ((size_t)b * H + h) * DV + lane * 16;
+#pragma unroll
+  for (int e = 0; e < 16; e += 8) {
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      __nv_bfloat162 two = __floats2bfloat162_rn(acc[e + 2 * q] * inv, acc[e + 2 * q + 1] * inv);
+      w[q] = *(uint32_t*)&two;
+    }
+    *(uint4*)(o + e) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  if (lane == 0) p.lse[(size_t)b * H + h] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
+}
+
+}  // namespace ls

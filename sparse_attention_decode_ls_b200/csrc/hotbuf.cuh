@@ -1,0 +1,224 @@
+// a4 / a5. Hot-buffer resolve and miss gather (XM-Sparse, hot-buffer section: HBM
+// keeps a per-request hot KV buffer; after each step's sparse selection only the
+// selected KV that misses it is fetched from the full history).
+//
+// hotbuf_resolve: one CTA per request.  Classifies each selection as hit (resident)
+// or miss, compacts the misses in selection order, orders the unpinned slots by
+// (empty first, recent score, slot) with a shared-memory bitonic sort of 64-bit
+// composite keys, hands the i-th victim to the i-th miss, and updates both maps
+// and the recent scores in place.
+//
+// gather_misses: copies each missed 1,152-byte row from pinned host memory into its
+// slot; every thread moves 16-byte vectors, and each warp keeps several rows' loads
+// in flight so that the PCIe link, not latency, sets the pace.
+#pragma once
+#include "common.cuh"
+
+namespace ls {
+
+struct HotbufParams {
+  int B, k, n_slots, max_len;
+  const int* sel;
+  const float* sel_score;
+  int* pos_of_slot;
+  float* recent;
+  int* slot_of_pos;
+  int* sel_slot;
+  int* miss_pos;
+  int* miss_slot;
+  int* n_miss;
+};
+
+constexpr int kHbThreads = 1024;
+constexpr int kHbMaxSlots = 4096;
+
+__global__ void __launch_bounds__(kHbThreads, 1) hotbuf_resolve_kernel(const HotbufParams p) {
+  extern __shared__ unsigned long long keys[];       // [next pow2 >= n_slots] sort buffer
+  __shared__ uint8_t pinned[kHbMaxSlots];
+  __shared__ int miss_j[kHbMaxSlots];               // selection index of the i-th miss
+  __shared__ unsigned long long scan_tmp[32];
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int k = p.k, S = p.n_slots;
+  const int* sel = p.sel + (size_t)b * k;
+  int* pos_of_slot = p.pos_of_slot + (size_t)b * S;
+  float* recent = p.recent + (size_t)b * S;
+  int* slot_of_pos = p.slot_of_pos + (size_t)b * p.max_len;
+  int* sel_slot = p.sel_slot + (size_t)b * k;
+
+  for (int s = tid; s < S; s += kHbThreads) pinned[s] = 0;
+  __syncthreads();
+  // ---- classify (contiguous per-thread ranges keep selection order for the scan)
+  const int per = (k + kHbThreads - 1) / kHbThreads;  // <= 4
+  const int j0 = min(k, tid * per), j1 = min(k, j0 + per);
+  uint32_t my_miss = 0;
+  uint32_t miss_bits = 0;
+  for (int j = j0; j < j1; ++j) {
+    const int pos = sel[j];
+    int slot = -1;
+    bool is_miss = false;
+    if (pos >= 0) {
+      if (pos >= p.max_len) {
+        flag(LS_DEV_BOUNDS);
+      } else {
+        slot = slot_of_pos[pos];
+        if (slot >= S) {
+          flag(LS_DEV_BOUNDS);
+          slot = -1;
+        } else if (slot >= 0) {
+          pinned[slot] = 1;
+        } else {
+          is_miss = true;
+        }
+      }
+    }
+    sel_slot[j] = slot;
+    if (is_miss) {
+      miss_bits |= 1u << (j - j0);
+      ++my_miss;
+    }
+  }
+  unsigned long long total;
+  const uint32_t mpre = (uint32_t)block_excl_scan_u64(my_miss, scan_tmp, &total);
+  const int n_miss = (int)total;
+  {
+    uint32_t o = mpre;
+    for (int j = j0; j < j1; ++j) {
+      if (miss_bits >> (j - j0) & 1u) {
+        miss_j[o] = j;
+        p.miss_pos[(size_t)b * k + o] = sel[j];
+        ++o;
+      }
+    }
+  }
+  // ---- victim order: (class, recent-score key, slot); class 0 empty, 1 occupied, 2 pinned
+  int n_pow2 = 1;
+  while (n_pow2 < S) n_pow2 <<= 1;
+  __syncthreads();
+  for (int s = tid; s < n_pow2; s += kHbThreads) {
+    unsigned long long key;
+    if (s >= S) {
+      key = ~0ull;
+    } else if (pinned[s]) {
+      key = (2ull << 44) | s;
+    } else if (pos_of_slot[s] < 0) {
+      key = (unsigned long long)s;
+    } else {
+      key = (1ull << 44) | ((unsigned long long)float_key(recent[s]) << 12) | (unsigned long long)s;
+    }
+    keys[s] = key;
+  }
+  __syncthreads();
+  for (int size = 2; size <= n_pow2; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int t = tid; t < (n_pow2 >> 1); t += kHbThreads) {
+        const int lo = 2 * t - (t & (stride - 1));
+        const int hi = lo + stride;
+        const bool up = (lo & size) == 0;
+        const unsigned long long a = keys[lo], c = keys[hi];
+        if ((a > c) == up) {
+          keys[lo] = c;
+          keys[hi] = a;
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // ---- apply: the i-th miss takes the i-th victim
+  for (int i = tid; i < n_miss; i += kHbThreads) {
+    const unsigned long long key = keys[i];
+    const int v = (int)(key & 0xFFFull);
+    if ((key >> 44) >= 2ull) {  // ran out of unpinned slots
+      flag(LS_DEV_CAPACITY);
+      p.miss_slot[(size_t)b * k + i] = -1;
+      continue;
+    }
+    const int pos = sel[miss_j[i]];
+    const int old = pos_of_slot[v];
+    if (old >= 0 && old < p.max_len) slot_of_pos[old] = -1;
+    pos_of_slot[v] = pos;
+    slot_of_pos[pos] = v;
+    sel_slot[miss_j[i]] = v;
+    p.miss_slot[(size_t)b * k + i] = v;
+  }
+  for (int i = n_miss + tid; i < k; i += kHbThreads) {
+    p.miss_pos[(size_t)b * k + i] = -1;
+    p.miss_slot[(size_t)b * k + i] = -1;
+  }
+  __syncthreads();
+  for (int j = tid; j < k; j += kHbThreads) {
+    const int s = sel_slot[j];
+    if (s >= 0) recent[s] = p.sel_score[(size_t)b * k + j];
+  }
+  if (tid == 0) p.n_miss[b] = n_miss;
+}
+
+struct GatherParams {
+  int B, k, n_slots, max_pages;
+  long long row_bytes, num_pages;
+  const char* host;
+  const int* page_table;
+  const int* miss_pos;
+  const int* miss_slot;
+  const int* n_miss;
+  char* hbuf;
+};
+
+// grid (ctas_per_req, B), 256 threads.  A warp owns 4 rows at a time and issues all
+// their 16-byte loads before storing any.
+__global__ void __launch_bounds__(256) gather_misses_kernel(const GatherParams p) {
+  const int b = blockIdx.y;
+  const int warp = warp_id(), lane = lane_id();
+  const int nm = p.n_miss[b];
+  if (nm < 0 || nm > p.k) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) flag(LS_DEV_BOUNDS);
+    return;
+  }
+  const int chunks = (int)(p.row_bytes >> 4);
+  const int gw = blockIdx.x * 8 + warp, nw = gridDim.x * 8;
+  constexpr int R = 4;
+  for (int i0 = gw * R; i0 < nm; i0 += nw * R) {
+    const char* src[R];
+    char* dst[R];
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+      src[q] = nullptr;
+      dst[q] = nullptr;
+      const int i = i0 + q;
+      if (i < nm) {
+        const int pos = p.miss_pos[(size_t)b * p.k + i];
+        const int slot = p.miss_slot[(size_t)b * p.k + i];
+        const int lp = pos >> 6;
+        if (pos >= 0 && lp < p.max_pages && slot >= 0 && slot < p.n_slots) {
+          const int page = p.page_table[(size_t)b * p.max_pages + lp];
+          if (page >= 0 && page < p.num_pages) {
+            src[q] = p.host + ((long long)page * 64 + (pos & 63)) * p.row_bytes;
+            dst[q] = p.hbuf + ((long long)b * p.n_slots + slot) * p.row_bytes;
+          } else {
+            flag(LS_DEV_BOUNDS);
+          }
+        } else {
+          flag(LS_DEV_BOUNDS);
+        }
+      }
+    }
+    for (int c0 = 0; c0 < chunks; c0 += 32 * 3) {
+      uint4 v[R][3];
+#pragma unroll
+      for (int q = 0; q < R; ++q)
+#pragma unroll
+        for (int e = 0; e < 3; ++e) {
+          const int c = c0 + e * 32 + lane;
+          if (src[q] && c < chunks) v[q][e] = *(const uint4*)(src[q] + (size_t)c * 16);
+        }
+#pragma unroll
+      for (int q = 0; q < R; ++q)
+#pragma unroll
+        for (int e = 0; e < 3; ++e) {
+          const int c = c0 + e * 32 + lane;
+          if (dst[q] && c < chunks) *(uint4*)(dst[q] + (size_t)c * 16) = v[q][e];
+        }
+    }
+  }
+}
+
+}  // namespace ls

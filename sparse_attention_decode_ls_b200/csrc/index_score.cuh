@@ -1,0 +1,399 @@
+// a1. Indexer score kernels.
+//
+// score[b][s] = key_scale[s] * sum_h (w[b][h] * q_scale[b][h]) * ReLU(q8[b][h] . k8[s])
+//
+// (the DSA lightning-indexer form; LeanSparse, abstract, names indexer keys and
+// indexer scores).  Two kernels:
+//   * index_score_tc   tcgen05 fp8 MMA.  A 128-row tile of keys (two 64-token pages,
+//                      TMA-loaded with 128-byte swizzle) is the A operand (M = 128
+//                      tokens), the query's heads are the B operand (N = 64), so each
+//                      epilogue thread owns one token's TMEM row and reduces the heads
+//                      in registers: ReLU, head weights and the token scale are fused.
+//                      The same tile engine also computes the coarse-to-fine block
+//                      bound (K = 256 bytes: [kmax | kmin] rows against [q+ | q-]).
+//   * index_score_simt CUDA cores, fp32 (and an e4m3 cross-check variant).
+#pragma once
+#include "common.cuh"
+
+namespace ls {
+
+// =====================================================================================
+// CUDA-core kernel: one 64-token page per CTA, 256 threads (token = tid % 64,
+// head group = tid / 64).
+// =====================================================================================
+struct IdxSimtParams {
+  int B, H, D, max_pages, max_len;
+  long long num_pages;
+  const void* q;
+  const float* qs;
+  const void* w;
+  int w_bf16;
+  const void* keys;
+  const float* ks;
+  const int* page_table;
+  const int* lens;
+  float* out;
+};
+
+template <bool E4M3>
+__global__ void __launch_bounds__(256) index_score_simt(IdxSimtParams p) {
+  extern __shared__ __align__(16) float sm_simt[];
+  const int b = blockIdx.y, lp = blockIdx.x, tid = threadIdx.x;
+  const int L = p.lens[b];
+  if (L < 0 || L > p.max_len || L > p.max_pages * 64) {
+    if (lp == 0 && tid == 0) flag(LS_DEV_BOUNDS);
+    return;
+  }
+  if (lp * 64 >= L) return;
+  const int page = p.page_table[(size_t)b * p.max_pages + lp];
+  if (page < 0 || page >= p.num_pages) {
+    if (tid == 0) flag(LS_DEV_BOUNDS);
+    return;
+  }
+  const int H = p.H, D = p.D, Dp = D + 1;
+  float* q_s = sm_simt;             // [H][D]
+  float* k_s = q_s + H * D;         // [64][D+1]
+  float* coef = k_s + 64 * Dp;      // [H]
+  float* part = coef + H;           // [4][64]
+  for (int i = tid; i < H * D; i += 256) {
+    const size_t gi = (size_t)b * H * D + i;
+    q_s[i] = E4M3 ? e4m3_to_float(((const uint8_t*)p.q)[gi]) : ((const float*)p.q)[gi];
+  }
+  for (int h = tid; h < H; h += 256) {
+    const size_t gi = (size_t)b * H + h;
+    float wv = p.w_bf16 ? __bfloat162float(((const __nv_bfloat16*)p.w)[gi]) : ((const float*)p.w)[gi];
+    coef[h] = E4M3 ? wv * p.qs[gi] : wv;
+  }
+  for (int i = tid; i < 64 * D; i += 256) {
+    const int t = i / D, d = i - t * D;
+    const size_t gi = ((size_t)page * 64 + t) * D + d;
+    k_s[t * Dp + d] = E4M3 ? e4m3_to_float(((const uint8_t*)p.keys)[gi]) : ((const float*)p.keys)[gi];
+  }
+  __syncthreads();
+  const int t = tid & 63, g = tid >> 6;
+  float acc = 0.f;
+  for (int h = g; h < H; h += 4) {
+    float dot = 0.f;
+    const float* qh = q_s + h * D;
+    const float* kt = k_s + t * Dp;
+    for (int d = 0; d < D; ++d) dot = fmaf(qh[d], kt[d], dot);
+    acc = fmaf(coef[h], fmaxf(dot, 0.f), acc);
+  }
+  part[g * 64 + t] = acc;
+  __syncthreads();
+  if (g == 0) {
+    const int s = lp * 64 + t;
+    if (s < L) {
+      float v = part[t] + part[64 + t] + part[128 + t] + part[192 + t];
+      if (E4M3) v *= p.ks[(size_t)page * 64 + t];
+      p.out[(size_t)b * p.max_len + s] = v;
+    }
+  }
+}
+
+// =====================================================================================
+// tcgen05 kernel
+// =====================================================================================
+struct IdxTcParams {
+  int mode;              // 0: paged keys (dense, or a list of logical pages); 1: block summaries
+  int B, max_pages, max_len, max_blocks, ctas_per_req;
+  long long num_pages;
+  const uint8_t* q8;     // [B,64,128]
+  const float* qs;       // [B,64]
+  const void* w;         // [B,64]
+  int w_bf16;
+  const float* row_scale;  // mode 0: key scale pool [num_pages*64]; mode 1: block scale [B*max_blocks]
+  const int* page_table;
+  const int* lens;
+  const int* unit_list;    // mode 0 list: [B,list_stride] logical pages (ascending); NULL = every page
+  const int* unit_count;   // [B] length of each list
+  int list_stride;
+  float* out;              // [B,out_stride]
+  long long out_stride;
+  float* out_plain;        // mode 1: bound without margin (may be NULL)
+  float eps_rel;           // mode 1: margin relative to the block magnitude bound
+};
+
+template <int KP, int NCOL>
+struct IdxTc {
+  static constexpr int kThreads = 192;                 // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+  static constexpr int kPanel = 128 * 128;             // one 128-row x 128-byte K panel
+  static constexpr int kStageBytes = KP * kPanel;
+  static constexpr int kStages = (KP == 1) ? 6 : 3;
+  static constexpr int kAcc = 256 / NCOL;              // accumulators in 256 TMEM columns
+  static constexpr int kBBytes = KP * NCOL * 128;
+  static constexpr int kOffB = kStages * kStageBytes;
+  static constexpr int kOffCoef = kOffB + kBBytes;
+  static constexpr int kOffBar = kOffCoef + NCOL * 4 + 16;
+  static constexpr int kNumBars = 2 * kStages + 2 * kAcc;
+  static constexpr int kOffTmem = kOffBar + kNumBars * 8;
+  static constexpr int kSmem = 1024 + kOffTmem + 16;   // +1024: runtime alignment slack
+  static constexpr uint32_t kIdesc = make_idesc(0 /*e4m3*/, 128, NCOL, false, false);
+};
+
+// Row coordinate (in 64-row units of the tensor map) of one unit, or -1 if the unit
+// has no data to load.
+__device__ __forceinline__ int idx_unit_row(const IdxTcParams& p, int b, int u, int* lp_out) {
+  if (p.mode == 1) {
+    *lp_out = u;
+    return b * p.max_blocks + u * 64;
+  }
+  int lp = p.unit_list ? p.unit_list[(size_t)b * p.list_stride + u] : u;
+  *lp_out = lp;
+  if (lp < 0 || lp >= p.max_pages) return -1;
+  const int page = p.page_table[(size_t)b * p.max_pages + lp];
+  if (page < 0 || page >= p.num_pages) return -1;
+  return page * 64;
+}
+
+template <int KP, int NCOL>
+__global__ void __launch_bounds__(192, 1)
+    index_score_tc(const IdxTcParams p, const __grid_constant__ CUtensorMap tmap) {
+  using C = IdxTc<KP, NCOL>;
+  extern __shared__ uint8_t sm_raw[];
+  uint8_t* sm = (uint8_t*)(((uintptr_t)sm_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sA = sm;
+  uint8_t* sB = sm + C::kOffB;
+  float* coef = (float*)(sm + C::kOffCoef);
+  float* gmag = coef + NCOL;  // mode 1: sum_h |w'_h| * sum_d |q8_hd|
+  uint64_t* bars = (uint64_t*)(sm + C::kOffBar);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::kStages;
+  uint64_t* accf = bars + 2 * C::kStages;
+  uint64_t* acce = accf + C::kAcc;
+  uint32_t* tmem_slot = (uint32_t*)(sm + C::kOffTmem);
+  __shared__ int s_abort;
+
+  const int b = blockIdx.y, cta = blockIdx.x, tid = threadIdx.x, warp = warp_id(), lane = lane_id();
+  const int L = p.lens[b];
+  const bool len_ok = L >= 0 && L <= p.max_len && L <= p.max_pages * 64;
+  if (!len_ok) {
+    if (cta == 0 && tid == 0) flag(LS_DEV_BOUNDS);
+    return;
+  }
+  int n_units;
+  if (p.mode == 1) {
+    if (((L + 63) >> 6) > p.max_blocks) {
+      if (cta == 0 && tid == 0) flag(LS_DEV_BOUNDS);
+      return;
+    }
+    n_units = (((L + 63) >> 6) + 63) >> 6;
+  } else if (p.unit_list) {
+    n_units = p.unit_count[b];
+    if (n_units < 0 || n_units > p.list_stride) {
+      if (cta == 0 && tid == 0) flag(LS_DEV_BOUNDS);
+      return;
+    }
+  } else {
+    n_units = (L + 63) >> 6;
+  }
+  const int n_tiles = (n_units + 1) >> 1;
+  const int t_begin = (int)(((long long)n_tiles * cta) / p.ctas_per_req);
+  const int t_end = (int)(((long long)n_tiles * (cta + 1)) / p.ctas_per_req);
+  const int my_tiles = t_end - t_begin;
+  if (my_tiles <= 0) return;
+
+  // ---- prologue: B operand (query side) in 128-byte-swizzled K-major layout, coefficients
+  const uint8_t* q8 = p.q8 + (size_t)b * 64 * 128;
+  for (int i = tid; i < NCOL * 8 * KP; i += C::kThreads) {
+    // i enumerates 16-byte chunks: panel pk, row n, chunk j
+    const int pk = i / (NCOL * 8);
+    const int rem = i - pk * NCOL * 8;
+    const int n = rem >> 3, j = rem & 7;
+    uint4 v;
+    if (KP == 1) {
+      v = *(const uint4*)(q8 + n * 128 + j * 16);
+    } else {
+      // rows 0..63: [q+ | q-], rows 64..127: [q- | q+]  (q+ keeps codes with clear sign bit)
+      const int h = n & 63;
+      const bool want_pos = ((n < 64) == (pk == 0));
+      uint4 raw = *(const uint4*)(q8 + h * 128 + j * 16);
+      uint32_t* r = (uint32_t*)&raw;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        uint32_t x = r[e], out = 0;
+#pragma unroll
+        for (int by = 0; by < 4; ++by) {
+          uint32_t c = (x >> (8 * by)) & 0xFFu;
+          bool neg = (c & 0x80u) != 0;
+          if (neg != want_pos) out |= c << (8 * by);
+        }
+        r[e] = out;
+      }
+      v = raw;
+    }
+    const int off = pk * NCOL * 128 + n * 128 + ((j ^ (n & 7)) << 4);
+    *(uint4*)(sB + off) = v;
+  }
+  if (tid < 64) {
+    const size_t gi = (size_t)b * 64 + tid;
+    const float wv = p.w_bf16 ? __bfloat162float(((const __nv_bfloat16*)p.w)[gi]) : ((const float*)p.w)[gi];
+    const float wq = wv * p.qs[gi];
+    if (NCOL == 64) {
+      coef[tid] = wq;
+    } else {
+      coef[tid] = fmaxf(wq, 0.f);
+      coef[64 + tid] = fminf(wq, 0.f);
+    }
+  }
+  if (p.mode == 1 && warp == 0) {
+    // magnitude bound used for the pruning margin
+    float acc = 0.f;
+    for (int h = lane; h < 64; h += 32) {
+      float s = 0.f;
+      for (int d = 0; d < 128; ++d) s += fabsf(e4m3_to_float(q8[h * 128 + d]));
+      const size_t gi = (size_t)b * 64 + h;
+      const float wv = p.w_bf16 ? __bfloat162float(((const __nv_bfloat16*)p.w)[gi]) : ((const float*)p.w)[gi];
+      acc += fabsf(wv * p.qs[gi]) * s;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) gmag[0] = acc;
+  }
+  fence_proxy_async_smem();
+  if (tid == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < C::kAcc; ++a) {
+      mbar_init(&accf[a], 1);
+      mbar_init(&acce[a], 128);
+    }
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ================= TMA producer =================
+    if (lane == 0) {
+      prefetch_tmap(&tmap);
+      int issued = 0;
+      for (int i = 0; i < my_tiles; ++i) {
+        const int st = i % C::kStages;
+        if (i >= C::kStages && !mbar_wait(&empty[st], ((i / C::kStages) - 1) & 1)) {
+          s_abort = 1;
+          break;
+        }
+        if (*(volatile int*)&s_abort) break;
+        const int tile = t_begin + i;
+        int rows[2], lp;
+        uint32_t bytes = 0;
+        for (int uu = 0; uu < 2; ++uu) {
+          const int u = 2 * tile + uu;
+          rows[uu] = -1;
+          if (u < n_units) {
+            rows[uu] = idx_unit_row(p, b, u, &lp);
+            if (rows[uu] < 0) flag(LS_DEV_BOUNDS);
+            else bytes += KP * 64 * 128;
+          }
+        }
+        mbar_arrive_expect_tx(&full[st], bytes);
+        const uint32_t dst = smem_u32(sA + st * C::kStageBytes);
+        for (int uu = 0; uu < 2; ++uu) {
+          if (rows[uu] < 0) continue;
+          for (int pk = 0; pk < KP; ++pk)
+            tma_load_2d(dst + pk * C::kPanel + uu * 64 * 128, &tmap, &full[st], pk * 128, rows[uu]);
+        }
+        ++issued;
+      }
+      // never leave with copies in flight: wait for every stage still owned by TMA
+      const int first = issued > C::kStages ? issued - C::kStages : 0;
+      for (int i = first; i < issued; ++i) mbar_wait(&full[i % C::kStages], (i / C::kStages) & 1);
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer =================
+    if (lane == 0) {
+      const uint32_t b_base = smem_u32(sB);
+      for (int i = 0; i < my_tiles; ++i) {
+        const int st = i % C::kStages, a = i % C::kAcc;
+        if (!mbar_wait(&full[st], (i / C::kStages) & 1)) { s_abort = 1; break; }
+        if (i >= C::kAcc && !mbar_wait(&acce[a], ((i / C::kAcc) - 1) & 1)) { s_abort = 1; break; }
+        if (*(volatile int*)&s_abort) break;
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(sA + st * C::kStageBytes);
+#pragma unroll
+        for (int pk = 0; pk < KP; ++pk) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = make_sdesc(a_base + pk * C::kPanel + kk * 32, 16, 1024, kSwizzle128);
+            const uint64_t bd = make_sdesc(b_base + pk * NCOL * 128 + kk * 32, 16, 1024, kSwizzle128);
+            mma_f8(tmem + a * NCOL, ad, bd, C::kIdesc, (pk | kk) != 0);
+          }
+        }
+        tc_commit(&empty[st]);
+        tc_commit(&accf[a]);
+      }
+    }
+  } else {
+    // ================= epilogue: warps 2..5, thread = tile row =================
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const float mag = (p.mode == 1) ? gmag[0] : 0.f;
+    for (int i = 0; i < my_tiles; ++i) {
+      const int a = i % C::kAcc;
+      const int tile = t_begin + i;
+      const int u = 2 * tile + (r >> 6), rr = r & 63;
+      // which output does this row feed?
+      bool valid = false;
+      float scale = 0.f;
+      long long out_idx = 0;
+      if (u < n_units) {
+        if (p.mode == 1) {
+          const int j = u * 64 + rr;
+          if (j < ((L + 63) >> 6)) {
+            valid = true;
+            scale = p.row_scale[(size_t)b * p.max_blocks + j];
+            out_idx = j;
+          }
+        } else {
+          int lp;
+          const int row = idx_unit_row(p, b, u, &lp);
+          const int s = lp * 64 + rr;
+          if (row >= 0 && s < L) {
+            valid = true;
+            scale = p.row_scale[(size_t)row + rr];
+            out_idx = p.unit_list ? (long long)u * 64 + rr : s;
+          }
+        }
+      }
+      if (!mbar_wait(&accf[a], (i / C::kAcc) & 1)) { s_abort = 1; break; }
+      tc_fence_after();
+      float sum = 0.f;
+      const uint32_t tbase = tmem + ((uint32_t)(wq * 32) << 16) + a * NCOL;
+#pragma unroll
+      for (int c0 = 0; c0 < NCOL; c0 += 32) {
+        float v[32];
+        tmem_ld32(tbase + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) sum = fmaf(coef[c0 + c], fmaxf(v[c], 0.f), sum);
+      }
+      tc_fence_before();
+      mbar_arrive(&acce[a]);
+      if (valid) {
+        float* o = p.out + (size_t)b * p.out_stride;
+        if (p.mode == 1) {
+          const float ub = sum * scale;
+          if (p.out_plain) p.out_plain[(size_t)b * p.out_stride + out_idx] = ub;
+          o[out_idx] = ub + p.eps_rel * 448.f * scale * mag;
+        } else {
+          o[out_idx] = sum * scale;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace ls

@@ -1,0 +1,170 @@
+"""End-to-end ls_decode_step parity against the CPU oracle on every workload shape:
+the fp32 tiny config, the MLA batch at 128K (reduced, and at full size in the launch
+configuration the benchmark times), hot-buffer decode with 20% / 40% misses, the
+coarse-to-fine indexer at long context, and a ragged mixed batch."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle.ls_oracle as O
+from sparse_attention_decode_ls_b200 import binding as B
+from sparse_attention_decode_ls_b200 import synthetic as syn
+from sparse_attention_decode_ls_b200 import workload as W
+
+from gpu_helpers import DEV, assert_status_clean, bits16, check_topk_band, oracle_index_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_selection(inp, k):
+    scores = O.index_score(**oracle_index_inputs(inp))
+    idx = np.stack([O.topk_select(s, k)[0] for s in scores])
+    sel = np.stack([O.topk_select(s, k)[1] for s in scores])
+    return scores, idx, sel
+
+
+def _attn_on(wl, sel_idx, heads=None):
+    """Run the GPU attention stage alone on a given (oracle) selection."""
+    t = wl.tensors
+    o = torch.zeros_like(t["o"])
+    lse = torch.zeros_like(t["lse"])
+    a = B.attn_args(q=t["a_q"], k_rows=t["kv"], sel=torch.as_tensor(sel_idx, dtype=torch.int32, device=DEV),
+                    o=o, lse=lse, scale=wl.args.attn.softmax_scale, page_table=t["i_page_table"])
+    ws = torch.empty(max(1, B.ls_sparse_attn_workspace_size(a)), dtype=torch.uint8, device=DEV)
+    B.ls_sparse_attn_decode(a, ws)
+    torch.cuda.synchronize()
+    return o.float().cpu().numpy(), lse.cpu().numpy()
+
+
+def _check_mla_step(wl, inp, q, kv, k, heads_sample=None, full_ref=True):
+    wl.step()
+    torch.cuda.synchronize()
+    assert_status_clean()
+    scores, ref_idx, _ = _oracle_selection(inp, k)
+    gidx = wl.idx.cpu().numpy()
+    n_diff = sum(check_topk_band(gidx[b], scores[b], k) for b in range(wl.batch))
+    qb, kvb = bits16(q), bits16(kv)
+    pt = inp.page_table.numpy()
+    o_gpu = wl.o.float().cpu().numpy()
+    l_gpu = wl.lse.cpu().numpy()
+    if n_diff:
+        # the selections differ only inside the tie band: judge attention on the oracle's selection
+        o_gpu, l_gpu = _attn_on(wl, ref_idx)
+    for b in range(wl.batch):
+        rows = O.bf16_decode(O.selected_rows(kvb, pt[b], ref_idx[b]))
+        hs = slice(None) if heads_sample is None else heads_sample
+        o, l = O.sparse_attn_decode(O.bf16_decode(qb[b][hs]), rows, rows[:, :512], syn.softmax_scale(576))
+        assert np.abs(o_gpu[b][hs] - o).max() <= 2e-2, b
+        assert np.abs(l_gpu[b][hs] - l).max() <= 2e-2, b
+
+
+def test_decode_step_tiny_f32():
+    wl = W.tiny_f32()
+    wl.step()
+    torch.cuda.synchronize()
+    assert_status_clean()
+    inp = syn.indexer_f32([8192], heads=8, dim=64, seed=1001)
+    q, K, V = syn.f32_attention(1, 128, heads=16, d=128, seed=2001)
+    scores, ref_idx, _ = _oracle_selection(inp, 256)
+    gidx = wl.idx.cpu().numpy()[0]
+    check_topk_band(gidx, scores[0], 256)
+    pt = inp.page_table.numpy()[0]
+    kr = O.selected_rows(K.numpy().astype(np.float64), pt, gidx)
+    vr = O.selected_rows(V.numpy().astype(np.float64), pt, gidx)
+    if np.array_equal(gidx, ref_idx[0]):
+        o, l = O.sparse_attn_decode(q[0].double().numpy(), kr, vr, 1 / math.sqrt(128))
+        assert np.abs(wl.o.cpu().numpy()[0] - o).max() <= 1e-4
+        assert np.abs(wl.lse.cpu().numpy()[0] - l).max() <= 1e-4
+
+
+def test_decode_step_mla_reduced():
+    lens = [20000, 20000]
+    inp = syn.indexer_fp8(lens, seed=301)
+    q, kv = syn.mla_attention(2, inp.key_pool.shape[0], seed=302)
+    wl = W.build("mla_reduced", inp, k=2048, attn=dict(q=q, kv=kv, scale=syn.softmax_scale(576)))
+    _check_mla_step(wl, inp, q, kv, 2048)
+
+
+def test_decode_step_mla_full_size_bench_config():
+    """B=8 at 131,072 tokens, k=2,048: the configuration bench.py times.  Scores and
+    selections are checked for every request; attention on a sample of 16 heads."""
+    lens = [131072] * 8
+    inp = syn.indexer_fp8(lens, seed=1002)
+    q, kv = syn.mla_attention(8, inp.key_pool.shape[0], seed=2002)
+    wl = W.build("mla_full", inp, k=2048, attn=dict(q=q, kv=kv, scale=syn.softmax_scale(576)))
+    _check_mla_step(wl, inp, q, kv, 2048, heads_sample=slice(0, 128, 8))
+
+
+def _hotbuf_step(lens, miss_frac, seed):
+    Bn, k = len(lens), 2048
+    inp = syn.indexer_fp8(lens, seed=seed)
+    scores, ref_idx, ref_sel = _oracle_selection(inp, k)
+    ml = (max(lens) + 3) // 4 * 4
+    pos_of_slot, slot_of_pos, recent = syn.hot_buffer_state([r[r >= 0] for r in ref_idx], lens, n_slots=4096,
+                                                            miss_frac=miss_frac, seed=seed + 1, max_len=ml)
+    n_pool = inp.key_pool.shape[0]
+    q, kv = syn.mla_attention(Bn, n_pool, seed=seed + 2)
+    host = kv.view(torch.int16).pin_memory()
+    wl = W.build("hotbuf", inp, k=k, attn=dict(q=q, kv_host=True, scale=syn.softmax_scale(576)),
+                 hotbuf=dict(pos_of_slot=pos_of_slot, slot_of_pos=slot_of_pos, recent=recent,
+                             host_kv=host.view(torch.bfloat16)))
+    wl.step()
+    torch.cuda.synchronize()
+    assert_status_clean()
+    gidx = wl.idx.cpu().numpy()
+    for b in range(Bn):
+        check_topk_band(gidx[b], scores[b], k)
+    gsel = wl.tensors["sel"].cpu().numpy()
+    # the hot-buffer stage is checked bit-exactly on the oracle's own selection when the
+    # GPU chose the same set (no tie-band swap), which is the common case
+    qb = bits16(q)
+    kvb = bits16(kv)
+    pt = inp.page_table.numpy()
+    for b in range(Bn):
+        if not np.array_equal(gidx[b], ref_idx[b]):
+            continue
+        r = O.hotbuf_resolve(ref_idx[b], gsel[b] * 0 + ref_sel[b].astype(np.float32), pos_of_slot[b].numpy(),
+                             recent[b].numpy(), slot_of_pos[b].numpy())
+        assert int(wl.tensors["n_miss"][b]) == r["n_miss"]
+        assert r["n_miss"] == int(round(miss_frac * k))
+        assert np.array_equal(wl.tensors["pos_of_slot"][b].cpu().numpy(), r["pos_of_slot"])
+        assert np.array_equal(wl.tensors["slot_of_pos"][b].cpu().numpy(), r["slot_of_pos"])
+        # every selected row now sits in the hot buffer with the history's bytes
+        hb = wl.tensors["hbuf"][b].view(torch.int16).cpu().numpy()
+        for p in ref_idx[b][:64]:
+            s = r["slot_of_pos"][p]
+            assert np.array_equal(hb[s], kvb[pt[b, p // 64], p % 64])
+        rows = O.bf16_decode(O.selected_rows(kvb, pt[b], ref_idx[b]))
+        o, l = O.sparse_attn_decode(O.bf16_decode(qb[b]), rows, rows[:, :512], syn.softmax_scale(576))
+        assert np.abs(wl.o[b].float().cpu().numpy() - o).max() <= 2e-2
+        assert np.abs(wl.lse[b].cpu().numpy() - l).max() <= 2e-2
+
+
+@pytest.mark.parametrize("miss_frac", [0.2, 0.4])
+def test_decode_step_hot_buffer(miss_frac):
+    _hotbuf_step([131072, 131072], miss_frac, seed=401)
+
+
+def test_decode_step_ragged_hot_buffer():
+    lens = syn.ragged_lens(6, seed=1005)
+    _hotbuf_step(lens, 0.2, seed=501)
+
+
+def test_decode_step_coarse_to_fine():
+    from test_gpu_stages import _c2f_inputs
+    lens = [64 * 8192, 64 * 5000 + 7]
+    inp = _c2f_inputs(lens, seed=601, clustered=True)
+    q, kv = syn.mla_attention(2, inp.key_pool.shape[0], seed=602)
+    wl = W.build("c2f", inp, k=2048, attn=dict(q=q, kv=kv, scale=syn.softmax_scale(576)), c2f=True)
+    full = W.build("full", inp, k=2048, attn=dict(q=q, kv=kv, scale=syn.softmax_scale(576)))
+    wl.step()
+    full.step()
+    torch.cuda.synchronize()
+    assert_status_clean()
+    assert torch.equal(wl.idx, full.idx)
+    assert torch.equal(wl.o, full.o)
+    n = wl.tensors["n_survivors"].cpu().numpy()
+    assert (n < np.array([-(-L // 64) for L in lens]) * 0.5).all()
+    _check_mla_step(full, inp, q, kv, 2048, heads_sample=slice(0, 128, 16))
