@@ -135,7 +135,8 @@ ls_status validate_index(const ls_index_score_args* a, bool need_scores) {
       return fail(LS_ERR_UNSUPPORTED, "e4m3 indexer is built for 64 heads x 128 dims (got %d x %d)", a->heads,
                   a->dim);
     LS_REQUIRE(a->q_scale && a->key_scale, "q_scale and key_scale are required for e4m3 keys");
-    LS_REQUIRE(aligned16(a->q) && aligned16(a->key_pool), "q and key_pool must be 16-byte aligned");
+    LS_REQUIRE(aligned16(a->q) && aligned16(a->key_pool) && aligned16(a->key_scale),
+               "q, key_pool and key_scale must be 16-byte aligned");
   } else if (a->key_dtype == LS_F32) {
     if (a->heads < 1 || a->heads > 64 || a->dim < 1 || a->dim > 128 || (a->dim & 3))
       return fail(LS_ERR_UNSUPPORTED, "f32 indexer: heads in [1,64], dim in [4,128] multiple of 4");
@@ -212,8 +213,60 @@ ls_status launch_index_tc(const ls_index_score_args* a, int mode, const int* uni
 }
 
 // ---- top-k launch -------------------------------------------------------------------
-std::atomic<uint64_t> g_smem_topk{0};
-constexpr int kTopkCluster = 8;
+// One cluster per request: 16 CTAs where the device can co-schedule them (non-portable
+// cluster size), else the portable 8.
+std::atomic<uint64_t> g_smem_topk8{0}, g_smem_topk16{0};
+std::atomic<int> g_topk16_ok[64];  // per device: 0 unknown, 1 yes, -1 no
+
+template <int CL>
+cudaLaunchConfig_t topk_config(int B, int smem, cudaStream_t st, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(B * CL);
+  cfg.blockDim = dim3(ls::kTopkThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+bool topk16_supported(cudaStream_t st) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::atomic<int>& flag16 = g_topk16_ok[dev & 63];
+  int v = flag16.load();
+  if (v != 0) return v > 0;
+  bool ok = cudaFuncSetAttribute(ls::topk_cluster<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+            cudaSuccess;
+  if (ok) ok = allow_smem(ls::topk_cluster<16>, ls::kTopkCacheKeys * 4, g_smem_topk16) == cudaSuccess;
+  if (ok) {
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = topk_config<16>(1, ls::kTopkCacheKeys * 4, st, attr);
+    int n = 0;
+    ok = cudaOccupancyMaxActiveClusters(&n, ls::topk_cluster<16>, &cfg) == cudaSuccess && n >= 1;
+  }
+  cudaGetLastError();  // a refused probe leaves no sticky error
+  flag16.store(ok ? 1 : -1);
+  return ok;
+}
+
+template <int CL>
+ls_status launch_topk_cl(const ls::TopkParams& p0, int B, cudaStream_t st, std::atomic<uint64_t>& smem_done) {
+  ls::TopkParams p = p0;
+  const int lc = (((p.len_limit + CL - 1) / CL) + 3) & ~3;
+  p.cache_keys = lc <= ls::kTopkCacheKeys ? lc : 0;
+  if (allow_smem(ls::topk_cluster<CL>, ls::kTopkCacheKeys * 4, smem_done) != cudaSuccess)
+    return check_launch("topk attribute");
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = topk_config<CL>(B, p.cache_keys * 4, st, attr);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, ls::topk_cluster<CL>, p);
+  if (e != cudaSuccess) return fail(LS_ERR_CUDA, "topk_cluster: %s", cudaGetErrorString(e));
+  return check_launch("topk_cluster");
+}
 
 ls_status launch_topk(int B, int k, const float* scores, int stride, const int* lens, int len_mul, int len_div,
                       int len_limit, const int* unit_list, int list_stride, int* idx, float* sel, float* thr,
@@ -222,26 +275,8 @@ ls_status launch_topk(int B, int k, const float* scores, int stride, const int* 
   p.B = B; p.k = k; p.stride = stride; p.scores = scores; p.lens = lens; p.len_mul = len_mul;
   p.len_div = len_div; p.len_limit = len_limit; p.unit_list = unit_list; p.list_stride = list_stride;
   p.idx = idx; p.sel = sel; p.thr = thr;
-  const int lc = (((len_limit + kTopkCluster - 1) / kTopkCluster) + 3) & ~3;
-  p.cache_keys = lc <= ls::kTopkCacheKeys ? lc : 0;
-  const int smem = p.cache_keys * 4;
-  if (allow_smem(ls::topk_cluster<kTopkCluster>, ls::kTopkCacheKeys * 4, g_smem_topk) != cudaSuccess)
-    return check_launch("topk attribute");
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(B * kTopkCluster);
-  cfg.blockDim = dim3(ls::kTopkThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kTopkCluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, ls::topk_cluster<kTopkCluster>, p);
-  if (e != cudaSuccess) return fail(LS_ERR_CUDA, "topk_cluster: %s", cudaGetErrorString(e));
-  return check_launch("topk_cluster");
+  if (topk16_supported(st)) return launch_topk_cl<16>(p, B, st, g_smem_topk16);
+  return launch_topk_cl<8>(p, B, st, g_smem_topk8);
 }
 
 // ---- attention ------------------------------------------------------------------------

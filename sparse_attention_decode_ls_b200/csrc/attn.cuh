@@ -139,7 +139,7 @@ constexpr int kNumBars = 2 + 2 + 2 + 1 + 1 + 1;        // kv_full[2] kv_empty[2]
 constexpr int kOffTmem = kOffBar + kNumBars * 8;
 constexpr int kSmem = 1024 + kOffTmem + 16;
 constexpr int kThreads = 256;
-constexpr int kLoaders = 96;                           // warps 0, 1, 3
+constexpr int kLoaders = 32;                           // one warp per KV stage
 constexpr int kChunksPerRow = DK * 2 / 16;             // 72
 constexpr uint32_t kIdescS = make_idesc(1 /*bf16*/, 128, N, false, false);
 constexpr uint32_t kIdescO = make_idesc(1 /*bf16*/, 128, DVH, false, true);
@@ -161,7 +161,7 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
   uint32_t* tmem_slot = (uint32_t*)(sm + kOffTmem);
   __shared__ long long s_rowoff[2][N];  // byte offset of each row of a stage, -1 if absent
   __shared__ int s_abort;
-  __shared__ int s_loader_go;
+  __shared__ uint32_t s_mask[2];        // valid rows of the tile in each stage
 
   const int b = blockIdx.y;
   const int half = blockIdx.x & 1;
@@ -207,38 +207,38 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
   const uint32_t tm_o = tmem;          // columns [0, 256): O half
   const uint32_t tm_s = tmem + 256;    // columns [256, 320): S double buffer
 
-  if (warp == 0 || warp == 1 || warp == 3) {
-    // ================= loaders: gather the tile's rows =================
-    const int lt = (warp == 3) ? 64 + lane : warp * 32 + lane;
-    for (int i = 0; i < my_tiles; ++i) {
-      const int st = i & 1;
-      // one thread decides whether to go on, so the named barrier stays uniform
-      if (lt == 0) {
-        bool go = (i < 2) || mbar_wait(&kv_empty[st], ((i >> 1) - 1) & 1);
-        if (*(volatile int*)&s_abort) go = false;
+  if (warp == 0 || warp == 1) {
+    // ================= loaders: warp w fills stage w with tiles w, w+2, ... =================
+    // Lane r owns row r of a tile (its row offset and validity); the copies are spread
+    // over the warp chunk by chunk so consecutive lanes read consecutive bytes.
+    const int st = warp;
+    for (int i = st; i < my_tiles; i += 2) {
+      int go = 1;
+      if (lane == 0) {  // one lane decides, so the warp stays converged
+        go = (i < 2) || mbar_wait(&kv_empty[st], ((i >> 1) - 1) & 1);
+        if (*(volatile int*)&s_abort) go = 0;
         if (!go) s_abort = 1;
-        s_loader_go = go ? 1 : 0;
       }
-      const int j0 = (t0 + i) * N;
-      if (lt < N) {
-        const int j = j0 + lt;
-        long long off = -1;
-        if (j < p.k) {
-          const long long r = attn_row(p, b, p.sel[(size_t)b * p.k + j]);
-          if (r >= 0) off = r * p.row_stride * 2;
-        }
-        s_rowoff[st][lt] = off;
+      go = __shfl_sync(0xffffffffu, go, 0);
+      if (!go) break;
+      const int j = (t0 + i) * N + lane;
+      long long off = -1;
+      if (j < p.k) {
+        const long long r = attn_row(p, b, p.sel[(size_t)b * p.k + j]);
+        if (r >= 0) off = r * p.row_stride * 2;
       }
-      asm volatile("bar.sync 1, 96;" ::: "memory");
-      if (!s_loader_go) break;
+      const uint32_t vmask = __ballot_sync(0xffffffffu, off >= 0);
+      if (lane == 0) s_mask[st] = vmask;
+      s_rowoff[st][lane] = off;
+      __syncwarp();
       const uint32_t dst0 = sbase + kOffKv + st * kKvBytes;
-      for (int e = lt; e < N * kChunksPerRow; e += kLoaders) {
+      for (int e = lane; e < N * kChunksPerRow; e += 32) {
         const int r = e / kChunksPerRow, c = e - r * kChunksPerRow;
         const int pn = c >> 3, jj = c & 7;
         const uint32_t dst = dst0 + pn * kKvPanel + r * 128 + ((jj ^ (r & 7)) << 4);
-        const long long off = s_rowoff[st][r];
-        if (off >= 0) {
-          cp_async_16(dst, kv_base + off + c * 16);
+        const long long ro = s_rowoff[st][r];
+        if (ro >= 0) {
+          cp_async_16(dst, kv_base + ro + c * 16);
         } else {
           asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0) : "memory");
         }
@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
       cp_async_wait<0>();
       fence_proxy_async_smem();
       mbar_arrive(&kv_full[st]);
-      asm volatile("bar.sync 1, 96;" ::: "memory");  // s_rowoff / s_loader_go reusable
+      __syncwarp();
     }
   } else if (warp == 2) {
     // ================= MMA issuer =================
@@ -301,13 +301,9 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
     bool ok = true;
     for (int i = 0; i < my_tiles; ++i) {
       const int st = i & 1;
-      const int j0 = (t0 + i) * N;
-      uint32_t vmask = 0;
-#pragma unroll 4
-      for (int r = 0; r < N; ++r) {
-        const int j = j0 + r;
-        if (j < p.k && attn_row(p, b, p.sel[(size_t)b * p.k + j]) >= 0) vmask |= 1u << r;
-      }
+      // the loader published the tile's valid rows with its kv_full arrival
+      if (!mbar_wait(&kv_full[st], (i >> 1) & 1)) { ok = false; break; }
+      const uint32_t vmask = s_mask[st];
       if (!mbar_wait(&s_full[st], (i >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
       float s[N];
@@ -335,7 +331,9 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
         psum += pr[r];
       }
       if (i >= 1 && !mbar_wait(p_free, (i - 1) & 1)) { ok = false; break; }
-      if (rescale) {
+      // tcgen05.ld/st are warp-collective: the whole warp rescales when any lane must
+      // (lanes that need not have factor 1)
+      if (__any_sync(0xffffffffu, rescale)) {
         tc_fence_after();
 #pragma unroll 1
         for (int c0 = 0; c0 < DVH; c0 += 32) {
@@ -365,7 +363,9 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
       mbar_arrive(p_full);
     }
     // ---- epilogue
-    if (ok && my_tiles > 0 && mbar_wait(o_done, 0)) {
+    bool fin = ok && my_tiles > 0 && mbar_wait(o_done, 0);
+    fin = __all_sync(0xffffffffu, fin);  // the TMEM reads below are warp-collective
+    if (fin) {
       tc_fence_after();
       const bool single = p.nsplit == 1;
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;

@@ -110,7 +110,7 @@ struct IdxTcParams {
   int list_stride;
   float* out;              // [B,out_stride]
   long long out_stride;
-  float* out_plain;        // mode 1: bound without margin (may be NULL)
+  float* out_plain;        // mode 1: bound without margin, [B,max_blocks] (may be NULL)
   float eps_rel;           // mode 1: margin relative to the block magnitude bound
 };
 
@@ -123,7 +123,9 @@ struct IdxTc {
   static constexpr int kAcc = 256 / NCOL;              // accumulators in 256 TMEM columns
   static constexpr int kBBytes = KP * NCOL * 128;
   static constexpr int kOffB = kStages * kStageBytes;
-  static constexpr int kOffCoef = kOffB + kBBytes;
+  static constexpr int kOffScale = kOffB + kBBytes;                  // [kStages][128] row scales
+  static constexpr int kOffMeta = kOffScale + kStages * 128 * 4;     // [kStages][2] logical unit ids
+  static constexpr int kOffCoef = kOffMeta + ((kStages * 8 + 15) & ~15);
   static constexpr int kOffBar = kOffCoef + NCOL * 4 + 16;
   static constexpr int kNumBars = 2 * kStages + 2 * kAcc;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
@@ -154,6 +156,8 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sm = (uint8_t*)(((uintptr_t)sm_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = sm;
   uint8_t* sB = sm + C::kOffB;
+  float* s_scale = (float*)(sm + C::kOffScale);
+  int* s_meta = (int*)(sm + C::kOffMeta);
   float* coef = (float*)(sm + C::kOffCoef);
   float* gmag = coef + NCOL;  // mode 1: sum_h |w'_h| * sum_d |q8_hd|
   uint64_t* bars = (uint64_t*)(sm + C::kOffBar);
@@ -254,7 +258,7 @@ __global__ void __launch_bounds__(192, 1)
   if (tid == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], 1 + 128);  // MMA commit + every epilogue thread
     }
     for (int a = 0; a < C::kAcc; ++a) {
       mbar_init(&accf[a], 1);
@@ -271,6 +275,10 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 0) {
     // ================= TMA producer =================
+    // Per tile: the keys of its two 64-row units (TMA, 128-byte swizzle) and, for keys,
+    // their 64 token scales (bulk copy) into the stage, plus each unit's logical id.
+    // A stage is released only when the MMA has consumed it and the epilogue has read
+    // its scales and ids.
     if (lane == 0) {
       prefetch_tmap(&tmap);
       int issued = 0;
@@ -282,16 +290,22 @@ __global__ void __launch_bounds__(192, 1)
         }
         if (*(volatile int*)&s_abort) break;
         const int tile = t_begin + i;
-        int rows[2], lp;
+        int rows[2], lps[2];
         uint32_t bytes = 0;
         for (int uu = 0; uu < 2; ++uu) {
           const int u = 2 * tile + uu;
           rows[uu] = -1;
+          lps[uu] = -1;
           if (u < n_units) {
-            rows[uu] = idx_unit_row(p, b, u, &lp);
-            if (rows[uu] < 0) flag(LS_DEV_BOUNDS);
-            else bytes += KP * 64 * 128;
+            rows[uu] = idx_unit_row(p, b, u, &lps[uu]);
+            if (rows[uu] < 0) {
+              flag(LS_DEV_BOUNDS);
+              lps[uu] = -1;
+            } else {
+              bytes += KP * 64 * 128 + (p.mode == 0 ? 256 : 0);
+            }
           }
+          s_meta[st * 2 + uu] = lps[uu];
         }
         mbar_arrive_expect_tx(&full[st], bytes);
         const uint32_t dst = smem_u32(sA + st * C::kStageBytes);
@@ -299,6 +313,8 @@ __global__ void __launch_bounds__(192, 1)
           if (rows[uu] < 0) continue;
           for (int pk = 0; pk < KP; ++pk)
             tma_load_2d(dst + pk * C::kPanel + uu * 64 * 128, &tmap, &full[st], pk * 128, rows[uu]);
+          if (p.mode == 0)
+            bulk_load(smem_u32(s_scale + st * 128 + uu * 64), p.row_scale + rows[uu], 256, &full[st]);
         }
         ++issued;
       }
@@ -334,33 +350,30 @@ __global__ void __launch_bounds__(192, 1)
     // ================= epilogue: warps 2..5, thread = tile row =================
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
+    const int rr = r & 63;
     const float mag = (p.mode == 1) ? gmag[0] : 0.f;
+    const int nb = (L + 63) >> 6;
     for (int i = 0; i < my_tiles; ++i) {
-      const int a = i % C::kAcc;
+      const int st = i % C::kStages, a = i % C::kAcc;
       const int tile = t_begin + i;
-      const int u = 2 * tile + (r >> 6), rr = r & 63;
-      // which output does this row feed?
+      const int u = 2 * tile + (r >> 6);
+      // the stage's unit ids and scales (written by the producer / TMA) -- acquire them
+      if (!mbar_wait(&full[st], (i / C::kStages) & 1)) { s_abort = 1; break; }
+      const int lp = s_meta[st * 2 + (r >> 6)];
       bool valid = false;
       float scale = 0.f;
       long long out_idx = 0;
-      if (u < n_units) {
-        if (p.mode == 1) {
-          const int j = u * 64 + rr;
-          if (j < ((L + 63) >> 6)) {
-            valid = true;
-            scale = p.row_scale[(size_t)b * p.max_blocks + j];
-            out_idx = j;
-          }
-        } else {
-          int lp;
-          const int row = idx_unit_row(p, b, u, &lp);
-          const int s = lp * 64 + rr;
-          if (row >= 0 && s < L) {
-            valid = true;
-            scale = p.row_scale[(size_t)row + rr];
-            out_idx = p.unit_list ? (long long)u * 64 + rr : s;
-          }
+      if (p.mode == 1) {
+        const int j = u * 64 + rr;
+        if (lp >= 0 && j < nb) {
+          valid = true;
+          scale = p.row_scale[(size_t)b * p.max_blocks + j];
+          out_idx = j;
         }
+      } else if (lp >= 0 && lp * 64 + rr < L) {
+        valid = true;
+        scale = s_scale[st * 128 + r];
+        out_idx = p.unit_list ? (long long)u * 64 + rr : (long long)lp * 64 + rr;
       }
       if (!mbar_wait(&accf[a], (i / C::kAcc) & 1)) { s_abort = 1; break; }
       tc_fence_after();
@@ -376,11 +389,12 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc_fence_before();
       mbar_arrive(&acce[a]);
+      mbar_arrive(&empty[st]);
       if (valid) {
         float* o = p.out + (size_t)b * p.out_stride;
         if (p.mode == 1) {
           const float ub = sum * scale;
-          if (p.out_plain) p.out_plain[(size_t)b * p.out_stride + out_idx] = ub;
+          if (p.out_plain) p.out_plain[(size_t)b * p.max_blocks + out_idx] = ub;
           o[out_idx] = ub + p.eps_rel * 448.f * scale * mag;
         } else {
           o[out_idx] = sum * scale;

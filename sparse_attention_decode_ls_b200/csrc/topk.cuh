@@ -154,17 +154,24 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
   const uint32_t T = prefix;   // exact k-th largest key
   const uint32_t R = k_rem;    // how many keys == T are taken (lowest positions first)
 
-  // ---- emit: contiguous per-thread ranges keep position order
-  const int per_t = (m + kTopkThreads - 1) / kTopkThreads;
-  const int i0 = min(m, tid * per_t), i1 = min(m, i0 + per_t);
+  // ---- emit: each warp owns a contiguous segment (position order) and walks it 32 keys
+  // at a time, so shared-memory reads are conflict-free and ballots give the ranks
+  const int lane = lane_id(), warp = warp_id();
+  constexpr int kWarps = kTopkThreads / 32;
+  const int seg = ((m + kWarps * 32 - 1) / (kWarps * 32)) * 32;
+  const int i0 = min(m, warp * seg), i1 = min(m, i0 + seg);
   uint32_t n_gt = 0, n_eq = 0;
-  for (int i = i0; i < i1; ++i) {
-    const uint32_t key = key_at(i);
-    n_gt += key > T;
-    n_eq += key == T;
+  for (int base = i0; base < i1; base += 32) {
+    const int i = base + lane;
+    const uint32_t key = i < i1 ? key_at(i) : 0u;
+    n_gt += __popc(__ballot_sync(0xffffffffu, i < i1 && key > T));
+    n_eq += __popc(__ballot_sync(0xffffffffu, i < i1 && key == T));
   }
+  // warp totals -> exclusive prefix over warps (block scan on one value per thread)
+  const unsigned long long mine = lane == 0 ? (((unsigned long long)n_gt << 32) | n_eq) : 0ull;
   unsigned long long tot;
-  const unsigned long long pre = block_excl_scan_u64(((unsigned long long)n_gt << 32) | n_eq, scan_tmp, &tot);
+  const unsigned long long pre_t = block_excl_scan_u64(mine, scan_tmp, &tot);
+  const unsigned long long pre = __shfl_sync(0xffffffffu, pre_t, 0);
   if (tid == 0) cnt_pub = tot;
   __syncthreads();
   cluster.sync();
@@ -178,23 +185,26 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
   }
   const uint32_t eq_left = R > eq_before ? R - eq_before : 0u;  // ties this CTA may still take
   const uint32_t gt_pre = (uint32_t)(pre >> 32), eq_pre = (uint32_t)pre;
-  uint32_t eq_seen = eq_pre;
+  uint32_t eq_seen = eq_pre;  // keys == T before this lane's current key, CTA-wide
   uint32_t out = out_before + gt_pre + min(eq_pre, eq_left);
-  for (int i = i0; i < i1; ++i) {
-    const uint32_t key = key_at(i);
-    bool take = key > T;
-    if (key == T) {
-      take = eq_seen < eq_left;
-      ++eq_seen;
-    }
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int base = i0; base < i1; base += 32) {
+    const int i = base + lane;
+    const bool in = i < i1;
+    const uint32_t key = in ? key_at(i) : 0u;
+    const uint32_t eq_mask = __ballot_sync(0xffffffffu, in && key == T);
+    const bool take = in && (key > T || (key == T && eq_seen + __popc(eq_mask & lt_mask) < eq_left));
+    const uint32_t take_mask = __ballot_sync(0xffffffffu, take);
     if (take) {
-      const int gi = c0 + i;
-      if (out < (uint32_t)k) {
-        if (p.idx) p.idx[(size_t)b * k + out] = topk_pos(p, b, gi);
-        if (p.sel) p.sel[(size_t)b * k + out] = key_float(key);
+      const uint32_t o = out + __popc(take_mask & lt_mask);
+      if (o < (uint32_t)k) {
+        const int gi = c0 + i;
+        if (p.idx) p.idx[(size_t)b * k + o] = topk_pos(p, b, gi);
+        if (p.sel) p.sel[(size_t)b * k + o] = key_float(key);
       }
-      ++out;
     }
+    out += __popc(take_mask);
+    eq_seen += __popc(eq_mask);
   }
   if (p.thr && rank == 0 && tid == 0) p.thr[b] = key_float(T);
   cluster.sync();  // keep this CTA's shared memory alive until the cluster is done with it

@@ -132,7 +132,7 @@ def _hotbuf_step(lens, miss_frac, seed):
         assert np.array_equal(wl.tensors["pos_of_slot"][b].cpu().numpy(), r["pos_of_slot"])
         assert np.array_equal(wl.tensors["slot_of_pos"][b].cpu().numpy(), r["slot_of_pos"])
         # every selected row now sits in the hot buffer with the history's bytes
-        hb = wl.tensors["hbuf"][b].view(torch.int16).cpu().numpy()
+        hb = wl.tensors["hbuf"][b].view(torch.int16).cpu().numpy().view(np.uint16)
         for p in ref_idx[b][:64]:
             s = r["slot_of_pos"][p]
             assert np.array_equal(hb[s], kvb[pt[b, p // 64], p % 64])
