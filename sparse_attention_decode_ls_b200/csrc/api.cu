@@ -242,10 +242,10 @@ bool topk16_supported(cudaStream_t st) {
   if (v != 0) return v > 0;
   bool ok = cudaFuncSetAttribute(ls::topk_cluster<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
             cudaSuccess;
-  if (ok) ok = allow_smem(ls::topk_cluster<16>, ls::kTopkCacheKeys * 4, g_smem_topk16) == cudaSuccess;
+  if (ok) ok = allow_smem(ls::topk_cluster<16>, ls::kTopkCacheKeys * 4 + ls::kTopkExtraBytes, g_smem_topk16) == cudaSuccess;
   if (ok) {
     cudaLaunchAttribute attr[1];
-    cudaLaunchConfig_t cfg = topk_config<16>(1, ls::kTopkCacheKeys * 4, st, attr);
+    cudaLaunchConfig_t cfg = topk_config<16>(1, ls::kTopkCacheKeys * 4 + ls::kTopkExtraBytes, st, attr);
     int n = 0;
     ok = cudaOccupancyMaxActiveClusters(&n, ls::topk_cluster<16>, &cfg) == cudaSuccess && n >= 1;
   }
@@ -259,10 +259,10 @@ ls_status launch_topk_cl(const ls::TopkParams& p0, int B, cudaStream_t st, std::
   ls::TopkParams p = p0;
   const int lc = (((p.len_limit + CL - 1) / CL) + 3) & ~3;
   p.cache_keys = lc <= ls::kTopkCacheKeys ? lc : 0;
-  if (allow_smem(ls::topk_cluster<CL>, ls::kTopkCacheKeys * 4, smem_done) != cudaSuccess)
+  if (allow_smem(ls::topk_cluster<CL>, ls::kTopkCacheKeys * 4 + ls::kTopkExtraBytes, smem_done) != cudaSuccess)
     return check_launch("topk attribute");
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = topk_config<CL>(B, p.cache_keys * 4, st, attr);
+  cudaLaunchConfig_t cfg = topk_config<CL>(B, p.cache_keys * 4 + ls::kTopkExtraBytes, st, attr);
   cudaError_t e = cudaLaunchKernelEx(&cfg, ls::topk_cluster<CL>, p);
   if (e != cudaSuccess) return fail(LS_ERR_CUDA, "topk_cluster: %s", cudaGetErrorString(e));
   return check_launch("topk_cluster");
@@ -350,7 +350,7 @@ ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressi
     ls::attn_mla_tc<<<dim3(2 * ns, a->batch), ls::mla::kThreads, ls::mla::kSmem, st>>>(p);
     LS_TRY(check_launch("attn_mla_tc"));
     if (ns > 1) {
-      ls::attn_combine<<<(a->batch * ls::mla::H + 3) / 4, 128, 0, st>>>(p);
+      ls::attn_combine<<<dim3(ls::mla::DV / 32, a->batch), 128, 0, st>>>(p);
       LS_TRY(check_launch("attn_combine"));
     }
     return LS_OK;

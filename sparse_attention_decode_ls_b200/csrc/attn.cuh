@@ -37,7 +37,7 @@ struct AttnParams {
   void* o;
   float* lse;
   int nsplit;
-  float* part_o;     // [B,nsplit,H,dv] unnormalised partial outputs
+  float* part_o;     // [B,nsplit,dv,H] unnormalised partial outputs (head fastest)
   float* part_ml;    // [B,nsplit,H,2] running max (log2 domain) and sum
 };
 
@@ -159,7 +159,6 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
   uint64_t* p_free = bars + 7;
   uint64_t* o_done = bars + 8;
   uint32_t* tmem_slot = (uint32_t*)(sm + kOffTmem);
-  __shared__ long long s_rowoff[2][N];  // byte offset of each row of a stage, -1 if absent
   __shared__ int s_abort;
   __shared__ uint32_t s_mask[2];        // valid rows of the tile in each stage
 
@@ -229,18 +228,24 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
       }
       const uint32_t vmask = __ballot_sync(0xffffffffu, off >= 0);
       if (lane == 0) s_mask[st] = vmask;
-      s_rowoff[st][lane] = off;
-      __syncwarp();
+      // lane l copies chunks l, l+32, l+64 of every row (consecutive lanes, consecutive
+      // 16-byte pieces of one row); row offsets travel by shuffle
       const uint32_t dst0 = sbase + kOffKv + st * kKvBytes;
-      for (int e = lane; e < N * kChunksPerRow; e += 32) {
-        const int r = e / kChunksPerRow, c = e - r * kChunksPerRow;
-        const int pn = c >> 3, jj = c & 7;
-        const uint32_t dst = dst0 + pn * kKvPanel + r * 128 + ((jj ^ (r & 7)) << 4);
-        const long long ro = s_rowoff[st][r];
-        if (ro >= 0) {
-          cp_async_16(dst, kv_base + ro + c * 16);
-        } else {
-          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0) : "memory");
+#pragma unroll 4
+      for (int r = 0; r < N; ++r) {
+        const long long ro = __shfl_sync(0xffffffffu, off, r);
+        const uint32_t rbase = dst0 + r * 128;
+#pragma unroll
+        for (int q = 0; q < 3; ++q) {
+          const int c = lane + 32 * q;
+          if (c < kChunksPerRow) {
+            const uint32_t dst = rbase + (c >> 3) * kKvPanel + ((uint32_t)((c & 7) ^ (r & 7)) << 4);
+            if (ro >= 0) {
+              cp_async_16(dst, kv_base + ro + c * 16);
+            } else {
+              asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0) : "memory");
+            }
+          }
         }
       }
       cp_async_commit();
@@ -291,8 +296,8 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
       if (!ok) s_abort = 1;
       tc_commit(o_done);
     }
-  } else {
-    // ================= softmax: warps 4..7, thread = head =================
+  } else if (warp >= 4) {
+    // ================= softmax: warps 4..7, thread = head (warp 3 has no role) =================
     const int wq = warp & 3;
     const int h = wq * 32 + lane;
     const float sl2 = p.scale * kLog2e;
@@ -308,7 +313,6 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
       tc_fence_after();
       float s[N];
       tmem_ld32(tm_s + lane_off + st * N, s);
-      tmem_wait_ld();
       float tmax = -INFINITY;
 #pragma unroll
       for (int r = 0; r < N; ++r)
@@ -339,7 +343,6 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
         for (int c0 = 0; c0 < DVH; c0 += 32) {
           float v[32];
           tmem_ld32(tm_o + lane_off + c0, v);
-          tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 32; ++c) v[c] *= factor;
           tmem_st32(tm_o + lane_off + c0, v);
@@ -372,7 +375,6 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
       for (int c0 = 0; c0 < DVH; c0 += 32) {
         float v[32];
         tmem_ld32(tm_o + lane_off + c0, v);
-        tmem_wait_ld();
         if (single) {
           __nv_bfloat16* o = (__nv_bfloat16*)p.o + ((size_t)b * H + h) * DV + half * DVH + c0;
 #pragma unroll
@@ -386,11 +388,10 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
             *(uint4*)(o + c) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         } else {
-          float* o = p.part_o + (((size_t)b * p.nsplit + split) * H + h) * DV + half * DVH + c0;
+          // head-fastest layout [b][split][dim][head]: consecutive threads, consecutive words
+          float* o = p.part_o + (((size_t)b * p.nsplit + split) * DV + half * DVH + c0) * H + h;
 #pragma unroll
-          for (int c = 0; c < 32; c += 4)
-            *(float4*)(o + c) = make_float4(l_run > 0.f ? v[c] : 0.f, l_run > 0.f ? v[c + 1] : 0.f,
-                                            l_run > 0.f ? v[c + 2] : 0.f, l_run > 0.f ? v[c + 3] : 0.f);
+          for (int c = 0; c < 32; ++c) o[(size_t)c * H] = l_run > 0.f ? v[c] : 0.f;
         }
       }
       if (half == 0) {
@@ -403,8 +404,8 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
         }
       }
     } else if (my_tiles == 0 && p.nsplit > 1) {
-      float* o = p.part_o + (((size_t)b * p.nsplit + split) * H + h) * DV + half * DVH;
-      for (int c = 0; c < DVH; ++c) o[c] = 0.f;
+      float* o = p.part_o + (((size_t)b * p.nsplit + split) * DV + half * DVH) * H + h;
+      for (int c = 0; c < DVH; ++c) o[(size_t)c * H] = 0.f;
       if (half == 0) {
         float* ml = p.part_ml + (((size_t)b * p.nsplit + split) * H + h) * 2;
         ml[0] = -INFINITY;
@@ -412,6 +413,9 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
       }
     }
   }
+  // every warp must reach the barrier converged (the MMA warp's lane 0 arrives last);
+  // only then may TMEM be released
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 2) {
@@ -421,40 +425,33 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
 }
 
 // Merge split-KV partials: o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
-// One warp per (request, head); each lane owns 16 of the 512 output dims.
+// grid (DV / 32, B), 128 threads: thread = head, 32 output dims per CTA; every read of
+// the head-fastest partials is coalesced across the warp.
 __global__ void __launch_bounds__(128) attn_combine(const AttnParams p) {
   using namespace mla;
-  const int gw = blockIdx.x * 4 + warp_id();
-  const int lane = lane_id();
-  if (gw >= p.B * H) return;
-  const int b = gw / H, h = gw - b * H;
+  const int d0 = blockIdx.x * 32, b = blockIdx.y, h = threadIdx.x;
+  const float* ml = p.part_ml + (size_t)b * p.nsplit * H * 2;
   float M = -INFINITY;
-  for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, p.part_ml[(((size_t)b * p.nsplit + s) * H + h) * 2]);
-  float acc[16];
+  for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, ml[((size_t)s * H + h) * 2]);
+  float acc[32];
 #pragma unroll
-  for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+  for (int e = 0; e < 32; ++e) acc[e] = 0.f;
   float Lsum = 0.f;
   if (M != -INFINITY) {
     for (int s = 0; s < p.nsplit; ++s) {
-      const float* ml = p.part_ml + (((size_t)b * p.nsplit + s) * H + h) * 2;
-      if (ml[1] <= 0.f) continue;
-      const float wgt = exp2f(ml[0] - M);
-      Lsum += wgt * ml[1];
-      const float* po = p.part_o + (((size_t)b * p.nsplit + s) * H + h) * DV + lane * 16;
+      const float l = ml[((size_t)s * H + h) * 2 + 1];
+      if (l <= 0.f) continue;
+      const float wgt = exp2f(ml[((size_t)s * H + h) * 2] - M);
+      Lsum += wgt * l;
+      const float* po = p.part_o + (((size_t)b * p.nsplit + s) * DV + d0) * H + h;
 #pragma unroll
-      for (int e = 0; e < 16; e += 4) {
-        const float4 v = *(const float4*)(po + e);
-        acc[e] += wgt * v.x;
-        acc[e + 1] += wgt * v.y;
-        acc[e + 2] += wgt * v.z;
-        acc[e + 3] += wgt * v.w;
-      }
+      for (int e = 0; e < 32; ++e) acc[e] = fmaf(wgt, po[(size_t)e * H], acc[e]);
     }
   }
   const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-  __nv_bfloat16* o = (__nv_bfloat16*)p.o + ((size_t)b * H + h) * DV + lane * 16;
+  __nv_bfloat16* o = (__nv_bfloat16*)p.o + ((size_t)b * H + h) * DV + d0;
 #pragma unroll
-  for (int e = 0; e < 16; e += 8) {
+  for (int e = 0; e < 32; e += 8) {
     uint32_t w[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -463,7 +460,7 @@ __global__ void __launch_bounds__(128) attn_combine(const AttnParams p) {
     }
     *(uint4*)(o + e) = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  if (lane == 0) p.lse[(size_t)b * H + h] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
+  if (blockIdx.x == 0) p.lse[(size_t)b * H + h] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
 }
 
 }  // namespace ls

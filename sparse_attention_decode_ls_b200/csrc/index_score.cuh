@@ -279,46 +279,63 @@ __global__ void __launch_bounds__(192, 1)
     // their 64 token scales (bulk copy) into the stage, plus each unit's logical id.
     // A stage is released only when the MMA has consumed it and the epilogue has read
     // its scales and ids.
-    if (lane == 0) {
-      prefetch_tmap(&tmap);
-      int issued = 0;
-      for (int i = 0; i < my_tiles; ++i) {
-        const int st = i % C::kStages;
-        if (i >= C::kStages && !mbar_wait(&empty[st], ((i / C::kStages) - 1) & 1)) {
-          s_abort = 1;
-          break;
+    // The warp fetches the rows of 32 units (16 tiles) at a time, so the page-table
+    // reads are off the issue path; lane 0 waits for free stages and issues the copies.
+    if (lane == 0) prefetch_tmap(&tmap);
+    int issued = 0;
+    bool go = true;
+    for (int i0 = 0; go && i0 < my_tiles; i0 += 16) {
+      const int u_lane = 2 * (t_begin + i0) + lane;
+      int row_l = -1, lp_l = -1;
+      if (u_lane < n_units) {
+        row_l = idx_unit_row(p, b, u_lane, &lp_l);
+        if (row_l < 0) {
+          flag(LS_DEV_BOUNDS);
+          lp_l = -1;
         }
-        if (*(volatile int*)&s_abort) break;
-        const int tile = t_begin + i;
-        int rows[2], lps[2];
-        uint32_t bytes = 0;
-        for (int uu = 0; uu < 2; ++uu) {
-          const int u = 2 * tile + uu;
-          rows[uu] = -1;
-          lps[uu] = -1;
-          if (u < n_units) {
-            rows[uu] = idx_unit_row(p, b, u, &lps[uu]);
-            if (rows[uu] < 0) {
-              flag(LS_DEV_BOUNDS);
-              lps[uu] = -1;
-            } else {
-              bytes += KP * 64 * 128 + (p.mode == 0 ? 256 : 0);
+      }
+      const int nt = min(16, my_tiles - i0);
+      for (int ii = 0; ii < nt; ++ii) {
+        const int i = i0 + ii;
+        const int st = i % C::kStages;
+        const int row0 = __shfl_sync(0xffffffffu, row_l, 2 * ii);
+        const int row1 = __shfl_sync(0xffffffffu, row_l, 2 * ii + 1);
+        const int lp0 = __shfl_sync(0xffffffffu, lp_l, 2 * ii);
+        const int lp1 = __shfl_sync(0xffffffffu, lp_l, 2 * ii + 1);
+        int ok_i = 1;
+        if (lane == 0) {
+          if (i >= C::kStages && !mbar_wait(&empty[st], ((i / C::kStages) - 1) & 1)) ok_i = 0;
+          if (*(volatile int*)&s_abort) ok_i = 0;
+          if (!ok_i) {
+            s_abort = 1;
+          } else {
+            constexpr uint32_t kUnitBytes = KP * 64 * 128;
+            const uint32_t extra = p.mode == 0 ? 256u : 0u;
+            s_meta[st * 2 + 0] = lp0;
+            s_meta[st * 2 + 1] = lp1;
+            const uint32_t bytes = (row0 >= 0 ? kUnitBytes + extra : 0u) + (row1 >= 0 ? kUnitBytes + extra : 0u);
+            mbar_arrive_expect_tx(&full[st], bytes);
+            const uint32_t dst = smem_u32(sA + st * C::kStageBytes);
+            const int rows[2] = {row0, row1};
+            for (int uu = 0; uu < 2; ++uu) {
+              if (rows[uu] < 0) continue;
+              for (int pk = 0; pk < KP; ++pk)
+                tma_load_2d(dst + pk * C::kPanel + uu * 64 * 128, &tmap, &full[st], pk * 128, rows[uu]);
+              if (p.mode == 0)
+                bulk_load(smem_u32(s_scale + st * 128 + uu * 64), p.row_scale + rows[uu], 256, &full[st]);
             }
           }
-          s_meta[st * 2 + uu] = lps[uu];
         }
-        mbar_arrive_expect_tx(&full[st], bytes);
-        const uint32_t dst = smem_u32(sA + st * C::kStageBytes);
-        for (int uu = 0; uu < 2; ++uu) {
-          if (rows[uu] < 0) continue;
-          for (int pk = 0; pk < KP; ++pk)
-            tma_load_2d(dst + pk * C::kPanel + uu * 64 * 128, &tmap, &full[st], pk * 128, rows[uu]);
-          if (p.mode == 0)
-            bulk_load(smem_u32(s_scale + st * 128 + uu * 64), p.row_scale + rows[uu], 256, &full[st]);
+        ok_i = __shfl_sync(0xffffffffu, ok_i, 0);
+        if (!ok_i) {
+          go = false;
+          break;
         }
         ++issued;
       }
-      // never leave with copies in flight: wait for every stage still owned by TMA
+    }
+    // never leave with copies in flight: wait for every stage still owned by TMA
+    if (lane == 0) {
       const int first = issued > C::kStages ? issued - C::kStages : 0;
       for (int i = first; i < issued; ++i) mbar_wait(&full[i % C::kStages], (i / C::kStages) & 1);
     }
@@ -377,16 +394,24 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (!mbar_wait(&accf[a], (i / C::kAcc) & 1)) { s_abort = 1; break; }
       tc_fence_after();
-      float sum = 0.f;
+      // four independent partial sums (fixed order: the result is the same for a token
+      // wherever it is scored)
+      float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
       const uint32_t tbase = tmem + ((uint32_t)(wq * 32) << 16) + a * NCOL;
 #pragma unroll
-      for (int c0 = 0; c0 < NCOL; c0 += 32) {
-        float v[32];
-        tmem_ld32(tbase + c0, v);
-        tmem_wait_ld();
+      for (int c0 = 0; c0 < NCOL; c0 += 64) {
+        float v[64];
+        tmem_ld64(tbase + c0, v);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) sum = fmaf(coef[c0 + c], fmaxf(v[c], 0.f), sum);
+        for (int c = 0; c < 64; c += 4) {
+          const float4 cf = *(const float4*)(coef + c0 + c);
+          acc0 = fmaf(cf.x, fmaxf(v[c], 0.f), acc0);
+          acc1 = fmaf(cf.y, fmaxf(v[c + 1], 0.f), acc1);
+          acc2 = fmaf(cf.z, fmaxf(v[c + 2], 0.f), acc2);
+          acc3 = fmaf(cf.w, fmaxf(v[c + 3], 0.f), acc3);
+        }
       }
+      const float sum = (acc0 + acc1) + (acc2 + acc3);
       tc_fence_before();
       mbar_arrive(&acce[a]);
       mbar_arrive(&empty[st]);
@@ -402,6 +427,9 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   }
+  // every warp must reach the barrier converged (the MMA warp's lane 0 arrives last);
+  // only then may TMEM be released
+  __syncwarp();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -38,21 +38,33 @@ __device__ __forceinline__ int topk_pos(const TopkParams& p, int b, int i) {
   return p.unit_list[(size_t)b * p.list_stride + (i >> 6)] * 64 + (i & 63);
 }
 
+// Candidate buffers of the fast path (dynamic shared memory after the key cache).
+constexpr int kCandCap = 2048;    // per CTA: keys of the threshold bin and their slice index
+constexpr int kCandTotal = 6144;  // all candidates of a request, gathered by CTA 0
+constexpr int kTopkExtraBytes = kCandCap * 8 + kCandTotal * 4;
+
 template <int CL>
 __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams p) {
   cg::cluster_group cluster = cg::this_cluster();
-  extern __shared__ __align__(16) uint32_t sm_keys[];
+  extern __shared__ __align__(16) uint32_t sm_keys[];  // [cache_keys] then candidate buffers
   __shared__ uint32_t hist[2048];
   __shared__ uint32_t red[2048 / CL];
   __shared__ uint32_t ghist[2048];
   __shared__ unsigned long long scan_tmp[32];
-  __shared__ unsigned long long cnt_pub;  // this CTA's (n_gt << 32 | n_eq), read by the cluster
+  __shared__ unsigned long long cnt_pub;  // fallback path: this CTA's (n_gt << 32 | n_eq)
   __shared__ int s_found_bin;
   __shared__ uint32_t s_found_above;
+  // fast path
+  __shared__ uint32_t s_ncand, s_nabove, s_overflow;
+  __shared__ uint32_t s_warp_above[kTopkThreads / 32], s_warp_gt[kTopkThreads / 32], s_warp_eq[kTopkThreads / 32];
+  __shared__ uint32_t s_T, s_R;                      // CTA 0 publishes
+  __shared__ uint32_t s_cta_gt[CL], s_cta_eq[CL];    // CTA 0 publishes
+  __shared__ uint32_t s_off[CL + 1];
 
   const int b = blockIdx.x / CL;
   const int rank = (int)cluster.block_rank();
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
+  constexpr int kWarps = kTopkThreads / 32;
   const int k = p.k;
 
   long long nll = ((long long)p.lens[b] * p.len_mul + p.len_div - 1) / p.len_div;
@@ -65,6 +77,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
   const int m = c1 - c0;
   const bool cached = Lc <= p.cache_keys;
   const float* row = p.scores + (size_t)b * p.stride;
+  uint32_t* cand_key = sm_keys + p.cache_keys;
+  uint32_t* cand_idx = cand_key + kCandCap;
+  uint32_t* gbuf = cand_idx + kCandCap;
 
   auto key_at = [&](int i) -> uint32_t {  // i relative to c0
     return cached ? sm_keys[i] : float_key(row[c0 + i]);
@@ -99,47 +114,49 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
     for (int i = m4 + tid; i < m; i += kTopkThreads) sm_keys[i] = float_key(row[c0 + i]);
   }
 
+  // Find the bin (of `width` bits at `shift`) holding the k_rem-th largest key among the
+  // keys whose bits above the digit equal `prefix`; bins scanned high to low.  With
+  // `local`, only this CTA's `vals` are counted; otherwise the cluster's slices.
   uint32_t prefix = 0;
   uint32_t k_rem = (uint32_t)k;
-  const int shifts[3] = {21, 10, 0};
-  const int widths[3] = {11, 11, 10};
-  for (int pass = 0; pass < 3; ++pass) {
-    const int shift = shifts[pass], width = widths[pass];
+  auto radix_pass = [&](int shift, int width, bool local, const uint32_t* vals, int nvals) {
     const int nbins = 1 << width;
     const uint32_t dmask = (uint32_t)nbins - 1u;
-    const int hi_shift = shift + width;  // bits above this pass's digit must equal prefix
+    const int hi_shift = shift + width;
     for (int d = tid; d < 2048; d += kTopkThreads) hist[d] = 0;
     __syncthreads();
-    for (int i = tid; i < m; i += kTopkThreads) {
-      const uint32_t key = key_at(i);
+    for (int i = tid; i < nvals; i += kTopkThreads) {
+      const uint32_t key = vals ? vals[i] : key_at(i);
       const bool cand = (hi_shift >= 32) || ((key >> hi_shift) == prefix);
       if (cand) atomicAdd(&hist[(key >> shift) & dmask], 1u);
     }
     __syncthreads();
-    cluster.sync();
-    // reduce my slice of bins over the cluster
-    const int slice = 2048 / CL;
-    for (int d = tid; d < slice; d += kTopkThreads) {
-      const int gd = rank * slice + d;
-      uint32_t s = 0;
-      if (gd < nbins) {
+    const uint32_t* h_all = hist;
+    if (!local) {
+      cluster.sync();
+      const int slice = 2048 / CL;
+      for (int d = tid; d < slice; d += kTopkThreads) {
+        const int gd = rank * slice + d;
+        uint32_t s = 0;
+        if (gd < nbins) {
 #pragma unroll
-        for (int c = 0; c < CL; ++c) s += cluster.map_shared_rank(hist, c)[gd];
+          for (int c = 0; c < CL; ++c) s += cluster.map_shared_rank(hist, c)[gd];
+        }
+        red[d] = s;
       }
-      red[d] = s;
+      cluster.sync();
+      for (int d = tid; d < nbins; d += kTopkThreads) ghist[d] = cluster.map_shared_rank(red, d / slice)[d % slice];
+      __syncthreads();
+      h_all = ghist;
     }
-    cluster.sync();
-    for (int d = tid; d < nbins; d += kTopkThreads) ghist[d] = cluster.map_shared_rank(red, d / slice)[d % slice];
-    __syncthreads();
-    // find the bin holding the k_rem-th largest candidate (bins scanned high to low)
     const int per = nbins / kTopkThreads;  // 4 or 2 bins per thread
     uint32_t mine = 0;
-    for (int j = 0; j < per; ++j) mine += ghist[nbins - 1 - (tid * per + j)];
+    for (int j = 0; j < per; ++j) mine += h_all[nbins - 1 - (tid * per + j)];
     unsigned long long tot;
     uint32_t above = (uint32_t)block_excl_scan_u64(mine, scan_tmp, &tot);
     for (int j = 0; j < per; ++j) {
       const int d = nbins - 1 - (tid * per + j);
-      const uint32_t h = ghist[d];
+      const uint32_t h = h_all[d];
       if (above < k_rem && above + h >= k_rem) {
         s_found_bin = d;
         s_found_above = above;
@@ -150,44 +167,167 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
     prefix = (prefix << width) | (uint32_t)s_found_bin;
     k_rem -= s_found_above;
     __syncthreads();
-  }
-  const uint32_t T = prefix;   // exact k-th largest key
-  const uint32_t R = k_rem;    // how many keys == T are taken (lowest positions first)
+  };
 
-  // ---- emit: each warp owns a contiguous segment (position order) and walks it 32 keys
-  // at a time, so shared-memory reads are conflict-free and ballots give the ranks
-  const int lane = lane_id(), warp = warp_id();
-  constexpr int kWarps = kTopkThreads / 32;
+  // ---- pass 0 over the whole request: the top 11 bits
+  radix_pass(21, 11, false, nullptr, m);
+  const uint32_t t0 = prefix;
+
+  // ---- fast path: collect the keys of bin t0 (the only undecided ones).  Each warp
+  // walks a contiguous segment, the same one it emits later, and counts the keys above.
   const int seg = ((m + kWarps * 32 - 1) / (kWarps * 32)) * 32;
   const int i0 = min(m, warp * seg), i1 = min(m, i0 + seg);
-  uint32_t n_gt = 0, n_eq = 0;
-  for (int base = i0; base < i1; base += 32) {
-    const int i = base + lane;
-    const uint32_t key = i < i1 ? key_at(i) : 0u;
-    n_gt += __popc(__ballot_sync(0xffffffffu, i < i1 && key > T));
-    n_eq += __popc(__ballot_sync(0xffffffffu, i < i1 && key == T));
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  if (tid == 0) {
+    s_ncand = 0;
+    s_overflow = 0;
   }
-  // warp totals -> exclusive prefix over warps (block scan on one value per thread)
-  const unsigned long long mine = lane == 0 ? (((unsigned long long)n_gt << 32) | n_eq) : 0ull;
-  unsigned long long tot;
-  const unsigned long long pre_t = block_excl_scan_u64(mine, scan_tmp, &tot);
-  const unsigned long long pre = __shfl_sync(0xffffffffu, pre_t, 0);
-  if (tid == 0) cnt_pub = tot;
+  __syncthreads();
+  {
+    uint32_t above_w = 0;
+    for (int base = i0; base < i1; base += 32) {
+      const int i = base + lane;
+      const bool in = i < i1;
+      const uint32_t key = in ? key_at(i) : 0u;
+      above_w += __popc(__ballot_sync(0xffffffffu, in && (key >> 21) > t0));
+      const uint32_t cm = __ballot_sync(0xffffffffu, in && (key >> 21) == t0);
+      if (cm) {
+        uint32_t slot = 0;
+        if (lane == 0) slot = atomicAdd(&s_ncand, (uint32_t)__popc(cm));
+        slot = __shfl_sync(0xffffffffu, slot, 0);
+        if (cm >> lane & 1u) {
+          const uint32_t o = slot + __popc(cm & lt_mask);
+          if (o < (uint32_t)kCandCap) {
+            cand_key[o] = key;
+            cand_idx[o] = (uint32_t)i;
+          } else {
+            s_overflow = 1;
+          }
+        }
+      }
+    }
+    if (lane == 0) s_warp_above[warp] = above_w;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t a = 0;
+    for (int w = 0; w < kWarps; ++w) a += s_warp_above[w];
+    s_nabove = a;
+  }
   __syncthreads();
   cluster.sync();
-  uint32_t eq_before = 0, out_before = 0;
-  for (int c = 0; c < rank; ++c) {
-    const unsigned long long v = *cluster.map_shared_rank(&cnt_pub, c);
-    const uint32_t g = (uint32_t)(v >> 32), e = (uint32_t)v;
-    const uint32_t take = R > eq_before ? min(e, R - eq_before) : 0u;
-    out_before += g + take;
-    eq_before += e;
+  // every CTA reads the same counts, so the choice of path is uniform over the cluster
+  uint32_t total = 0, ovf = 0;
+  for (int c = 0; c < CL; ++c) {
+    total += *cluster.map_shared_rank(&s_ncand, c);
+    ovf |= *cluster.map_shared_rank(&s_overflow, c);
   }
+  const bool fast = !ovf && total <= (uint32_t)kCandTotal;
+
+  uint32_t T, R, out_before = 0, eq_before = 0;
+  unsigned long long pre;
+  if (fast) {
+    if (rank == 0) {
+      // gather every CTA's candidates and finish the selection on them alone
+      if (tid == 0) {
+        uint32_t o = 0;
+        for (int c = 0; c < CL; ++c) {
+          s_off[c] = o;
+          o += *cluster.map_shared_rank(&s_ncand, c);
+        }
+        s_off[CL] = o;
+      }
+      __syncthreads();
+      for (int c = 0; c < CL; ++c) {
+        const uint32_t nc = s_off[c + 1] - s_off[c];
+        const uint32_t* src = cluster.map_shared_rank(cand_key, c);
+        for (uint32_t j = tid; j < nc; j += kTopkThreads) gbuf[s_off[c] + j] = src[j];
+      }
+      __syncthreads();
+      radix_pass(10, 11, true, gbuf, (int)total);
+      radix_pass(0, 10, true, gbuf, (int)total);
+      if (tid < CL) {
+        s_cta_gt[tid] = *cluster.map_shared_rank(&s_nabove, tid);
+        s_cta_eq[tid] = 0;
+      }
+      __syncthreads();
+      for (uint32_t j = tid; j < total; j += kTopkThreads) {
+        int c = 0;
+        while (j >= s_off[c + 1]) ++c;
+        const uint32_t key = gbuf[j];
+        if (key > prefix) atomicAdd(&s_cta_gt[c], 1u);
+        else if (key == prefix) atomicAdd(&s_cta_eq[c], 1u);
+      }
+      if (tid == 0) {
+        s_T = prefix;
+        s_R = k_rem;
+      }
+      __syncthreads();
+    }
+    cluster.sync();
+    T = *cluster.map_shared_rank(&s_T, 0);
+    R = *cluster.map_shared_rank(&s_R, 0);
+    for (int c = 0; c < rank; ++c) {
+      const uint32_t g = *cluster.map_shared_rank(&s_cta_gt[c], 0);
+      const uint32_t e = *cluster.map_shared_rank(&s_cta_eq[c], 0);
+      const uint32_t take = R > eq_before ? min(e, R - eq_before) : 0u;
+      out_before += g + take;
+      eq_before += e;
+    }
+    // per-warp counts: the keys above bin t0 plus this CTA's candidates above / at T
+    if (tid < kWarps) {
+      s_warp_gt[tid] = s_warp_above[tid];
+      s_warp_eq[tid] = 0;
+    }
+    __syncthreads();
+    const uint32_t nmine = min(s_ncand, (uint32_t)kCandCap);
+    for (uint32_t j = tid; j < nmine; j += kTopkThreads) {
+      const uint32_t key = cand_key[j];
+      const int w = (int)(cand_idx[j] / (uint32_t)max(seg, 1));
+      if (key > T) atomicAdd(&s_warp_gt[w], 1u);
+      else if (key == T) atomicAdd(&s_warp_eq[w], 1u);
+    }
+    __syncthreads();
+    const unsigned long long mine =
+        lane == 0 ? (((unsigned long long)s_warp_gt[warp] << 32) | s_warp_eq[warp]) : 0ull;
+    unsigned long long tot;
+    const unsigned long long pre_t = block_excl_scan_u64(mine, scan_tmp, &tot);
+    pre = __shfl_sync(0xffffffffu, pre_t, 0);
+  } else {
+    // ---- general path (too many keys share bin t0): two more cluster-wide passes
+    radix_pass(10, 11, false, nullptr, m);
+    radix_pass(0, 10, false, nullptr, m);
+    T = prefix;
+    R = k_rem;
+    uint32_t n_gt = 0, n_eq = 0;
+    for (int base = i0; base < i1; base += 32) {
+      const int i = base + lane;
+      const uint32_t key = i < i1 ? key_at(i) : 0u;
+      n_gt += __popc(__ballot_sync(0xffffffffu, i < i1 && key > T));
+      n_eq += __popc(__ballot_sync(0xffffffffu, i < i1 && key == T));
+    }
+    const unsigned long long mine = lane == 0 ? (((unsigned long long)n_gt << 32) | n_eq) : 0ull;
+    unsigned long long tot;
+    const unsigned long long pre_t = block_excl_scan_u64(mine, scan_tmp, &tot);
+    pre = __shfl_sync(0xffffffffu, pre_t, 0);
+    if (tid == 0) cnt_pub = tot;
+    __syncthreads();
+    cluster.sync();
+    for (int c = 0; c < rank; ++c) {
+      const unsigned long long v = *cluster.map_shared_rank(&cnt_pub, c);
+      const uint32_t g = (uint32_t)(v >> 32), e = (uint32_t)v;
+      const uint32_t take = R > eq_before ? min(e, R - eq_before) : 0u;
+      out_before += g + take;
+      eq_before += e;
+    }
+  }
+
+  // ---- emit: each warp walks its segment 32 keys at a time in position order;
+  // ballots give every taken key its output slot (ties: lower position first)
   const uint32_t eq_left = R > eq_before ? R - eq_before : 0u;  // ties this CTA may still take
   const uint32_t gt_pre = (uint32_t)(pre >> 32), eq_pre = (uint32_t)pre;
   uint32_t eq_seen = eq_pre;  // keys == T before this lane's current key, CTA-wide
   uint32_t out = out_before + gt_pre + min(eq_pre, eq_left);
-  const uint32_t lt_mask = (1u << lane) - 1u;
   for (int base = i0; base < i1; base += 32) {
     const int i = base + lane;
     const bool in = i < i1;
