@@ -307,6 +307,31 @@ ls_status ls_sparse_attn_decode(const ls_sparse_attn_args* args, void* workspace
                                 size_t workspace_bytes, ls_stream_t stream);
 
 /* ------------------------------------------------------------------------------
+ * Allocation-free variant of ls_sparse_attn_decode (no counterpart in the paper).
+ *
+ * For callers that cannot allocate device memory and so cannot hand in a
+ * workspace: for example code that runs inside another engine whose memory
+ * manager has already reserved the GPU's free HBM for its own pools (a further
+ * cudaMalloc there fails or fragments those pools), or a plain C caller that has
+ * no device allocator of its own at the point where it decodes.
+ *
+ * Same arguments, semantics and results as ls_sparse_attn_decode, except that the
+ * split-KV partial outputs go to a scratch array built into the library instead of
+ * a caller workspace.  The call allocates and frees nothing.
+ *   - The scratch holds 20 MiB; every GPU that loads the library holds it until the
+ *     process exits.  A configuration whose partials need more returns
+ *     LS_ERR_INVALID_ARG with a message (ls_sparse_attn_workspace_size() gives the
+ *     need); one that needs none does not touch the scratch.
+ *   - The first call on a device looks up the scratch's device address, with that
+ *     device current; make that first call before any stream capture.
+ *   - All calls on a device share the one array, which keeps the last call's
+ *     contents.  Nothing in it has to start at zero: each call writes every partial
+ *     before it reads it.  Calls whose kernels overlap on the GPU (for example on two
+ *     streams with no ordering between them) race on the array.
+ * --------------------------------------------------------------------------- */
+ls_status ls_sparse_attn_decode_noalloc(const ls_sparse_attn_args* args, ls_stream_t stream);
+
+/* ------------------------------------------------------------------------------
  * a7. One decode step: indexer (or coarse-to-fine indexer) -> top-k -> [hot-buffer
  * resolve -> miss gather] -> sparse attention, all on `stream`, with no allocation
  * (the caller provides the workspace) and no host synchronisation.

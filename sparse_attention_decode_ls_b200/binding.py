@@ -109,6 +109,8 @@ def lib():
             f = getattr(L, name)
             f.argtypes = [P(st)]
             f.restype = C.c_size_t
+        L.ls_sparse_attn_decode_noalloc.argtypes = [P(SparseAttnArgs), _p]
+        L.ls_sparse_attn_decode_noalloc.restype = C.c_int
         L.ls_build_block_summaries.argtypes = [P(IndexScoreArgs), _p, _p, _i32, _p]
         L.ls_build_block_summaries.restype = C.c_int
         L.ls_get_error_string.restype = C.c_char_p
@@ -265,6 +267,12 @@ def ls_sparse_attn_workspace_size(a: SparseAttnArgs) -> int:
 def ls_sparse_attn_decode(a: SparseAttnArgs, workspace=None, stream=None):
     _check(lib().ls_sparse_attn_decode(C.byref(a), _ptr(workspace),
                                        0 if workspace is None else workspace.numel(), _stream(stream)))
+
+
+def ls_sparse_attn_decode_noalloc(a: SparseAttnArgs, stream=None):
+    """Allocation-free attention: the split-KV partials use the library's built-in
+    scratch instead of a caller workspace (see include/ls.h)."""
+    _check(lib().ls_sparse_attn_decode_noalloc(C.byref(a), _stream(stream)))
 
 
 # ------------------------------------------------------------------------------- a7

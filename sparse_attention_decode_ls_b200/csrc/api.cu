@@ -747,3 +747,63 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
 }
 
 }  // extern "C"
+
+// =========================================================================================
+// Allocation-free attention: the split-KV scratch lives in a fixed device array that the
+// library itself provides, for callers that cannot allocate device memory.
+// =========================================================================================
+namespace {
+
+// Largest split-KV scratch the allocation-free entry point supports.  With 148 SMs the
+// split count is floor(148 / (2 * batch)), so the partials of any batch fit in
+// 74 * 128 * 512 * 4 B + 74 * 128 * 8 B (about 19 MB).
+constexpr size_t kStaticAttnScratchBytes = 20u << 20;
+
+}  // namespace
+
+// One copy per GPU that loads the library, alive until the process exits.
+static __device__ __align__(256) unsigned char g_attn_scratch[kStaticAttnScratchBytes];
+
+namespace {
+
+// Device address of g_attn_scratch on the current device.  In host code the symbol is
+// only a host-side stand-in, so the address is asked for once per device (with that
+// device current) and cached.
+ls_status static_scratch(void** out) {
+  static std::atomic<void*> cache[64];
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(LS_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= 64) return fail(LS_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  void* p = cache[dev].load();
+  if (!p) {
+    std::lock_guard<std::mutex> lock(mu);
+    p = cache[dev].load();
+    if (!p) {
+      e = cudaGetSymbolAddress(&p, g_attn_scratch);
+      if (e != cudaSuccess || !p)
+        return fail(LS_ERR_CUDA, "cudaGetSymbolAddress(attention scratch): %s", cudaGetErrorString(e));
+      cache[dev].store(p);
+    }
+  }
+  *out = p;
+  return LS_OK;
+}
+
+}  // namespace
+
+extern "C" ls_status ls_sparse_attn_decode_noalloc(const ls_sparse_attn_args* a, ls_stream_t stream) {
+  LS_TRY(validate_attn(a, true));
+  const size_t need = attn_ws_bytes(a);
+  if (need > kStaticAttnScratchBytes)
+    return fail(LS_ERR_INVALID_ARG,
+                "allocation-free attention needs %zu bytes of scratch; the built-in scratch holds %zu bytes "
+                "(use ls_sparse_attn_decode with a caller workspace)",
+                need, kStaticAttnScratchBytes);
+  void* ws = nullptr;
+  if (need > 0) LS_TRY(static_scratch(&ws));
+  LS_TRY(launch_attn(a, a->sel, a->addressing, a->page_table, a->max_pages, a->n_slots, nullptr, a->num_rows, ws,
+                     need > 0 ? kStaticAttnScratchBytes : 0, (cudaStream_t)stream));
+  return ok();
+}
