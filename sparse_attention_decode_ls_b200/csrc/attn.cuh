@@ -10,9 +10,10 @@
 //       accumulators.  O for all 512 V dims would fill the whole 512-column TMEM,
 //       so each CTA owns one 256-wide half of V (the pair recomputes S) and keeps
 //       O_half (256 columns) + a double-buffered S (2 x 32 columns) in TMEM.
-//     - Rows are gathered through the page table or the hot-buffer slots by
-//       cp.async 16-byte copies straight into 128-byte-swizzled panels; the same
-//       panels serve as the K-major B operand of S and the MN-major B operand of PV.
+//     - Rows are gathered through the page table or the hot-buffer slots by TMA: one
+//       128-byte box per (row, 64-dim panel), landing swizzled in the row's line of
+//       the panel; the same panels serve as the K-major B operand of S and the
+//       MN-major B operand of PV.
 //     - Online softmax in the exp2 domain with lazy rescaling (O is only rescaled
 //       when the running max grows by more than 2^8).
 //     - Split-KV across CTAs (enough CTAs to fill the GPU at small batch), merged
@@ -139,7 +140,7 @@ constexpr int kNumBars = 2 + 2 + 2 + 1 + 1 + 1;        // kv_full[2] kv_empty[2]
 constexpr int kOffTmem = kOffBar + kNumBars * 8;
 constexpr int kSmem = 1024 + kOffTmem + 16;
 constexpr int kThreads = 256;
-constexpr int kLoaders = 32;                           // one warp per KV stage
+constexpr int kLoaders = 32;                           // one warp per KV stage (TMA issue)
 constexpr int kChunksPerRow = DK * 2 / 16;             // 72
 constexpr uint32_t kIdescS = make_idesc(1 /*bf16*/, 128, N, false, false);
 constexpr uint32_t kIdescO = make_idesc(1 /*bf16*/, 128, DVH, false, true);
@@ -147,7 +148,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 }  // namespace mla
 
-__global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
+__global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p, const __grid_constant__ CUtensorMap kv_map) {
   using namespace mla;
   extern __shared__ uint8_t sm_raw_a[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)sm_raw_a + 1023) & ~(uintptr_t)1023);
@@ -171,7 +172,6 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
   const int t1 = (int)(((long long)T_all * (split + 1)) / p.nsplit);
   const int my_tiles = t1 - t0;
   const uint32_t sbase = smem_u32(sm);
-  const char* kv_base = (const char*)p.krows;
 
   // ---- Q (128 heads x 576) into nine 128-byte-swizzled K-major panels
   {
@@ -184,8 +184,8 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
     cp_async_commit();
   }
   if (tid == 0) {
-    mbar_init(&kv_full[0], kLoaders);
-    mbar_init(&kv_full[1], kLoaders);
+    mbar_init(&kv_full[0], 1);  // the loader lane 0 arrives with the expected bytes
+    mbar_init(&kv_full[1], 1);
     mbar_init(&kv_empty[0], 1);
     mbar_init(&kv_empty[1], 1);
     mbar_init(&s_full[0], 1);
@@ -208,9 +208,12 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
 
   if (warp == 0 || warp == 1) {
     // ================= loaders: warp w fills stage w with tiles w, w+2, ... =================
-    // Lane r owns row r of a tile (its row offset and validity); the copies are spread
-    // over the warp chunk by chunk so consecutive lanes read consecutive bytes.
+    // Lane r owns row r of a tile: it resolves the row and issues the row's nine
+    // 128-byte TMA boxes (one per 64-dim panel, landing swizzled at line r of each
+    // panel).  Rows that are padding are zeroed with plain stores instead.  The stage
+    // completes when its valid rows' bytes have arrived.
     const int st = warp;
+    int last = -1;
     for (int i = st; i < my_tiles; i += 2) {
       int go = 1;
       if (lane == 0) {  // one lane decides, so the warp stays converged
@@ -221,39 +224,35 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p) {
       go = __shfl_sync(0xffffffffu, go, 0);
       if (!go) break;
       const int j = (t0 + i) * N + lane;
-      long long off = -1;
-      if (j < p.k) {
-        const long long r = attn_row(p, b, p.sel[(size_t)b * p.k + j]);
-        if (r >= 0) off = r * p.row_stride * 2;
-      }
-      const uint32_t vmask = __ballot_sync(0xffffffffu, off >= 0);
-      if (lane == 0) s_mask[st] = vmask;
-      // lane l copies chunks l, l+32, l+64 of every row (consecutive lanes, consecutive
-      // 16-byte pieces of one row); row offsets travel by shuffle
-      const uint32_t dst0 = sbase + kOffKv + st * kKvBytes;
-#pragma unroll 4
-      for (int r = 0; r < N; ++r) {
-        const long long ro = __shfl_sync(0xffffffffu, off, r);
-        const uint32_t rbase = dst0 + r * 128;
+      long long row = -1;
+      if (j < p.k) row = attn_row(p, b, p.sel[(size_t)b * p.k + j]);
+      const uint32_t vmask = __ballot_sync(0xffffffffu, row >= 0);
+      const uint32_t dst0 = sbase + kOffKv + st * kKvBytes + lane * 128;
+      if (row < 0) {
+#pragma unroll 1
+        for (int pn = 0; pn < kPanels; ++pn)
 #pragma unroll
-        for (int q = 0; q < 3; ++q) {
-          const int c = lane + 32 * q;
-          if (c < kChunksPerRow) {
-            const uint32_t dst = rbase + (c >> 3) * kKvPanel + ((uint32_t)((c & 7) ^ (r & 7)) << 4);
-            if (ro >= 0) {
-              cp_async_16(dst, kv_base + ro + c * 16);
-            } else {
-              asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0) : "memory");
-            }
-          }
-        }
+          for (int c = 0; c < 8; ++c)
+            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst0 + pn * kKvPanel + c * 16), "r"(0)
+                         : "memory");
+        fence_proxy_async_smem();
       }
-      cp_async_commit();
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
-      mbar_arrive(&kv_full[st]);
       __syncwarp();
+      if (lane == 0) {
+        s_mask[st] = vmask;
+        mbar_arrive_expect_tx(&kv_full[st], (uint32_t)__popc(vmask) * (uint32_t)(DK * 2));
+      }
+      __syncwarp();
+      if (row >= 0) {
+#pragma unroll
+        for (int pn = 0; pn < kPanels; ++pn)
+          tma_load_2d(dst0 + pn * kKvPanel, &kv_map, &kv_full[st], pn * 64, (int)row);
+      }
+      last = i;
     }
+    // never leave with copies in flight
+    if (lane == 0 && last >= 0) mbar_wait(&kv_full[st], (last >> 1) & 1);
+    __syncwarp();
   } else if (warp == 2) {
     // ================= MMA issuer =================
     if (lane == 0 && my_tiles > 0) {

@@ -127,7 +127,7 @@ struct IdxTc {
   static constexpr int kOffMeta = kOffScale + kStages * 128 * 4;     // [kStages][2] logical unit ids
   static constexpr int kOffCoef = kOffMeta + ((kStages * 8 + 15) & ~15);
   static constexpr int kOffBar = kOffCoef + NCOL * 4 + 16;
-  static constexpr int kNumBars = 2 * kStages + 2 * kAcc;
+  static constexpr int kNumBars = 2 * kStages + 2 * kAcc + 1;  // + b_ready
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kSmem = 1024 + kOffTmem + 16;   // +1024: runtime alignment slack
   static constexpr uint32_t kIdesc = make_idesc(0 /*e4m3*/, 128, NCOL, false, false);
@@ -165,6 +165,7 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* empty = bars + C::kStages;
   uint64_t* accf = bars + 2 * C::kStages;
   uint64_t* acce = accf + C::kAcc;
+  uint64_t* b_ready = acce + C::kAcc;
   uint32_t* tmem_slot = (uint32_t*)(sm + C::kOffTmem);
   __shared__ int s_abort;
 
@@ -197,9 +198,12 @@ __global__ void __launch_bounds__(192, 1)
   const int my_tiles = t_end - t_begin;
   if (my_tiles <= 0) return;
 
-  // ---- prologue: B operand (query side) in 128-byte-swizzled K-major layout, coefficients
+  // ---- query side: B operand in 128-byte-swizzled K-major layout, coefficients and, for
+  // the bound, the magnitude used by the margin.  The epilogue warps build it while the
+  // producer's first loads are in flight; the MMA waits for it on b_ready.
   const uint8_t* q8 = p.q8 + (size_t)b * 64 * 128;
-  for (int i = tid; i < NCOL * 8 * KP; i += C::kThreads) {
+  auto build_query_side = [&](int et) {  // et: epilogue thread index in [0, 128)
+  for (int i = et; i < NCOL * 8 * KP; i += 128) {
     // i enumerates 16-byte chunks: panel pk, row n, chunk j
     const int pk = i / (NCOL * 8);
     const int rem = i - pk * NCOL * 8;
@@ -229,21 +233,21 @@ __global__ void __launch_bounds__(192, 1)
     const int off = pk * NCOL * 128 + n * 128 + ((j ^ (n & 7)) << 4);
     *(uint4*)(sB + off) = v;
   }
-  if (tid < 64) {
-    const size_t gi = (size_t)b * 64 + tid;
+  if (et < 64) {
+    const size_t gi = (size_t)b * 64 + et;
     const float wv = p.w_bf16 ? __bfloat162float(((const __nv_bfloat16*)p.w)[gi]) : ((const float*)p.w)[gi];
     const float wq = wv * p.qs[gi];
     if (NCOL == 64) {
-      coef[tid] = wq;
+      coef[et] = wq;
     } else {
-      coef[tid] = fmaxf(wq, 0.f);
-      coef[64 + tid] = fminf(wq, 0.f);
+      coef[et] = fmaxf(wq, 0.f);
+      coef[64 + et] = fminf(wq, 0.f);
     }
   }
-  if (p.mode == 1 && warp == 0) {
+  if (p.mode == 1 && et < 32) {
     // magnitude bound used for the pruning margin
     float acc = 0.f;
-    for (int h = lane; h < 64; h += 32) {
+    for (int h = et; h < 64; h += 32) {
       float s = 0.f;
       for (int d = 0; d < 128; ++d) s += fabsf(e4m3_to_float(q8[h * 128 + d]));
       const size_t gi = (size_t)b * 64 + h;
@@ -252,9 +256,10 @@ __global__ void __launch_bounds__(192, 1)
     }
 #pragma unroll
     for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) gmag[0] = acc;
+    if (et == 0) gmag[0] = acc;
   }
   fence_proxy_async_smem();
+  };
   if (tid == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -264,6 +269,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&accf[a], 1);
       mbar_init(&acce[a], 128);
     }
+    mbar_init(b_ready, 128);
     s_abort = 0;
     fence_mbar_init();
   }
@@ -343,7 +349,9 @@ __global__ void __launch_bounds__(192, 1)
     // ================= MMA issuer =================
     if (lane == 0) {
       const uint32_t b_base = smem_u32(sB);
-      for (int i = 0; i < my_tiles; ++i) {
+      const bool have_b = mbar_wait(b_ready, 0);
+      if (!have_b) s_abort = 1;
+      for (int i = 0; have_b && i < my_tiles; ++i) {
         const int st = i % C::kStages, a = i % C::kAcc;
         if (!mbar_wait(&full[st], (i / C::kStages) & 1)) { s_abort = 1; break; }
         if (i >= C::kAcc && !mbar_wait(&acce[a], ((i / C::kAcc) - 1) & 1)) { s_abort = 1; break; }
@@ -365,6 +373,9 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ================= epilogue: warps 2..5, thread = tile row =================
+    build_query_side(tid - 64);
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // coefficients visible to all epilogue warps
+    mbar_arrive(b_ready);
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const int rr = r & 63;

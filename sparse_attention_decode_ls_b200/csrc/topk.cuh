@@ -43,6 +43,30 @@ constexpr int kCandCap = 2048;    // per CTA: keys of the threshold bin and thei
 constexpr int kCandTotal = 6144;  // all candidates of a request, gathered by CTA 0
 constexpr int kTopkExtraBytes = kCandCap * 8 + kCandTotal * 4;
 
+
+// Warp 0: lane c holds CTA c's count of keys above the threshold key (g) and equal to
+// it (e).  Ties are taken by lower position, i.e. by lower CTA first, R in all.  The lane
+// of this CTA's rank stores how many outputs and how many ties precede the CTA.
+#define cluster_prefix(g_, e_, R_, rank_, lane_)                                        \
+  do {                                                                                  \
+    uint32_t _e_incl = (e_);                                                            \
+    _Pragma("unroll") for (int _o = 1; _o < 32; _o <<= 1) {                             \
+      const uint32_t _y = __shfl_up_sync(0xffffffffu, _e_incl, _o);                     \
+      if ((lane_) >= _o) _e_incl += _y;                                                 \
+    }                                                                                   \
+    const uint32_t _eqb = _e_incl - (e_);                                               \
+    const uint32_t _take = (R_) > _eqb ? min((e_), (R_) - _eqb) : 0u;                   \
+    uint32_t _o_incl = (g_) + _take;                                                    \
+    _Pragma("unroll") for (int _o = 1; _o < 32; _o <<= 1) {                             \
+      const uint32_t _y = __shfl_up_sync(0xffffffffu, _o_incl, _o);                     \
+      if ((lane_) >= _o) _o_incl += _y;                                                 \
+    }                                                                                   \
+    if ((lane_) == (rank_)) {                                                           \
+      s_out_before = _o_incl - ((g_) + _take);                                          \
+      s_eq_before = _eqb;                                                               \
+    }                                                                                   \
+  } while (0)
+
 template <int CL>
 __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams p) {
   cg::cluster_group cluster = cg::this_cluster();
@@ -60,6 +84,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
   __shared__ uint32_t s_T, s_R;                      // CTA 0 publishes
   __shared__ uint32_t s_cta_gt[CL], s_cta_eq[CL];    // CTA 0 publishes
   __shared__ uint32_t s_off[CL + 1];
+  __shared__ uint32_t s_total, s_fast, s_Tb, s_Rb, s_out_before, s_eq_before;
 
   const int b = blockIdx.x / CL;
   const int rank = (int)cluster.block_rank();
@@ -83,6 +108,24 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
 
   auto key_at = [&](int i) -> uint32_t {  // i relative to c0
     return cached ? sm_keys[i] : float_key(row[c0 + i]);
+  };
+  // keys i..i+3 (i a multiple of 4; entries at or beyond `end` are 0)
+  auto key4 = [&](int i, int end, uint32_t* kq) {
+    if (i + 3 < m) {
+      if (cached) {
+        const uint4 v = *(const uint4*)(sm_keys + i);
+        kq[0] = v.x; kq[1] = v.y; kq[2] = v.z; kq[3] = v.w;
+      } else {
+        const float4 v = *(const float4*)(row + c0 + i);
+        kq[0] = float_key(v.x); kq[1] = float_key(v.y); kq[2] = float_key(v.z); kq[3] = float_key(v.w);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) kq[e] = i + e < m ? key_at(i + e) : 0u;
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (i + e >= end) kq[e] = 0u;
   };
 
   if (n < k) {
@@ -125,10 +168,21 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
     const int hi_shift = shift + width;
     for (int d = tid; d < 2048; d += kTopkThreads) hist[d] = 0;
     __syncthreads();
-    for (int i = tid; i < nvals; i += kTopkThreads) {
-      const uint32_t key = vals ? vals[i] : key_at(i);
-      const bool cand = (hi_shift >= 32) || ((key >> hi_shift) == prefix);
-      if (cand) atomicAdd(&hist[(key >> shift) & dmask], 1u);
+    if (vals) {
+      for (int i = tid; i < nvals; i += kTopkThreads) {
+        const uint32_t key = vals[i];
+        if ((hi_shift >= 32) || ((key >> hi_shift) == prefix)) atomicAdd(&hist[(key >> shift) & dmask], 1u);
+      }
+    } else {
+      for (int i = tid * 4; i < nvals; i += kTopkThreads * 4) {
+        uint32_t kq[4];
+        key4(i, nvals, kq);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if (i + e < nvals && ((hi_shift >= 32) || ((kq[e] >> hi_shift) == prefix)))
+            atomicAdd(&hist[(kq[e] >> shift) & dmask], 1u);
+        }
+      }
     }
     __syncthreads();
     const uint32_t* h_all = hist;
@@ -174,8 +228,9 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
   const uint32_t t0 = prefix;
 
   // ---- fast path: collect the keys of bin t0 (the only undecided ones).  Each warp
-  // walks a contiguous segment, the same one it emits later, and counts the keys above.
-  const int seg = ((m + kWarps * 32 - 1) / (kWarps * 32)) * 32;
+  // walks a contiguous segment (a multiple of 128 keys; the same one it emits later),
+  // four keys per thread per step, and counts the keys above bin t0.
+  const int seg = ((m + kWarps * 128 - 1) / (kWarps * 128)) * 128;
   const int i0 = min(m, warp * seg), i1 = min(m, i0 + seg);
   const uint32_t lt_mask = (1u << lane) - 1u;
   if (tid == 0) {
@@ -184,29 +239,29 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
   }
   __syncthreads();
   {
-    uint32_t above_w = 0;
-    for (int base = i0; base < i1; base += 32) {
-      const int i = base + lane;
-      const bool in = i < i1;
-      const uint32_t key = in ? key_at(i) : 0u;
-      above_w += __popc(__ballot_sync(0xffffffffu, in && (key >> 21) > t0));
-      const uint32_t cm = __ballot_sync(0xffffffffu, in && (key >> 21) == t0);
-      if (cm) {
-        uint32_t slot = 0;
-        if (lane == 0) slot = atomicAdd(&s_ncand, (uint32_t)__popc(cm));
-        slot = __shfl_sync(0xffffffffu, slot, 0);
-        if (cm >> lane & 1u) {
-          const uint32_t o = slot + __popc(cm & lt_mask);
+    uint32_t above = 0;
+    for (int base = i0; base < i1; base += 128) {
+      const int i = base + 4 * lane;
+      uint32_t kq[4];
+      key4(i, i1, kq);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (i + e >= i1) continue;
+        const uint32_t bin = kq[e] >> 21;
+        above += bin > t0;
+        if (bin == t0) {
+          const uint32_t o = atomicAdd(&s_ncand, 1u);
           if (o < (uint32_t)kCandCap) {
-            cand_key[o] = key;
-            cand_idx[o] = (uint32_t)i;
+            cand_key[o] = kq[e];
+            cand_idx[o] = (uint32_t)(i + e);
           } else {
             s_overflow = 1;
           }
         }
       }
     }
-    if (lane == 0) s_warp_above[warp] = above_w;
+    above = __reduce_add_sync(0xffffffffu, above);
+    if (lane == 0) s_warp_above[warp] = above;
   }
   __syncthreads();
   if (tid == 0) {
@@ -216,32 +271,42 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
   }
   __syncthreads();
   cluster.sync();
-  // every CTA reads the same counts, so the choice of path is uniform over the cluster
-  uint32_t total = 0, ovf = 0;
-  for (int c = 0; c < CL; ++c) {
-    total += *cluster.map_shared_rank(&s_ncand, c);
-    ovf |= *cluster.map_shared_rank(&s_overflow, c);
+  // lane c of warp 0 reads CTA c's counts: one distributed-shared-memory round trip;
+  // every CTA reads the same values, so the choice of path is uniform over the cluster
+  if (warp == 0) {
+    uint32_t nc = 0, ov = 0;
+    if (lane < CL) {
+      nc = *cluster.map_shared_rank(&s_ncand, lane);
+      ov = *cluster.map_shared_rank(&s_overflow, lane);
+    }
+    const uint32_t tot = __reduce_add_sync(0xffffffffu, nc);
+    const bool anyov = __any_sync(0xffffffffu, ov != 0);
+    uint32_t incl = nc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane < CL) s_off[lane] = incl - nc;
+    if (lane == 0) {
+      s_off[CL] = tot;
+      s_total = tot;
+      s_fast = (!anyov && tot <= (uint32_t)kCandTotal) ? 1u : 0u;
+    }
   }
-  const bool fast = !ovf && total <= (uint32_t)kCandTotal;
+  __syncthreads();
+  const uint32_t total = s_total;
+  const bool fast = s_fast != 0;
 
-  uint32_t T, R, out_before = 0, eq_before = 0;
+  uint32_t T, R, out_before, eq_before;
   unsigned long long pre;
   if (fast) {
     if (rank == 0) {
-      // gather every CTA's candidates and finish the selection on them alone
-      if (tid == 0) {
-        uint32_t o = 0;
-        for (int c = 0; c < CL; ++c) {
-          s_off[c] = o;
-          o += *cluster.map_shared_rank(&s_ncand, c);
-        }
-        s_off[CL] = o;
-      }
-      __syncthreads();
-      for (int c = 0; c < CL; ++c) {
-        const uint32_t nc = s_off[c + 1] - s_off[c];
-        const uint32_t* src = cluster.map_shared_rank(cand_key, c);
-        for (uint32_t j = tid; j < nc; j += kTopkThreads) gbuf[s_off[c] + j] = src[j];
+      // gather every CTA's candidates (all loads independent) and finish the selection alone
+      for (uint32_t j = tid; j < total; j += kTopkThreads) {
+        int c = 0;
+        while (j >= s_off[c + 1]) ++c;
+        gbuf[j] = cluster.map_shared_rank(cand_key, c)[j - s_off[c]];
       }
       __syncthreads();
       radix_pass(10, 11, true, gbuf, (int)total);
@@ -265,15 +330,25 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
       __syncthreads();
     }
     cluster.sync();
-    T = *cluster.map_shared_rank(&s_T, 0);
-    R = *cluster.map_shared_rank(&s_R, 0);
-    for (int c = 0; c < rank; ++c) {
-      const uint32_t g = *cluster.map_shared_rank(&s_cta_gt[c], 0);
-      const uint32_t e = *cluster.map_shared_rank(&s_cta_eq[c], 0);
-      const uint32_t take = R > eq_before ? min(e, R - eq_before) : 0u;
-      out_before += g + take;
-      eq_before += e;
+    if (warp == 0) {
+      uint32_t g = 0, e = 0;
+      if (lane < CL) {
+        g = *cluster.map_shared_rank(&s_cta_gt[lane], 0);
+        e = *cluster.map_shared_rank(&s_cta_eq[lane], 0);
+      }
+      const uint32_t Tv = *cluster.map_shared_rank(&s_T, 0);
+      const uint32_t Rv = *cluster.map_shared_rank(&s_R, 0);
+      cluster_prefix(g, e, Rv, rank, lane);
+      if (lane == 0) {
+        s_Tb = Tv;
+        s_Rb = Rv;
+      }
     }
+    __syncthreads();
+    T = s_Tb;
+    R = s_Rb;
+    out_before = s_out_before;
+    eq_before = s_eq_before;
     // per-warp counts: the keys above bin t0 plus this CTA's candidates above / at T
     if (tid < kWarps) {
       s_warp_gt[tid] = s_warp_above[tid];
@@ -313,13 +388,13 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
     if (tid == 0) cnt_pub = tot;
     __syncthreads();
     cluster.sync();
-    for (int c = 0; c < rank; ++c) {
-      const unsigned long long v = *cluster.map_shared_rank(&cnt_pub, c);
-      const uint32_t g = (uint32_t)(v >> 32), e = (uint32_t)v;
-      const uint32_t take = R > eq_before ? min(e, R - eq_before) : 0u;
-      out_before += g + take;
-      eq_before += e;
+    if (warp == 0) {
+      const unsigned long long v = lane < CL ? *cluster.map_shared_rank(&cnt_pub, lane) : 0ull;
+      cluster_prefix((uint32_t)(v >> 32), (uint32_t)v, R, rank, lane);
     }
+    __syncthreads();
+    out_before = s_out_before;
+    eq_before = s_eq_before;
   }
 
   // ---- emit: each warp walks its segment 32 keys at a time in position order;
