@@ -130,6 +130,25 @@ def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
+def _hold(a, *objs):
+    """Keep the tensors whose addresses an argument struct holds alive for as long as the
+    struct: without this, a temporary such as ``x.to("cuda")`` passed to a builder is
+    freed on return and its memory handed to the next allocation (often the workspace)
+    before the kernel that reads it runs.  Nested structs bring their own references."""
+    refs = list(getattr(a, "_refs", ()))
+    for o in objs:
+        if o is None:
+            continue
+        if isinstance(o, dict):
+            refs.extend(v for v in o.values() if v is not None)
+        elif isinstance(o, C.Structure):
+            refs.extend(getattr(o, "_refs", ()))
+        else:
+            refs.append(o)
+    a._refs = refs
+    return a
+
+
 def _stream(stream):
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
@@ -162,7 +181,7 @@ def index_args(*, q, w, key_pool, page_table, lens, scores=None, q_scale=None, k
     a.q, a.q_scale, a.w = _ptr(q), _ptr(q_scale), _ptr(w)
     a.key_pool, a.key_scale = _ptr(key_pool), _ptr(key_scale)
     a.page_table, a.lens, a.scores = _ptr(page_table), _ptr(lens), _ptr(scores)
-    return a
+    return _hold(a, q, q_scale, w, key_pool, key_scale, page_table, lens, scores)
 
 
 def ls_index_score(*, q, w, key_pool, page_table, lens, scores, q_scale=None, key_scale=None, variant=0,
@@ -199,7 +218,7 @@ def c2f_args(*, index: IndexScoreArgs, k, summaries, block_scale, idx, sel_score
     a.summaries, a.block_scale = _ptr(summaries), _ptr(block_scale)
     a.idx, a.sel_score, a.survivors = _ptr(idx), _ptr(sel_score), _ptr(survivors)
     a.n_survivors, a.ub = _ptr(n_survivors), _ptr(ub)
-    return a
+    return _hold(a, index, summaries, block_scale, idx, sel_score, survivors, n_survivors, ub)
 
 
 def ls_block_bound_prune_workspace_size(a: BlockBoundPruneArgs) -> int:
@@ -257,7 +276,7 @@ def attn_args(*, q, k_rows, v_rows=None, sel=None, o, lse, scale, page_table=Non
     a.num_rows = k_rows.numel() // k_rows.shape[-1]
     a.q, a.k_rows, a.v_rows = _ptr(q), _ptr(k_rows), _ptr(v_rows)
     a.page_table, a.sel, a.o, a.lse = _ptr(page_table), _ptr(sel), _ptr(o), _ptr(lse)
-    return a
+    return _hold(a, q, k_rows, v_rows, page_table, sel, o, lse)
 
 
 def ls_sparse_attn_workspace_size(a: SparseAttnArgs) -> int:
@@ -300,7 +319,7 @@ def decode_step_args(*, index: IndexScoreArgs, k, attn: SparseAttnArgs, c2f=None
         a.hbuf, a.n_miss = _ptr(hotbuf["hbuf"]), _ptr(hotbuf.get("n_miss"))
     a.idx, a.sel_score = _ptr(idx), _ptr(sel_score)
     a.events = None if events is None else C.cast(events, C.c_void_p).value
-    return a
+    return _hold(a, index, attn, c2f, hotbuf, idx, sel_score, events)
 
 
 def ls_decode_step_workspace_size(a: DecodeStepArgs) -> int:

@@ -120,14 +120,16 @@ ls_status make_tmap_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_
   return LS_OK;
 }
 
-// 2D bf16 rows [rows][inner] (row stride in bytes), one-row boxes of 64 elements (128
-// bytes), 128-byte swizzle: used to gather single rows into swizzled panels.
-ls_status make_tmap_bf16_rows(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t stride) {
+// 2D bf16 rows [rows][inner] (row stride in bytes), boxes of 64 elements (128 bytes) x
+// `box_rows` rows, 128-byte swizzle.  One-row boxes gather single rows into swizzled
+// panels; 128-row boxes load a whole K-major operand panel.
+ls_status make_tmap_bf16_rows(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t stride,
+                              uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {stride};
-  cuuint32_t box[2] = {64, 1};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
@@ -363,9 +365,11 @@ ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressi
     }
     if (allow_smem(ls::attn_mla_tc, ls::mla::kSmem, g_smem_attn_tc) != cudaSuccess)
       return check_launch("attn_mla_tc attribute");
-    CUtensorMap kv_map;
-    LS_TRY(make_tmap_bf16_rows(&kv_map, p.krows, ls::mla::DK, (uint64_t)num_rows, (uint64_t)a->row_stride * 2));
-    ls::attn_mla_tc<<<dim3(2 * ns, a->batch), ls::mla::kThreads, ls::mla::kSmem, st>>>(p, kv_map);
+    CUtensorMap q_map, kv_map;
+    LS_TRY(make_tmap_bf16_rows(&q_map, a->q, ls::mla::DK, (uint64_t)a->batch * ls::mla::H, ls::mla::DK * 2,
+                               ls::mla::H));
+    LS_TRY(make_tmap_bf16_rows(&kv_map, p.krows, ls::mla::DK, (uint64_t)num_rows, (uint64_t)a->row_stride * 2, 1));
+    ls::attn_mla_tc<<<dim3(2 * ns, a->batch), ls::mla::kThreads, ls::mla::kSmem, st>>>(p, q_map, kv_map);
     LS_TRY(check_launch("attn_mla_tc"));
     if (ns > 1) {
       ls::attn_combine<<<dim3(ls::mla::DV / 32, a->batch), 128, 0, st>>>(p);

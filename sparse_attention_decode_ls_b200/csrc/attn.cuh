@@ -136,19 +136,32 @@ constexpr int kOffKv = kQBytes;
 constexpr int kOffP = kOffKv + 2 * kKvBytes;           // 221184
 constexpr int kPBytes = H * N * 2;                     // 8192
 constexpr int kOffBar = kOffP + kPBytes;               // 229376
-constexpr int kNumBars = 2 + 2 + 2 + 1 + 1 + 1;        // kv_full[2] kv_empty[2] s_full[2] p_full p_free o_done
+// kv_full[2] kv_empty[2] s_full[2] p_full p_free o_done q_full
+constexpr int kNumBars = 2 + 2 + 2 + 1 + 1 + 1 + 1;
 constexpr int kOffTmem = kOffBar + kNumBars * 8;
 constexpr int kSmem = 1024 + kOffTmem + 16;
-constexpr int kThreads = 256;
-constexpr int kLoaders = 32;                           // one warp per KV stage (TMA issue)
-constexpr int kChunksPerRow = DK * 2 / 16;             // 72
+// warps 0-3 softmax (warp w reads TMEM lanes 32w..32w+31), warp 4 MMA issue,
+// warps 5.. loaders: kLoadWarps per KV stage
+constexpr int kMmaWarp = 4;
+constexpr int kLoadWarps = 4;
+constexpr int kThreads = (kMmaWarp + 1 + 2 * kLoadWarps) * 32;          // 416
+constexpr int kBoxes = N * kPanels;                                     // 288 row boxes per tile
+constexpr int kBoxesPerLane = (kBoxes + kLoadWarps * 32 - 1) / (kLoadWarps * 32);  // 3
 constexpr uint32_t kIdescS = make_idesc(1 /*bf16*/, 128, N, false, false);
 constexpr uint32_t kIdescO = make_idesc(1 /*bf16*/, 128, DVH, false, true);
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 }  // namespace mla
 
-__global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p, const __grid_constant__ CUtensorMap kv_map) {
+// One CTA = (request b, KV split, output half).  The CTA keeps Q (128 heads x 576) in
+// shared memory, streams its share of the selected rows through two KV stages, forms
+// S = Q K^T (128 x 32 per tile) in TMEM, runs the online softmax on CUDA cores (one
+// thread per head), writes P (bf16) to shared memory and accumulates O_half += P V_half
+// in TMEM (256 columns).  Q is loaded by TMA (nine 128-row boxes); each KV tile is
+// gathered by TMA one 128-byte row box at a time, spread over four warps per stage.
+__global__ void __launch_bounds__(mla::kThreads, 1)
+    attn_mla_tc(const AttnParams p, const __grid_constant__ CUtensorMap q_map,
+                const __grid_constant__ CUtensorMap kv_map) {
   using namespace mla;
   extern __shared__ uint8_t sm_raw_a[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)sm_raw_a + 1023) & ~(uintptr_t)1023);
@@ -159,6 +172,7 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p, const 
   uint64_t* p_full = bars + 6;
   uint64_t* p_free = bars + 7;
   uint64_t* o_done = bars + 8;
+  uint64_t* q_full = bars + 9;
   uint32_t* tmem_slot = (uint32_t*)(sm + kOffTmem);
   __shared__ int s_abort;
   __shared__ uint32_t s_mask[2];        // valid rows of the tile in each stage
@@ -166,26 +180,16 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p, const 
   const int b = blockIdx.y;
   const int half = blockIdx.x & 1;
   const int split = blockIdx.x >> 1;
-  const int tid = threadIdx.x, warp = warp_id(), lane = lane_id();
+  const int warp = warp_id(), lane = lane_id();
   const int T_all = (p.k + N - 1) / N;
   const int t0 = (int)(((long long)T_all * split) / p.nsplit);
   const int t1 = (int)(((long long)T_all * (split + 1)) / p.nsplit);
   const int my_tiles = t1 - t0;
   const uint32_t sbase = smem_u32(sm);
 
-  // ---- Q (128 heads x 576) into nine 128-byte-swizzled K-major panels
-  {
-    const char* q = (const char*)p.q + (size_t)b * H * DK * 2;
-    for (int e = tid; e < H * kChunksPerRow; e += kThreads) {
-      const int h = e / kChunksPerRow, c = e - h * kChunksPerRow;
-      const int pn = c >> 3, j = c & 7;
-      cp_async_16(sbase + pn * (H * 128) + h * 128 + ((j ^ (h & 7)) << 4), q + (size_t)h * DK * 2 + c * 16);
-    }
-    cp_async_commit();
-  }
-  if (tid == 0) {
-    mbar_init(&kv_full[0], 1);  // the loader lane 0 arrives with the expected bytes
-    mbar_init(&kv_full[1], 1);
+  if (threadIdx.x == 0) {
+    mbar_init(&kv_full[0], kLoadWarps);  // one arrival per loader warp, with its bytes
+    mbar_init(&kv_full[1], kLoadWarps);
     mbar_init(&kv_empty[0], 1);
     mbar_init(&kv_empty[1], 1);
     mbar_init(&s_full[0], 1);
@@ -193,12 +197,11 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p, const 
     mbar_init(p_full, 128);
     mbar_init(p_free, 1);
     mbar_init(o_done, 1);
+    mbar_init(q_full, 1);
     s_abort = 0;
     fence_mbar_init();
   }
-  if (warp == 2) tmem_alloc(tmem_slot, 512);
-  cp_async_wait<0>();
-  fence_proxy_async_smem();
+  if (warp == kMmaWarp) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -206,13 +209,16 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p, const 
   const uint32_t tm_o = tmem;          // columns [0, 256): O half
   const uint32_t tm_s = tmem + 256;    // columns [256, 320): S double buffer
 
-  if (warp == 0 || warp == 1) {
-    // ================= loaders: warp w fills stage w with tiles w, w+2, ... =================
-    // Lane r owns row r of a tile: it resolves the row and issues the row's nine
-    // 128-byte TMA boxes (one per 64-dim panel, landing swizzled at line r of each
-    // panel).  Rows that are padding are zeroed with plain stores instead.  The stage
-    // completes when its valid rows' bytes have arrived.
-    const int st = warp;
+  if (warp > kMmaWarp) {
+    // ================= loaders: stage st holds tiles st, st+2, ... =================
+    // Every loader warp of a stage resolves the tile's 32 rows (lane r -> row r); the
+    // tile's 288 (row, panel) boxes are dealt round-robin over the stage's warps and
+    // lanes, each a 128-byte TMA box landing swizzled at line r of its panel.  Boxes
+    // of padding rows are zeroed with plain stores instead.  The stage completes when
+    // every loader warp has arrived (announcing its own bytes) and those bytes landed.
+    const int lw = warp - (kMmaWarp + 1);
+    const int st = lw / kLoadWarps, sub = lw - st * kLoadWarps;
+    const uint32_t stage = sbase + kOffKv + st * kKvBytes;
     int last = -1;
     for (int i = st; i < my_tiles; i += 2) {
       int go = 1;
@@ -227,85 +233,118 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p, const 
       long long row = -1;
       if (j < p.k) row = attn_row(p, b, p.sel[(size_t)b * p.k + j]);
       const uint32_t vmask = __ballot_sync(0xffffffffu, row >= 0);
-      const uint32_t dst0 = sbase + kOffKv + st * kKvBytes + lane * 128;
-      if (row < 0) {
-#pragma unroll 1
-        for (int pn = 0; pn < kPanels; ++pn)
+      long long brow[kBoxesPerLane];
+      bool zeroed = false;
+      int nbox = 0;  // boxes this lane copies
+#pragma unroll
+      for (int it = 0; it < kBoxesPerLane; ++it) {
+        const int e = sub + kLoadWarps * (lane + 32 * it);
+        const int r = min(e / kPanels, N - 1);
+        brow[it] = __shfl_sync(0xffffffffu, row, r);
+        nbox += (e < kBoxes && brow[it] >= 0) ? 1 : 0;
+        if (e < kBoxes && brow[it] < 0) {
+          const uint32_t dst = stage + (e - (e / kPanels) * kPanels) * kKvPanel + r * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c)
-            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst0 + pn * kKvPanel + c * 16), "r"(0)
-                         : "memory");
-        fence_proxy_async_smem();
+            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst + c * 16), "r"(0) : "memory");
+          zeroed = true;
+        }
       }
+      if (zeroed) fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
-        s_mask[st] = vmask;
-        mbar_arrive_expect_tx(&kv_full[st], (uint32_t)__popc(vmask) * (uint32_t)(DK * 2));
-      }
-      __syncwarp();
-      if (row >= 0) {
+      // each warp announces its own bytes before issuing its copies, so the stage's
+      // transaction count never runs ahead of what has been announced
 #pragma unroll
-        for (int pn = 0; pn < kPanels; ++pn)
-          tma_load_2d(dst0 + pn * kKvPanel, &kv_map, &kv_full[st], pn * 64, (int)row);
+      for (int o = 16; o > 0; o >>= 1) nbox += __shfl_xor_sync(0xffffffffu, nbox, o);
+      if (lane == 0) {
+        if (sub == 0) s_mask[st] = vmask;
+        mbar_arrive_expect_tx(&kv_full[st], (uint32_t)nbox * 128u);
+      }
+      __syncwarp();
+#pragma unroll
+      for (int it = 0; it < kBoxesPerLane; ++it) {
+        const int e = sub + kLoadWarps * (lane + 32 * it);
+        if (e < kBoxes && brow[it] >= 0) {
+          const int r = e / kPanels, pn = e - r * kPanels;
+          tma_load_2d(stage + pn * kKvPanel + r * 128, &kv_map, &kv_full[st], pn * 64, (int)brow[it]);
+        }
       }
       last = i;
     }
     // never leave with copies in flight
     if (lane == 0 && last >= 0) mbar_wait(&kv_full[st], (last >> 1) & 1);
     __syncwarp();
-  } else if (warp == 2) {
-    // ================= MMA issuer =================
+  } else if (warp == kMmaWarp) {
+    // ================= MMA issuer: event driven =================
+    // PV(i) goes out as soon as P(i) is ready and S(i) as soon as tile i has landed
+    // (with S(i-2)'s buffer consumed), so neither waits behind the other's inputs.
     if (lane == 0 && my_tiles > 0) {
       const uint32_t q_addr = sbase;
       const uint32_t p_addr = sbase + kOffP;
-      auto issue_s = [&](int i) -> bool {
-        const int st = i & 1;
-        if (!mbar_wait(&kv_full[st], (i >> 1) & 1)) return false;
-        tc_fence_after();
-        const uint32_t kv = sbase + kOffKv + st * kKvBytes;
+      mbar_arrive_expect_tx(q_full, kQBytes);
 #pragma unroll 1
-        for (int pn = 0; pn < kPanels; ++pn) {
+      for (int pn = 0; pn < kPanels; ++pn) tma_load_2d(q_addr + pn * (H * 128), &q_map, q_full, pn * 64, b * H);
+      bool ok = mbar_wait(q_full, 0);
+      int ns = 0, npv = 0;
+      uint64_t idle_since = 0;
+      while (ok && npv < my_tiles) {
+        bool progressed = false;
+        if (npv < ns && mbar_test_wait(p_full, npv & 1)) {
+          tc_fence_after();
+          const uint32_t v = sbase + kOffKv + (npv & 1) * kKvBytes + half * 4 * kKvPanel;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = make_sdesc(q_addr + pn * (H * 128) + kk * 32, 16, 1024, kSwizzle128);
-            const uint64_t bd = make_sdesc(kv + pn * kKvPanel + kk * 32, 16, 1024, kSwizzle128);
-            mma_bf16(tm_s + st * N, ad, bd, kIdescS, (pn | kk) != 0);
+          for (int kk = 0; kk < 2; ++kk) {
+            const uint64_t ad = make_sdesc(p_addr + kk * 2 * 2048, 2048, 128, kSwizzleNone);
+            const uint64_t bd = make_sdesc(v + kk * 16 * 128, kKvPanel, 1024, kSwizzle128);
+            mma_bf16(tm_o, ad, bd, kIdescO, (npv > 0 || kk > 0));
+          }
+          tc_commit(&kv_empty[npv & 1]);
+          tc_commit(p_free);
+          ++npv;
+          progressed = true;
+        }
+        if (ns < my_tiles && ns < npv + 2 && mbar_test_wait(&kv_full[ns & 1], (ns >> 1) & 1)) {
+          tc_fence_after();
+          const int st = ns & 1;
+          const uint32_t kv = sbase + kOffKv + st * kKvBytes;
+#pragma unroll 1
+          for (int pn = 0; pn < kPanels; ++pn) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = make_sdesc(q_addr + pn * (H * 128) + kk * 32, 16, 1024, kSwizzle128);
+              const uint64_t bd = make_sdesc(kv + pn * kKvPanel + kk * 32, 16, 1024, kSwizzle128);
+              mma_bf16(tm_s + st * N, ad, bd, kIdescS, (pn | kk) != 0);
+            }
+          }
+          tc_commit(&s_full[st]);
+          ++ns;
+          progressed = true;
+        }
+        if (progressed) {
+          idle_since = 0;
+        } else {
+          const uint64_t now = globaltimer();
+          if (idle_since == 0) {
+            idle_since = now;
+          } else if (now - idle_since > kWaitLimitNs) {
+            flag(LS_DEV_TIMEOUT);
+            ok = false;
           }
         }
-        tc_commit(&s_full[st]);
-        return true;
-      };
-      bool ok = issue_s(0);
-      if (ok && my_tiles > 1) ok = issue_s(1);
-      for (int i = 0; ok && i < my_tiles; ++i) {
-        const int st = i & 1;
-        if (!mbar_wait(p_full, i & 1)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t v = sbase + kOffKv + st * kKvBytes + half * 4 * kKvPanel;
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          const uint64_t ad = make_sdesc(p_addr + kk * 2 * 2048, 2048, 128, kSwizzleNone);
-          const uint64_t bd = make_sdesc(v + kk * 16 * 128, kKvPanel, 1024, kSwizzle128);
-          mma_bf16(tm_o, ad, bd, kIdescO, (i > 0 || kk > 0));
-        }
-        tc_commit(&kv_empty[st]);
-        tc_commit(p_free);
-        if (i + 2 < my_tiles) ok = issue_s(i + 2);
       }
       if (!ok) s_abort = 1;
       tc_commit(o_done);
     }
-  } else if (warp >= 4) {
-    // ================= softmax: warps 4..7, thread = head (warp 3 has no role) =================
-    const int wq = warp & 3;
-    const int h = wq * 32 + lane;
+  } else {
+    // ================= softmax: warps 0..3, thread = head =================
+    const int h = warp * 32 + lane;
     const float sl2 = p.scale * kLog2e;
-    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int i = 0; i < my_tiles; ++i) {
       const int st = i & 1;
-      // the loader published the tile's valid rows with its kv_full arrival
+      // the loaders published the tile's valid rows with their kv_full arrivals
       if (!mbar_wait(&kv_full[st], (i >> 1) & 1)) { ok = false; break; }
       const uint32_t vmask = s_mask[st];
       if (!mbar_wait(&s_full[st], (i >> 1) & 1)) { ok = false; break; }
@@ -417,7 +456,7 @@ __global__ void __launch_bounds__(256, 1) attn_mla_tc(const AttnParams p, const 
   __syncwarp();
   tc_fence_before();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

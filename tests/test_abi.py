@@ -120,3 +120,34 @@ def test_host_checks_reject_bad_arguments(lib):
     s.batch = 8
     assert lib.ls_sparse_attn_workspace_size(C.byref(s)) > 0
     assert _err(lib, lib.ls_sparse_attn_decode(C.byref(s), None, 0, None)) == B.LS_ERR_INVALID_ARG
+
+
+def test_arg_structs_keep_their_tensors_alive():
+    """A builder given temporaries (x.to(device) inside the call) must hold them until
+    the struct goes away; otherwise their memory is reused before the kernel reads it."""
+    import gc
+    import weakref
+
+    import torch
+
+    made = []
+
+    def tmp(*shape, dtype=torch.float32):
+        t = torch.zeros(*shape, dtype=dtype)
+        made.append(weakref.ref(t))
+        return t
+
+    a = B.attn_args(q=tmp(2, 128, 576, dtype=torch.bfloat16), k_rows=tmp(4, 64, 576, dtype=torch.bfloat16),
+                    sel=tmp(2, 64, dtype=torch.int32), o=tmp(2, 128, 512, dtype=torch.bfloat16), lse=tmp(2, 128),
+                    scale=0.1, page_table=tmp(2, 4, dtype=torch.int32))
+    ia = B.index_args(q=tmp(2, 64, 128), w=tmp(2, 64), key_pool=tmp(3, 64, 128),
+                      page_table=tmp(2, 4, dtype=torch.int32), lens=tmp(2, dtype=torch.int32), scores=tmp(2, 256))
+    c = B.c2f_args(index=ia, k=64, summaries=tmp(2, 4, 256, dtype=torch.uint8), block_scale=tmp(2, 4),
+                   idx=tmp(2, 64, dtype=torch.int32))
+    d = B.decode_step_args(index=ia, k=64, attn=a, idx=tmp(2, 64, dtype=torch.int32))
+    del ia, a
+    gc.collect()
+    assert all(r() is not None for r in made)
+    del c, d
+    gc.collect()
+    assert all(r() is None for r in made)
