@@ -233,9 +233,11 @@ def run_ours(args):
         wl.step()
     torch.cuda.synchronize()
     B.ls_check_device_status()
-    stage_ev = [new_events(6) for _ in range(K)]
+    # timed steps: only the indexer (the roofline kernel) is bracketed by events, so the
+    # later kernels of the step still start as programmatic dependents of one another
+    idx_ev = [new_events(2) for _ in range(K)]
     step_ev = [new_events(2) for _ in range(K)]
-    arrs = [B.event_array(s) for s in stage_ev]
+    arrs = [B.event_array([e[0], e[1], None, None, None, None]) for e in idx_ev]
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
@@ -252,7 +254,14 @@ def run_ours(args):
     torch.cuda.synchronize()
     status = B.ls_check_device_status()
     step_ms = [s[0].elapsed_time(s[1]) for s in step_ev]
-    idx_ms = [s[0].elapsed_time(s[1]) for s in stage_ev]
+    idx_ms = [s[0].elapsed_time(s[1]) for s in idx_ev]
+    # stage breakdown (not part of the timed number): every stage boundary recorded
+    nb = min(K, 100)
+    stage_ev = [new_events(6) for _ in range(nb)]
+    for i in range(nb):
+        flush.zero_()
+        wl.step(events=B.event_array(stage_ev[i]))
+    torch.cuda.synchronize()
     topk_ms = [s[1].elapsed_time(s[4]) for s in stage_ev]
     attn_ms = [s[4].elapsed_time(s[5]) for s in stage_ev]
     total_ms = sum(step_ms)
@@ -310,7 +319,9 @@ def run_ours(args):
                         "algorithmic_bytes_per_launch": idx_bytes,
                         "indexer_ms": idx_mean_ms, "topk_ms": statistics.mean(topk_ms),
                         "attn_ms": statistics.mean(attn_ms),
-                        "indexer_plus_attn_GBps": combined, "indexer_plus_attn_frac": combined / peak},
+                        "indexer_plus_attn_GBps": combined, "indexer_plus_attn_frac": combined / peak,
+                        "stage_note": "indexer_ms from the timed steps; topk_ms and attn_ms from a separate "
+                                      "pass with every stage boundary recorded"},
            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d_bytes,
                    "d2h_bytes_per_step": d2h_bytes},
            "clocks": clk.summary(), "gpu_launches": K * wl.kernels_per_step, "device_status": status}

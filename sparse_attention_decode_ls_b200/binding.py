@@ -341,8 +341,9 @@ def ls_check_device_status(stream=None) -> int:
 
 
 def event_array(events):
-    """ctypes array of raw cudaEvent_t handles from torch.cuda.Event objects."""
+    """ctypes array of raw cudaEvent_t handles from torch.cuda.Event objects (None:
+    that stage boundary is not recorded)."""
     arr = (C.c_void_p * len(events))()
     for i, e in enumerate(events):
-        arr[i] = e.cuda_event
+        arr[i] = None if e is None else e.cuda_event
     return arr

@@ -121,8 +121,7 @@ ls_status make_tmap_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_
 }
 
 // 2D bf16 rows [rows][inner] (row stride in bytes), boxes of 64 elements (128 bytes) x
-// `box_rows` rows, 128-byte swizzle.  One-row boxes gather single rows into swizzled
-// panels; 128-row boxes load a whole K-major operand panel.
+// `box_rows` rows, 128-byte swizzle: 128-row boxes load a whole K-major operand panel.
 ls_status make_tmap_bf16_rows(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t stride,
                               uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
@@ -247,8 +246,12 @@ cudaLaunchConfig_t topk_config(int B, int smem, cudaStream_t st, cudaLaunchAttri
   attr[0].val.clusterDim.x = CL;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // the kernel waits (griddepcontrol.wait) before reading anything, so it may always be
+  // launched as a programmatic dependent of the kernel before
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cfg;
 }
 
@@ -262,7 +265,7 @@ bool topk16_supported(cudaStream_t st) {
             cudaSuccess;
   if (ok) ok = allow_smem(ls::topk_cluster<16>, ls::kTopkCacheKeys * 4 + ls::kTopkExtraBytes, g_smem_topk16) == cudaSuccess;
   if (ok) {
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = topk_config<16>(1, ls::kTopkCacheKeys * 4 + ls::kTopkExtraBytes, st, attr);
     int n = 0;
     ok = cudaOccupancyMaxActiveClusters(&n, ls::topk_cluster<16>, &cfg) == cudaSuccess && n >= 1;
@@ -279,7 +282,7 @@ ls_status launch_topk_cl(const ls::TopkParams& p0, int B, cudaStream_t st, std::
   p.cache_keys = lc <= ls::kTopkCacheKeys ? lc : 0;
   if (allow_smem(ls::topk_cluster<CL>, ls::kTopkCacheKeys * 4 + ls::kTopkExtraBytes, smem_done) != cudaSuccess)
     return check_launch("topk attribute");
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cudaLaunchConfig_t cfg = topk_config<CL>(B, p.cache_keys * 4 + ls::kTopkExtraBytes, st, attr);
   cudaError_t e = cudaLaunchKernelEx(&cfg, ls::topk_cluster<CL>, p);
   if (e != cudaSuccess) return fail(LS_ERR_CUDA, "topk_cluster: %s", cudaGetErrorString(e));
@@ -345,9 +348,27 @@ ls_status validate_attn(const ls_sparse_attn_args* a, bool need_sel) {
 
 std::atomic<uint64_t> g_smem_attn_tc{0}, g_smem_attn_simt_f{0}, g_smem_attn_simt_b{0};
 
+// Programmatic dependent launch: the kernel may start while the one before it finishes
+// (it waits for it with griddepcontrol.wait before touching its output).
+cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, size_t smem, cudaStream_t st, cudaLaunchAttribute* attr,
+                              bool pdl) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cfg;
+}
+
+// `pdl`: launched right behind another kernel of the same decode step, whose outputs
+// (selection, or gathered rows) the attention reads; Q is not among them.
 ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressing, const int* page_table,
                       int max_pages, int n_slots, const void* rows, long long num_rows, void* ws, size_t ws_bytes,
-                      cudaStream_t st) {
+                      cudaStream_t st, bool pdl) {
   ls::AttnParams p{};
   p.B = a->batch; p.H = a->heads; p.dk = a->dk; p.dv = a->dv; p.k = a->k; p.scale = a->softmax_scale;
   p.addressing = addressing; p.max_pages = max_pages; p.n_slots = n_slots; p.row_stride = a->row_stride;
@@ -365,14 +386,19 @@ ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressi
     }
     if (allow_smem(ls::attn_mla_tc, ls::mla::kSmem, g_smem_attn_tc) != cudaSuccess)
       return check_launch("attn_mla_tc attribute");
-    CUtensorMap q_map, kv_map;
+    CUtensorMap q_map;
     LS_TRY(make_tmap_bf16_rows(&q_map, a->q, ls::mla::DK, (uint64_t)a->batch * ls::mla::H, ls::mla::DK * 2,
                                ls::mla::H));
-    LS_TRY(make_tmap_bf16_rows(&kv_map, p.krows, ls::mla::DK, (uint64_t)num_rows, (uint64_t)a->row_stride * 2, 1));
-    ls::attn_mla_tc<<<dim3(2 * ns, a->batch), ls::mla::kThreads, ls::mla::kSmem, st>>>(p, q_map, kv_map);
+    p.early_q = pdl ? 1 : 0;
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = pdl_config(dim3(2 * ns, a->batch), dim3(ls::mla::kThreads), ls::mla::kSmem, st, attr, pdl);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, ls::attn_mla_tc, p, q_map);
+    if (e != cudaSuccess) return fail(LS_ERR_CUDA, "attn_mla_tc: %s", cudaGetErrorString(e));
     LS_TRY(check_launch("attn_mla_tc"));
     if (ns > 1) {
-      ls::attn_combine<<<dim3(ls::mla::DV / 32, a->batch), 128, 0, st>>>(p);
+      cudaLaunchConfig_t cc = pdl_config(dim3(ls::mla::DV / 32, a->batch), dim3(128), 0, st, attr, true);
+      e = cudaLaunchKernelEx(&cc, ls::attn_combine, p);
+      if (e != cudaSuccess) return fail(LS_ERR_CUDA, "attn_combine: %s", cudaGetErrorString(e));
       LS_TRY(check_launch("attn_combine"));
     }
     return LS_OK;
@@ -675,7 +701,7 @@ ls_status ls_sparse_attn_decode(const ls_sparse_attn_args* a, void* workspace, s
                                 ls_stream_t stream) {
   LS_TRY(validate_attn(a, true));
   LS_TRY(launch_attn(a, a->sel, a->addressing, a->page_table, a->max_pages, a->n_slots, nullptr, a->num_rows,
-                     workspace, workspace_bytes, (cudaStream_t)stream));
+                     workspace, workspace_bytes, (cudaStream_t)stream, false));
   return ok();
 }
 
@@ -755,14 +781,14 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
     LS_TRY(launch_gather(&g, st));
     rec(4);
     LS_TRY(launch_attn(&at, sel_slot, LS_ROWS_SLOTS, nullptr, 0, a->n_slots, a->hbuf,
-                       (long long)ix->batch * a->n_slots, attn_ws, attn_ws_b, st));
+                       (long long)ix->batch * a->n_slots, attn_ws, attn_ws_b, st, true));
   } else {
     rec(2);
     rec(3);
     rec(4);
     const int* pt = at.page_table ? at.page_table : ix->page_table;
     const int mp = at.page_table ? at.max_pages : ix->max_pages;
-    LS_TRY(launch_attn(&at, idx, LS_ROWS_PAGED, pt, mp, 0, nullptr, at.num_rows, attn_ws, attn_ws_b, st));
+    LS_TRY(launch_attn(&at, idx, LS_ROWS_PAGED, pt, mp, 0, nullptr, at.num_rows, attn_ws, attn_ws_b, st, true));
   }
   rec(5);
   return ok();
@@ -826,6 +852,6 @@ extern "C" ls_status ls_sparse_attn_decode_noalloc(const ls_sparse_attn_args* a,
   void* ws = nullptr;
   if (need > 0) LS_TRY(static_scratch(&ws));
   LS_TRY(launch_attn(a, a->sel, a->addressing, a->page_table, a->max_pages, a->n_slots, nullptr, a->num_rows, ws,
-                     need > 0 ? kStaticAttnScratchBytes : 0, (cudaStream_t)stream));
+                     need > 0 ? kStaticAttnScratchBytes : 0, (cudaStream_t)stream, false));
   return ok();
 }

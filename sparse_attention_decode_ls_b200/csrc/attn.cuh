@@ -40,6 +40,7 @@ struct AttnParams {
   int nsplit;
   float* part_o;     // [B,nsplit,dv,H] unnormalised partial outputs (head fastest)
   float* part_ml;    // [B,nsplit,H,2] running max (log2 domain) and sum
+  int early_q;       // tensor-core kernel: load Q before waiting for the kernel before
 };
 
 // Row index of selection value sv of request b, or -1 (padding or out of range).
@@ -145,23 +146,33 @@ constexpr int kSmem = 1024 + kOffTmem + 16;
 constexpr int kMmaWarp = 4;
 constexpr int kLoadWarps = 4;
 constexpr int kThreads = (kMmaWarp + 1 + 2 * kLoadWarps) * 32;          // 416
-constexpr int kBoxes = N * kPanels;                                     // 288 row boxes per tile
-constexpr int kBoxesPerLane = (kBoxes + kLoadWarps * 32 - 1) / (kLoadWarps * 32);  // 3
+constexpr int kChunksPerRow = DK * 2 / 16;                              // 72 16-byte chunks
+constexpr int kChunksPerThread = N * kChunksPerRow / (kLoadWarps * 32);  // 18
+static_assert(N * kChunksPerRow % (kLoadWarps * 32) == 0, "chunks must split evenly");
 constexpr uint32_t kIdescS = make_idesc(1 /*bf16*/, 128, N, false, false);
 constexpr uint32_t kIdescO = make_idesc(1 /*bf16*/, 128, DVH, false, true);
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 }  // namespace mla
 
+// Q of request b (128 heads x 576) as nine 128-row TMA boxes, one 128-byte-swizzled
+// K-major panel each.  One thread.
+__device__ __forceinline__ void issue_q_load(uint32_t q_smem, const CUtensorMap* q_map, uint64_t* bar, int b) {
+  using namespace mla;
+  mbar_arrive_expect_tx(bar, kQBytes);
+#pragma unroll 1
+  for (int pn = 0; pn < kPanels; ++pn) tma_load_2d(q_smem + pn * (H * 128), q_map, bar, pn * 64, b * H);
+}
+
 // One CTA = (request b, KV split, output half).  The CTA keeps Q (128 heads x 576) in
 // shared memory, streams its share of the selected rows through two KV stages, forms
 // S = Q K^T (128 x 32 per tile) in TMEM, runs the online softmax on CUDA cores (one
 // thread per head), writes P (bf16) to shared memory and accumulates O_half += P V_half
 // in TMEM (256 columns).  Q is loaded by TMA (nine 128-row boxes); each KV tile is
-// gathered by TMA one 128-byte row box at a time, spread over four warps per stage.
+// gathered with 16-byte cp.async copies by four warps per stage (a row gather would
+// need one TMA box per 128 bytes, and the TMA unit issues those too slowly).
 __global__ void __launch_bounds__(mla::kThreads, 1)
-    attn_mla_tc(const AttnParams p, const __grid_constant__ CUtensorMap q_map,
-                const __grid_constant__ CUtensorMap kv_map) {
+    attn_mla_tc(const AttnParams p, const __grid_constant__ CUtensorMap q_map) {
   using namespace mla;
   extern __shared__ uint8_t sm_raw_a[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)sm_raw_a + 1023) & ~(uintptr_t)1023);
@@ -188,7 +199,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   const uint32_t sbase = smem_u32(sm);
 
   if (threadIdx.x == 0) {
-    mbar_init(&kv_full[0], kLoadWarps);  // one arrival per loader warp, with its bytes
+    mbar_init(&kv_full[0], kLoadWarps);  // one arrival per loader warp, after its copies
     mbar_init(&kv_full[1], kLoadWarps);
     mbar_init(&kv_empty[0], 1);
     mbar_init(&kv_empty[1], 1);
@@ -200,27 +211,44 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     mbar_init(q_full, 1);
     s_abort = 0;
     fence_mbar_init();
+    if (p.early_q && my_tiles > 0) issue_q_load(sbase, &q_map, q_full, b);
   }
   if (warp == kMmaWarp) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // under programmatic dependent launch everything above overlaps the kernel before;
+  // the selection, the rows and the outputs are touched only after it has finished
+  griddep_wait();
+  griddep_launch_dependents();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tm_o = tmem;          // columns [0, 256): O half
   const uint32_t tm_s = tmem + 256;    // columns [256, 320): S double buffer
 
   if (warp > kMmaWarp) {
     // ================= loaders: stage st holds tiles st, st+2, ... =================
-    // Every loader warp of a stage resolves the tile's 32 rows (lane r -> row r); the
-    // tile's 288 (row, panel) boxes are dealt round-robin over the stage's warps and
-    // lanes, each a 128-byte TMA box landing swizzled at line r of its panel.  Boxes
-    // of padding rows are zeroed with plain stores instead.  The stage completes when
-    // every loader warp has arrived (announcing its own bytes) and those bytes landed.
+    // Every loader warp of a stage resolves the tile's 32 rows (lane r -> row r).  The
+    // tile's 32 x 72 16-byte chunks are dealt over the stage's 128 threads in row-major
+    // order (consecutive threads, consecutive chunks of a row: coalesced), each copied
+    // with cp.async to its 128-byte-swizzled place in its panel; chunks of padding rows
+    // are zeroed instead.  A thread waits for its own copies, makes them visible to the
+    // tensor core (proxy fence), and the warp arrives on the stage's barrier.
     const int lw = warp - (kMmaWarp + 1);
-    const int st = lw / kLoadWarps, sub = lw - st * kLoadWarps;
+    const int st = lw / kLoadWarps;
+    const int t = (lw - st * kLoadWarps) * 32 + lane;  // thread within the stage
     const uint32_t stage = sbase + kOffKv + st * kKvBytes;
-    int last = -1;
+    const char* kv_base = (const char*)p.krows;
+    const long long row_bytes = p.row_stride * 2;
+    // row of tile i for this lane; resolved one tile ahead, so the two dependent loads
+    // (selection, page table) overlap the wait for the stage
+    auto tile_row = [&](int i) -> long long {
+      const int j = (t0 + i) * N + lane;
+      return (i < my_tiles && j < p.k) ? attn_row(p, b, p.sel[(size_t)b * p.k + j]) : -1;
+    };
+    long long row_next = tile_row(st);
     for (int i = st; i < my_tiles; i += 2) {
+      const long long row = row_next;
+      row_next = tile_row(i + 2);
       int go = 1;
       if (lane == 0) {  // one lane decides, so the warp stays converged
         go = (i < 2) || mbar_wait(&kv_empty[st], ((i >> 1) - 1) & 1);
@@ -229,50 +257,27 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
       }
       go = __shfl_sync(0xffffffffu, go, 0);
       if (!go) break;
-      const int j = (t0 + i) * N + lane;
-      long long row = -1;
-      if (j < p.k) row = attn_row(p, b, p.sel[(size_t)b * p.k + j]);
       const uint32_t vmask = __ballot_sync(0xffffffffu, row >= 0);
-      long long brow[kBoxesPerLane];
-      bool zeroed = false;
-      int nbox = 0;  // boxes this lane copies
-#pragma unroll
-      for (int it = 0; it < kBoxesPerLane; ++it) {
-        const int e = sub + kLoadWarps * (lane + 32 * it);
-        const int r = min(e / kPanels, N - 1);
-        brow[it] = __shfl_sync(0xffffffffu, row, r);
-        nbox += (e < kBoxes && brow[it] >= 0) ? 1 : 0;
-        if (e < kBoxes && brow[it] < 0) {
-          const uint32_t dst = stage + (e - (e / kPanels) * kPanels) * kKvPanel + r * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst + c * 16), "r"(0) : "memory");
-          zeroed = true;
-        }
+#pragma unroll 6
+      for (int it = 0; it < kChunksPerThread; ++it) {
+        const int e = t + kLoadWarps * 32 * it;
+        const int r = e / kChunksPerRow, c = e - r * kChunksPerRow;
+        const long long rr = __shfl_sync(0xffffffffu, row, r);
+        const uint32_t dst = stage + (c >> 3) * kKvPanel + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+        if (rr >= 0)
+          cp_async_16(dst, kv_base + rr * row_bytes + c * 16);
+        else
+          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0) : "memory");
       }
-      if (zeroed) fence_proxy_async_smem();
+      cp_async_commit();
+      cp_async_wait<0>();
+      fence_proxy_async_smem();
       __syncwarp();
-      // each warp announces its own bytes before issuing its copies, so the stage's
-      // transaction count never runs ahead of what has been announced
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) nbox += __shfl_xor_sync(0xffffffffu, nbox, o);
       if (lane == 0) {
-        if (sub == 0) s_mask[st] = vmask;
-        mbar_arrive_expect_tx(&kv_full[st], (uint32_t)nbox * 128u);
+        if (t == 0) s_mask[st] = vmask;
+        mbar_arrive(&kv_full[st]);
       }
-      __syncwarp();
-#pragma unroll
-      for (int it = 0; it < kBoxesPerLane; ++it) {
-        const int e = sub + kLoadWarps * (lane + 32 * it);
-        if (e < kBoxes && brow[it] >= 0) {
-          const int r = e / kPanels, pn = e - r * kPanels;
-          tma_load_2d(stage + pn * kKvPanel + r * 128, &kv_map, &kv_full[st], pn * 64, (int)brow[it]);
-        }
-      }
-      last = i;
     }
-    // never leave with copies in flight
-    if (lane == 0 && last >= 0) mbar_wait(&kv_full[st], (last >> 1) & 1);
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ================= MMA issuer: event driven =================
@@ -281,10 +286,10 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     if (lane == 0 && my_tiles > 0) {
       const uint32_t q_addr = sbase;
       const uint32_t p_addr = sbase + kOffP;
-      mbar_arrive_expect_tx(q_full, kQBytes);
-#pragma unroll 1
-      for (int pn = 0; pn < kPanels; ++pn) tma_load_2d(q_addr + pn * (H * 128), &q_map, q_full, pn * 64, b * H);
+      if (!p.early_q) issue_q_load(sbase, &q_map, q_full, b);
       bool ok = mbar_wait(q_full, 0);
+      // S(i) goes out whole once tile i has landed (and S(i-2)'s buffer is consumed),
+      // PV(i) as soon as P(i) is ready; each is checked without blocking on the other
       int ns = 0, npv = 0;
       uint64_t idle_since = 0;
       while (ok && npv < my_tiles) {
@@ -468,6 +473,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
 __global__ void __launch_bounds__(128) attn_combine(const AttnParams p) {
   using namespace mla;
   const int d0 = blockIdx.x * 32, b = blockIdx.y, h = threadIdx.x;
+  griddep_wait();  // the partials come from the kernel before
   const float* ml = p.part_ml + (size_t)b * p.nsplit * H * 2;
   float M = -INFINITY;
   for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, ml[((size_t)s * H + h) * 2]);

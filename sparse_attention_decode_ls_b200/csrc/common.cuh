@@ -98,6 +98,18 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // ---------------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the kernel before it is still running; it must call
+// griddep_wait() (every thread that touches that kernel's output, or that writes memory
+// the earlier kernel may still read) before doing so.  Without the launch attribute both
+// calls are no-ops.
+// ---------------------------------------------------------------------------------
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------------
 // Proxy fences and async copies
 // ---------------------------------------------------------------------------------
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy

@@ -170,6 +170,7 @@ __global__ void __launch_bounds__(192, 1)
   __shared__ int s_abort;
 
   const int b = blockIdx.y, cta = blockIdx.x, tid = threadIdx.x, warp = warp_id(), lane = lane_id();
+  griddep_launch_dependents();  // the next kernel may be scheduled now; it waits for this one
   const int L = p.lens[b];
   const bool len_ok = L >= 0 && L <= p.max_len && L <= p.max_pages * 64;
   if (!len_ok) {

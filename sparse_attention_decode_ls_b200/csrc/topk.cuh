@@ -91,6 +91,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
   const int tid = threadIdx.x, lane = lane_id(), warp = warp_id();
   constexpr int kWarps = kTopkThreads / 32;
   const int k = p.k;
+  griddep_wait();  // the scores come from the kernel before
+  griddep_launch_dependents();
 
   long long nll = ((long long)p.lens[b] * p.len_mul + p.len_div - 1) / p.len_div;
   bool bad = nll < 0 || nll > p.len_limit;
