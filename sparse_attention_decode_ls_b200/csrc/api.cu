@@ -396,7 +396,8 @@ ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressi
     if (e != cudaSuccess) return fail(LS_ERR_CUDA, "attn_mla_tc: %s", cudaGetErrorString(e));
     LS_TRY(check_launch("attn_mla_tc"));
     if (ns > 1) {
-      cudaLaunchConfig_t cc = pdl_config(dim3(ls::mla::DV / 32, a->batch), dim3(128), 0, st, attr, true);
+      cudaLaunchConfig_t cc = pdl_config(dim3(ls::mla::H * ls::mla::DV / 8 / ls::kCombineThreads, a->batch),
+                                         dim3(ls::kCombineThreads), 0, st, attr, true);
       e = cudaLaunchKernelEx(&cc, ls::attn_combine, p);
       if (e != cudaSuccess) return fail(LS_ERR_CUDA, "attn_combine: %s", cudaGetErrorString(e));
       LS_TRY(check_launch("attn_combine"));

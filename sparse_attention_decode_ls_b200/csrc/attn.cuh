@@ -38,7 +38,7 @@ struct AttnParams {
   void* o;
   float* lse;
   int nsplit;
-  float* part_o;     // [B,nsplit,dv,H] unnormalised partial outputs (head fastest)
+  float* part_o;     // [B,nsplit,H,dv] unnormalised partial outputs (dim fastest)
   float* part_ml;    // [B,nsplit,H,2] running max (log2 domain) and sum
   int early_q;       // tensor-core kernel: load Q before waiting for the kernel before
 };
@@ -431,10 +431,12 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
             *(uint4*)(o + c) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         } else {
-          // head-fastest layout [b][split][dim][head]: consecutive threads, consecutive words
-          float* o = p.part_o + (((size_t)b * p.nsplit + split) * DV + half * DVH + c0) * H + h;
+          // layout [b][split][head][dim]: each thread stores 128 contiguous bytes
+          float4* o = (float4*)(p.part_o + (((size_t)b * p.nsplit + split) * H + h) * DV + half * DVH + c0);
+          const bool any = l_run > 0.f;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[(size_t)c * H] = l_run > 0.f ? v[c] : 0.f;
+          for (int c = 0; c < 32; c += 4)
+            o[c / 4] = any ? make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
       if (half == 0) {
@@ -447,8 +449,8 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
         }
       }
     } else if (my_tiles == 0 && p.nsplit > 1) {
-      float* o = p.part_o + (((size_t)b * p.nsplit + split) * DV + half * DVH) * H + h;
-      for (int c = 0; c < DVH; ++c) o[(size_t)c * H] = 0.f;
+      float4* o = (float4*)(p.part_o + (((size_t)b * p.nsplit + split) * H + h) * DV + half * DVH);
+      for (int c = 0; c < DVH / 4; ++c) o[c] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (half == 0) {
         float* ml = p.part_ml + (((size_t)b * p.nsplit + split) * H + h) * 2;
         ml[0] = -INFINITY;
@@ -468,43 +470,48 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
 }
 
 // Merge split-KV partials: o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
-// grid (DV / 32, B), 128 threads: thread = head, 32 output dims per CTA; every read of
-// the head-fastest partials is coalesced across the warp.
-__global__ void __launch_bounds__(128) attn_combine(const AttnParams p) {
+// One thread per (request, head, 8 consecutive dims); grid (H * DV / 8 / 256, B), 256
+// threads.  A warp covers 256 contiguous dims of one head, so every partial read is a
+// coalesced 1 KB run and every output store a 512-byte run; the 2 x nsplit 16-byte loads
+// of a thread are independent of one another.
+constexpr int kCombineThreads = 256;
+__global__ void __launch_bounds__(kCombineThreads) attn_combine(const AttnParams p) {
   using namespace mla;
-  const int d0 = blockIdx.x * 32, b = blockIdx.y, h = threadIdx.x;
   griddep_wait();  // the partials come from the kernel before
-  const float* ml = p.part_ml + (size_t)b * p.nsplit * H * 2;
+  const int b = blockIdx.y;
+  const int item = blockIdx.x * kCombineThreads + threadIdx.x;
+  const int h = item / (DV / 8), d0 = (item - h * (DV / 8)) * 8;
+  const float* ml = p.part_ml + (size_t)b * p.nsplit * H * 2 + (size_t)h * 2;
   float M = -INFINITY;
-  for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, ml[((size_t)s * H + h) * 2]);
-  float acc[32];
+  for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, ml[(size_t)s * H * 2]);
+  float acc[8];
 #pragma unroll
-  for (int e = 0; e < 32; ++e) acc[e] = 0.f;
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
   float Lsum = 0.f;
   if (M != -INFINITY) {
+#pragma unroll 4
     for (int s = 0; s < p.nsplit; ++s) {
-      const float l = ml[((size_t)s * H + h) * 2 + 1];
-      if (l <= 0.f) continue;
-      const float wgt = exp2f(ml[((size_t)s * H + h) * 2] - M);
+      const float l = ml[(size_t)s * H * 2 + 1];
+      if (!(l > 0.f)) continue;
+      const float wgt = exp2f(ml[(size_t)s * H * 2] - M);
       Lsum += wgt * l;
-      const float* po = p.part_o + (((size_t)b * p.nsplit + s) * DV + d0) * H + h;
-#pragma unroll
-      for (int e = 0; e < 32; ++e) acc[e] = fmaf(wgt, po[(size_t)e * H], acc[e]);
+      const float4* po = (const float4*)(p.part_o + (((size_t)b * p.nsplit + s) * H + h) * DV + d0);
+      const float4 x = po[0], y = po[1];
+      acc[0] = fmaf(wgt, x.x, acc[0]); acc[1] = fmaf(wgt, x.y, acc[1]);
+      acc[2] = fmaf(wgt, x.z, acc[2]); acc[3] = fmaf(wgt, x.w, acc[3]);
+      acc[4] = fmaf(wgt, y.x, acc[4]); acc[5] = fmaf(wgt, y.y, acc[5]);
+      acc[6] = fmaf(wgt, y.z, acc[6]); acc[7] = fmaf(wgt, y.w, acc[7]);
     }
   }
   const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-  __nv_bfloat16* o = (__nv_bfloat16*)p.o + ((size_t)b * H + h) * DV + d0;
+  uint32_t w[4];
 #pragma unroll
-  for (int e = 0; e < 32; e += 8) {
-    uint32_t w[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      __nv_bfloat162 two = __floats2bfloat162_rn(acc[e + 2 * q] * inv, acc[e + 2 * q + 1] * inv);
-      w[q] = *(uint32_t*)&two;
-    }
-    *(uint4*)(o + e) = make_uint4(w[0], w[1], w[2], w[3]);
+  for (int q = 0; q < 4; ++q) {
+    __nv_bfloat162 two = __floats2bfloat162_rn(acc[2 * q] * inv, acc[2 * q + 1] * inv);
+    w[q] = *(uint32_t*)&two;
   }
-  if (blockIdx.x == 0) p.lse[(size_t)b * H + h] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
+  *(uint4*)((__nv_bfloat16*)p.o + ((size_t)b * H + h) * DV + d0) = make_uint4(w[0], w[1], w[2], w[3]);
+  if (d0 == 0) p.lse[(size_t)b * H + h] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
 }
 
 }  // namespace ls
