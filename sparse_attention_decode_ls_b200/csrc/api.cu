@@ -390,8 +390,14 @@ ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressi
     LS_TRY(make_tmap_bf16_rows(&q_map, a->q, ls::mla::DK, (uint64_t)a->batch * ls::mla::H, ls::mla::DK * 2,
                                ls::mla::H));
     p.early_q = pdl ? 1 : 0;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = pdl_config(dim3(2 * ns, a->batch), dim3(ls::mla::kThreads), ls::mla::kSmem, st, attr, pdl);
+    // the two CTAs of an (request, split) pair form a cluster
+    attr[cfg.numAttrs].id = cudaLaunchAttributeClusterDimension;
+    attr[cfg.numAttrs].val.clusterDim.x = 2;
+    attr[cfg.numAttrs].val.clusterDim.y = 1;
+    attr[cfg.numAttrs].val.clusterDim.z = 1;
+    cfg.numAttrs += 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, ls::attn_mla_tc, p, q_map);
     if (e != cudaSuccess) return fail(LS_ERR_CUDA, "attn_mla_tc: %s", cudaGetErrorString(e));
     LS_TRY(check_launch("attn_mla_tc"));

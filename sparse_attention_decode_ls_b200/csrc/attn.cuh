@@ -38,7 +38,7 @@ struct AttnParams {
   void* o;
   float* lse;
   int nsplit;
-  float* part_o;     // [B,nsplit,H,dv] unnormalised partial outputs (dim fastest)
+  float* part_o;     // [B,nsplit,dv/4,H,4] unnormalised partial outputs (4-dim granules, head next)
   float* part_ml;    // [B,nsplit,H,2] running max (log2 domain) and sum
   int early_q;       // tensor-core kernel: load Q before waiting for the kernel before
 };
@@ -130,47 +130,59 @@ __global__ void __launch_bounds__(256) attn_simt(const AttnParams p) {
 namespace mla {
 constexpr int H = 128, DK = 576, DV = 512, DVH = 256, N = 32;
 constexpr int kPanels = DK / 64;                       // 9 panels of 64 bf16 (128 bytes)
-constexpr int kQBytes = kPanels * H * 128;             // 147456
+// The two CTAs of a pair split the latent dims of S = Q K^T: rank 0 takes panels 0-4,
+// rank 1 panels 5-8.  Each loads panels 4r .. 4r+4 of every row (its S panels plus its
+// half of V: panels 0-3 or 4-7).
+constexpr int kLocalPanels = 5;
+__host__ __device__ constexpr int s_panels(int rank) { return rank == 0 ? 5 : 4; }  // S panels per rank
+constexpr int kQBytes = 5 * H * 128;                   // 81920 (rank 1 uses 65536)
 constexpr int kKvPanel = N * 128;                      // 4096
-constexpr int kKvBytes = kPanels * kKvPanel;           // 36864
+constexpr int kStageBytes = kLocalPanels * kKvPanel;   // 20480
+constexpr int kStages = 4;
 constexpr int kOffKv = kQBytes;
-constexpr int kOffP = kOffKv + 2 * kKvBytes;           // 221184
+constexpr int kOffP = kOffKv + kStages * kStageBytes;  // 163840
 constexpr int kPBytes = H * N * 2;                     // 8192
-constexpr int kOffBar = kOffP + kPBytes;               // 229376
-// kv_full[2] kv_empty[2] s_full[2] p_full p_free o_done q_full
-constexpr int kNumBars = 2 + 2 + 2 + 1 + 1 + 1 + 1;
+constexpr int kOffX = kOffP + kPBytes;                 // 172032: the peer's S partials
+constexpr int kXBytes = H * N * 4;                     // 16384 per buffer, two buffers
+constexpr int kOffBar = kOffX + 2 * kXBytes;           // 204800
+// kv_full[kStages] kv_empty[kStages] s_full[2] x_full[2] sx_full[2] p_full p_free o_done q_full
+constexpr int kNumBars = 2 * kStages + 2 + 2 + 2 + 4;
 constexpr int kOffTmem = kOffBar + kNumBars * 8;
 constexpr int kSmem = 1024 + kOffTmem + 16;
-// warps 0-3 softmax (warp w reads TMEM lanes 32w..32w+31), warp 4 MMA issue,
-// warps 5.. loaders: kLoadWarps per KV stage
-constexpr int kMmaWarp = 4;
-constexpr int kLoadWarps = 4;
-constexpr int kThreads = (kMmaWarp + 1 + 2 * kLoadWarps) * 32;          // 416
-constexpr int kChunksPerRow = DK * 2 / 16;                              // 72 16-byte chunks
-constexpr int kChunksPerThread = N * kChunksPerRow / (kLoadWarps * 32);  // 18
+// warps 0-3 softmax and 4-7 S exchange (warp w reads TMEM lanes 32(w%4) .. +31),
+// warp 8 MMA issue, warps 9.. loaders: kLoadWarps per KV stage
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarps = 2;
+constexpr int kThreads = (kMmaWarp + 1 + kStages * kLoadWarps) * 32;    // 544
+constexpr int kChunksPerRow = kLocalPanels * 8;                         // 40 16-byte chunks
+constexpr int kChunksPerThread = N * kChunksPerRow / (kLoadWarps * 32);  // 20
 static_assert(N * kChunksPerRow % (kLoadWarps * 32) == 0, "chunks must split evenly");
+static_assert(kSmem <= 227 * 1024, "shared memory budget");
 constexpr uint32_t kIdescS = make_idesc(1 /*bf16*/, 128, N, false, false);
 constexpr uint32_t kIdescO = make_idesc(1 /*bf16*/, 128, DVH, false, true);
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 }  // namespace mla
 
-// Q of request b (128 heads x 576) as nine 128-row TMA boxes, one 128-byte-swizzled
-// K-major panel each.  One thread.
-__device__ __forceinline__ void issue_q_load(uint32_t q_smem, const CUtensorMap* q_map, uint64_t* bar, int b) {
+// This rank's Q panels of request b as 128-row TMA boxes (one 128-byte-swizzled K-major
+// panel each).  One thread.
+__device__ __forceinline__ void issue_q_load(uint32_t q_smem, const CUtensorMap* q_map, uint64_t* bar, int b,
+                                             int rank) {
   using namespace mla;
-  mbar_arrive_expect_tx(bar, kQBytes);
+  const int np = s_panels(rank), p0 = rank * s_panels(0);
+  mbar_arrive_expect_tx(bar, (uint32_t)np * H * 128);
 #pragma unroll 1
-  for (int pn = 0; pn < kPanels; ++pn) tma_load_2d(q_smem + pn * (H * 128), q_map, bar, pn * 64, b * H);
+  for (int i = 0; i < np; ++i) tma_load_2d(q_smem + i * (H * 128), q_map, bar, (p0 + i) * 64, b * H);
 }
 
-// One CTA = (request b, KV split, output half).  The CTA keeps Q (128 heads x 576) in
-// shared memory, streams its share of the selected rows through two KV stages, forms
-// S = Q K^T (128 x 32 per tile) in TMEM, runs the online softmax on CUDA cores (one
-// thread per head), writes P (bf16) to shared memory and accumulates O_half += P V_half
-// in TMEM (256 columns).  Q is loaded by TMA (nine 128-row boxes); each KV tile is
-// gathered with 16-byte cp.async copies by four warps per stage (a row gather would
-// need one TMA box per 128 bytes, and the TMA unit issues those too slowly).
+// One cluster of two CTAs = (request b, KV split); rank r of the pair produces output
+// dims [256r, 256r + 256).  Per 32-row tile, each CTA gathers its five 64-dim panels of
+// the selected rows (cp.async, four stages), forms its part of S = Q K^T over its latent
+// dims in TMEM, sends that 128 x 32 partial to the other CTA through distributed shared
+// memory and adds the one it receives, so both hold the same S (fp32 addition commutes,
+// so the two sums are bit-identical) and run the same online softmax (one thread per
+// head).  P goes to shared memory as bf16 and O_half += P V_half accumulates in TMEM
+// (256 columns).
 __global__ void __launch_bounds__(mla::kThreads, 1)
     attn_mla_tc(const AttnParams p, const __grid_constant__ CUtensorMap q_map) {
   using namespace mla;
@@ -178,18 +190,20 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   uint8_t* sm = (uint8_t*)(((uintptr_t)sm_raw_a + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = (uint64_t*)(sm + kOffBar);
   uint64_t* kv_full = bars;
-  uint64_t* kv_empty = bars + 2;
-  uint64_t* s_full = bars + 4;
-  uint64_t* p_full = bars + 6;
-  uint64_t* p_free = bars + 7;
-  uint64_t* o_done = bars + 8;
-  uint64_t* q_full = bars + 9;
+  uint64_t* kv_empty = bars + kStages;
+  uint64_t* s_full = bars + 2 * kStages;
+  uint64_t* x_full = s_full + 2;
+  uint64_t* sx_full = x_full + 2;
+  uint64_t* p_full = sx_full + 2;
+  uint64_t* p_free = p_full + 1;
+  uint64_t* o_done = p_full + 2;
+  uint64_t* q_full = p_full + 3;
   uint32_t* tmem_slot = (uint32_t*)(sm + kOffTmem);
   __shared__ int s_abort;
-  __shared__ uint32_t s_mask[2];        // valid rows of the tile in each stage
+  __shared__ uint32_t s_mask[kStages];  // valid rows of the tile in each stage
 
   const int b = blockIdx.y;
-  const int half = blockIdx.x & 1;
+  const int rank = (int)cluster_rank();  // == blockIdx.x & 1
   const int split = blockIdx.x >> 1;
   const int warp = warp_id(), lane = lane_id();
   const int T_all = (p.k + N - 1) / N;
@@ -199,23 +213,27 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   const uint32_t sbase = smem_u32(sm);
 
   if (threadIdx.x == 0) {
-    mbar_init(&kv_full[0], kLoadWarps);  // one arrival per loader warp, after its copies
-    mbar_init(&kv_full[1], kLoadWarps);
-    mbar_init(&kv_empty[0], 1);
-    mbar_init(&kv_empty[1], 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&kv_full[s], kLoadWarps);  // one arrival per loader warp, after its copies
+      mbar_init(&kv_empty[s], 1);
+    }
     mbar_init(&s_full[0], 1);
     mbar_init(&s_full[1], 1);
+    mbar_init(&x_full[0], 128);  // the other CTA's softmax threads, remotely
+    mbar_init(&x_full[1], 128);
+    mbar_init(&sx_full[0], 128);  // this CTA's exchange threads: full S is in TMEM
+    mbar_init(&sx_full[1], 128);
     mbar_init(p_full, 128);
     mbar_init(p_free, 1);
     mbar_init(o_done, 1);
     mbar_init(q_full, 1);
     s_abort = 0;
     fence_mbar_init();
-    if (p.early_q && my_tiles > 0) issue_q_load(sbase, &q_map, q_full, b);
+    if (p.early_q && my_tiles > 0) issue_q_load(sbase, &q_map, q_full, b, rank);
   }
   if (warp == kMmaWarp) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers exist before any remote arrival
   tc_fence_after();
   // under programmatic dependent launch everything above overlaps the kernel before;
   // the selection, the rows and the outputs are touched only after it has finished
@@ -226,39 +244,39 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   const uint32_t tm_s = tmem + 256;    // columns [256, 320): S double buffer
 
   if (warp > kMmaWarp) {
-    // ================= loaders: stage st holds tiles st, st+2, ... =================
-    // Every loader warp of a stage resolves the tile's 32 rows (lane r -> row r).  The
-    // tile's 32 x 72 16-byte chunks are dealt over the stage's 128 threads in row-major
-    // order (consecutive threads, consecutive chunks of a row: coalesced), each copied
-    // with cp.async to its 128-byte-swizzled place in its panel; chunks of padding rows
-    // are zeroed instead.  A thread waits for its own copies, makes them visible to the
-    // tensor core (proxy fence), and the warp arrives on the stage's barrier.
+    // ================= loaders: stage st holds tiles st, st + kStages, ... =================
+    // Both warps of a stage resolve the tile's 32 rows (lane r -> row r).  The tile's
+    // 32 x 40 16-byte chunks (this rank's five panels) are dealt over the stage's 64
+    // threads in row-major order (consecutive threads, consecutive chunks of a row), each
+    // copied with cp.async to its 128-byte-swizzled place; chunks of padding rows are
+    // zeroed instead.  A thread waits for its own copies and makes them visible to the
+    // tensor core (proxy fence); then its warp arrives on the stage's barrier.
     const int lw = warp - (kMmaWarp + 1);
     const int st = lw / kLoadWarps;
     const int t = (lw - st * kLoadWarps) * 32 + lane;  // thread within the stage
-    const uint32_t stage = sbase + kOffKv + st * kKvBytes;
-    const char* kv_base = (const char*)p.krows;
+    const uint32_t stage = sbase + kOffKv + st * kStageBytes;
+    const char* kv_base = (const char*)p.krows + rank * 4 * 128;  // first dim of panel 4r
     const long long row_bytes = p.row_stride * 2;
-    // row of tile i for this lane; resolved one tile ahead, so the two dependent loads
+    // row of tile i for this lane; resolved one round ahead, so the two dependent loads
     // (selection, page table) overlap the wait for the stage
     auto tile_row = [&](int i) -> long long {
       const int j = (t0 + i) * N + lane;
       return (i < my_tiles && j < p.k) ? attn_row(p, b, p.sel[(size_t)b * p.k + j]) : -1;
     };
     long long row_next = tile_row(st);
-    for (int i = st; i < my_tiles; i += 2) {
+    for (int i = st; i < my_tiles; i += kStages) {
       const long long row = row_next;
-      row_next = tile_row(i + 2);
+      row_next = tile_row(i + kStages);
       int go = 1;
       if (lane == 0) {  // one lane decides, so the warp stays converged
-        go = (i < 2) || mbar_wait(&kv_empty[st], ((i >> 1) - 1) & 1);
+        go = (i < kStages) || mbar_wait(&kv_empty[st], ((i / kStages) - 1) & 1);
         if (*(volatile int*)&s_abort) go = 0;
         if (!go) s_abort = 1;
       }
       go = __shfl_sync(0xffffffffu, go, 0);
       if (!go) break;
       const uint32_t vmask = __ballot_sync(0xffffffffu, row >= 0);
-#pragma unroll 6
+#pragma unroll 5
       for (int it = 0; it < kChunksPerThread; ++it) {
         const int e = t + kLoadWarps * 32 * it;
         const int r = e / kChunksPerRow, c = e - r * kChunksPerRow;
@@ -281,47 +299,48 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ================= MMA issuer: event driven =================
-    // PV(i) goes out as soon as P(i) is ready and S(i) as soon as tile i has landed
-    // (with S(i-2)'s buffer consumed), so neither waits behind the other's inputs.
+    // S(i) (this rank's panels) goes out whole once tile i has landed and S(i-2)'s
+    // buffer is consumed; PV(i) as soon as P(i) is ready.  Neither blocks the other.
     if (lane == 0 && my_tiles > 0) {
       const uint32_t q_addr = sbase;
       const uint32_t p_addr = sbase + kOffP;
-      if (!p.early_q) issue_q_load(sbase, &q_map, q_full, b);
+      const int nsp = s_panels(rank);
+      const int lp0 = rank;  // first local panel used by S: rank 1 skips panel 4 (V only)
+      if (!p.early_q) issue_q_load(sbase, &q_map, q_full, b, rank);
       bool ok = mbar_wait(q_full, 0);
-      // S(i) goes out whole once tile i has landed (and S(i-2)'s buffer is consumed),
-      // PV(i) as soon as P(i) is ready; each is checked without blocking on the other
       int ns = 0, npv = 0;
       uint64_t idle_since = 0;
       while (ok && npv < my_tiles) {
         bool progressed = false;
         if (npv < ns && mbar_test_wait(p_full, npv & 1)) {
           tc_fence_after();
-          const uint32_t v = sbase + kOffKv + (npv & 1) * kKvBytes + half * 4 * kKvPanel;
+          // this rank's V half is local panels 0-3 of the stage
+          const uint32_t v = sbase + kOffKv + (npv % kStages) * kStageBytes;
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk) {
             const uint64_t ad = make_sdesc(p_addr + kk * 2 * 2048, 2048, 128, kSwizzleNone);
             const uint64_t bd = make_sdesc(v + kk * 16 * 128, kKvPanel, 1024, kSwizzle128);
             mma_bf16(tm_o, ad, bd, kIdescO, (npv > 0 || kk > 0));
           }
-          tc_commit(&kv_empty[npv & 1]);
+          tc_commit(&kv_empty[npv % kStages]);
           tc_commit(p_free);
           ++npv;
           progressed = true;
         }
-        if (ns < my_tiles && ns < npv + 2 && mbar_test_wait(&kv_full[ns & 1], (ns >> 1) & 1)) {
+        if (ns < my_tiles && ns < npv + 2 && mbar_test_wait(&kv_full[ns % kStages], (ns / kStages) & 1)) {
           tc_fence_after();
-          const int st = ns & 1;
-          const uint32_t kv = sbase + kOffKv + st * kKvBytes;
+          const uint32_t kv = sbase + kOffKv + (ns % kStages) * kStageBytes + lp0 * kKvPanel;
+          const uint32_t sb = tm_s + (ns & 1) * N;
 #pragma unroll 1
-          for (int pn = 0; pn < kPanels; ++pn) {
+          for (int pn = 0; pn < nsp; ++pn) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t ad = make_sdesc(q_addr + pn * (H * 128) + kk * 32, 16, 1024, kSwizzle128);
               const uint64_t bd = make_sdesc(kv + pn * kKvPanel + kk * 32, 16, 1024, kSwizzle128);
-              mma_bf16(tm_s + st * N, ad, bd, kIdescS, (pn | kk) != 0);
+              mma_bf16(sb, ad, bd, kIdescS, (pn | kk) != 0);
             }
           }
-          tc_commit(&s_full[st]);
+          tc_commit(&s_full[ns & 1]);
           ++ns;
           progressed = true;
         }
@@ -340,6 +359,42 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
       if (!ok) s_abort = 1;
       tc_commit(o_done);
     }
+  } else if (warp >= 4) {
+    // ================= S exchange: warps 4..7, thread = head =================
+    // Per tile: this rank's partial S from TMEM goes to the other CTA, the other rank's
+    // partial is added, and the full S is written back over the partial in TMEM for the
+    // softmax warps.  Runs a tile ahead of the softmax.
+    const int q = warp & 3;
+    const int h = q * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    // partials are stored chunk-major (chunk c of head h at c * 2048 + h * 16), so a
+    // warp's 16-byte accesses are consecutive
+    const uint32_t x_peer = dsmem_map(sbase + kOffX, (uint32_t)(rank ^ 1));
+    const uint32_t xfull_peer = dsmem_map(smem_u32(x_full), (uint32_t)(rank ^ 1));
+    for (int i = 0; i < my_tiles; ++i) {
+      const int sb = i & 1;
+      if (!mbar_wait(&s_full[sb], (i >> 1) & 1)) break;
+      tc_fence_after();
+      float s[N];
+      tmem_ld32(tm_s + lane_off + sb * N, s);
+#pragma unroll
+      for (int c = 0; c < N / 4; ++c)
+        st_cluster_v4(x_peer + sb * kXBytes + c * 2048 + h * 16, s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]);
+      mbar_arrive_remote(xfull_peer + sb * 8);
+      if (!mbar_wait_cluster(&x_full[sb], (i >> 1) & 1)) break;
+#pragma unroll
+      for (int c = 0; c < N / 4; ++c) {
+        const float4 o = *(const float4*)(sm + kOffX + sb * kXBytes + c * 2048 + h * 16);
+        s[4 * c] += o.x;
+        s[4 * c + 1] += o.y;
+        s[4 * c + 2] += o.z;
+        s[4 * c + 3] += o.w;
+      }
+      tmem_st32(tm_s + lane_off + sb * N, s);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sx_full[sb]);
+    }
   } else {
     // ================= softmax: warps 0..3, thread = head =================
     const int h = warp * 32 + lane;
@@ -348,14 +403,15 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int i = 0; i < my_tiles; ++i) {
-      const int st = i & 1;
+      const int st = i % kStages, sb = i & 1;
       // the loaders published the tile's valid rows with their kv_full arrivals
-      if (!mbar_wait(&kv_full[st], (i >> 1) & 1)) { ok = false; break; }
+      if (!mbar_wait(&kv_full[st], (i / kStages) & 1)) { ok = false; break; }
       const uint32_t vmask = s_mask[st];
-      if (!mbar_wait(&s_full[st], (i >> 1) & 1)) { ok = false; break; }
+      // full S = both ranks' partials, summed by the exchange warps
+      if (!mbar_wait(&sx_full[sb], (i >> 1) & 1)) { ok = false; break; }
       tc_fence_after();
       float s[N];
-      tmem_ld32(tm_s + lane_off + st * N, s);
+      tmem_ld32(tm_s + lane_off + sb * N, s);
       float tmax = -INFINITY;
 #pragma unroll
       for (int r = 0; r < N; ++r)
@@ -419,7 +475,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
         float v[32];
         tmem_ld32(tm_o + lane_off + c0, v);
         if (single) {
-          __nv_bfloat16* o = (__nv_bfloat16*)p.o + ((size_t)b * H + h) * DV + half * DVH + c0;
+          __nv_bfloat16* o = (__nv_bfloat16*)p.o + ((size_t)b * H + h) * DV + rank * DVH + c0;
 #pragma unroll
           for (int c = 0; c < 32; c += 8) {
             uint32_t w[4];
@@ -431,15 +487,15 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
             *(uint4*)(o + c) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         } else {
-          // layout [b][split][head][dim]: each thread stores 128 contiguous bytes
-          float4* o = (float4*)(p.part_o + (((size_t)b * p.nsplit + split) * H + h) * DV + half * DVH + c0);
+          // layout [b][split][dim / 4][head][4]: a warp's store is 512 contiguous bytes
+          float4* o = (float4*)p.part_o + (((size_t)b * p.nsplit + split) * (DV / 4) + (rank * DVH + c0) / 4) * H + h;
           const bool any = l_run > 0.f;
 #pragma unroll
           for (int c = 0; c < 32; c += 4)
-            o[c / 4] = any ? make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+            o[(size_t)(c / 4) * H] = any ? make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
-      if (half == 0) {
+      if (rank == 0) {  // both ranks hold the same running max and sum
         if (single) {
           p.lse[(size_t)b * H + h] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
         } else {
@@ -449,20 +505,21 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
         }
       }
     } else if (my_tiles == 0 && p.nsplit > 1) {
-      float4* o = (float4*)(p.part_o + (((size_t)b * p.nsplit + split) * H + h) * DV + half * DVH);
-      for (int c = 0; c < DVH / 4; ++c) o[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (half == 0) {
+      float4* o = (float4*)p.part_o + (((size_t)b * p.nsplit + split) * (DV / 4) + rank * DVH / 4) * H + h;
+      for (int c = 0; c < DVH / 4; ++c) o[(size_t)c * H] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (rank == 0) {
         float* ml = p.part_ml + (((size_t)b * p.nsplit + split) * H + h) * 2;
         ml[0] = -INFINITY;
         ml[1] = 0.f;
       }
     }
   }
-  // every warp must reach the barrier converged (the MMA warp's lane 0 arrives last);
-  // only then may TMEM be released
+  // every warp must reach the barrier converged (the MMA warp's lane 0 arrives last).
+  // The cluster-wide barrier also keeps this CTA's shared memory alive until the other
+  // CTA has made its last remote write and arrival; only then may TMEM be released.
   __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -471,8 +528,8 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
 
 // Merge split-KV partials: o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
 // One thread per (request, head, 8 consecutive dims); grid (H * DV / 8 / 256, B), 256
-// threads.  A warp covers 256 contiguous dims of one head, so every partial read is a
-// coalesced 1 KB run and every output store a 512-byte run; the 2 x nsplit 16-byte loads
+// threads.  A warp covers 32 consecutive heads at the same dims, so each of its partial
+// reads is a 512-byte run of the [dim / 4][head][4] layout; the 2 x nsplit 16-byte loads
 // of a thread are independent of one another.
 constexpr int kCombineThreads = 256;
 __global__ void __launch_bounds__(kCombineThreads) attn_combine(const AttnParams p) {
@@ -480,7 +537,7 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine(const AttnParams
   griddep_wait();  // the partials come from the kernel before
   const int b = blockIdx.y;
   const int item = blockIdx.x * kCombineThreads + threadIdx.x;
-  const int h = item / (DV / 8), d0 = (item - h * (DV / 8)) * 8;
+  const int g = item / H, h = item - g * H, d0 = g * 8;
   const float* ml = p.part_ml + (size_t)b * p.nsplit * H * 2 + (size_t)h * 2;
   float M = -INFINITY;
   for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, ml[(size_t)s * H * 2]);
@@ -495,8 +552,8 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine(const AttnParams
       if (!(l > 0.f)) continue;
       const float wgt = exp2f(ml[(size_t)s * H * 2] - M);
       Lsum += wgt * l;
-      const float4* po = (const float4*)(p.part_o + (((size_t)b * p.nsplit + s) * H + h) * DV + d0);
-      const float4 x = po[0], y = po[1];
+      const float4* po = (const float4*)p.part_o + (((size_t)b * p.nsplit + s) * (DV / 4) + d0 / 4) * H + h;
+      const float4 x = po[0], y = po[H];
       acc[0] = fmaf(wgt, x.x, acc[0]); acc[1] = fmaf(wgt, x.y, acc[1]);
       acc[2] = fmaf(wgt, x.z, acc[2]); acc[3] = fmaf(wgt, x.w, acc[3]);
       acc[4] = fmaf(wgt, y.x, acc[4]); acc[5] = fmaf(wgt, y.y, acc[5]);
