@@ -120,15 +120,14 @@ ls_status make_tmap_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_
   return LS_OK;
 }
 
-// 2D bf16 rows [rows][inner] (row stride in bytes), boxes of 64 elements (128 bytes) x
-// `box_rows` rows, 128-byte swizzle: 128-row boxes load a whole K-major operand panel.
-ls_status make_tmap_bf16_rows(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t stride,
-                              uint32_t box_rows) {
+// 2D bf16 rows [rows][inner] (row stride in bytes), one-row boxes of 64 elements (128
+// bytes), 128-byte swizzle: row gathers (tile::gather4) into K-major operand panels.
+ls_status make_tmap_bf16_rows(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t stride) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {stride};
-  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t box[2] = {64, 1};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
@@ -333,6 +332,7 @@ ls_status validate_attn(const ls_sparse_attn_args* a, bool need_sel) {
     if (a->variant == 0) {
       LS_REQUIRE(a->k_rows == a->v_rows, "MLA attention reads V from the latent rows (v_rows == k_rows)");
       LS_REQUIRE(a->row_stride >= 576 && (a->row_stride % 8) == 0, "row_stride must be >= 576 and % 8 == 0");
+      LS_REQUIRE(a->num_rows < 0x7fffffffLL, "num_rows must be below 2^31 - 1");
       LS_REQUIRE(aligned16(a->k_rows) && aligned16(a->q), "k_rows and q must be 16-byte aligned");
     }
   } else if (a->dtype != LS_F32) {
@@ -386,9 +386,6 @@ ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressi
     }
     if (allow_smem(ls::attn_mla_tc, ls::mla::kSmem, g_smem_attn_tc) != cudaSuccess)
       return check_launch("attn_mla_tc attribute");
-    CUtensorMap q_map;
-    LS_TRY(make_tmap_bf16_rows(&q_map, a->q, ls::mla::DK, (uint64_t)a->batch * ls::mla::H, ls::mla::DK * 2,
-                               ls::mla::H));
     p.early_q = pdl ? 1 : 0;
     cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = pdl_config(dim3(2 * ns, a->batch), dim3(ls::mla::kThreads), ls::mla::kSmem, st, attr, pdl);
@@ -398,7 +395,9 @@ ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressi
     attr[cfg.numAttrs].val.clusterDim.y = 1;
     attr[cfg.numAttrs].val.clusterDim.z = 1;
     cfg.numAttrs += 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, ls::attn_mla_tc, p, q_map);
+    CUtensorMap kv_map;
+    LS_TRY(make_tmap_bf16_rows(&kv_map, p.krows, ls::mla::DK, (uint64_t)num_rows, (uint64_t)a->row_stride * 2));
+    cudaError_t e = cudaLaunchKernelEx(&cfg, ls::attn_mla_tc, p, kv_map);
     if (e != cudaSuccess) return fail(LS_ERR_CUDA, "attn_mla_tc: %s", cudaGetErrorString(e));
     LS_TRY(check_launch("attn_mla_tc"));
     if (ns > 1) {

@@ -40,8 +40,16 @@ struct AttnParams {
   int nsplit;
   float* part_o;     // [B,nsplit,dv/4,H,4] unnormalised partial outputs (4-dim granules, head next)
   float* part_ml;    // [B,nsplit,H,2] running max (log2 domain) and sum
-  int early_q;       // tensor-core kernel: load Q before waiting for the kernel before
+  int early_q;       // tensor-core kernel: read Q before waiting for the kernel before
 };
+
+// 2^x with the hardware approximation (relative error about 2^-22; results below the
+// smallest normal flush to zero, which the softmax weights tolerate).
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 // Row index of selection value sv of request b, or -1 (padding or out of range).
 __device__ __forceinline__ long long attn_row(const AttnParams& p, int b, int sv) {
@@ -135,28 +143,36 @@ constexpr int kPanels = DK / 64;                       // 9 panels of 64 bf16 (1
 // half of V: panels 0-3 or 4-7).
 constexpr int kLocalPanels = 5;
 __host__ __device__ constexpr int s_panels(int rank) { return rank == 0 ? 5 : 4; }  // S panels per rank
-constexpr int kQBytes = 5 * H * 128;                   // 81920 (rank 1 uses 65536)
 constexpr int kKvPanel = N * 128;                      // 4096
 constexpr int kStageBytes = kLocalPanels * kKvPanel;   // 20480
-constexpr int kStages = 4;
-constexpr int kOffKv = kQBytes;
+constexpr int kStages = 8;
+constexpr int kOffKv = 0;
 constexpr int kOffP = kOffKv + kStages * kStageBytes;  // 163840
 constexpr int kPBytes = H * N * 2;                     // 8192
 constexpr int kOffX = kOffP + kPBytes;                 // 172032: the peer's S partials
 constexpr int kXBytes = H * N * 4;                     // 16384 per buffer, two buffers
-constexpr int kOffBar = kOffX + 2 * kXBytes;           // 204800
-// kv_full[kStages] kv_empty[kStages] s_full[2] x_full[2] sx_full[2] p_full p_free o_done q_full
-constexpr int kNumBars = 2 * kStages + 2 + 2 + 2 + 4;
+constexpr int kMaxRows = 4096;                         // k <= 4096: a CTA's rows, resolved once
+constexpr int kOffRows = kOffX + 2 * kXBytes;
+constexpr int kOffBar = kOffRows + kMaxRows * 4;
+constexpr int kSBufs = 3;                              // S tiles in TMEM (32 columns each)
+// TMEM columns: O half [0, 256), S tiles [256, 352), this rank's Q [352, 512)
+constexpr int kTmemS = DVH, kTmemQ = DVH + kSBufs * N;
+static_assert(kTmemQ + 5 * 32 <= 512, "TMEM budget");
+// kv_full[kStages] kv_empty[kStages] s_full[kSBufs] s_read[kSBufs] x_full[2] x_free[2]
+// x_read[2] p_full p_free o_done q_full
+constexpr int kNumBars = 2 * kStages + 2 * kSBufs + 2 + 2 + 2 + 4;
 constexpr int kOffTmem = kOffBar + kNumBars * 8;
 constexpr int kSmem = 1024 + kOffTmem + 16;
-// warps 0-3 softmax and 4-7 S exchange (warp w reads TMEM lanes 32(w%4) .. +31),
-// warp 8 MMA issue, warps 9.. loaders: kLoadWarps per KV stage
+// warps 0-3 softmax and 4-7 S senders (warp w reads TMEM lanes 32(w%4) .. +31),
+// warp 8 MMA issue, warp 9 credit forwarding, warps 10-13 row gathers
 constexpr int kMmaWarp = 8;
-constexpr int kLoadWarps = 2;
-constexpr int kThreads = (kMmaWarp + 1 + kStages * kLoadWarps) * 32;    // 544
-constexpr int kChunksPerRow = kLocalPanels * 8;                         // 40 16-byte chunks
-constexpr int kChunksPerThread = N * kChunksPerRow / (kLoadWarps * 32);  // 20
-static_assert(N * kChunksPerRow % (kLoadWarps * 32) == 0, "chunks must split evenly");
+constexpr int kFwdWarp = 9;
+constexpr int kLoadWarp0 = 10;
+constexpr int kLoadWarps = 4;  // a warp issues its TMA ops one lane at a time: spread them
+constexpr int kThreads = (kLoadWarp0 + kLoadWarps) * 32;               // 448
+constexpr int kGathers = (N / 4) * kLocalPanels;                        // 40 gather4 per tile
+constexpr int kGathersPerWarp = kGathers / kLoadWarps;                  // 10
+static_assert(kGathers % kLoadWarps == 0 && kGathersPerWarp <= 32, "gathers per warp");
 static_assert(kSmem <= 227 * 1024, "shared memory budget");
 constexpr uint32_t kIdescS = make_idesc(1 /*bf16*/, 128, N, false, false);
 constexpr uint32_t kIdescO = make_idesc(1 /*bf16*/, 128, DVH, false, true);
@@ -164,37 +180,49 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 }  // namespace mla
 
-// This rank's Q panels of request b as 128-row TMA boxes (one 128-byte-swizzled K-major
-// panel each).  One thread.
-__device__ __forceinline__ void issue_q_load(uint32_t q_smem, const CUtensorMap* q_map, uint64_t* bar, int b,
-                                             int rank) {
+// This rank's Q panels (head h's row) into TMEM lane h as the MMA's A operand: 64 dims
+// = 32 columns per panel, two bf16 per column.  Every thread of warps 0-3, converged.
+__device__ __forceinline__ void load_q_tmem(const AttnParams& p, int b, int rank, int h, uint32_t t_row) {
   using namespace mla;
-  const int np = s_panels(rank), p0 = rank * s_panels(0);
-  mbar_arrive_expect_tx(bar, (uint32_t)np * H * 128);
+  const uint4* src = (const uint4*)((const char*)p.q + ((size_t)b * H + h) * DK * 2 + rank * s_panels(0) * 128);
 #pragma unroll 1
-  for (int i = 0; i < np; ++i) tma_load_2d(q_smem + i * (H * 128), q_map, bar, (p0 + i) * 64, b * H);
+  for (int c = 0; c < s_panels(rank); ++c) {
+    float f[32];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint4 v = src[c * 8 + j];
+      f[4 * j] = __uint_as_float(v.x);
+      f[4 * j + 1] = __uint_as_float(v.y);
+      f[4 * j + 2] = __uint_as_float(v.z);
+      f[4 * j + 3] = __uint_as_float(v.w);
+    }
+    tmem_st32(t_row + c * 32, f);
+  }
+  tmem_wait_st();
 }
 
 // One cluster of two CTAs = (request b, KV split); rank r of the pair produces output
 // dims [256r, 256r + 256).  Per 32-row tile, each CTA gathers its five 64-dim panels of
-// the selected rows (cp.async, four stages), forms its part of S = Q K^T over its latent
-// dims in TMEM, sends that 128 x 32 partial to the other CTA through distributed shared
+// the selected rows (TMA gather4, eight stages), forms its part of S = Q K^T over its latent
+// dims in TMEM (Q, the A operand, also lives in TMEM), sends that 128 x 32 partial to the other CTA through distributed shared
 // memory and adds the one it receives, so both hold the same S (fp32 addition commutes,
 // so the two sums are bit-identical) and run the same online softmax (one thread per
 // head).  P goes to shared memory as bf16 and O_half += P V_half accumulates in TMEM
 // (256 columns).
 __global__ void __launch_bounds__(mla::kThreads, 1)
-    attn_mla_tc(const AttnParams p, const __grid_constant__ CUtensorMap q_map) {
+    attn_mla_tc(const AttnParams p, const __grid_constant__ CUtensorMap kv_map) {
   using namespace mla;
   extern __shared__ uint8_t sm_raw_a[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)sm_raw_a + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = (uint64_t*)(sm + kOffBar);
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = bars + kStages;
-  uint64_t* s_full = bars + 2 * kStages;
-  uint64_t* x_full = s_full + 2;
-  uint64_t* sx_full = x_full + 2;
-  uint64_t* p_full = sx_full + 2;
+  uint64_t* s_full = bars + 2 * kStages;   // S partial of the tile in TMEM buffer i % kSBufs
+  uint64_t* s_read = s_full + kSBufs;      // ... and the sender warps have read it
+  uint64_t* x_full = s_read + kSBufs;      // the other rank's partial has arrived here
+  uint64_t* x_free = x_full + 2;           // the other rank has read our partial (credit)
+  uint64_t* x_read = x_free + 2;           // our softmax has read receive buffer b
+  uint64_t* p_full = x_read + 2;
   uint64_t* p_free = p_full + 1;
   uint64_t* o_done = p_full + 2;
   uint64_t* q_full = p_full + 3;
@@ -214,59 +242,67 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&kv_full[s], kLoadWarps);  // one arrival per loader warp, after its copies
+      mbar_init(&kv_full[s], kLoadWarps);  // each gather warp arrives with its bytes
       mbar_init(&kv_empty[s], 1);
     }
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(&x_full[0], 128);  // the other CTA's softmax threads, remotely
-    mbar_init(&x_full[1], 128);
-    mbar_init(&sx_full[0], 128);  // this CTA's exchange threads: full S is in TMEM
-    mbar_init(&sx_full[1], 128);
+    for (int s = 0; s < kSBufs; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_read[s], 128);  // this CTA's sender threads
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&x_full[s], 1);  // armed with the partial's bytes; the other CTA's stores land on it
+      mbar_init(&x_free[s], 1);    // the other CTA's forwarding thread, remotely
+      mbar_init(&x_read[s], 128);  // this CTA's softmax threads
+    }
     mbar_init(p_full, 128);
     mbar_init(p_free, 1);
     mbar_init(o_done, 1);
-    mbar_init(q_full, 1);
+    mbar_init(q_full, 128);  // the softmax threads, once Q is in TMEM
     s_abort = 0;
     fence_mbar_init();
-    if (p.early_q && my_tiles > 0) issue_q_load(sbase, &q_map, q_full, b, rank);
+    // arm the receive buffers for tiles 0 and 1 before the other CTA can send
+    for (int s = 0; s < 2 && s < my_tiles; ++s) mbar_arrive_expect_tx(&x_full[s], kXBytes);
   }
   if (warp == kMmaWarp) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
   cluster_sync_all();  // both CTAs' barriers exist before any remote arrival
   tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tm_o = tmem;          // columns [0, 256): O half
+  const uint32_t tm_s = tmem + kTmemS;  // kSBufs S tiles
+  const uint32_t tm_q = tmem + kTmemQ;  // this rank's Q panels
+  if (warp < 4 && p.early_q && my_tiles > 0) {  // Q is not written by the kernel before
+    load_q_tmem(p, b, rank, threadIdx.x, tm_q + ((uint32_t)(warp * 32) << 16));
+    tc_fence_before();
+    mbar_arrive(q_full);
+  }
   // under programmatic dependent launch everything above overlaps the kernel before;
   // the selection, the rows and the outputs are touched only after it has finished
   griddep_wait();
   griddep_launch_dependents();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t tm_o = tmem;          // columns [0, 256): O half
-  const uint32_t tm_s = tmem + 256;    // columns [256, 320): S double buffer
 
-  if (warp > kMmaWarp) {
-    // ================= loaders: stage st holds tiles st, st + kStages, ... =================
-    // Both warps of a stage resolve the tile's 32 rows (lane r -> row r).  The tile's
-    // 32 x 40 16-byte chunks (this rank's five panels) are dealt over the stage's 64
-    // threads in row-major order (consecutive threads, consecutive chunks of a row), each
-    // copied with cp.async to its 128-byte-swizzled place; chunks of padding rows are
-    // zeroed instead.  A thread waits for its own copies and makes them visible to the
-    // tensor core (proxy fence); then its warp arrives on the stage's barrier.
-    const int lw = warp - (kMmaWarp + 1);
-    const int st = lw / kLoadWarps;
-    const int t = (lw - st * kLoadWarps) * 32 + lane;  // thread within the stage
-    const uint32_t stage = sbase + kOffKv + st * kStageBytes;
-    const char* kv_base = (const char*)p.krows + rank * 4 * 128;  // first dim of panel 4r
-    const long long row_bytes = p.row_stride * 2;
-    // row of tile i for this lane; resolved one round ahead, so the two dependent loads
-    // (selection, page table) overlap the wait for the stage
-    auto tile_row = [&](int i) -> long long {
-      const int j = (t0 + i) * N + lane;
-      return (i < my_tiles && j < p.k) ? attn_row(p, b, p.sel[(size_t)b * p.k + j]) : -1;
-    };
-    long long row_next = tile_row(st);
-    for (int i = st; i < my_tiles; i += kStages) {
-      const long long row = row_next;
-      row_next = tile_row(i + kStages);
+  if (warp >= kLoadWarp0) {
+    // ================= row gathers: tile i goes to stage i % kStages =================
+    // The gather warps first resolve all of this CTA's rows (selection -> page table) into
+    // shared memory.  A tile's 8 groups of 4 rows x 5 panels are then 40 TMA gather4
+    // loads; gather e (group e % 8, panel e / 8) is
+    // issued by lane e % 10 of gather warp e / 10, each landing as four 128-byte-swizzled
+    // lines of its panel.  Padding rows point one past the pool, which the TMA unit fills
+    // with zeros; the softmax masks them.
+    const int lw = warp - kLoadWarp0;
+    const int e = lw * kGathersPerWarp + lane;  // this lane's gather (if lane < 10)
+    const int lx = e & 7, lp = e >> 3;
+    // resolve all of this CTA's rows once (out-of-range marker: one past the pool)
+    int* s_rows = (int*)(sm + kOffRows);
+    const int nrows = my_tiles * N;
+    for (int r = lw * 32 + lane; r < nrows; r += kLoadWarps * 32) {
+      const int j = t0 * N + r;
+      const long long row = j < p.k ? attn_row(p, b, p.sel[(size_t)b * p.k + j]) : -1;
+      s_rows[r] = row >= 0 ? (int)row : (int)p.num_rows;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kLoadWarps * 32) : "memory");  // the gather warps only
+    for (int i = 0; i < my_tiles; ++i) {
+      const int st = i % kStages;
       int go = 1;
       if (lane == 0) {  // one lane decides, so the warp stays converged
         go = (i < kStages) || mbar_wait(&kv_empty[st], ((i / kStages) - 1) & 1);
@@ -275,39 +311,46 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
       }
       go = __shfl_sync(0xffffffffu, go, 0);
       if (!go) break;
-      const uint32_t vmask = __ballot_sync(0xffffffffu, row >= 0);
-#pragma unroll 5
-      for (int it = 0; it < kChunksPerThread; ++it) {
-        const int e = t + kLoadWarps * 32 * it;
-        const int r = e / kChunksPerRow, c = e - r * kChunksPerRow;
-        const long long rr = __shfl_sync(0xffffffffu, row, r);
-        const uint32_t dst = stage + (c >> 3) * kKvPanel + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-        if (rr >= 0)
-          cp_async_16(dst, kv_base + rr * row_bytes + c * 16);
-        else
-          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0) : "memory");
-      }
-      cp_async_commit();
-      cp_async_wait<0>();
-      fence_proxy_async_smem();
-      __syncwarp();
+      const uint32_t vmask = __ballot_sync(0xffffffffu, s_rows[i * N + lane] < (int)p.num_rows);
       if (lane == 0) {
-        if (t == 0) s_mask[st] = vmask;
-        mbar_arrive(&kv_full[st]);
+        if (lw == 0) s_mask[st] = vmask;
+        mbar_arrive_expect_tx(&kv_full[st], kGathersPerWarp * 512);
+      }
+      __syncwarp();
+      if (lane < kGathersPerWarp) {
+        const int* rr = s_rows + i * N + 4 * lx;
+        tma_gather4(sbase + kOffKv + st * kStageBytes + lp * kKvPanel + lx * 512, &kv_map, &kv_full[st],
+                    (rank * 4 + lp) * 64, rr[0], rr[1], rr[2], rr[3]);
       }
     }
+    // never leave with copies in flight (the tiles of the last kStages loads)
+    if (lane == 0)
+      for (int i = max(0, my_tiles - kStages); i < my_tiles; ++i) mbar_wait(&kv_full[i % kStages], (i / kStages) & 1);
     __syncwarp();
+  } else if (warp == kFwdWarp) {
+    // ================= credit forwarding =================
+    // Once this CTA's softmax has read receive buffer b (tile j), re-arm its barrier for
+    // tile j + 2 and tell the other CTA's senders they may write it.  The remote arrival
+    // (a cluster-scope release) is slow, so it is kept off the softmax warps.
+    if (lane == 0) {
+      const uint32_t xfree_peer = dsmem_map(smem_u32(x_free), (uint32_t)(rank ^ 1));
+      for (int j = 0; j + 2 < my_tiles; ++j) {
+        const int xb = j & 1;
+        if (!mbar_wait(&x_read[xb], (j >> 1) & 1)) break;
+        mbar_arrive_expect_tx(&x_full[xb], kXBytes);
+        mbar_arrive_remote(xfree_peer + xb * 8);
+      }
+    }
   } else if (warp == kMmaWarp) {
     // ================= MMA issuer: event driven =================
-    // S(i) (this rank's panels) goes out whole once tile i has landed and S(i-2)'s
+    // S(i) (this rank's panels) goes out whole once tile i has landed and S(i-kSBufs)'s
     // buffer is consumed; PV(i) as soon as P(i) is ready.  Neither blocks the other.
     if (lane == 0 && my_tiles > 0) {
-      const uint32_t q_addr = sbase;
       const uint32_t p_addr = sbase + kOffP;
       const int nsp = s_panels(rank);
       const int lp0 = rank;  // first local panel used by S: rank 1 skips panel 4 (V only)
-      if (!p.early_q) issue_q_load(sbase, &q_map, q_full, b, rank);
       bool ok = mbar_wait(q_full, 0);
+      tc_fence_after();
       int ns = 0, npv = 0;
       uint64_t idle_since = 0;
       while (ok && npv < my_tiles) {
@@ -327,20 +370,22 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
           ++npv;
           progressed = true;
         }
-        if (ns < my_tiles && ns < npv + 2 && mbar_test_wait(&kv_full[ns % kStages], (ns / kStages) & 1)) {
+        // S(i): this rank's 20 (or 16) K steps into TMEM buffer i % kSBufs.  Each MMA
+        // waits on the previous one (same accumulator), so S costs about as many MMA
+        // latencies as it has K steps, whatever N is.
+        if (ns < my_tiles && ns < npv + kSBufs && mbar_test_wait(&kv_full[ns % kStages], (ns / kStages) & 1)) {
           tc_fence_after();
           const uint32_t kv = sbase + kOffKv + (ns % kStages) * kStageBytes + lp0 * kKvPanel;
-          const uint32_t sb = tm_s + (ns & 1) * N;
+          const uint32_t sb = tm_s + (ns % kSBufs) * N;
 #pragma unroll 1
           for (int pn = 0; pn < nsp; ++pn) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = make_sdesc(q_addr + pn * (H * 128) + kk * 32, 16, 1024, kSwizzle128);
               const uint64_t bd = make_sdesc(kv + pn * kKvPanel + kk * 32, 16, 1024, kSwizzle128);
-              mma_bf16(sb, ad, bd, kIdescS, (pn | kk) != 0);
+              mma_bf16_ta(sb, tm_q + pn * 32 + kk * 8, bd, kIdescS, (pn | kk) != 0);
             }
           }
-          tc_commit(&s_full[ns & 1]);
+          tc_commit(&s_full[ns % kSBufs]);
           ++ns;
           progressed = true;
         }
@@ -360,58 +405,66 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
       tc_commit(o_done);
     }
   } else if (warp >= 4) {
-    // ================= S exchange: warps 4..7, thread = head =================
-    // Per tile: this rank's partial S from TMEM goes to the other CTA, the other rank's
-    // partial is added, and the full S is written back over the partial in TMEM for the
-    // softmax warps.  Runs a tile ahead of the softmax.
+    // ================= S senders: warps 4..7, thread = head =================
+    // This rank's partial S of each tile goes from TMEM to the other CTA as asynchronous
+    // stores that count their bytes on the receiver's barrier (armed by the receiver for
+    // each tile).  Receive buffer i % 2 of the other CTA is written only after that CTA's
+    // softmax has read tile i-2 from it and its forwarding thread has re-armed the barrier
+    // (x_free credit), so the senders run ahead of both softmaxes by up to two tiles.
     const int q = warp & 3;
     const int h = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const uint32_t peer = (uint32_t)(rank ^ 1);
     // partials are stored chunk-major (chunk c of head h at c * 2048 + h * 16), so a
     // warp's 16-byte accesses are consecutive
-    const uint32_t x_peer = dsmem_map(sbase + kOffX, (uint32_t)(rank ^ 1));
-    const uint32_t xfull_peer = dsmem_map(smem_u32(x_full), (uint32_t)(rank ^ 1));
+    const uint32_t x_peer = dsmem_map(sbase + kOffX, peer);
+    const uint32_t xfull_peer = dsmem_map(smem_u32(x_full), peer);
     for (int i = 0; i < my_tiles; ++i) {
-      const int sb = i & 1;
-      if (!mbar_wait(&s_full[sb], (i >> 1) & 1)) break;
+      const int sb = i % kSBufs, xb = i & 1;
+      if (!mbar_wait(&s_full[sb], (i / kSBufs) & 1)) break;
       tc_fence_after();
-      float s[N];
-      tmem_ld32(tm_s + lane_off + sb * N, s);
+      float cur[N];
+      tmem_ld32(tm_s + lane_off + sb * N, cur);
+      tc_fence_before();
+      mbar_arrive(&s_read[sb]);
+      if (i >= 2 && !mbar_wait_cluster(&x_free[xb], ((i >> 1) - 1) & 1)) break;
 #pragma unroll
       for (int c = 0; c < N / 4; ++c)
-        st_cluster_v4(x_peer + sb * kXBytes + c * 2048 + h * 16, s[4 * c], s[4 * c + 1], s[4 * c + 2], s[4 * c + 3]);
-      mbar_arrive_remote(xfull_peer + sb * 8);
-      if (!mbar_wait_cluster(&x_full[sb], (i >> 1) & 1)) break;
-#pragma unroll
-      for (int c = 0; c < N / 4; ++c) {
-        const float4 o = *(const float4*)(sm + kOffX + sb * kXBytes + c * 2048 + h * 16);
-        s[4 * c] += o.x;
-        s[4 * c + 1] += o.y;
-        s[4 * c + 2] += o.z;
-        s[4 * c + 3] += o.w;
-      }
-      tmem_st32(tm_s + lane_off + sb * N, s);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&sx_full[sb]);
+        st_async_v4(x_peer + xb * kXBytes + c * 2048 + h * 16, cur[4 * c], cur[4 * c + 1], cur[4 * c + 2],
+                    cur[4 * c + 3], xfull_peer + xb * 8);
     }
   } else {
     // ================= softmax: warps 0..3, thread = head =================
     const int h = warp * 32 + lane;
     const float sl2 = p.scale * kLog2e;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    if (!p.early_q && my_tiles > 0) {
+      load_q_tmem(p, b, rank, h, tm_q + lane_off);
+      tc_fence_before();
+      mbar_arrive(q_full);
+    }
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int i = 0; i < my_tiles; ++i) {
-      const int st = i % kStages, sb = i & 1;
+      const int st = i % kStages, sb = i % kSBufs, xb = i & 1;
       // the loaders published the tile's valid rows with their kv_full arrivals
       if (!mbar_wait(&kv_full[st], (i / kStages) & 1)) { ok = false; break; }
       const uint32_t vmask = s_mask[st];
-      // full S = both ranks' partials, summed by the exchange warps
-      if (!mbar_wait(&sx_full[sb], (i >> 1) & 1)) { ok = false; break; }
+      // S = this rank's partial (TMEM) + the other rank's (receive buffer xb)
+      if (!mbar_wait(&s_full[sb], (i / kSBufs) & 1)) { ok = false; break; }
       tc_fence_after();
       float s[N];
       tmem_ld32(tm_s + lane_off + sb * N, s);
+      if (!mbar_wait_cluster(&x_full[xb], (i >> 1) & 1)) { ok = false; break; }
+#pragma unroll
+      for (int c = 0; c < N / 4; ++c) {
+        const float4 o = *(const float4*)(sm + kOffX + xb * kXBytes + c * 2048 + h * 16);
+        s[4 * c] += o.x;
+        s[4 * c + 1] += o.y;
+        s[4 * c + 2] += o.z;
+        s[4 * c + 3] += o.w;
+      }
+      mbar_arrive(&x_read[xb]);  // the forwarding thread re-arms buffer xb and passes the credit
       float tmax = -INFINITY;
 #pragma unroll
       for (int r = 0; r < N; ++r)
@@ -430,7 +483,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
       float psum = 0.f;
 #pragma unroll
       for (int r = 0; r < N; ++r) {
-        pr[r] = (vmask >> r & 1u) ? exp2f(fmaf(s[r], sl2, -m_run)) : 0.f;
+        pr[r] = (vmask >> r & 1u) ? ex2_ftz(fmaf(s[r], sl2, -m_run)) : 0.f;
         psum += pr[r];
       }
       if (i >= 1 && !mbar_wait(p_free, (i - 1) & 1)) { ok = false; break; }
@@ -449,6 +502,8 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
         tmem_wait_st();
       }
       l_run = l_run * factor + psum;
+      // PV(i) lets S(i + kSBufs) into this TMEM buffer: the senders must have read it
+      if (!mbar_wait(&s_read[sb], (i / kSBufs) & 1)) { ok = false; break; }
       uint8_t* pbuf = sm + kOffP;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {

@@ -84,9 +84,9 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete; gives up after kWaitLimitNs,
-// raising LS_DEV_TIMEOUT.  Returns false on timeout.
-__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait(bar, parity)) return true;
+// raising LS_DEV_TIMEOUT.  Returns false on timeout.  The polling loop is out of line;
+// a phase that has already completed costs one inline probe.
+__device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -95,6 +95,9 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  return mbar_try_wait(bar, parity) || mbar_wait_slow(bar, parity);
 }
 
 // ---------------------------------------------------------------------------------
@@ -118,6 +121,16 @@ __device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, f
                : "memory");
 }
 
+// Asynchronous 16-byte store into another CTA's shared memory; its bytes are counted
+// (complete_tx) on that CTA's mbarrier `cluster_bar` when they land.
+__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, float a, float b, float c, float d,
+                                            uint32_t cluster_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   cluster_addr),
+               "f"(a), "f"(b), "f"(c), "f"(d), "r"(cluster_bar)
+               : "memory");
+}
+
 // Arrive on an mbarrier of another CTA of the cluster; this thread's earlier writes
 // (remote ones included) are released to whoever waits on it with cluster scope.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
@@ -136,8 +149,7 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 }
 
 // As mbar_wait, with acquire at cluster scope (the arrivals come from another CTA).
-__device__ __noinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
-  if (mbar_try_wait_cluster(bar, parity)) return true;
+__device__ __noinline__ bool mbar_wait_cluster_slow(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
@@ -146,6 +158,9 @@ __device__ __noinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
+  return mbar_try_wait_cluster(bar, parity) || mbar_wait_cluster_slow(bar, parity);
 }
 
 // All threads of all CTAs of the cluster; every warp must arrive converged.
@@ -190,6 +205,18 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst_smem, const CUtensorMap
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
       "[%2];" ::"r"(dst_smem),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// TMA gather (tile::gather4, no multicast): columns [x, x + box width) of rows r0..r3 of
+// a 2D tensor whose box is one row high, landing as four consecutive box rows at
+// dst_smem; completes on `bar`.  Rows outside the tensor read as zeros.
+__device__ __forceinline__ void tma_gather4(uint32_t dst_smem, const CUtensorMap* map, uint64_t* bar, int x, int r0,
+                                            int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3, %4, %5, %6}], [%7];" ::"r"(dst_smem),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -247,6 +274,16 @@ __device__ __forceinline__ void mma_bf16(uint32_t d, uint64_t a, uint64_t b, uin
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}" ::"r"(d),
       "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0), "r"(0), "r"(0), "r"(0)
+      : "memory");
+}
+
+// As mma_bf16, with A read from tensor memory at `a_tmem` (M rows = lanes, the K
+// elements of a row packed two per 32-bit column); B from shared memory.
+__device__ __forceinline__ void mma_bf16_ta(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
 
