@@ -31,17 +31,18 @@ struct TopkParams {
 };
 
 constexpr int kTopkThreads = 512;
-constexpr int kTopkCacheKeys = 40960;  // at most 160 KB of cached keys per CTA
+constexpr int kTopkCacheKeys = 36864;  // at most 144 KB of cached keys per CTA
 
 __device__ __forceinline__ int topk_pos(const TopkParams& p, int b, int i) {
   if (!p.unit_list) return i;
   return p.unit_list[(size_t)b * p.list_stride + (i >> 6)] * 64 + (i & 63);
 }
 
-// Candidate buffers of the fast path (dynamic shared memory after the key cache).
-constexpr int kCandCap = 2048;    // per CTA: keys of the threshold bin and their slice index
-constexpr int kCandTotal = 6144;  // all candidates of a request, gathered by CTA 0
-constexpr int kTopkExtraBytes = kCandCap * 8 + kCandTotal * 4;
+// Buffers of the fast path (dynamic shared memory after the key cache).
+constexpr int kCandCap = 2048;    // per CTA: keys of the threshold bin
+constexpr int kCandTotal = 8192;  // all candidates of a request, gathered by CTA 0
+constexpr int kWarpList = 512;    // per warp: its keys at or above the threshold bin, in order
+constexpr int kTopkExtraBytes = kCandCap * 4 + kCandTotal * 4 + (kTopkThreads / 32) * kWarpList * 2;
 
 
 // Warp 0: lane c holds CTA c's count of keys above the threshold key (g) and equal to
@@ -105,8 +106,8 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
   const bool cached = Lc <= p.cache_keys;
   const float* row = p.scores + (size_t)b * p.stride;
   uint32_t* cand_key = sm_keys + p.cache_keys;
-  uint32_t* cand_idx = cand_key + kCandCap;
-  uint32_t* gbuf = cand_idx + kCandCap;
+  uint32_t* gbuf = cand_key + kCandCap;
+  uint16_t* wlists = (uint16_t*)(gbuf + kCandTotal);
 
   auto key_at = [&](int i) -> uint32_t {  // i relative to c0
     return cached ? sm_keys[i] : float_key(row[c0 + i]);
@@ -170,20 +171,24 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
     const int hi_shift = shift + width;
     for (int d = tid; d < 2048; d += kTopkThreads) hist[d] = 0;
     __syncthreads();
+    // scores crowd into few bins, so lanes of a warp that hit the same bin add once
+    auto count = [&](bool ok, uint32_t key) {
+      if (ok) atomicAdd(&hist[(key >> shift) & dmask], 1u);
+    };
     if (vals) {
-      for (int i = tid; i < nvals; i += kTopkThreads) {
-        const uint32_t key = vals[i];
-        if ((hi_shift >= 32) || ((key >> hi_shift) == prefix)) atomicAdd(&hist[(key >> shift) & dmask], 1u);
+      for (int i0 = 0; i0 < nvals; i0 += kTopkThreads) {  // whole warps step together
+        const int i = i0 + tid;
+        const uint32_t key = i < nvals ? vals[i] : 0u;
+        count(i < nvals && ((hi_shift >= 32) || ((key >> hi_shift) == prefix)), key);
       }
     } else {
-      for (int i = tid * 4; i < nvals; i += kTopkThreads * 4) {
+      for (int i0 = 0; i0 < nvals; i0 += kTopkThreads * 4) {
+        const int i = i0 + tid * 4;
         uint32_t kq[4];
         key4(i, nvals, kq);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if (i + e < nvals && ((hi_shift >= 32) || ((kq[e] >> hi_shift) == prefix)))
-            atomicAdd(&hist[(kq[e] >> shift) & dmask], 1u);
-        }
+        for (int e = 0; e < 4; ++e)
+          count(i + e < nvals && ((hi_shift >= 32) || ((kq[e] >> hi_shift) == prefix)), kq[e]);
       }
     }
     __syncthreads();
@@ -229,47 +234,64 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
   radix_pass(21, 11, false, nullptr, m);
   const uint32_t t0 = prefix;
 
-  // ---- fast path: collect the keys of bin t0 (the only undecided ones).  Each warp
-  // walks a contiguous segment (a multiple of 128 keys; the same one it emits later),
-  // four keys per thread per step, and counts the keys above bin t0.
+  // ---- collect.  Each warp walks a contiguous segment of the slice (the one it emits
+  // from) 32 keys at a time in position order and keeps, in order, the offsets of its
+  // keys at or above bin t0 -- every output comes from these lists.  The keys of bin t0
+  // (the only undecided ones) also go to the CTA's candidate buffer.
   const int seg = ((m + kWarps * 128 - 1) / (kWarps * 128)) * 128;
   const int i0 = min(m, warp * seg), i1 = min(m, i0 + seg);
   const uint32_t lt_mask = (1u << lane) - 1u;
+  uint16_t* wl = wlists + warp * kWarpList;
   if (tid == 0) {
     s_ncand = 0;
-    s_overflow = 0;
+    s_overflow = seg > 65535 ? 1u : 0u;  // offsets are 16-bit
   }
   __syncthreads();
+  uint32_t nl = 0;  // length of this warp's list
   {
-    uint32_t above = 0;
-    for (int base = i0; base < i1; base += 128) {
-      const int i = base + 4 * lane;
-      uint32_t kq[4];
-      key4(i, i1, kq);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        if (i + e >= i1) continue;
-        const uint32_t bin = kq[e] >> 21;
-        above += bin > t0;
-        if (bin == t0) {
-          const uint32_t o = atomicAdd(&s_ncand, 1u);
-          if (o < (uint32_t)kCandCap) {
-            cand_key[o] = kq[e];
-            cand_idx[o] = (uint32_t)(i + e);
-          } else {
-            s_overflow = 1;
-          }
+    uint32_t nc = 0;  // keys of bin t0 in this warp's segment
+    for (int base = i0; base < i1; base += 32) {
+      const int i = base + lane;
+      const bool in = i < i1;
+      const uint32_t key = in ? key_at(i) : 0u;
+      const uint32_t bin = key >> 21;
+      const bool sel = in && bin >= t0;
+      const uint32_t selm = __ballot_sync(0xffffffffu, sel);
+      if (sel) {
+        const uint32_t o = nl + __popc(selm & lt_mask);
+        if (o < (uint32_t)kWarpList) wl[o] = (uint16_t)(i - i0);
+      }
+      nl += __popc(selm);
+      nc += __popc(__ballot_sync(0xffffffffu, in && bin == t0));
+    }
+    // one reservation per warp, then the candidates straight from the (complete) list
+    uint32_t cb = 0;
+    if (lane == 0) {
+      s_warp_above[warp] = nl - nc;
+      if (nl > (uint32_t)kWarpList) s_overflow = 1;
+      cb = atomicAdd(&s_ncand, nc);
+    }
+    cb = __shfl_sync(0xffffffffu, cb, 0);
+    if (nl <= (uint32_t)kWarpList) {
+      for (uint32_t jb = 0; jb < nl; jb += 32) {
+        const uint32_t j = jb + lane;
+        const uint32_t key = j < nl ? key_at(i0 + wl[j]) : 0u;
+        const bool cand = j < nl && (key >> 21) == t0;
+        const uint32_t cm = __ballot_sync(0xffffffffu, cand);
+        if (cand) {
+          const uint32_t o = cb + __popc(cm & lt_mask);
+          if (o < (uint32_t)kCandCap) cand_key[o] = key;
         }
+        cb += __popc(cm);
       }
     }
-    above = __reduce_add_sync(0xffffffffu, above);
-    if (lane == 0) s_warp_above[warp] = above;
   }
   __syncthreads();
   if (tid == 0) {
     uint32_t a = 0;
     for (int w = 0; w < kWarps; ++w) a += s_warp_above[w];
     s_nabove = a;
+    if (s_ncand > (uint32_t)kCandCap) s_overflow = 1;
   }
   __syncthreads();
   cluster.sync();
@@ -304,26 +326,43 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
   unsigned long long pre;
   if (fast) {
     if (rank == 0) {
-      // gather every CTA's candidates (all loads independent) and finish the selection alone
-      for (uint32_t j = tid; j < total; j += kTopkThreads) {
-        int c = 0;
-        while (j >= s_off[c + 1]) ++c;
-        gbuf[j] = cluster.map_shared_rank(cand_key, c)[j - s_off[c]];
+      // warp c brings CTA c's candidates (one source per warp, loads independent), then
+      // this CTA finishes the selection alone
+      if (warp < CL) {
+        const uint32_t* src = cluster.map_shared_rank(cand_key, warp);
+        const uint32_t o = s_off[warp], cnt = s_off[warp + 1] - o;
+        for (uint32_t jb = 0; jb < cnt; jb += 8 * 32) {  // eight remote loads in flight per lane
+          uint32_t v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t j = jb + u * 32 + lane;
+            v[u] = j < cnt ? src[j] : 0u;
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint32_t j = jb + u * 32 + lane;
+            if (j < cnt) gbuf[o + j] = v[u];
+          }
+        }
       }
       __syncthreads();
       radix_pass(10, 11, true, gbuf, (int)total);
       radix_pass(0, 10, true, gbuf, (int)total);
-      if (tid < CL) {
-        s_cta_gt[tid] = *cluster.map_shared_rank(&s_nabove, tid);
-        s_cta_eq[tid] = 0;
-      }
-      __syncthreads();
-      for (uint32_t j = tid; j < total; j += kTopkThreads) {
-        int c = 0;
-        while (j >= s_off[c + 1]) ++c;
-        const uint32_t key = gbuf[j];
-        if (key > prefix) atomicAdd(&s_cta_gt[c], 1u);
-        else if (key == prefix) atomicAdd(&s_cta_eq[c], 1u);
+      // warp c counts CTA c's keys above the k-th key T (all keys above bin t0 are) and equal to it
+      if (warp < CL) {
+        const uint32_t o = s_off[warp], cnt = s_off[warp + 1] - o;
+        uint32_t g = 0, e = 0;
+        for (uint32_t j = lane; j < cnt; j += 32) {
+          const uint32_t key = gbuf[o + j];
+          g += key > prefix ? 1u : 0u;
+          e += key == prefix ? 1u : 0u;
+        }
+        g = __reduce_add_sync(0xffffffffu, g);
+        e = __reduce_add_sync(0xffffffffu, e);
+        if (lane == 0) {
+          s_cta_gt[warp] = g + *cluster.map_shared_rank(&s_nabove, warp);
+          s_cta_eq[warp] = e;
+        }
       }
       if (tid == 0) {
         s_T = prefix;
@@ -351,18 +390,20 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
     R = s_Rb;
     out_before = s_out_before;
     eq_before = s_eq_before;
-    // per-warp counts: the keys above bin t0 plus this CTA's candidates above / at T
-    if (tid < kWarps) {
-      s_warp_gt[tid] = s_warp_above[tid];
-      s_warp_eq[tid] = 0;
-    }
-    __syncthreads();
-    const uint32_t nmine = min(s_ncand, (uint32_t)kCandCap);
-    for (uint32_t j = tid; j < nmine; j += kTopkThreads) {
-      const uint32_t key = cand_key[j];
-      const int w = (int)(cand_idx[j] / (uint32_t)max(seg, 1));
-      if (key > T) atomicAdd(&s_warp_gt[w], 1u);
-      else if (key == T) atomicAdd(&s_warp_eq[w], 1u);
+    // per-warp counts over the warp's list, then their prefix over the CTA
+    {
+      uint32_t g = 0, e = 0;
+      for (uint32_t j = lane; j < nl; j += 32) {
+        const uint32_t key = key_at(i0 + wl[j]);
+        g += key > T ? 1u : 0u;
+        e += key == T ? 1u : 0u;
+      }
+      g = __reduce_add_sync(0xffffffffu, g);
+      e = __reduce_add_sync(0xffffffffu, e);
+      if (lane == 0) {
+        s_warp_gt[warp] = g;
+        s_warp_eq[warp] = e;
+      }
     }
     __syncthreads();
     const unsigned long long mine =
@@ -370,6 +411,31 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
     unsigned long long tot;
     const unsigned long long pre_t = block_excl_scan_u64(mine, scan_tmp, &tot);
     pre = __shfl_sync(0xffffffffu, pre_t, 0);
+    // ---- emit from the list: ballots give every taken key its output slot (ties: lower
+    // position first)
+    const uint32_t eq_left = R > eq_before ? R - eq_before : 0u;  // ties this CTA may still take
+    const uint32_t gt_pre = (uint32_t)(pre >> 32), eq_pre = (uint32_t)pre;
+    uint32_t eq_seen = eq_pre;  // keys == T before this lane's current key, CTA-wide
+    uint32_t out = out_before + gt_pre + min(eq_pre, eq_left);
+    for (uint32_t jb = 0; jb < nl; jb += 32) {
+      const uint32_t j = jb + lane;
+      const bool in = j < nl;
+      const int i = in ? i0 + wl[j] : 0;
+      const uint32_t key = in ? key_at(i) : 0u;
+      const uint32_t eq_mask = __ballot_sync(0xffffffffu, in && key == T);
+      const bool take = in && (key > T || (key == T && eq_seen + __popc(eq_mask & lt_mask) < eq_left));
+      const uint32_t take_mask = __ballot_sync(0xffffffffu, take);
+      if (take) {
+        const uint32_t o = out + __popc(take_mask & lt_mask);
+        if (o < (uint32_t)k) {
+          const int gi = c0 + i;
+          if (p.idx) p.idx[(size_t)b * k + o] = topk_pos(p, b, gi);
+          if (p.sel) p.sel[(size_t)b * k + o] = key_float(key);
+        }
+      }
+      out += __popc(take_mask);
+      eq_seen += __popc(eq_mask);
+    }
   } else {
     // ---- general path (too many keys share bin t0): two more cluster-wide passes
     radix_pass(10, 11, false, nullptr, m);
@@ -397,31 +463,29 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
     __syncthreads();
     out_before = s_out_before;
     eq_before = s_eq_before;
-  }
-
-  // ---- emit: each warp walks its segment 32 keys at a time in position order;
-  // ballots give every taken key its output slot (ties: lower position first)
-  const uint32_t eq_left = R > eq_before ? R - eq_before : 0u;  // ties this CTA may still take
-  const uint32_t gt_pre = (uint32_t)(pre >> 32), eq_pre = (uint32_t)pre;
-  uint32_t eq_seen = eq_pre;  // keys == T before this lane's current key, CTA-wide
-  uint32_t out = out_before + gt_pre + min(eq_pre, eq_left);
-  for (int base = i0; base < i1; base += 32) {
-    const int i = base + lane;
-    const bool in = i < i1;
-    const uint32_t key = in ? key_at(i) : 0u;
-    const uint32_t eq_mask = __ballot_sync(0xffffffffu, in && key == T);
-    const bool take = in && (key > T || (key == T && eq_seen + __popc(eq_mask & lt_mask) < eq_left));
-    const uint32_t take_mask = __ballot_sync(0xffffffffu, take);
-    if (take) {
-      const uint32_t o = out + __popc(take_mask & lt_mask);
-      if (o < (uint32_t)k) {
-        const int gi = c0 + i;
-        if (p.idx) p.idx[(size_t)b * k + o] = topk_pos(p, b, gi);
-        if (p.sel) p.sel[(size_t)b * k + o] = key_float(key);
+    // ---- emit: each warp walks its segment 32 keys at a time in position order
+    const uint32_t eq_left = R > eq_before ? R - eq_before : 0u;
+    const uint32_t gt_pre = (uint32_t)(pre >> 32), eq_pre = (uint32_t)pre;
+    uint32_t eq_seen = eq_pre;
+    uint32_t out = out_before + gt_pre + min(eq_pre, eq_left);
+    for (int base = i0; base < i1; base += 32) {
+      const int i = base + lane;
+      const bool in = i < i1;
+      const uint32_t key = in ? key_at(i) : 0u;
+      const uint32_t eq_mask = __ballot_sync(0xffffffffu, in && key == T);
+      const bool take = in && (key > T || (key == T && eq_seen + __popc(eq_mask & lt_mask) < eq_left));
+      const uint32_t take_mask = __ballot_sync(0xffffffffu, take);
+      if (take) {
+        const uint32_t o = out + __popc(take_mask & lt_mask);
+        if (o < (uint32_t)k) {
+          const int gi = c0 + i;
+          if (p.idx) p.idx[(size_t)b * k + o] = topk_pos(p, b, gi);
+          if (p.sel) p.sel[(size_t)b * k + o] = key_float(key);
+        }
       }
+      out += __popc(take_mask);
+      eq_seen += __popc(eq_mask);
     }
-    out += __popc(take_mask);
-    eq_seen += __popc(eq_mask);
   }
   if (p.thr && rank == 0 && tid == 0) p.thr[b] = key_float(T);
   cluster.sync();  // keep this CTA's shared memory alive until the cluster is done with it
