@@ -136,27 +136,27 @@ __global__ void __launch_bounds__(256) attn_simt(const AttnParams p) {
 // tcgen05 MLA kernel
 // =====================================================================================
 namespace mla {
-constexpr int H = 128, DK = 576, DV = 512, DVH = 256, N = 32;
+constexpr int H = 128, DK = 576, DV = 512, DVH = 256, N = 64;  // N: selected rows per tile
 constexpr int kPanels = DK / 64;                       // 9 panels of 64 bf16 (128 bytes)
 // The two CTAs of a pair split the latent dims of S = Q K^T: rank 0 takes panels 0-4,
 // rank 1 panels 5-8.  Each loads panels 4r .. 4r+4 of every row (its S panels plus its
 // half of V: panels 0-3 or 4-7).
 constexpr int kLocalPanels = 5;
 __host__ __device__ constexpr int s_panels(int rank) { return rank == 0 ? 5 : 4; }  // S panels per rank
-constexpr int kKvPanel = N * 128;                      // 4096
-constexpr int kStageBytes = kLocalPanels * kKvPanel;   // 20480
-constexpr int kStages = 8;
+constexpr int kKvPanel = N * 128;                      // 8192
+constexpr int kStageBytes = kLocalPanels * kKvPanel;   // 40960
+constexpr int kStages = 3;
 constexpr int kOffKv = 0;
-constexpr int kOffP = kOffKv + kStages * kStageBytes;  // 163840
-constexpr int kPBytes = H * N * 2;                     // 8192
-constexpr int kOffX = kOffP + kPBytes;                 // 172032: the peer's S partials
-constexpr int kXBytes = H * N * 4;                     // 16384 per buffer, two buffers
+constexpr int kOffX = kOffKv + kStages * kStageBytes;  // the peer's S partials
+constexpr int kXBytes = H * N * 4;                     // 32768 per buffer, two buffers
 constexpr int kMaxRows = 4096;                         // k <= 4096: a CTA's rows, resolved once
 constexpr int kOffRows = kOffX + 2 * kXBytes;
 constexpr int kOffBar = kOffRows + kMaxRows * 4;
-constexpr int kSBufs = 3;                              // S tiles in TMEM (32 columns each)
-// TMEM columns: O half [0, 256), S tiles [256, 352), this rank's Q [352, 512)
-constexpr int kTmemS = DVH, kTmemQ = DVH + kSBufs * N;
+// One S tile in TMEM: every MMA instruction costs about the same whatever its N, so the
+// tile is as wide as the TMEM budget allows.  TMEM columns: O half [0, 256), S [256, 320),
+// P as bf16 pairs [320, 352), this rank's Q [352, 512).
+constexpr int kSBufs = 1;
+constexpr int kTmemS = DVH, kTmemP = kTmemS + kSBufs * N, kTmemQ = kTmemP + N / 2;
 static_assert(kTmemQ + 5 * 32 <= 512, "TMEM budget");
 // kv_full[kStages] kv_empty[kStages] s_full[kSBufs] s_read[kSBufs] x_full[2] x_free[2]
 // x_read[2] p_full p_free o_done q_full
@@ -170,8 +170,8 @@ constexpr int kFwdWarp = 9;
 constexpr int kLoadWarp0 = 10;
 constexpr int kLoadWarps = 4;  // a warp issues its TMA ops one lane at a time: spread them
 constexpr int kThreads = (kLoadWarp0 + kLoadWarps) * 32;               // 448
-constexpr int kGathers = (N / 4) * kLocalPanels;                        // 40 gather4 per tile
-constexpr int kGathersPerWarp = kGathers / kLoadWarps;                  // 10
+constexpr int kGathers = (N / 4) * kLocalPanels;                        // 80 gather4 per tile
+constexpr int kGathersPerWarp = kGathers / kLoadWarps;                  // 20
 static_assert(kGathers % kLoadWarps == 0 && kGathersPerWarp <= 32, "gathers per warp");
 static_assert(kSmem <= 227 * 1024, "shared memory budget");
 constexpr uint32_t kIdescS = make_idesc(1 /*bf16*/, 128, N, false, false);
@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = bars + kStages;
   uint64_t* s_full = bars + 2 * kStages;   // S partial of the tile in TMEM buffer i % kSBufs
-  uint64_t* s_read = s_full + kSBufs;      // ... and the sender warps have read it
+  uint64_t* s_read = s_full + kSBufs;      // ... and the senders and the softmax have read it
   uint64_t* x_full = s_read + kSBufs;      // the other rank's partial has arrived here
   uint64_t* x_free = x_full + 2;           // the other rank has read our partial (credit)
   uint64_t* x_read = x_free + 2;           // our softmax has read receive buffer b
@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   uint64_t* q_full = p_full + 3;
   uint32_t* tmem_slot = (uint32_t*)(sm + kOffTmem);
   __shared__ int s_abort;
-  __shared__ uint32_t s_mask[kStages];  // valid rows of the tile in each stage
+  __shared__ uint64_t s_mask[kStages];  // valid rows of the tile in each stage
 
   const int b = blockIdx.y;
   const int rank = (int)cluster_rank();  // == blockIdx.x & 1
@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     }
     for (int s = 0; s < kSBufs; ++s) {
       mbar_init(&s_full[s], 1);
-      mbar_init(&s_read[s], 128);  // this CTA's sender threads
+      mbar_init(&s_read[s], 256);  // this CTA's sender and softmax threads
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&x_full[s], 1);  // armed with the partial's bytes; the other CTA's stores land on it
@@ -270,6 +270,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tm_o = tmem;          // columns [0, 256): O half
   const uint32_t tm_s = tmem + kTmemS;  // kSBufs S tiles
+  const uint32_t tm_p = tmem + kTmemP;  // P of the current tile, bf16 pairs (PV's A operand)
   const uint32_t tm_q = tmem + kTmemQ;  // this rank's Q panels
   if (warp < 4 && p.early_q && my_tiles > 0) {  // Q is not written by the kernel before
     load_q_tmem(p, b, rank, threadIdx.x, tm_q + ((uint32_t)(warp * 32) << 16));
@@ -284,14 +285,13 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   if (warp >= kLoadWarp0) {
     // ================= row gathers: tile i goes to stage i % kStages =================
     // The gather warps first resolve all of this CTA's rows (selection -> page table) into
-    // shared memory.  A tile's 8 groups of 4 rows x 5 panels are then 40 TMA gather4
-    // loads; gather e (group e % 8, panel e / 8) is
-    // issued by lane e % 10 of gather warp e / 10, each landing as four 128-byte-swizzled
-    // lines of its panel.  Padding rows point one past the pool, which the TMA unit fills
+    // shared memory.  A tile's 16 groups of 4 rows x 5 panels are then 80 TMA gather4
+    // loads; gather e (group e % 16, panel e / 16) is issued by lane e % 20 of gather warp
+    // e / 20, each landing as four 128-byte-swizzled lines of its panel.  Padding rows point one past the pool, which the TMA unit fills
     // with zeros; the softmax masks them.
     const int lw = warp - kLoadWarp0;
     const int e = lw * kGathersPerWarp + lane;  // this lane's gather (if lane < 10)
-    const int lx = e & 7, lp = e >> 3;
+    const int lx = e % (N / 4), lp = e / (N / 4);
     // resolve all of this CTA's rows once (out-of-range marker: one past the pool)
     int* s_rows = (int*)(sm + kOffRows);
     const int nrows = my_tiles * N;
@@ -311,7 +311,10 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
       }
       go = __shfl_sync(0xffffffffu, go, 0);
       if (!go) break;
-      const uint32_t vmask = __ballot_sync(0xffffffffu, s_rows[i * N + lane] < (int)p.num_rows);
+      uint64_t vmask = 0;
+#pragma unroll
+      for (int h32 = 0; h32 < N / 32; ++h32)
+        vmask |= (uint64_t)__ballot_sync(0xffffffffu, s_rows[i * N + h32 * 32 + lane] < (int)p.num_rows) << (32 * h32);
       if (lane == 0) {
         if (lw == 0) s_mask[st] = vmask;
         mbar_arrive_expect_tx(&kv_full[st], kGathersPerWarp * 512);
@@ -343,10 +346,10 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ================= MMA issuer: event driven =================
-    // S(i) (this rank's panels) goes out whole once tile i has landed and S(i-kSBufs)'s
-    // buffer is consumed; PV(i) as soon as P(i) is ready.  Neither blocks the other.
+    // S(i) (this rank's panels) goes out whole once tile i has landed and S(i-kSBufs) has
+    // been read out of its TMEM buffer; PV(i) as soon as P(i) is ready.  Neither blocks
+    // the other.
     if (lane == 0 && my_tiles > 0) {
-      const uint32_t p_addr = sbase + kOffP;
       const int nsp = s_panels(rank);
       const int lp0 = rank;  // first local panel used by S: rank 1 skips panel 4 (V only)
       bool ok = mbar_wait(q_full, 0);
@@ -360,10 +363,9 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
           // this rank's V half is local panels 0-3 of the stage
           const uint32_t v = sbase + kOffKv + (npv % kStages) * kStageBytes;
 #pragma unroll
-          for (int kk = 0; kk < 2; ++kk) {
-            const uint64_t ad = make_sdesc(p_addr + kk * 2 * 2048, 2048, 128, kSwizzleNone);
+          for (int kk = 0; kk < N / 16; ++kk) {
             const uint64_t bd = make_sdesc(v + kk * 16 * 128, kKvPanel, 1024, kSwizzle128);
-            mma_bf16(tm_o, ad, bd, kIdescO, (npv > 0 || kk > 0));
+            mma_bf16_ta(tm_o, tm_p + kk * 8, bd, kIdescO, (npv > 0 || kk > 0));
           }
           tc_commit(&kv_empty[npv % kStages]);
           tc_commit(p_free);
@@ -373,7 +375,8 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
         // S(i): this rank's 20 (or 16) K steps into TMEM buffer i % kSBufs.  Each MMA
         // waits on the previous one (same accumulator), so S costs about as many MMA
         // latencies as it has K steps, whatever N is.
-        if (ns < my_tiles && ns < npv + kSBufs && mbar_test_wait(&kv_full[ns % kStages], (ns / kStages) & 1)) {
+        if (ns < my_tiles && (ns < kSBufs || mbar_test_wait(&s_read[ns % kSBufs], ((ns / kSBufs) - 1) & 1)) &&
+            mbar_test_wait(&kv_full[ns % kStages], (ns / kStages) & 1)) {
           tc_fence_after();
           const uint32_t kv = sbase + kOffKv + (ns % kStages) * kStageBytes + lp0 * kKvPanel;
           const uint32_t sb = tm_s + (ns % kSBufs) * N;
@@ -424,7 +427,8 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
       if (!mbar_wait(&s_full[sb], (i / kSBufs) & 1)) break;
       tc_fence_after();
       float cur[N];
-      tmem_ld32(tm_s + lane_off + sb * N, cur);
+#pragma unroll
+      for (int c = 0; c < N; c += 32) tmem_ld32(tm_s + lane_off + sb * N + c, cur + c);
       tc_fence_before();
       mbar_arrive(&s_read[sb]);
       if (i >= 2 && !mbar_wait_cluster(&x_free[xb], ((i >> 1) - 1) & 1)) break;
@@ -449,12 +453,15 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
       const int st = i % kStages, sb = i % kSBufs, xb = i & 1;
       // the loaders published the tile's valid rows with their kv_full arrivals
       if (!mbar_wait(&kv_full[st], (i / kStages) & 1)) { ok = false; break; }
-      const uint32_t vmask = s_mask[st];
+      const uint64_t vmask = s_mask[st];
       // S = this rank's partial (TMEM) + the other rank's (receive buffer xb)
       if (!mbar_wait(&s_full[sb], (i / kSBufs) & 1)) { ok = false; break; }
       tc_fence_after();
       float s[N];
-      tmem_ld32(tm_s + lane_off + sb * N, s);
+#pragma unroll
+      for (int c = 0; c < N; c += 32) tmem_ld32(tm_s + lane_off + sb * N + c, s + c);
+      tc_fence_before();
+      mbar_arrive(&s_read[sb]);  // with the senders' reads, this frees the S buffer
       if (!mbar_wait_cluster(&x_full[xb], (i >> 1) & 1)) { ok = false; break; }
 #pragma unroll
       for (int c = 0; c < N / 4; ++c) {
@@ -468,7 +475,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
       float tmax = -INFINITY;
 #pragma unroll
       for (int r = 0; r < N; ++r)
-        if (vmask >> r & 1u) tmax = fmaxf(tmax, s[r]);
+        if ((vmask >> r) & 1u) tmax = fmaxf(tmax, s[r]);
       const float mt = tmax * sl2;
       float factor = 1.f;
       bool rescale = false;
@@ -479,12 +486,11 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
         }
         m_run = mt;
       }
-      float pr[N];
-      float psum = 0.f;
+      float psum = 0.f;  // s becomes P in place
 #pragma unroll
       for (int r = 0; r < N; ++r) {
-        pr[r] = (vmask >> r & 1u) ? ex2_ftz(fmaf(s[r], sl2, -m_run)) : 0.f;
-        psum += pr[r];
+        s[r] = ((vmask >> r) & 1u) ? ex2_ftz(fmaf(s[r], sl2, -m_run)) : 0.f;
+        psum += s[r];
       }
       if (i >= 1 && !mbar_wait(p_free, (i - 1) & 1)) { ok = false; break; }
       // tcgen05.ld/st are warp-collective: the whole warp rescales when any lane must
@@ -502,20 +508,15 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
         tmem_wait_st();
       }
       l_run = l_run * factor + psum;
-      // PV(i) lets S(i + kSBufs) into this TMEM buffer: the senders must have read it
-      if (!mbar_wait(&s_read[sb], (i / kSBufs) & 1)) { ok = false; break; }
-      uint8_t* pbuf = sm + kOffP;
+      // P(i) into TMEM lane h: column c holds rows 2c, 2c+1 as bf16 (PV(i-1) has read P(i-1))
+      float pw[N / 2];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          __nv_bfloat162 two = __floats2bfloat162_rn(pr[c * 8 + 2 * e], pr[c * 8 + 2 * e + 1]);
-          w[e] = *(uint32_t*)&two;
-        }
-        *(uint4*)(pbuf + h * 16 + c * 2048) = make_uint4(w[0], w[1], w[2], w[3]);
+      for (int c = 0; c < N / 2; ++c) {
+        __nv_bfloat162 two = __floats2bfloat162_rn(s[2 * c], s[2 * c + 1]);
+        pw[c] = __uint_as_float(*(uint32_t*)&two);
       }
-      fence_proxy_async_smem();
+      tmem_st32(tm_p + lane_off, pw);
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(p_full);
     }
