@@ -82,8 +82,7 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
   // fast path
   __shared__ uint32_t s_ncand, s_nabove, s_overflow;
   __shared__ uint32_t s_warp_above[kTopkThreads / 32], s_warp_gt[kTopkThreads / 32], s_warp_eq[kTopkThreads / 32];
-  __shared__ uint32_t s_T, s_R;                      // CTA 0 publishes
-  __shared__ uint32_t s_cta_gt[CL], s_cta_eq[CL];    // CTA 0 publishes
+  __shared__ uint32_t s_cta_gt[CL], s_cta_eq[CL];    // per CTA of the cluster: keys above / at T
   __shared__ uint32_t s_off[CL + 1];
   __shared__ uint32_t s_total, s_fast, s_Tb, s_Rb, s_out_before, s_eq_before;
 
@@ -298,10 +297,12 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
   // lane c of warp 0 reads CTA c's counts: one distributed-shared-memory round trip;
   // every CTA reads the same values, so the choice of path is uniform over the cluster
   if (warp == 0) {
-    uint32_t nc = 0, ov = 0;
+    uint32_t nc = 0, ov = 0, na = 0;
     if (lane < CL) {
       nc = *cluster.map_shared_rank(&s_ncand, lane);
       ov = *cluster.map_shared_rank(&s_overflow, lane);
+      na = *cluster.map_shared_rank(&s_nabove, lane);
+      s_cta_gt[lane] = na;  // keys above bin t0 (all above T), completed below
     }
     const uint32_t tot = __reduce_add_sync(0xffffffffu, nc);
     const bool anyov = __any_sync(0xffffffffu, ov != 0);
@@ -325,64 +326,52 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
   uint32_t T, R, out_before, eq_before;
   unsigned long long pre;
   if (fast) {
-    if (rank == 0) {
-      // warp c brings CTA c's candidates (one source per warp, loads independent), then
-      // this CTA finishes the selection alone
-      if (warp < CL) {
-        const uint32_t* src = cluster.map_shared_rank(cand_key, warp);
-        const uint32_t o = s_off[warp], cnt = s_off[warp + 1] - o;
-        for (uint32_t jb = 0; jb < cnt; jb += 8 * 32) {  // eight remote loads in flight per lane
-          uint32_t v[8];
+    // every CTA brings all candidates (warp c from CTA c, eight loads in flight per lane)
+    // and finishes the selection itself: the same T and counts everywhere, and no second
+    // round of publishing and reading
+    if (warp < CL) {
+      const uint32_t* src = cluster.map_shared_rank(cand_key, warp);
+      const uint32_t o = s_off[warp], cnt = s_off[warp + 1] - o;
+      for (uint32_t jb = 0; jb < cnt; jb += 8 * 32) {
+        uint32_t v[8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const uint32_t j = jb + u * 32 + lane;
-            v[u] = j < cnt ? src[j] : 0u;
-          }
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t j = jb + u * 32 + lane;
+          v[u] = j < cnt ? src[j] : 0u;
+        }
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const uint32_t j = jb + u * 32 + lane;
-            if (j < cnt) gbuf[o + j] = v[u];
-          }
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t j = jb + u * 32 + lane;
+          if (j < cnt) gbuf[o + j] = v[u];
         }
       }
-      __syncthreads();
-      radix_pass(10, 11, true, gbuf, (int)total);
-      radix_pass(0, 10, true, gbuf, (int)total);
-      // warp c counts CTA c's keys above the k-th key T (all keys above bin t0 are) and equal to it
-      if (warp < CL) {
-        const uint32_t o = s_off[warp], cnt = s_off[warp + 1] - o;
-        uint32_t g = 0, e = 0;
-        for (uint32_t j = lane; j < cnt; j += 32) {
-          const uint32_t key = gbuf[o + j];
-          g += key > prefix ? 1u : 0u;
-          e += key == prefix ? 1u : 0u;
-        }
-        g = __reduce_add_sync(0xffffffffu, g);
-        e = __reduce_add_sync(0xffffffffu, e);
-        if (lane == 0) {
-          s_cta_gt[warp] = g + *cluster.map_shared_rank(&s_nabove, warp);
-          s_cta_eq[warp] = e;
-        }
-      }
-      if (tid == 0) {
-        s_T = prefix;
-        s_R = k_rem;
-      }
-      __syncthreads();
     }
-    cluster.sync();
-    if (warp == 0) {
+    __syncthreads();
+    radix_pass(10, 11, true, gbuf, (int)total);
+    radix_pass(0, 10, true, gbuf, (int)total);
+    // warp c counts CTA c's candidates above the k-th key T and equal to it
+    if (warp < CL) {
+      const uint32_t o = s_off[warp], cnt = s_off[warp + 1] - o;
       uint32_t g = 0, e = 0;
-      if (lane < CL) {
-        g = *cluster.map_shared_rank(&s_cta_gt[lane], 0);
-        e = *cluster.map_shared_rank(&s_cta_eq[lane], 0);
+      for (uint32_t j = lane; j < cnt; j += 32) {
+        const uint32_t key = gbuf[o + j];
+        g += key > prefix ? 1u : 0u;
+        e += key == prefix ? 1u : 0u;
       }
-      const uint32_t Tv = *cluster.map_shared_rank(&s_T, 0);
-      const uint32_t Rv = *cluster.map_shared_rank(&s_R, 0);
-      cluster_prefix(g, e, Rv, rank, lane);
+      g = __reduce_add_sync(0xffffffffu, g);
+      e = __reduce_add_sync(0xffffffffu, e);
       if (lane == 0) {
-        s_Tb = Tv;
-        s_Rb = Rv;
+        s_cta_gt[warp] += g;
+        s_cta_eq[warp] = e;
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      const uint32_t g = lane < CL ? s_cta_gt[lane] : 0u, e = lane < CL ? s_cta_eq[lane] : 0u;
+      cluster_prefix(g, e, k_rem, rank, lane);
+      if (lane == 0) {
+        s_Tb = prefix;
+        s_Rb = k_rem;
       }
     }
     __syncthreads();
