@@ -271,6 +271,24 @@ def run_ours(args):
     torch.cuda.synchronize()
     topk_ms = [s[1].elapsed_time(s[4]) for s in stage_ev]
     attn_ms = [s[4].elapsed_time(s[5]) for s in stage_ev]
+    # the indexer kernel's own duration: launch after launch through ls_index_score (its
+    # 143 MB of keys and scales exceed the 126 MB L2, so nothing is reused between launches;
+    # inside a flushed step the events also enclose the launch gap after the flush)
+    t = wl.tensors
+    scores = torch.empty((BATCH, wl.args.index.max_len), dtype=torch.float32, device="cuda")
+    def run_indexer():
+        B.ls_index_score(q=t["i_q"], w=t["i_w"], key_pool=t["i_key_pool"], page_table=t["i_page_table"],
+                         lens=t["i_lens"], scores=scores, q_scale=t["i_q_scale"], key_scale=t["i_key_scale"])
+    for _ in range(Wm):
+        run_indexer()
+    kb = new_events(2)
+    torch.cuda.synchronize()
+    kb[0].record(stream)
+    for _ in range(K):
+        run_indexer()
+    kb[1].record(stream)
+    torch.cuda.synchronize()
+    idx_kernel_ms = kb[0].elapsed_time(kb[1]) / K
     total_ms = sum(step_ms)
     if dist:
         t = torch.tensor([total_ms], device="cuda")
@@ -313,9 +331,9 @@ def run_ours(args):
     peak, peak_kind = measured_peaks()
     idx_bytes = BATCH * CTX * INDEX_BYTES_PER_TOKEN
     idx_mean_ms = statistics.mean(idx_ms)
-    achieved = idx_bytes / (idx_mean_ms / 1e3) / 1e9
+    achieved = idx_bytes / (idx_kernel_ms / 1e3) / 1e9
     attn_bytes = BATCH * TOPK * ATTN_ROW_BYTES + BATCH * 128 * (576 + 512) * 2
-    combined = (idx_bytes + attn_bytes) / ((idx_mean_ms + statistics.mean(attn_ms)) / 1e3) / 1e9
+    combined = (idx_bytes + attn_bytes) / ((idx_kernel_ms + statistics.mean(attn_ms)) / 1e3) / 1e9
     traffic = profile_traffic()
     out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": Wm,
            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -324,12 +342,15 @@ def run_ours(args):
            "roofline": {"bound": "hbm", "kernel": "index_score_tc", "achieved": achieved, "peak": peak,
                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak, "traffic": traffic,
                         "algorithmic_bytes_per_launch": idx_bytes,
-                        "indexer_ms": idx_mean_ms, "topk_ms": statistics.mean(topk_ms),
+                        "indexer_ms": idx_kernel_ms, "indexer_ms_in_step": idx_mean_ms,
+                        "topk_ms": statistics.mean(topk_ms),
                         "attn_ms": statistics.mean(attn_ms),
                         "indexer_plus_attn_GBps": combined, "indexer_plus_attn_frac": combined / peak,
-                        "stage_note": "value from steps with no events inside them; indexer_ms from a second "
-                                      "timed pass of the same steps with the indexer bracketed by events; "
-                                      "topk_ms and attn_ms from a pass with every stage boundary recorded"},
+                        "stage_note": "value from steps with no events inside them; indexer_ms (achieved) "
+                                      "from K back-to-back indexer launches between two events; "
+                                      "indexer_ms_in_step from a timed pass of the steps with the indexer "
+                                      "bracketed by events; topk_ms and attn_ms from a pass with every "
+                                      "stage boundary recorded"},
            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d_bytes,
                    "d2h_bytes_per_step": d2h_bytes},
            "clocks": clk.summary(), "gpu_launches": K * wl.kernels_per_step, "device_status": status}
