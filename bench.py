@@ -40,7 +40,8 @@ WORKLOAD = "mla_decode_b8_ctx131072_top2048"
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "index_score_tc_mla_decode_b8_ctx131072.md")
 CONFIG = {"workload": WORKLOAD, "batch": BATCH, "ctx": CTX, "topk": TOPK, "indexer": "64x128 e4m3",
           "attention": "MLA 128 heads x 576 (V 512) bf16", "page": 64,
-          "l2": "flushed between timed steps (256 MB write)"}
+          "l2": "flushed before every step: 256 MB written, then a second 256 MB buffer read so the "
+                "flush's own dirty lines are written back before the step starts"}
 
 
 def rank_env():
@@ -219,7 +220,17 @@ def run_ours(args):
 
     wl = W.mla_decode(batch=BATCH, ctx=CTX, k=TOPK, seed=1002 + 7919 * rank, device="cuda")
     stream = torch.cuda.current_stream()
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush_r = torch.ones(64 << 20, dtype=torch.float32, device="cuda")
+    flush_sink = torch.empty((), dtype=torch.float32, device="cuda")
+
+    class _Flush:  # evicts L2: write a buffer larger than L2, then read another one
+        @staticmethod
+        def zero_():
+            flush_w.zero_()
+            torch.sum(flush_r, dim=0, out=flush_sink)
+
+    flush = _Flush()
     K, Wm = args.steps, args.warmup
 
     def new_events(n):
@@ -273,7 +284,7 @@ def run_ours(args):
     attn_ms = [s[4].elapsed_time(s[5]) for s in stage_ev]
     # the indexer kernel's own duration: launch after launch through ls_index_score (its
     # 143 MB of keys and scales exceed the 126 MB L2, so nothing is reused between launches;
-    # inside a flushed step the events also enclose the launch gap after the flush)
+    # inside a flushed step the events also enclose the launch gap before the kernel)
     t = wl.tensors
     scores = torch.empty((BATCH, wl.args.index.max_len), dtype=torch.float32, device="cuda")
     def run_indexer():
