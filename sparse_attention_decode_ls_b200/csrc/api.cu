@@ -308,8 +308,10 @@ int attn_nsplit(const ls_sparse_attn_args* a) {
   return ns;
 }
 
-size_t attn_ws_bytes(const ls_sparse_attn_args* a) {
-  const int ns = attn_nsplit(a);
+// Split-KV partials of `npasses` launches over the same requests (each with
+// attn_nsplit splits), merged by one combine.
+size_t attn_ws_bytes(const ls_sparse_attn_args* a, int npasses = 1) {
+  const int ns = attn_nsplit(a) * npasses;
   if (ns <= 1) return 0;
   return align256((size_t)a->batch * ns * a->heads * a->dv * 4) + align256((size_t)a->batch * ns * a->heads * 8);
 }
@@ -365,10 +367,14 @@ cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, size_t smem, cudaStream_t s
 }
 
 // `pdl`: launched right behind another kernel of the same decode step, whose outputs
-// (selection, or gathered rows) the attention reads; Q is not among them.
+// (selection, or gathered rows) the attention reads; Q is not among them.  `compacted`:
+// every request's valid selection entries come first.  Pass `pass` of `npasses`
+// (tensor-core path): the launch fills its own range of split-KV partials; `combine`
+// merges all passes' partials into o and lse.
 ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressing, const int* page_table,
                       int max_pages, int n_slots, const void* rows, long long num_rows, void* ws, size_t ws_bytes,
-                      cudaStream_t st, bool pdl) {
+                      cudaStream_t st, bool pdl, bool compacted = false, int pass = 0, int npasses = 1,
+                      bool combine = true) {
   ls::AttnParams p{};
   p.B = a->batch; p.H = a->heads; p.dk = a->dk; p.dv = a->dv; p.k = a->k; p.scale = a->softmax_scale;
   p.addressing = addressing; p.max_pages = max_pages; p.n_slots = n_slots; p.row_stride = a->row_stride;
@@ -376,13 +382,17 @@ ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressi
   p.page_table = page_table; p.sel = sel; p.o = a->o; p.lse = a->lse;
   if (a->dtype == LS_BF16 && a->variant == 0) {
     const int ns = attn_nsplit(a);
+    const int total = ns * npasses;
     p.nsplit = ns;
-    if (ns > 1) {
-      const size_t need = attn_ws_bytes(a);
+    p.split_base = pass * ns;
+    p.nsplit_total = total;
+    p.compacted = compacted ? 1 : 0;
+    if (total > 1) {
+      const size_t need = attn_ws_bytes(a, npasses);
       LS_REQUIRE(ws && ws_bytes >= need, "attention workspace too small (%zu < %zu bytes)", ws_bytes, need);
       LS_REQUIRE(((uintptr_t)ws & 255) == 0, "workspace must be 256-byte aligned");
       p.part_o = (float*)ws;
-      p.part_ml = (float*)((char*)ws + align256((size_t)a->batch * ns * a->heads * a->dv * 4));
+      p.part_ml = (float*)((char*)ws + align256((size_t)a->batch * total * a->heads * a->dv * 4));
     }
     if (allow_smem(ls::attn_mla_tc, ls::mla::kSmem, g_smem_attn_tc) != cudaSuccess)
       return check_launch("attn_mla_tc attribute");
@@ -400,7 +410,7 @@ ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressi
     cudaError_t e = cudaLaunchKernelEx(&cfg, ls::attn_mla_tc, p, kv_map);
     if (e != cudaSuccess) return fail(LS_ERR_CUDA, "attn_mla_tc: %s", cudaGetErrorString(e));
     LS_TRY(check_launch("attn_mla_tc"));
-    if (ns > 1) {
+    if (total > 1 && combine) {
       cudaLaunchConfig_t cc = pdl_config(dim3(ls::mla::H * ls::mla::DV / 8 / ls::kCombineThreads, a->batch),
                                          dim3(ls::kCombineThreads), 0, st, attr, true);
       e = cudaLaunchKernelEx(&cc, ls::attn_combine, p);
@@ -439,8 +449,9 @@ ls_status validate_hotbuf(const ls_hotbuf_args* a) {
   return LS_OK;
 }
 
-ls_status launch_hotbuf(const ls_hotbuf_args* a, cudaStream_t st) {
+ls_status launch_hotbuf(const ls_hotbuf_args* a, cudaStream_t st, int* hit_slot = nullptr) {
   ls::HotbufParams p{};
+  p.hit_slot = hit_slot;
   p.B = a->batch; p.k = a->k; p.n_slots = a->n_slots; p.max_len = a->max_len; p.sel = a->sel;
   p.sel_score = a->sel_score; p.pos_of_slot = a->pos_of_slot; p.recent = a->recent_score;
   p.slot_of_pos = a->slot_of_pos; p.sel_slot = a->sel_slot; p.miss_pos = a->miss_pos; p.miss_slot = a->miss_slot;
@@ -562,7 +573,8 @@ ls_status run_c2f(const ls_block_bound_prune_args* a, void* ws, size_t ws_bytes,
 
 // ---- decode step workspace ------------------------------------------------------------
 struct StepLayout {
-  size_t off_scores, off_idx, off_sel, off_selslot, off_mpos, off_mslot, off_nmiss, off_attn, off_c2f, total;
+  size_t off_scores, off_idx, off_sel, off_selslot, off_mpos, off_mslot, off_nmiss, off_hitslot, off_attn, off_c2f,
+      total;
 };
 
 ls_block_bound_prune_args step_c2f_args(const ls_decode_step_args* a, int* idx, float* sel) {
@@ -579,6 +591,47 @@ ls_block_bound_prune_args step_c2f_args(const ls_decode_step_args* a, int* idx, 
   c.n_survivors = a->n_survivors;
   c.ub = nullptr;
   return c;
+}
+
+// Merge the split-KV partials of `npasses` tensor-core attention launches into o and lse.
+ls_status launch_attn_combine(const ls_sparse_attn_args* a, void* ws, int npasses, cudaStream_t st) {
+  ls::AttnParams p{};
+  p.B = a->batch; p.H = a->heads; p.dk = a->dk; p.dv = a->dv; p.k = a->k; p.o = a->o; p.lse = a->lse;
+  const int ns = attn_nsplit(a), total = ns * npasses;
+  p.nsplit = ns;
+  p.nsplit_total = total;
+  p.part_o = (float*)ws;
+  p.part_ml = (float*)((char*)ws + align256((size_t)a->batch * total * a->heads * a->dv * 4));
+  ls::attn_combine<<<dim3(ls::mla::H * ls::mla::DV / 8 / ls::kCombineThreads, a->batch), ls::kCombineThreads, 0,
+                     st>>>(p);
+  return check_launch("attn_combine");
+}
+
+// Whether the hot-buffer step attends to the resident rows while the misses are being
+// gathered (tensor-core attention), or strictly after the gather.
+bool overlap_misses(const ls_sparse_attn_args* at) { return at->dtype == LS_BF16 && at->variant == 0; }
+
+// A second stream of this host thread on the current device, and two events, for the
+// fork and join of the overlapped hot-buffer step (created once, reused).
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+ls_status side_stream(SideStream** out) {
+  thread_local SideStream per_dev[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  SideStream& ss = per_dev[dev & 63];
+  if (!ss.s) {
+    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+      ss.s = nullptr;
+      return check_launch("side stream");
+    }
+  }
+  *out = &ss;
+  return LS_OK;
 }
 
 ls_sparse_attn_args step_attn_args(const ls_decode_step_args* a) {
@@ -601,7 +654,9 @@ StepLayout step_layout(const ls_decode_step_args* a) {
   l.off_mslot = take(a->use_hotbuf ? (size_t)B * k * 4 : 0);
   l.off_nmiss = take(a->use_hotbuf ? (size_t)B * 4 : 0);
   ls_sparse_attn_args t = step_attn_args(a);
-  l.off_attn = take(attn_ws_bytes(&t));
+  const bool two_pass = a->use_hotbuf && overlap_misses(&t);
+  l.off_hitslot = take(two_pass ? (size_t)B * k * 4 : 0);
+  l.off_attn = take(attn_ws_bytes(&t, two_pass ? 2 : 1));
   if (a->use_c2f) {
     ls_block_bound_prune_args c = step_c2f_args(a, nullptr, nullptr);
     l.off_c2f = take(c2f_layout(&c).total);
@@ -766,19 +821,33 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
                        nullptr, st));
   }
   void* attn_ws = w + l.off_attn;
-  const size_t attn_ws_b = attn_ws_bytes(&at);
   if (a->use_hotbuf) {
     int* sel_slot = (int*)(w + l.off_selslot);
     int* mpos = (int*)(w + l.off_mpos);
     int* mslot = (int*)(w + l.off_mslot);
     int* nmiss = a->n_miss ? a->n_miss : (int*)(w + l.off_nmiss);
+    const bool two_pass = overlap_misses(&at);
+    int* hit_slot = two_pass ? (int*)(w + l.off_hitslot) : nullptr;
+    const size_t attn_ws_b = attn_ws_bytes(&at, two_pass ? 2 : 1);
+    const long long n_rows = (long long)ix->batch * a->n_slots;
     rec(2);
     ls_hotbuf_args h{};
     h.batch = ix->batch; h.k = a->k; h.n_slots = a->n_slots; h.max_len = ix->max_len; h.sel = idx;
     h.sel_score = sel; h.pos_of_slot = a->pos_of_slot; h.recent_score = a->recent_score;
     h.slot_of_pos = a->slot_of_pos; h.sel_slot = sel_slot; h.miss_pos = mpos; h.miss_slot = mslot; h.n_miss = nmiss;
-    LS_TRY(launch_hotbuf(&h, st));
+    LS_TRY(launch_hotbuf(&h, st, hit_slot));
     rec(3);
+    SideStream* ss = nullptr;
+    if (two_pass) {
+      // the resident rows are attended to on a second stream while the misses are copied
+      // from the host into their victim slots (victims are never resident selected rows)
+      LS_TRY(side_stream(&ss));
+      cudaEventRecord(ss->fork, st);
+      cudaStreamWaitEvent(ss->s, ss->fork, 0);
+      LS_TRY(launch_attn(&at, hit_slot, LS_ROWS_SLOTS, nullptr, 0, a->n_slots, a->hbuf, n_rows, attn_ws, attn_ws_b,
+                         ss->s, false, false, 0, 2, false));
+      cudaEventRecord(ss->join, ss->s);
+    }
     ls_gather_args g{};
     g.batch = ix->batch; g.k = a->k; g.n_slots = a->n_slots; g.max_pages = ix->max_pages;
     g.row_bytes = at.row_stride * (at.dtype == LS_BF16 ? 2 : 4); g.num_pages = a->host_num_pages;
@@ -786,15 +855,25 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
     g.n_miss = nmiss; g.hbuf = a->hbuf;
     LS_TRY(launch_gather(&g, st));
     rec(4);
-    LS_TRY(launch_attn(&at, sel_slot, LS_ROWS_SLOTS, nullptr, 0, a->n_slots, a->hbuf,
-                       (long long)ix->batch * a->n_slots, attn_ws, attn_ws_b, st, true));
+    if (two_pass) {
+      // then the misses (a compacted list), and one merge of both passes' partials
+      LS_TRY(launch_attn(&at, mslot, LS_ROWS_SLOTS, nullptr, 0, a->n_slots, a->hbuf, n_rows, attn_ws, attn_ws_b, st,
+                         true, true, 1, 2, false));
+      cudaStreamWaitEvent(st, ss->join, 0);
+      LS_TRY(launch_attn_combine(&at, attn_ws, 2, st));
+    } else {
+      LS_TRY(launch_attn(&at, sel_slot, LS_ROWS_SLOTS, nullptr, 0, a->n_slots, a->hbuf, n_rows, attn_ws, attn_ws_b,
+                         st, true));
+    }
   } else {
+    const size_t attn_ws_b = attn_ws_bytes(&at);
     rec(2);
     rec(3);
     rec(4);
     const int* pt = at.page_table ? at.page_table : ix->page_table;
     const int mp = at.page_table ? at.max_pages : ix->max_pages;
-    LS_TRY(launch_attn(&at, idx, LS_ROWS_PAGED, pt, mp, 0, nullptr, at.num_rows, attn_ws, attn_ws_b, st, true));
+    LS_TRY(launch_attn(&at, idx, LS_ROWS_PAGED, pt, mp, 0, nullptr, at.num_rows, attn_ws, attn_ws_b, st, true,
+                       true));
   }
   rec(5);
   return ok();

@@ -41,6 +41,9 @@ struct AttnParams {
   float* part_o;     // [B,nsplit,dv/4,H,4] unnormalised partial outputs (4-dim granules, head next)
   float* part_ml;    // [B,nsplit,H,2] running max (log2 domain) and sum
   int early_q;       // tensor-core kernel: read Q before waiting for the kernel before
+  int split_base;    // tensor-core kernel: this launch's splits are partial slots
+  int nsplit_total;  //   [split_base, split_base + nsplit) of nsplit_total per request
+  int compacted;     // the valid entries of every request's selection come first
 };
 
 // 2^x with the hardware approximation (relative error about 2^-22; results below the
@@ -237,7 +240,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   const int T_all = (p.k + N - 1) / N;
   const int t0 = (int)(((long long)T_all * split) / p.nsplit);
   const int t1 = (int)(((long long)T_all * (split + 1)) / p.nsplit);
-  const int my_tiles = t1 - t0;
+  const int my_tiles0 = t1 - t0;  // tiles of this CTA's share of the selection
   const uint32_t sbase = smem_u32(sm);
 
   if (threadIdx.x == 0) {
@@ -261,7 +264,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     s_abort = 0;
     fence_mbar_init();
     // arm the receive buffers for tiles 0 and 1 before the other CTA can send
-    for (int s = 0; s < 2 && s < my_tiles; ++s) mbar_arrive_expect_tx(&x_full[s], kXBytes);
+    for (int s = 0; s < 2 && s < my_tiles0; ++s) mbar_arrive_expect_tx(&x_full[s], kXBytes);
   }
   if (warp == kMmaWarp) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
@@ -272,7 +275,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   const uint32_t tm_s = tmem + kTmemS;  // kSBufs S tiles
   const uint32_t tm_p = tmem + kTmemP;  // P of the current tile, bf16 pairs (PV's A operand)
   const uint32_t tm_q = tmem + kTmemQ;  // this rank's Q panels
-  if (warp < 4 && p.early_q && my_tiles > 0) {  // Q is not written by the kernel before
+  if (warp < 4 && p.early_q && my_tiles0 > 0) {  // Q is not written by the kernel before
     load_q_tmem(p, b, rank, threadIdx.x, tm_q + ((uint32_t)(warp * 32) << 16));
     tc_fence_before();
     mbar_arrive(q_full);
@@ -281,6 +284,11 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   // the selection, the rows and the outputs are touched only after it has finished
   griddep_wait();
   griddep_launch_dependents();
+  // in a compacted selection a share that starts with padding holds no row at all (the
+  // tail of a miss list): such a CTA only writes an empty partial
+  const int my_tiles =
+      (p.compacted && my_tiles0 > 0 && p.sel[(size_t)b * p.k + (size_t)t0 * N] < 0) ? 0 : my_tiles0;
+  const size_t pslot = (size_t)b * p.nsplit_total + p.split_base + split;  // partial slot
 
   if (warp >= kLoadWarp0) {
     // ================= row gathers: tile i goes to stage i % kStages =================
@@ -525,7 +533,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     fin = __all_sync(0xffffffffu, fin);  // the TMEM reads below are warp-collective
     if (fin) {
       tc_fence_after();
-      const bool single = p.nsplit == 1;
+      const bool single = p.nsplit_total == 1;
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
       for (int c0 = 0; c0 < DVH; c0 += 32) {
         float v[32];
@@ -544,7 +552,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
           }
         } else {
           // layout [b][split][dim / 4][head][4]: a warp's store is 512 contiguous bytes
-          float4* o = (float4*)p.part_o + (((size_t)b * p.nsplit + split) * (DV / 4) + (rank * DVH + c0) / 4) * H + h;
+          float4* o = (float4*)p.part_o + (pslot * (DV / 4) + (rank * DVH + c0) / 4) * H + h;
           const bool any = l_run > 0.f;
 #pragma unroll
           for (int c = 0; c < 32; c += 4)
@@ -555,16 +563,16 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
         if (single) {
           p.lse[(size_t)b * H + h] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
         } else {
-          float* ml = p.part_ml + (((size_t)b * p.nsplit + split) * H + h) * 2;
+          float* ml = p.part_ml + (pslot * H + h) * 2;
           ml[0] = l_run > 0.f ? m_run : -INFINITY;
           ml[1] = l_run;
         }
       }
-    } else if (my_tiles == 0 && p.nsplit > 1) {
-      float4* o = (float4*)p.part_o + (((size_t)b * p.nsplit + split) * (DV / 4) + rank * DVH / 4) * H + h;
+    } else if (my_tiles == 0 && p.nsplit_total > 1) {
+      float4* o = (float4*)p.part_o + (pslot * (DV / 4) + rank * DVH / 4) * H + h;
       for (int c = 0; c < DVH / 4; ++c) o[(size_t)c * H] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (rank == 0) {
-        float* ml = p.part_ml + (((size_t)b * p.nsplit + split) * H + h) * 2;
+        float* ml = p.part_ml + (pslot * H + h) * 2;
         ml[0] = -INFINITY;
         ml[1] = 0.f;
       }
@@ -594,21 +602,21 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine(const AttnParams
   const int b = blockIdx.y;
   const int item = blockIdx.x * kCombineThreads + threadIdx.x;
   const int g = item / H, h = item - g * H, d0 = g * 8;
-  const float* ml = p.part_ml + (size_t)b * p.nsplit * H * 2 + (size_t)h * 2;
+  const float* ml = p.part_ml + (size_t)b * p.nsplit_total * H * 2 + (size_t)h * 2;
   float M = -INFINITY;
-  for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, ml[(size_t)s * H * 2]);
+  for (int s = 0; s < p.nsplit_total; ++s) M = fmaxf(M, ml[(size_t)s * H * 2]);
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
   float Lsum = 0.f;
   if (M != -INFINITY) {
 #pragma unroll 4
-    for (int s = 0; s < p.nsplit; ++s) {
+    for (int s = 0; s < p.nsplit_total; ++s) {
       const float l = ml[(size_t)s * H * 2 + 1];
       if (!(l > 0.f)) continue;
       const float wgt = exp2f(ml[(size_t)s * H * 2] - M);
       Lsum += wgt * l;
-      const float4* po = (const float4*)p.part_o + (((size_t)b * p.nsplit + s) * (DV / 4) + d0 / 4) * H + h;
+      const float4* po = (const float4*)p.part_o + (((size_t)b * p.nsplit_total + s) * (DV / 4) + d0 / 4) * H + h;
       const float4 x = po[0], y = po[H];
       acc[0] = fmaf(wgt, x.x, acc[0]); acc[1] = fmaf(wgt, x.y, acc[1]);
       acc[2] = fmaf(wgt, x.z, acc[2]); acc[3] = fmaf(wgt, x.w, acc[3]);

@@ -24,6 +24,7 @@ struct HotbufParams {
   float* recent;
   int* slot_of_pos;
   int* sel_slot;
+  int* hit_slot;   // optional: the slot of every selected position already resident, else -1
   int* miss_pos;
   int* miss_slot;
   int* n_miss;
@@ -72,6 +73,7 @@ __global__ void __launch_bounds__(kHbThreads, 1) hotbuf_resolve_kernel(const Hot
       }
     }
     sel_slot[j] = slot;
+    if (p.hit_slot) p.hit_slot[(size_t)b * k + j] = is_miss ? -1 : slot;
     if (is_miss) {
       miss_bits |= 1u << (j - j0);
       ++my_miss;

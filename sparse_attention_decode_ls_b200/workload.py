@@ -145,7 +145,9 @@ def kernels_per_step(wl: DecodeWorkload, *, c2f: bool, hotbuf: bool, mla: bool) 
     n = 8 if c2f else 2
     if hotbuf:
         n += 2
-    if mla:
+    if mla and hotbuf:
+        n += 3   # resident-row pass, miss pass, merge of both passes
+    elif mla:
         n += 2 if B.ls_sparse_attn_workspace_size(wl.args.attn) > 0 else 1
     else:
         n += 1
@@ -163,6 +165,36 @@ def mla_decode(batch=8, ctx=131072, k=2048, seed=1002, device="cuda", kv_on_devi
     q, kv = syn.mla_attention(batch, n_pool, seed=seed + 1000, device=device if kv_on_device else "cpu")
     return build(f"mla_decode_b{batch}_ctx{ctx}", ind, k=k, device=device,
                  attn=dict(q=q, kv=kv, scale=syn.softmax_scale(576)))
+
+
+def mla_hotbuf_decode(batch=36, ctx=131072, k=2048, miss_frac=0.2, n_slots=4096, seed=1003,
+                      device="cuda") -> DecodeWorkload:
+    """The hot-buffer configuration: the full KV history in pinned host memory, a
+    4,096-slot hot buffer per request in HBM holding all but a seeded ``miss_frac`` of this
+    step's selection (the selection of the GPU's own indexer and top-k), filled up with
+    other positions.  Restore the buffer state (``restore_hotbuf``) before every step."""
+    lens = [ctx] * batch
+    ind = syn.indexer_fp8(lens, seed=seed)
+    n_pool = ind.key_pool.shape[0]
+    q, kv_dev = syn.mla_attention(batch, n_pool, seed=seed + 1000, device=device)
+    host = torch.empty(kv_dev.shape, dtype=torch.bfloat16, pin_memory=True)
+    host.copy_(kv_dev)
+    del kv_dev
+    ml = _round4(ctx)
+    d = {key: getattr(ind, key).to(device) for key in ("q", "q_scale", "w", "key_pool", "key_scale", "page_table",
+                                                      "lens")}
+    scores = torch.empty((batch, ml), dtype=torch.float32, device=device)
+    idx = torch.empty((batch, k), dtype=torch.int32, device=device)
+    B.ls_index_score(q=d["q"], w=d["w"], key_pool=d["key_pool"], page_table=d["page_table"], lens=d["lens"],
+                     scores=scores, q_scale=d["q_scale"], key_scale=d["key_scale"])
+    B.ls_topk_select(scores=scores, lens=d["lens"], idx=idx)
+    sel = idx.cpu()
+    del d, scores
+    pos_of_slot, slot_of_pos, recent = syn.hot_buffer_state([r[r >= 0] for r in sel], lens, n_slots=n_slots,
+                                                            miss_frac=miss_frac, seed=seed + 2000, max_len=ml)
+    return build(f"mla_hotbuf_b{batch}_ctx{ctx}_miss{int(round(miss_frac * 100))}", ind, k=k, device=device,
+                 attn=dict(q=q, kv_host=True, scale=syn.softmax_scale(576)),
+                 hotbuf=dict(pos_of_slot=pos_of_slot, slot_of_pos=slot_of_pos, recent=recent, host_kv=host))
 
 
 def tiny_f32(device="cuda") -> DecodeWorkload:

@@ -37,3 +37,46 @@ def test_decode_step_graph_replay_matches_eager():
         assert torch.equal(wl.o, o_ref)
         assert torch.equal(wl.lse, lse_ref)
     assert B.ls_check_device_status() == 0
+
+
+def test_hot_buffer_step_graph_replay_matches_eager():
+    """The hot-buffer step forks the resident-row attention onto a second stream while the
+    misses are copied in from pinned host memory; the fork and join are captured too."""
+    lens = [40000, 64 * 300 + 5]
+    inp = syn.indexer_fp8(lens, seed=911)
+    n_pool = inp.key_pool.shape[0]
+    q, kv = syn.mla_attention(len(lens), n_pool, seed=912)
+    host = kv.view(torch.int16).pin_memory().view(torch.bfloat16)
+    ml = (max(lens) + 3) // 4 * 4
+    # a buffer that holds a seeded half of some other positions: most of the selection misses
+    g0 = torch.Generator().manual_seed(913)
+    other = [torch.randperm(L, generator=g0)[:1024] for L in lens]
+    pos_of_slot, slot_of_pos, recent = syn.hot_buffer_state(other, lens, n_slots=4096, miss_frac=0.5, seed=914,
+                                                            max_len=ml)
+    wl = W.build("graph_hotbuf", inp, k=2048, attn=dict(q=q, kv_host=True, scale=syn.softmax_scale(576)),
+                 hotbuf=dict(pos_of_slot=pos_of_slot, slot_of_pos=slot_of_pos, recent=recent, host_kv=host))
+    state = ("pos_of_slot", "slot_of_pos", "hbuf", "n_miss")
+    wl.restore_hotbuf()
+    wl.step()
+    torch.cuda.synchronize()
+    ref = {key: wl.tensors[key].clone() for key in ("o", "lse", "idx") + state}
+    assert int(ref["n_miss"].min()) > 0
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        wl.restore_hotbuf()
+        wl.step()  # warm up on the capture stream
+    torch.cuda.current_stream().wait_stream(s)
+    with torch.cuda.graph(g):
+        wl.step()
+    for _ in range(3):
+        wl.restore_hotbuf()
+        wl.o.zero_()
+        wl.idx.fill_(-5)
+        wl.tensors["n_miss"].fill_(-1)
+        g.replay()
+        torch.cuda.synchronize()
+        for key, val in ref.items():
+            assert torch.equal(wl.tensors[key], val), key
+    assert B.ls_check_device_status() == 0
