@@ -416,6 +416,9 @@ def run_hotbuf(args):
     # then the miss pass and the merge (the resident-row pass runs beside the gather)
     stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(min(args.steps, 20))]
     for evs in stage_ev:
+        for e in evs:
+            e.record(stream)   # created by torch; the library records them again inside the step
+    for evs in stage_ev:
         prep()
         wl.step(events=B.event_array(evs))
     torch.cuda.synchronize()

@@ -86,6 +86,22 @@ cudaError_t allow_smem(K kernel, int bytes, std::atomic<uint64_t>& done) {
   return e;
 }
 
+// Ask for the SM's full shared-memory carve-out for a kernel that needs little of it: an
+// SM's split between L1 and shared memory changes only when the SM is idle, so a small
+// kernel that left its SMs in an L1-heavy split would keep the attention CTAs (about
+// 206 KB of shared memory each) that run beside it off those SMs.
+template <typename K>
+cudaError_t keep_smem_carveout(K kernel, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done.load() & bit) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                       (int)cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess) done.fetch_or(bit);
+  return e;
+}
+
 // ---- TMA descriptor ----------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -374,7 +390,7 @@ cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, size_t smem, cudaStream_t s
 ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressing, const int* page_table,
                       int max_pages, int n_slots, const void* rows, long long num_rows, void* ws, size_t ws_bytes,
                       cudaStream_t st, bool pdl, bool compacted = false, int pass = 0, int npasses = 1,
-                      bool combine = true) {
+                      bool combine = true, const int* n_valid = nullptr) {
   ls::AttnParams p{};
   p.B = a->batch; p.H = a->heads; p.dk = a->dk; p.dv = a->dv; p.k = a->k; p.scale = a->softmax_scale;
   p.addressing = addressing; p.max_pages = max_pages; p.n_slots = n_slots; p.row_stride = a->row_stride;
@@ -387,6 +403,7 @@ ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressi
     p.split_base = pass * ns;
     p.nsplit_total = total;
     p.compacted = compacted ? 1 : 0;
+    p.n_valid = n_valid;
     if (total > 1) {
       const size_t need = attn_ws_bytes(a, npasses);
       LS_REQUIRE(ws && ws_bytes >= need, "attention workspace too small (%zu < %zu bytes)", ws_bytes, need);
@@ -435,7 +452,7 @@ ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressi
 }
 
 // ---- hot buffer -------------------------------------------------------------------------
-std::atomic<uint64_t> g_smem_hb{0};
+std::atomic<uint64_t> g_smem_hb{0}, g_carve_hb{0}, g_carve_gather{0}, g_carve_classify{0}, g_carve_copy{0};
 
 ls_status validate_hotbuf(const ls_hotbuf_args* a) {
   LS_REQUIRE(a, "args is NULL");
@@ -449,9 +466,8 @@ ls_status validate_hotbuf(const ls_hotbuf_args* a) {
   return LS_OK;
 }
 
-ls_status launch_hotbuf(const ls_hotbuf_args* a, cudaStream_t st, int* hit_slot = nullptr) {
+ls_status launch_hotbuf(const ls_hotbuf_args* a, cudaStream_t st) {
   ls::HotbufParams p{};
-  p.hit_slot = hit_slot;
   p.B = a->batch; p.k = a->k; p.n_slots = a->n_slots; p.max_len = a->max_len; p.sel = a->sel;
   p.sel_score = a->sel_score; p.pos_of_slot = a->pos_of_slot; p.recent = a->recent_score;
   p.slot_of_pos = a->slot_of_pos; p.sel_slot = a->sel_slot; p.miss_pos = a->miss_pos; p.miss_slot = a->miss_slot;
@@ -459,7 +475,8 @@ ls_status launch_hotbuf(const ls_hotbuf_args* a, cudaStream_t st, int* hit_slot 
   int pow2 = 1;
   while (pow2 < a->n_slots) pow2 <<= 1;
   const int smem = pow2 * 8;
-  if (allow_smem(ls::hotbuf_resolve_kernel, ls::kHbMaxSlots * 8, g_smem_hb) != cudaSuccess)
+  if (allow_smem(ls::hotbuf_resolve_kernel, ls::kHbMaxSlots * 8, g_smem_hb) != cudaSuccess ||
+      keep_smem_carveout(ls::hotbuf_resolve_kernel, g_carve_hb) != cudaSuccess)
     return check_launch("hotbuf attribute");
   ls::hotbuf_resolve_kernel<<<a->batch, ls::kHbThreads, smem, st>>>(p);
   return check_launch("hotbuf_resolve");
@@ -476,16 +493,50 @@ ls_status validate_gather(const ls_gather_args* a) {
   return LS_OK;
 }
 
-ls_status launch_gather(const ls_gather_args* a, cudaStream_t st) {
+ls_status launch_gather(const ls_gather_args* a, cudaStream_t st, void* stage = nullptr) {
   ls::GatherParams p{};
   p.B = a->batch; p.k = a->k; p.n_slots = a->n_slots; p.max_pages = a->max_pages; p.row_bytes = a->row_bytes;
   p.num_pages = a->num_pages; p.host = (const char*)a->host_kv; p.page_table = a->page_table;
   p.miss_pos = a->miss_pos; p.miss_slot = a->miss_slot; p.n_miss = a->n_miss; p.hbuf = (char*)a->hbuf;
-  const int rows_per_cta = 8 * 4;
+  p.stage = (char*)stage;
+  // small CTAs on about a quarter of the SMs: 144 warps with two rows each in flight keep
+  // the host link busy (measured: as fast as one CTA per SM), and the attention on the
+  // resident rows, which runs beside the gather in the decode step, is slowed far less
+  // by a gather CTA on its SM
+  const int rows_per_cta = (ls::kGatherThreads / 32) * 2;
   int g = (a->k + rows_per_cta - 1) / rows_per_cta;
-  g = std::max(1, std::min(g, (8 * device_sms()) / a->batch + 1));
-  ls::gather_misses_kernel<<<dim3(g, a->batch), 256, 0, st>>>(p);
+  g = std::max(1, std::min(g, device_sms() / (4 * a->batch)));
+  if (keep_smem_carveout(ls::gather_misses_kernel, g_carve_gather) != cudaSuccess)
+    return check_launch("gather attribute");
+  ls::gather_misses_kernel<<<dim3(g, a->batch), ls::kGatherThreads, 0, st>>>(p);
   return check_launch("gather_misses");
+}
+
+// The decode step's classification of the selection (resident slots; misses compacted
+// in selection order) ahead of the full resolve.
+ls_status launch_classify(const ls_hotbuf_args* a, int* hit_slot, int* n_hit, int* miss_pos, int* miss_row,
+                          int* n_miss, cudaStream_t st) {
+  ls::ClassifyParams p{};
+  p.B = a->batch; p.k = a->k; p.n_slots = a->n_slots; p.max_len = a->max_len; p.sel = a->sel;
+  p.slot_of_pos = a->slot_of_pos; p.hit_slot = hit_slot; p.n_hit = n_hit; p.miss_pos = miss_pos; p.miss_row = miss_row;
+  p.n_miss = n_miss;
+  if (keep_smem_carveout(ls::hotbuf_classify_kernel, g_carve_classify) != cudaSuccess)
+    return check_launch("classify attribute");
+  ls::hotbuf_classify_kernel<<<a->batch, ls::kHbThreads, 0, st>>>(p);
+  return check_launch("hotbuf_classify");
+}
+
+// Staged miss rows into the victim slots the resolve chose.
+ls_status launch_copy_staged(const ls_gather_args* g, const void* stage, cudaStream_t st) {
+  ls::StageCopyParams p{};
+  p.B = g->batch; p.k = g->k; p.n_slots = g->n_slots; p.row_bytes = g->row_bytes; p.stage = (const char*)stage;
+  p.miss_slot = g->miss_slot; p.n_miss = g->n_miss; p.hbuf = (char*)g->hbuf;
+  int c = (g->k + 7) / 8;
+  c = std::max(1, std::min(c, (4 * device_sms()) / g->batch + 1));
+  if (keep_smem_carveout(ls::copy_staged_kernel, g_carve_copy) != cudaSuccess)
+    return check_launch("copy_staged attribute");
+  ls::copy_staged_kernel<<<dim3(c, g->batch), 256, 0, st>>>(p);
+  return check_launch("copy_staged");
 }
 
 // ---- coarse-to-fine ---------------------------------------------------------------------
@@ -573,8 +624,8 @@ ls_status run_c2f(const ls_block_bound_prune_args* a, void* ws, size_t ws_bytes,
 
 // ---- decode step workspace ------------------------------------------------------------
 struct StepLayout {
-  size_t off_scores, off_idx, off_sel, off_selslot, off_mpos, off_mslot, off_nmiss, off_hitslot, off_attn, off_c2f,
-      total;
+  size_t off_scores, off_idx, off_sel, off_selslot, off_mpos, off_mslot, off_nmiss, off_hitslot, off_cpos, off_crow,
+      off_cnmiss, off_cnhit, off_stage, off_attn, off_c2f, total;
 };
 
 ls_block_bound_prune_args step_c2f_args(const ls_decode_step_args* a, int* idx, float* sel) {
@@ -611,23 +662,28 @@ ls_status launch_attn_combine(const ls_sparse_attn_args* a, void* ws, int npasse
 // gathered (tensor-core attention), or strictly after the gather.
 bool overlap_misses(const ls_sparse_attn_args* at) { return at->dtype == LS_BF16 && at->variant == 0; }
 
-// A second stream of this host thread on the current device, and two events, for the
-// fork and join of the overlapped hot-buffer step (created once, reused).
+// Two more streams of this host thread on the current device, and the events for the
+// fork and joins of the overlapped hot-buffer step (created once, reused).
 struct SideStream {
-  cudaStream_t s = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaStream_t s[2] = {nullptr, nullptr};
+  cudaEvent_t fork = nullptr, gathered = nullptr, join[2] = {nullptr, nullptr};
 };
 ls_status side_stream(SideStream** out) {
   thread_local SideStream per_dev[64];
   int dev = 0;
   cudaGetDevice(&dev);
   SideStream& ss = per_dev[dev & 63];
-  if (!ss.s) {
-    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
-      ss.s = nullptr;
-      return check_launch("side stream");
+  if (!ss.s[1]) {
+    bool good = true;
+    for (int i = 0; i < 2; ++i) {
+      if (!ss.s[i]) good = good && cudaStreamCreateWithFlags(&ss.s[i], cudaStreamNonBlocking) == cudaSuccess;
+      if (!ss.join[i]) good = good && cudaEventCreateWithFlags(&ss.join[i], cudaEventDisableTiming) == cudaSuccess;
+    }
+    if (!ss.fork) good = good && cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) == cudaSuccess;
+    if (!ss.gathered) good = good && cudaEventCreateWithFlags(&ss.gathered, cudaEventDisableTiming) == cudaSuccess;
+    if (!good) {
+      ss.s[1] = nullptr;
+      return check_launch("side streams");
     }
   }
   *out = &ss;
@@ -656,6 +712,11 @@ StepLayout step_layout(const ls_decode_step_args* a) {
   ls_sparse_attn_args t = step_attn_args(a);
   const bool two_pass = a->use_hotbuf && overlap_misses(&t);
   l.off_hitslot = take(two_pass ? (size_t)B * k * 4 : 0);
+  l.off_cpos = take(two_pass ? (size_t)B * k * 4 : 0);
+  l.off_crow = take(two_pass ? (size_t)B * k * 4 : 0);
+  l.off_cnmiss = take(two_pass ? (size_t)B * 4 : 0);
+  l.off_cnhit = take(two_pass ? (size_t)B * 4 : 0);
+  l.off_stage = take(two_pass ? (size_t)B * k * t.row_stride * 2 : 0);
   l.off_attn = take(attn_ws_bytes(&t, two_pass ? 2 : 1));
   if (a->use_c2f) {
     ls_block_bound_prune_args c = step_c2f_args(a, nullptr, nullptr);
@@ -827,7 +888,6 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
     int* mslot = (int*)(w + l.off_mslot);
     int* nmiss = a->n_miss ? a->n_miss : (int*)(w + l.off_nmiss);
     const bool two_pass = overlap_misses(&at);
-    int* hit_slot = two_pass ? (int*)(w + l.off_hitslot) : nullptr;
     const size_t attn_ws_b = attn_ws_bytes(&at, two_pass ? 2 : 1);
     const long long n_rows = (long long)ix->batch * a->n_slots;
     rec(2);
@@ -835,33 +895,54 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
     h.batch = ix->batch; h.k = a->k; h.n_slots = a->n_slots; h.max_len = ix->max_len; h.sel = idx;
     h.sel_score = sel; h.pos_of_slot = a->pos_of_slot; h.recent_score = a->recent_score;
     h.slot_of_pos = a->slot_of_pos; h.sel_slot = sel_slot; h.miss_pos = mpos; h.miss_slot = mslot; h.n_miss = nmiss;
-    LS_TRY(launch_hotbuf(&h, st, hit_slot));
-    rec(3);
-    SideStream* ss = nullptr;
-    if (two_pass) {
-      // the resident rows are attended to on a second stream while the misses are copied
-      // from the host into their victim slots (victims are never resident selected rows)
-      LS_TRY(side_stream(&ss));
-      cudaEventRecord(ss->fork, st);
-      cudaStreamWaitEvent(ss->s, ss->fork, 0);
-      LS_TRY(launch_attn(&at, hit_slot, LS_ROWS_SLOTS, nullptr, 0, a->n_slots, a->hbuf, n_rows, attn_ws, attn_ws_b,
-                         ss->s, false, false, 0, 2, false));
-      cudaEventRecord(ss->join, ss->s);
-    }
     ls_gather_args g{};
     g.batch = ix->batch; g.k = a->k; g.n_slots = a->n_slots; g.max_pages = ix->max_pages;
     g.row_bytes = at.row_stride * (at.dtype == LS_BF16 ? 2 : 4); g.num_pages = a->host_num_pages;
     g.host_kv = a->host_kv; g.page_table = ix->page_table; g.miss_pos = mpos; g.miss_slot = mslot;
     g.n_miss = nmiss; g.hbuf = a->hbuf;
-    LS_TRY(launch_gather(&g, st));
-    rec(4);
     if (two_pass) {
-      // then the misses (a compacted list), and one merge of both passes' partials
-      LS_TRY(launch_attn(&at, mslot, LS_ROWS_SLOTS, nullptr, 0, a->n_slots, a->hbuf, n_rows, attn_ws, attn_ws_b, st,
-                         true, true, 1, 2, false));
-      cudaStreamWaitEvent(st, ss->join, 0);
+      // critical path: classify -> fetch the misses over the host link into staging rows
+      // -> attend to them there -> merge.  Beside it: the resident rows' attention, and
+      // the victim choice + map update, then the staged rows into their victim slots
+      // (victims are never resident selected rows, so nothing here races).
+      int* hit_slot = (int*)(w + l.off_hitslot);
+      int* cpos = (int*)(w + l.off_cpos);
+      int* crow = (int*)(w + l.off_crow);
+      int* cn = (int*)(w + l.off_cnmiss);
+      int* chit = (int*)(w + l.off_cnhit);
+      void* stage = w + l.off_stage;
+      LS_TRY(launch_classify(&h, hit_slot, chit, cpos, crow, cn, st));
+      rec(3);
+      SideStream* ss = nullptr;
+      LS_TRY(side_stream(&ss));
+      cudaEventRecord(ss->fork, st);
+      cudaStreamWaitEvent(ss->s[0], ss->fork, 0);
+      cudaStreamWaitEvent(ss->s[1], ss->fork, 0);
+      LS_TRY(launch_hotbuf(&h, ss->s[0]));
+      LS_TRY(launch_attn(&at, hit_slot, LS_ROWS_SLOTS, nullptr, 0, a->n_slots, a->hbuf, n_rows, attn_ws, attn_ws_b,
+                         ss->s[1], false, true, 0, 2, false, chit));
+      cudaEventRecord(ss->join[1], ss->s[1]);
+      ls_gather_args gs = g;
+      gs.miss_pos = cpos;
+      gs.n_miss = cn;
+      LS_TRY(launch_gather(&gs, st, stage));
+      rec(4);
+      // the staging area as rows: request b's i-th miss at row b*k + i (launched straight
+      // after the gather, so that its prologue overlaps the gather's end)
+      LS_TRY(launch_attn(&at, crow, LS_ROWS_SLOTS, nullptr, 0, a->k, stage, (long long)ix->batch * a->k, attn_ws,
+                         attn_ws_b, st, true, true, 1, 2, false, cn));
+      cudaEventRecord(ss->gathered, st);
+      cudaStreamWaitEvent(ss->s[0], ss->gathered, 0);
+      LS_TRY(launch_copy_staged(&g, stage, ss->s[0]));
+      cudaEventRecord(ss->join[0], ss->s[0]);
+      cudaStreamWaitEvent(st, ss->join[1], 0);
       LS_TRY(launch_attn_combine(&at, attn_ws, 2, st));
+      cudaStreamWaitEvent(st, ss->join[0], 0);
     } else {
+      LS_TRY(launch_hotbuf(&h, st));
+      rec(3);
+      LS_TRY(launch_gather(&g, st));
+      rec(4);
       LS_TRY(launch_attn(&at, sel_slot, LS_ROWS_SLOTS, nullptr, 0, a->n_slots, a->hbuf, n_rows, attn_ws, attn_ws_b,
                          st, true));
     }

@@ -44,6 +44,8 @@ struct AttnParams {
   int split_base;    // tensor-core kernel: this launch's splits are partial slots
   int nsplit_total;  //   [split_base, split_base + nsplit) of nsplit_total per request
   int compacted;     // the valid entries of every request's selection come first
+  const int* n_valid;  // optional [B]: and there are n_valid[b] of them; the splits share
+                       //   those rows instead of all k entries
 };
 
 // 2^x with the hardware approximation (relative error about 2^-22; results below the
@@ -241,6 +243,9 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   const int t0 = (int)(((long long)T_all * split) / p.nsplit);
   const int t1 = (int)(((long long)T_all * (split + 1)) / p.nsplit);
   const int my_tiles0 = t1 - t0;  // tiles of this CTA's share of the selection
+  // with n_valid the share is known only after the kernel before has finished: what runs
+  // ahead of that is sized for the most tiles a share can get
+  const int my_tiles_max = p.n_valid ? (T_all + p.nsplit - 1) / p.nsplit : my_tiles0;
   const uint32_t sbase = smem_u32(sm);
 
   if (threadIdx.x == 0) {
@@ -263,8 +268,9 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     mbar_init(q_full, 128);  // the softmax threads, once Q is in TMEM
     s_abort = 0;
     fence_mbar_init();
-    // arm the receive buffers for tiles 0 and 1 before the other CTA can send
-    for (int s = 0; s < 2 && s < my_tiles0; ++s) mbar_arrive_expect_tx(&x_full[s], kXBytes);
+    // arm the receive buffers for tiles 0 and 1 before the other CTA can send (an armed
+    // buffer that no tile uses is never waited on)
+    for (int s = 0; s < 2 && s < my_tiles_max; ++s) mbar_arrive_expect_tx(&x_full[s], kXBytes);
   }
   if (warp == kMmaWarp) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
@@ -275,7 +281,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   const uint32_t tm_s = tmem + kTmemS;  // kSBufs S tiles
   const uint32_t tm_p = tmem + kTmemP;  // P of the current tile, bf16 pairs (PV's A operand)
   const uint32_t tm_q = tmem + kTmemQ;  // this rank's Q panels
-  if (warp < 4 && p.early_q && my_tiles0 > 0) {  // Q is not written by the kernel before
+  if (warp < 4 && p.early_q && my_tiles_max > 0) {  // Q is not written by the kernel before
     load_q_tmem(p, b, rank, threadIdx.x, tm_q + ((uint32_t)(warp * 32) << 16));
     tc_fence_before();
     mbar_arrive(q_full);
@@ -286,8 +292,15 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   griddep_launch_dependents();
   // in a compacted selection a share that starts with padding holds no row at all (the
   // tail of a miss list): such a CTA only writes an empty partial
-  const int my_tiles =
-      (p.compacted && my_tiles0 > 0 && p.sel[(size_t)b * p.k + (size_t)t0 * N] < 0) ? 0 : my_tiles0;
+  int tb = t0, my_tiles = my_tiles0;
+  if (p.n_valid) {
+    const int nv = min(max(p.n_valid[b], 0), p.k);
+    const int tv = (nv + N - 1) / N;
+    tb = (int)(((long long)tv * split) / p.nsplit);
+    my_tiles = min((int)(((long long)tv * (split + 1)) / p.nsplit) - tb, my_tiles_max);
+  } else if (p.compacted && my_tiles0 > 0 && p.sel[(size_t)b * p.k + (size_t)t0 * N] < 0) {
+    my_tiles = 0;
+  }
   const size_t pslot = (size_t)b * p.nsplit_total + p.split_base + split;  // partial slot
 
   if (warp >= kLoadWarp0) {
@@ -304,7 +317,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     int* s_rows = (int*)(sm + kOffRows);
     const int nrows = my_tiles * N;
     for (int r = lw * 32 + lane; r < nrows; r += kLoadWarps * 32) {
-      const int j = t0 * N + r;
+      const int j = tb * N + r;
       const long long row = j < p.k ? attn_row(p, b, p.sel[(size_t)b * p.k + j]) : -1;
       s_rows[r] = row >= 0 ? (int)row : (int)p.num_rows;
     }

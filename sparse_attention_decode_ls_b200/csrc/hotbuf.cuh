@@ -9,8 +9,15 @@
 // and the recent scores in place.
 //
 // gather_misses: copies each missed 1,152-byte row from pinned host memory into its
-// slot; every thread moves 16-byte vectors, and each warp keeps several rows' loads
-// in flight so that the PCIe link, not latency, sets the pace.
+// slot (or, in the decode step, into a staging row in miss order); every thread moves
+// 16-byte vectors, and each warp keeps several rows' loads in flight so that the PCIe
+// link, not latency, sets the pace.
+//
+// hotbuf_classify + copy_staged: the decode step's split of the same work.  The
+// classify pass (which selections are resident, the misses in selection order) is all
+// the host-link fetch needs, so the fetch starts into staging rows while the victim
+// order is still being sorted; once both are done the staged rows are copied into
+// their victim slots.
 #pragma once
 #include "common.cuh"
 
@@ -24,7 +31,6 @@ struct HotbufParams {
   float* recent;
   int* slot_of_pos;
   int* sel_slot;
-  int* hit_slot;   // optional: the slot of every selected position already resident, else -1
   int* miss_pos;
   int* miss_slot;
   int* n_miss;
@@ -73,7 +79,6 @@ __global__ void __launch_bounds__(kHbThreads, 1) hotbuf_resolve_kernel(const Hot
       }
     }
     sel_slot[j] = slot;
-    if (p.hit_slot) p.hit_slot[(size_t)b * k + j] = is_miss ? -1 : slot;
     if (is_miss) {
       miss_bits |= 1u << (j - j0);
       ++my_miss;
@@ -154,6 +159,74 @@ __global__ void __launch_bounds__(kHbThreads, 1) hotbuf_resolve_kernel(const Hot
   if (tid == 0) p.n_miss[b] = n_miss;
 }
 
+struct ClassifyParams {
+  int B, k, n_slots, max_len;
+  const int* sel;
+  const int* slot_of_pos;
+  int* hit_slot;   // [B,k] the slots of the resident selections in selection order, -1 after them
+  int* n_hit;      // [B]
+  int* miss_pos;   // [B,k] the missing positions in selection order, -1 after them
+  int* miss_row;   // [B,k] i at the i-th miss, -1 after them (rows of the staging area)
+  int* n_miss;     // [B]
+};
+
+// One CTA per request; the same classification as the resolve's first phase, without
+// touching the maps.
+__global__ void __launch_bounds__(kHbThreads, 1) hotbuf_classify_kernel(const ClassifyParams p) {
+  __shared__ unsigned long long scan_tmp[32];
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int k = p.k, S = p.n_slots;
+  const int* sel = p.sel + (size_t)b * k;
+  const int* slot_of_pos = p.slot_of_pos + (size_t)b * p.max_len;
+  const int per = (k + kHbThreads - 1) / kHbThreads;  // <= 4
+  const int j0 = min(k, tid * per), j1 = min(k, j0 + per);
+  int pos[4], slot[4];
+  uint32_t n_m = 0, n_h = 0;
+  for (int j = j0; j < j1; ++j) {
+    const int q = j - j0;
+    pos[q] = sel[j];
+    slot[q] = -2;  // neither (padding or out of range)
+    if (pos[q] >= 0) {
+      if (pos[q] >= p.max_len) {
+        flag(LS_DEV_BOUNDS);
+      } else {
+        slot[q] = slot_of_pos[pos[q]];
+        if (slot[q] >= S) {
+          flag(LS_DEV_BOUNDS);
+          slot[q] = -2;
+        }
+      }
+    }
+    n_m += slot[q] == -1;
+    n_h += slot[q] >= 0;
+  }
+  // one scan of both counts: misses in the low half, hits in the high half
+  unsigned long long total;
+  const unsigned long long pre = block_excl_scan_u64(((unsigned long long)n_h << 32) | n_m, scan_tmp, &total);
+  uint32_t om = (uint32_t)pre, oh = (uint32_t)(pre >> 32);
+  for (int j = j0; j < j1; ++j) {
+    const int q = j - j0;
+    if (slot[q] == -1) {
+      p.miss_pos[(size_t)b * k + om] = pos[q];
+      p.miss_row[(size_t)b * k + om] = (int)om;
+      ++om;
+    } else if (slot[q] >= 0) {
+      p.hit_slot[(size_t)b * k + oh] = slot[q];
+      ++oh;
+    }
+  }
+  const int n_miss = (int)(uint32_t)total, n_hit = (int)(total >> 32);
+  for (int i = n_miss + tid; i < k; i += kHbThreads) {
+    p.miss_pos[(size_t)b * k + i] = -1;
+    p.miss_row[(size_t)b * k + i] = -1;
+  }
+  for (int i = n_hit + tid; i < k; i += kHbThreads) p.hit_slot[(size_t)b * k + i] = -1;
+  if (tid == 0) {
+    p.n_miss[b] = n_miss;
+    p.n_hit[b] = n_hit;
+  }
+}
+
 struct GatherParams {
   int B, k, n_slots, max_pages;
   long long row_bytes, num_pages;
@@ -163,11 +236,14 @@ struct GatherParams {
   const int* miss_slot;
   const int* n_miss;
   char* hbuf;
+  char* stage;   // optional: the i-th miss goes to staging row b*k + i (miss_slot unused)
 };
 
-// grid (ctas_per_req, B), 256 threads.  A warp owns 4 rows at a time and issues all
-// their 16-byte loads before storing any.
-__global__ void __launch_bounds__(256) gather_misses_kernel(const GatherParams p) {
+// grid (ctas_per_req, B), 128 threads and at most 64 registers each, so that a gather
+// CTA fits beside an attention CTA on one SM.  A warp owns 2 rows at a time and issues
+// all their 16-byte loads before storing any.
+constexpr int kGatherThreads = 128;
+__global__ void __launch_bounds__(kGatherThreads, 8) gather_misses_kernel(const GatherParams p) {
   const int b = blockIdx.y;
   const int warp = warp_id(), lane = lane_id();
   const int nm = p.n_miss[b];
@@ -176,8 +252,9 @@ __global__ void __launch_bounds__(256) gather_misses_kernel(const GatherParams p
     return;
   }
   const int chunks = (int)(p.row_bytes >> 4);
-  const int gw = blockIdx.x * 8 + warp, nw = gridDim.x * 8;
-  constexpr int R = 4;
+  constexpr int kWarps = kGatherThreads / 32;
+  const int gw = blockIdx.x * kWarps + warp, nw = gridDim.x * kWarps;
+  constexpr int R = 2;
   for (int i0 = gw * R; i0 < nm; i0 += nw * R) {
     const char* src[R];
     char* dst[R];
@@ -188,13 +265,14 @@ __global__ void __launch_bounds__(256) gather_misses_kernel(const GatherParams p
       const int i = i0 + q;
       if (i < nm) {
         const int pos = p.miss_pos[(size_t)b * p.k + i];
-        const int slot = p.miss_slot[(size_t)b * p.k + i];
+        const int slot = p.stage ? 0 : p.miss_slot[(size_t)b * p.k + i];
         const int lp = pos >> 6;
         if (pos >= 0 && lp < p.max_pages && slot >= 0 && slot < p.n_slots) {
           const int page = p.page_table[(size_t)b * p.max_pages + lp];
           if (page >= 0 && page < p.num_pages) {
             src[q] = p.host + ((long long)page * 64 + (pos & 63)) * p.row_bytes;
-            dst[q] = p.hbuf + ((long long)b * p.n_slots + slot) * p.row_bytes;
+            dst[q] = p.stage ? p.stage + ((long long)b * p.k + i) * p.row_bytes
+                             : p.hbuf + ((long long)b * p.n_slots + slot) * p.row_bytes;
           } else {
             flag(LS_DEV_BOUNDS);
           }
@@ -220,6 +298,31 @@ __global__ void __launch_bounds__(256) gather_misses_kernel(const GatherParams p
           if (dst[q] && c < chunks) *(uint4*)(dst[q] + (size_t)c * 16) = v[q][e];
         }
     }
+  }
+}
+
+struct StageCopyParams {
+  int B, k, n_slots;
+  long long row_bytes;
+  const char* stage;     // [B,k,row_bytes]: the i-th miss of request b at row b*k + i
+  const int* miss_slot;  // [B,k] the i-th miss's victim slot (-1: none)
+  const int* n_miss;     // [B]
+  char* hbuf;            // [B,n_slots,row_bytes]
+};
+
+// grid (ctas_per_req, B), 256 threads: a warp per row, 16-byte vectors.
+__global__ void __launch_bounds__(256) copy_staged_kernel(const StageCopyParams p) {
+  const int b = blockIdx.y;
+  const int nm = p.n_miss[b];
+  if (nm < 0 || nm > p.k) return;  // the resolve has flagged it
+  const int chunks = (int)(p.row_bytes >> 4);
+  const int gw = blockIdx.x * 8 + warp_id(), nw = gridDim.x * 8, lane = lane_id();
+  for (int i = gw; i < nm; i += nw) {
+    const int slot = p.miss_slot[(size_t)b * p.k + i];
+    if (slot < 0 || slot >= p.n_slots) continue;  // out of capacity: flagged by the resolve
+    const uint4* src = (const uint4*)(p.stage + ((long long)b * p.k + i) * p.row_bytes);
+    uint4* dst = (uint4*)(p.hbuf + ((long long)b * p.n_slots + slot) * p.row_bytes);
+    for (int c = lane; c < chunks; c += 32) dst[c] = src[c];
   }
 }
 

@@ -143,10 +143,12 @@ def kernels_per_step(wl: DecodeWorkload, *, c2f: bool, hotbuf: bool, mla: bool) 
     """How many of the library's kernels one ls_decode_step launches."""
     # indexer + top-k; coarse-to-fine: bound, top-k, phase 1, rescore, top-k, survivors, rescore, top-k
     n = 8 if c2f else 2
-    if hotbuf:
-        n += 2
     if mla and hotbuf:
-        n += 3   # resident-row pass, miss pass, merge of both passes
+        # classify, resolve, gather into staging, staged rows into slots; resident-row
+        # pass, miss pass, merge of both passes
+        n += 4 + 3
+    elif hotbuf:
+        n += 2 + 1   # resolve, gather; attention
     elif mla:
         n += 2 if B.ls_sparse_attn_workspace_size(wl.args.attn) > 0 else 1
     else:
