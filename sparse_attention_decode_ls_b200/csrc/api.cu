@@ -138,12 +138,13 @@ ls_status make_tmap_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_
 
 // 2D bf16 rows [rows][inner] (row stride in bytes), one-row boxes of 64 elements (128
 // bytes), 128-byte swizzle: row gathers (tile::gather4) into K-major operand panels.
-ls_status make_tmap_bf16_rows(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t stride) {
+ls_status make_tmap_bf16_rows(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t stride,
+                              uint32_t box_rows = 1) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(LS_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {stride};
-  cuuint32_t box[2] = {64, 1};
+  cuuint32_t box[2] = {64, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
@@ -413,7 +414,6 @@ ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressi
     }
     if (allow_smem(ls::attn_mla_tc, ls::mla::kSmem, g_smem_attn_tc) != cudaSuccess)
       return check_launch("attn_mla_tc attribute");
-    p.early_q = pdl ? 1 : 0;
     cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = pdl_config(dim3(2 * ns, a->batch), dim3(ls::mla::kThreads), ls::mla::kSmem, st, attr, pdl);
     // the two CTAs of an (request, split) pair form a cluster
@@ -424,7 +424,10 @@ ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressi
     cfg.numAttrs += 1;
     CUtensorMap kv_map;
     LS_TRY(make_tmap_bf16_rows(&kv_map, p.krows, ls::mla::DK, (uint64_t)num_rows, (uint64_t)a->row_stride * 2));
-    cudaError_t e = cudaLaunchKernelEx(&cfg, ls::attn_mla_tc, p, kv_map);
+    CUtensorMap q_map;  // [B*128 heads, 576] bf16, one 128-head x 64-dim box per panel
+    LS_TRY(make_tmap_bf16_rows(&q_map, p.q, ls::mla::DK, (uint64_t)a->batch * ls::mla::H, ls::mla::DK * 2,
+                               ls::mla::H));
+    cudaError_t e = cudaLaunchKernelEx(&cfg, ls::attn_mla_tc, p, kv_map, q_map);
     if (e != cudaSuccess) return fail(LS_ERR_CUDA, "attn_mla_tc: %s", cudaGetErrorString(e));
     LS_TRY(check_launch("attn_mla_tc"));
     if (total > 1 && combine) {

@@ -40,7 +40,6 @@ struct AttnParams {
   int nsplit;
   float* part_o;     // [B,nsplit,dv/4,H,4] unnormalised partial outputs (4-dim granules, head next)
   float* part_ml;    // [B,nsplit,H,2] running max (log2 domain) and sum
-  int early_q;       // tensor-core kernel: read Q before waiting for the kernel before
   int split_base;    // tensor-core kernel: this launch's splits are partial slots
   int nsplit_total;  //   [split_base, split_base + nsplit) of nsplit_total per request
   int compacted;     // the valid entries of every request's selection come first
@@ -164,8 +163,12 @@ constexpr int kSBufs = 1;
 constexpr int kTmemS = DVH, kTmemP = kTmemS + kSBufs * N, kTmemQ = kTmemP + N / 2;
 static_assert(kTmemQ + 5 * 32 <= 512, "TMEM budget");
 // kv_full[kStages] kv_empty[kStages] s_full[kSBufs] s_read[kSBufs] x_full[2] x_free[2]
-// x_read[2] p_full p_free o_done q_full
-constexpr int kNumBars = 2 * kStages + 2 * kSBufs + 2 + 2 + 2 + 4;
+// x_read[2] p_full p_free o_done q_full q_tma
+constexpr int kNumBars = 2 * kStages + 2 * kSBufs + 2 + 2 + 2 + 5;
+// Q arrives by TMA (one 128-head x 64-dim box per panel, 128-byte swizzle) in the KV
+// stage buffers, which the row gathers use only once Q has moved on into TMEM
+constexpr int kQPanelBytes = H * 128;
+static_assert(5 * kQPanelBytes <= kStages * kStageBytes, "Q staging fits the KV stages");
 constexpr int kOffTmem = kOffBar + kNumBars * 8;
 constexpr int kSmem = 1024 + kOffTmem + 16;
 // warps 0-3 softmax and 4-7 S senders (warp w reads TMEM lanes 32(w%4) .. +31),
@@ -185,17 +188,19 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 }  // namespace mla
 
-// This rank's Q panels (head h's row) into TMEM lane h as the MMA's A operand: 64 dims
-// = 32 columns per panel, two bf16 per column.  Every thread of warps 0-3, converged.
-__device__ __forceinline__ void load_q_tmem(const AttnParams& p, int b, int rank, int h, uint32_t t_row) {
+// This rank's Q panels (head h's row), staged in shared memory by TMA (128-byte swizzle:
+// 16-byte chunk j of row h sits at chunk j ^ (h & 7)), into TMEM lane h as the MMA's A
+// operand: 64 dims = 32 columns per panel, two bf16 per column.  Every thread of warps
+// 0-3, converged.
+__device__ __forceinline__ void load_q_tmem(const uint8_t* q_smem, int rank, int h, uint32_t t_row) {
   using namespace mla;
-  const uint4* src = (const uint4*)((const char*)p.q + ((size_t)b * H + h) * DK * 2 + rank * s_panels(0) * 128);
 #pragma unroll 1
   for (int c = 0; c < s_panels(rank); ++c) {
+    const uint4* row = (const uint4*)(q_smem + c * kQPanelBytes + h * 128);
     float f[32];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const uint4 v = src[c * 8 + j];
+      const uint4 v = row[j ^ (h & 7)];
       f[4 * j] = __uint_as_float(v.x);
       f[4 * j + 1] = __uint_as_float(v.y);
       f[4 * j + 2] = __uint_as_float(v.z);
@@ -215,7 +220,8 @@ __device__ __forceinline__ void load_q_tmem(const AttnParams& p, int b, int rank
 // head).  P goes to shared memory as bf16 and O_half += P V_half accumulates in TMEM
 // (256 columns).
 __global__ void __launch_bounds__(mla::kThreads, 1)
-    attn_mla_tc(const AttnParams p, const __grid_constant__ CUtensorMap kv_map) {
+    attn_mla_tc(const AttnParams p, const __grid_constant__ CUtensorMap kv_map,
+                const __grid_constant__ CUtensorMap q_map) {
   using namespace mla;
   extern __shared__ uint8_t sm_raw_a[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)sm_raw_a + 1023) & ~(uintptr_t)1023);
@@ -231,6 +237,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   uint64_t* p_free = p_full + 1;
   uint64_t* o_done = p_full + 2;
   uint64_t* q_full = p_full + 3;
+  uint64_t* q_tma = p_full + 4;
   uint32_t* tmem_slot = (uint32_t*)(sm + kOffTmem);
   __shared__ int s_abort;
   __shared__ uint64_t s_mask[kStages];  // valid rows of the tile in each stage
@@ -265,31 +272,65 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     mbar_init(p_full, 128);
     mbar_init(p_free, 1);
     mbar_init(o_done, 1);
-    mbar_init(q_full, 128);  // the softmax threads, once Q is in TMEM
+    mbar_init(q_full, 128);  // the softmax threads, once Q is in TMEM (and out of the stages)
+    mbar_init(q_tma, 1);
     s_abort = 0;
     fence_mbar_init();
+    // Q is an input of the step, never written by the kernel before: fetch it at once
+    if (my_tiles_max > 0) {
+      mbar_arrive_expect_tx(q_tma, s_panels(rank) * kQPanelBytes);
+      for (int c = 0; c < s_panels(rank); ++c)
+        tma_load_2d(sbase + kOffKv + c * kQPanelBytes, &q_map, q_tma, (rank * s_panels(0) + c) * 64, b * H);
+    }
     // arm the receive buffers for tiles 0 and 1 before the other CTA can send (an armed
     // buffer that no tile uses is never waited on)
     for (int s = 0; s < 2 && s < my_tiles_max; ++s) mbar_arrive_expect_tx(&x_full[s], kXBytes);
   }
   if (warp == kMmaWarp) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
-  cluster_sync_all();  // both CTAs' barriers exist before any remote arrival
+  __syncthreads();
+  // the other CTA may address this one's barriers and receive buffers once it has seen
+  // this arrival; only the warps that write to the other CTA wait for it early (the rest
+  // wait before the final barrier), so the row gathers need not
+  cluster_arrive();
+  bool cluster_waited = false;
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tm_o = tmem;          // columns [0, 256): O half
   const uint32_t tm_s = tmem + kTmemS;  // kSBufs S tiles
   const uint32_t tm_p = tmem + kTmemP;  // P of the current tile, bf16 pairs (PV's A operand)
   const uint32_t tm_q = tmem + kTmemQ;  // this rank's Q panels
-  if (warp < 4 && p.early_q && my_tiles_max > 0) {  // Q is not written by the kernel before
-    load_q_tmem(p, b, rank, threadIdx.x, tm_q + ((uint32_t)(warp * 32) << 16));
-    tc_fence_before();
+  if (warp < 4 && my_tiles_max > 0) {
+    // a wait that gives up (recorded in the device status) aborts the whole CTA
+    if (mbar_wait(q_tma, 0)) {
+      load_q_tmem(sm + kOffKv, rank, threadIdx.x, tm_q + ((uint32_t)(warp * 32) << 16));
+      tc_fence_before();
+    } else if (threadIdx.x == 0) {
+      s_abort = 1;
+    }
     mbar_arrive(q_full);
+  }
+  if (warp >= kLoadWarp0 && p.addressing == LS_ROWS_PAGED) {
+    // the page table is an input of the step: warm its rows for this request in L2
+    const int* pt = p.page_table + (size_t)b * p.max_pages;
+    for (int i = ((warp - kLoadWarp0) * 32 + lane) * 32; i < p.max_pages; i += kLoadWarps * 32 * 32)
+      prefetch_l2(pt + i);
   }
   // under programmatic dependent launch everything above overlaps the kernel before;
   // the selection, the rows and the outputs are touched only after it has finished
   griddep_wait();
   griddep_launch_dependents();
+  // the gather warps load the selections of their first rows (for the usual tile range)
+  // while the tile range is settled below, so that the two loads overlap
+  constexpr int kRStep = kLoadWarps * 32;
+  int spec_sv[4];
+  if (warp >= kLoadWarp0) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = (warp - kLoadWarp0) * 32 + lane + u * kRStep, j = t0 * N + r;
+      spec_sv[u] = (r < my_tiles0 * N && j < p.k) ? p.sel[(size_t)b * p.k + j] : -1;
+    }
+  }
   // in a compacted selection a share that starts with padding holds no row at all (the
   // tail of a miss list): such a CTA only writes an empty partial
   int tb = t0, my_tiles = my_tiles0;
@@ -316,17 +357,28 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     // resolve all of this CTA's rows once (out-of-range marker: one past the pool)
     int* s_rows = (int*)(sm + kOffRows);
     const int nrows = my_tiles * N;
-    for (int r = lw * 32 + lane; r < nrows; r += kLoadWarps * 32) {
-      const int j = tb * N + r;
-      const long long row = j < p.k ? attn_row(p, b, p.sel[(size_t)b * p.k + j]) : -1;
-      s_rows[r] = row >= 0 ? (int)row : (int)p.num_rows;
+    for (int r0 = lw * 32 + lane; r0 < nrows; r0 += 4 * kRStep) {
+      int sv[4];  // four rows' selections, then their page-table lookups, in flight together
+      const bool spec = r0 < kRStep && tb == t0 && my_tiles <= my_tiles0;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int r = r0 + u * kRStep, j = tb * N + r;
+        sv[u] = (r < nrows && j < p.k) ? (spec ? spec_sv[u] : p.sel[(size_t)b * p.k + j]) : -1;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int r = r0 + u * kRStep;
+        const long long row = attn_row(p, b, sv[u]);
+        if (r < nrows) s_rows[r] = row >= 0 ? (int)row : (int)p.num_rows;
+      }
     }
     asm volatile("bar.sync 1, %0;" ::"n"(kLoadWarps * 32) : "memory");  // the gather warps only
     for (int i = 0; i < my_tiles; ++i) {
       const int st = i % kStages;
       int go = 1;
       if (lane == 0) {  // one lane decides, so the warp stays converged
-        go = (i < kStages) || mbar_wait(&kv_empty[st], ((i / kStages) - 1) & 1);
+        // the first tiles land where Q was staged: only once Q is in TMEM
+        go = i >= kStages ? mbar_wait(&kv_empty[st], ((i / kStages) - 1) & 1) : (i > 0 || mbar_wait(q_full, 0));
         if (*(volatile int*)&s_abort) go = 0;
         if (!go) s_abort = 1;
       }
@@ -356,6 +408,8 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     // Once this CTA's softmax has read receive buffer b (tile j), re-arm its barrier for
     // tile j + 2 and tell the other CTA's senders they may write it.  The remote arrival
     // (a cluster-scope release) is slow, so it is kept off the softmax warps.
+    cluster_wait();
+    cluster_waited = true;
     if (lane == 0) {
       const uint32_t xfree_peer = dsmem_map(smem_u32(x_free), (uint32_t)(rank ^ 1));
       for (int j = 0; j + 2 < my_tiles; ++j) {
@@ -443,6 +497,8 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     // warp's 16-byte accesses are consecutive
     const uint32_t x_peer = dsmem_map(sbase + kOffX, peer);
     const uint32_t xfull_peer = dsmem_map(smem_u32(x_full), peer);
+    cluster_wait();
+    cluster_waited = true;
     for (int i = 0; i < my_tiles; ++i) {
       const int sb = i % kSBufs, xb = i & 1;
       if (!mbar_wait(&s_full[sb], (i / kSBufs) & 1)) break;
@@ -463,11 +519,6 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     const int h = warp * 32 + lane;
     const float sl2 = p.scale * kLog2e;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    if (!p.early_q && my_tiles > 0) {
-      load_q_tmem(p, b, rank, h, tm_q + lane_off);
-      tc_fence_before();
-      mbar_arrive(q_full);
-    }
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int i = 0; i < my_tiles; ++i) {
@@ -595,6 +646,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   // The cluster-wide barrier also keeps this CTA's shared memory alive until the other
   // CTA has made its last remote write and arrival; only then may TMEM be released.
   __syncwarp();
+  if (!cluster_waited) cluster_wait();
   tc_fence_before();
   cluster_sync_all();
   if (warp == kMmaWarp) {
