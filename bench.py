@@ -287,9 +287,12 @@ def run_ours(args):
     # inside a flushed step the events also enclose the launch gap before the kernel)
     t = wl.tensors
     scores = torch.empty((BATCH, wl.args.index.max_len), dtype=torch.float32, device="cuda")
-    def run_indexer():
-        B.ls_index_score(q=t["i_q"], w=t["i_w"], key_pool=t["i_key_pool"], page_table=t["i_page_table"],
-                         lens=t["i_lens"], scores=scores, q_scale=t["i_q_scale"], key_scale=t["i_key_scale"])
+    ia = B.index_args(q=t["i_q"], w=t["i_w"], key_pool=t["i_key_pool"], page_table=t["i_page_table"],
+                      lens=t["i_lens"], scores=scores, q_scale=t["i_q_scale"], key_scale=t["i_key_scale"])
+    lib, ia_ref, st_handle = B.lib(), B.C.byref(ia), stream.cuda_stream
+    def run_indexer():  # arguments built once: the host keeps ahead of the GPU
+        if lib.ls_index_score(ia_ref, st_handle) != 0:
+            raise RuntimeError(lib.ls_get_error_string().decode())
     for _ in range(Wm):
         run_indexer()
     kb = new_events(2)
