@@ -180,6 +180,15 @@ ls_status ls_build_block_summaries(const ls_index_score_args* keys, uint8_t* sum
  * indexer (heads 64, dim 128).  idx/sel_score as in ls_topk_select.  survivors
  * receives each request's surviving block ids (ascending), n_survivors the count.
  * Needs a workspace of ls_block_bound_prune_workspace_size() bytes (256-aligned).
+ *
+ * Host-resident original keys (LeanSparse, abstract: keeping the full indexer keys
+ * on the GPU limits decode concurrency): with keys_on_host != 0, index.key_pool and
+ * index.key_scale are pinned host memory (cudaHostAlloc / cudaHostRegister, device-
+ * accessible); only the summaries stay in HBM.  Steps 2 and 4 first copy the listed
+ * blocks' keys and scales (8,448 bytes per block) over the host link into workspace
+ * staging of stage_blocks blocks per request, then score them there; survivors beyond
+ * stage_blocks take further passes of the same size.  The result is identical to
+ * keys in HBM.
  * --------------------------------------------------------------------------- */
 typedef struct ls_block_bound_prune_args {
   ls_index_score_args index;  /* a1 inputs; index.scores is ignored */
@@ -194,6 +203,9 @@ typedef struct ls_block_bound_prune_args {
   int32_t* survivors;         /* [B,max_blocks] out */
   int32_t* n_survivors;       /* [B] out */
   float* ub;                  /* [B,max_blocks] out, may be NULL */
+  int32_t keys_on_host;       /* != 0: index.key_pool / key_scale are pinned host memory */
+  int32_t stage_blocks;       /* keys_on_host: staging blocks per request and pass
+                                 (0 = 2048; at least ceil(k/64)+1 are used) */
 } ls_block_bound_prune_args;
 
 size_t ls_block_bound_prune_workspace_size(const ls_block_bound_prune_args* args);
@@ -358,6 +370,8 @@ typedef struct ls_decode_step_args {
   const float* block_scale;
   int32_t* survivors;         /* c2f: [B,max_blocks] out, may be NULL (workspace) */
   int32_t* n_survivors;       /* c2f: [B] out, may be NULL (workspace) */
+  int32_t c2f_keys_on_host;   /* c2f: keys_on_host / stage_blocks of ls_block_bound_prune_args */
+  int32_t c2f_stage_blocks;
   ls_sparse_attn_args attn;
   int32_t use_hotbuf;
   int32_t n_slots;

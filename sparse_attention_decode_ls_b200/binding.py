@@ -38,7 +38,7 @@ class TopkArgs(C.Structure):
 class BlockBoundPruneArgs(C.Structure):
     _fields_ = [("index", IndexScoreArgs), ("k", _i32), ("max_blocks", _i32), ("eps_rel", _f32),
                 ("summaries", _p), ("block_scale", _p), ("idx", _p), ("sel_score", _p), ("survivors", _p),
-                ("n_survivors", _p), ("ub", _p)]
+                ("n_survivors", _p), ("ub", _p), ("keys_on_host", _i32), ("stage_blocks", _i32)]
 
 
 class HotbufArgs(C.Structure):
@@ -63,7 +63,8 @@ class SparseAttnArgs(C.Structure):
 class DecodeStepArgs(C.Structure):
     _fields_ = [("index", IndexScoreArgs), ("k", _i32), ("use_c2f", _i32), ("max_blocks", _i32),
                 ("eps_rel", _f32), ("summaries", _p), ("block_scale", _p), ("survivors", _p),
-                ("n_survivors", _p), ("attn", SparseAttnArgs), ("use_hotbuf", _i32), ("n_slots", _i32),
+                ("n_survivors", _p), ("c2f_keys_on_host", _i32), ("c2f_stage_blocks", _i32),
+                ("attn", SparseAttnArgs), ("use_hotbuf", _i32), ("n_slots", _i32),
                 ("pos_of_slot", _p), ("recent_score", _p), ("slot_of_pos", _p), ("host_kv", _p),
                 ("host_num_pages", _i64), ("hbuf", _p), ("n_miss", _p), ("idx", _p), ("sel_score", _p),
                 ("events", _p)]
@@ -209,8 +210,12 @@ def ls_build_block_summaries(*, q, w, key_pool, key_scale, q_scale, page_table, 
 
 
 def c2f_args(*, index: IndexScoreArgs, k, summaries, block_scale, idx, sel_score=None, survivors=None,
-             n_survivors=None, ub=None, eps_rel=0.0) -> BlockBoundPruneArgs:
+             n_survivors=None, ub=None, eps_rel=0.0, keys_on_host=False, stage_blocks=0) -> BlockBoundPruneArgs:
+    """keys_on_host: index's key_pool / key_scale are pinned CPU tensors (only the summaries
+    are on the GPU); stage_blocks: staging capacity per request and pass (0: default)."""
     a = BlockBoundPruneArgs()
+    a.keys_on_host = 1 if keys_on_host else 0
+    a.stage_blocks = stage_blocks
     a.index = index
     a.k = k
     a.max_blocks = summaries.shape[1]
@@ -297,7 +302,8 @@ def ls_sparse_attn_decode_noalloc(a: SparseAttnArgs, stream=None):
 # ------------------------------------------------------------------------------- a7
 def decode_step_args(*, index: IndexScoreArgs, k, attn: SparseAttnArgs, c2f=None, hotbuf=None, idx=None,
                      sel_score=None, events=None) -> DecodeStepArgs:
-    """c2f: dict(summaries, block_scale, survivors=None, n_survivors=None, eps_rel=0.0);
+    """c2f: dict(summaries, block_scale, survivors=None, n_survivors=None, eps_rel=0.0,
+    keys_on_host=False, stage_blocks=0);
     hotbuf: dict(pos_of_slot, recent_score, slot_of_pos, host_kv, hbuf, n_miss=None).
     events: optional ctypes array of 6 cudaEvent_t handles."""
     a = DecodeStepArgs()
@@ -310,6 +316,8 @@ def decode_step_args(*, index: IndexScoreArgs, k, attn: SparseAttnArgs, c2f=None
         a.eps_rel = c2f.get("eps_rel", 0.0)
         a.summaries, a.block_scale = _ptr(c2f["summaries"]), _ptr(c2f["block_scale"])
         a.survivors, a.n_survivors = _ptr(c2f.get("survivors")), _ptr(c2f.get("n_survivors"))
+        a.c2f_keys_on_host = 1 if c2f.get("keys_on_host") else 0
+        a.c2f_stage_blocks = int(c2f.get("stage_blocks", 0))
     if hotbuf is not None:
         a.use_hotbuf = 1
         a.n_slots = hotbuf["pos_of_slot"].shape[1]

@@ -206,8 +206,12 @@ ls_status launch_index_simt(const ls_index_score_args* a, cudaStream_t st) {
 // tcgen05 tile engine over keys (mode 0) or block summaries (mode 1).
 ls_status launch_index_tc(const ls_index_score_args* a, int mode, const int* unit_list, const int* unit_count,
                           int list_stride, float* out, long long out_stride, const uint8_t* summ,
-                          const float* bscale, int max_blocks, float* out_plain, float eps_rel, cudaStream_t st) {
+                          const float* bscale, int max_blocks, float* out_plain, float eps_rel, cudaStream_t st,
+                          int staged_base = -1, int stage_cap = 0) {
   ls::IdxTcParams p{};
+  p.staged = staged_base >= 0 ? 1 : 0;  // list entries [staged_base, + stage_cap) from staging units
+  p.unit_base = staged_base >= 0 ? staged_base : 0;
+  p.stage_cap = stage_cap;
   p.mode = mode; p.B = a->batch; p.max_pages = a->max_pages; p.max_len = a->max_len; p.max_blocks = max_blocks;
   p.num_pages = a->num_pages; p.q8 = (const uint8_t*)a->q; p.qs = a->q_scale; p.w = a->w;
   p.w_bf16 = a->w_dtype == LS_BF16; p.page_table = a->page_table; p.lens = a->lens;
@@ -219,7 +223,8 @@ ls_status launch_index_tc(const ls_index_score_args* a, int mode, const int* uni
   if (mode == 0) {
     p.row_scale = a->key_scale;
     LS_TRY(make_tmap_u8(&tmap, a->key_pool, 128, (uint64_t)a->num_pages * 64, 128));
-    max_units = unit_list ? list_stride : (a->max_len + 63) / 64;
+    max_units = unit_list ? (staged_base >= 0 ? std::min(list_stride, stage_cap) : list_stride)
+                          : (a->max_len + 63) / 64;
   } else {
     p.row_scale = bscale;
     LS_TRY(make_tmap_u8(&tmap, summ, 256, (uint64_t)a->batch * max_blocks, 256));
@@ -544,8 +549,9 @@ ls_status launch_copy_staged(const ls_gather_args* g, const void* stage, cudaStr
 
 // ---- coarse-to-fine ---------------------------------------------------------------------
 struct C2fLayout {
-  int nb0, ub_stride;
-  size_t off_ub, off_blk, off_cnt1, off_clen1, off_tau, off_clen2, off_nsurv, off_surv, off_c1, off_c2, total;
+  int nb0, ub_stride, cap;
+  size_t off_ub, off_blk, off_cnt1, off_clen1, off_tau, off_clen2, off_nsurv, off_surv, off_c1, off_c2, off_skeys,
+      off_sscales, total;
 };
 
 C2fLayout c2f_layout(const ls_block_bound_prune_args* a) {
@@ -565,6 +571,12 @@ C2fLayout c2f_layout(const ls_block_bound_prune_args* a) {
   l.off_surv = take((size_t)B * a->max_blocks * 4);
   l.off_c1 = take((size_t)B * l.nb0 * 64 * 4);
   l.off_c2 = take((size_t)B * a->max_blocks * 64 * 4);
+  l.cap = 0;
+  if (a->keys_on_host) {  // staging for the keys fetched from the host, per pass
+    l.cap = std::min(a->max_blocks, std::max(l.nb0, a->stage_blocks > 0 ? a->stage_blocks : 2048));
+    l.off_skeys = take((size_t)B * l.cap * 8192);
+    l.off_sscales = take((size_t)B * l.cap * 256);
+  }
   l.total = o;
   return l;
 }
@@ -578,7 +590,47 @@ ls_status validate_c2f(const ls_block_bound_prune_args* a) {
   LS_REQUIRE((long long)a->max_blocks * 64 <= (1ll << 30), "max_blocks too large");
   LS_REQUIRE(a->summaries && a->block_scale && a->idx, "summaries, block_scale and idx are required");
   LS_REQUIRE(aligned16(a->summaries), "summaries must be 16-byte aligned");
+  LS_REQUIRE(a->stage_blocks >= 0, "stage_blocks must be >= 0");
   return LS_OK;
+}
+
+// Device addresses of host-resident keys and scales: both must be pinned host memory.
+ls_status host_key_ptrs(const ls_index_score_args* ix, const uint8_t** keys, const float** scales) {
+  const void* src[2] = {ix->key_pool, ix->key_scale};
+  void* dev[2] = {nullptr, nullptr};
+  for (int i = 0; i < 2; ++i) {
+    cudaPointerAttributes at{};
+    if (cudaPointerGetAttributes(&at, src[i]) != cudaSuccess || at.type != cudaMemoryTypeHost || !at.devicePointer) {
+      cudaGetLastError();
+      return fail(LS_ERR_INVALID_ARG, "keys_on_host: index.%s is not pinned host memory",
+                  i == 0 ? "key_pool" : "key_scale");
+    }
+    dev[i] = at.devicePointer;
+  }
+  *keys = (const uint8_t*)dev[0];
+  *scales = (const float*)dev[1];
+  return LS_OK;
+}
+
+// List entries [base, base + cap) of each request: their keys over the host link into
+// staging, then their exact scores into out (at the entries' own positions).
+ls_status fetch_and_score(const ls_index_score_args* ix, const uint8_t* hkeys, const float* hscales,
+                          const int* list, const int* count, int list_stride, int base, int cap, uint8_t* skeys,
+                          float* sscales, float* out, long long out_stride, cudaStream_t st) {
+  ls::FetchParams f{};
+  f.B = ix->batch; f.max_pages = ix->max_pages; f.list_stride = list_stride; f.base = base; f.cap = cap;
+  f.num_pages = ix->num_pages; f.host_keys = hkeys; f.host_scales = hscales; f.page_table = ix->page_table;
+  f.list = list; f.count = count; f.stage_keys = skeys; f.stage_scales = sscales;
+  // small CTAs on about a quarter of the SMs keep enough loads in flight for the link
+  const int g = std::max(1, std::min((cap + 3) / 4, device_sms() / (4 * ix->batch)));
+  ls::fetch_blocks_kernel<<<dim3(g, ix->batch), 128, 0, st>>>(f);
+  LS_TRY(check_launch("fetch_blocks"));
+  ls_index_score_args tmp = *ix;
+  tmp.key_pool = skeys;
+  tmp.key_scale = sscales;
+  tmp.num_pages = (int64_t)ix->batch * cap;
+  return launch_index_tc(&tmp, 0, list, count, list_stride, out, out_stride, nullptr, nullptr, 0, nullptr, 0.f, st,
+                         base, cap);
 }
 
 ls_status run_c2f(const ls_block_bound_prune_args* a, void* ws, size_t ws_bytes, int* survivors, int* n_surv,
@@ -600,6 +652,11 @@ ls_status run_c2f(const ls_block_bound_prune_args* a, void* ws, size_t ws_bytes,
   const ls_index_score_args* ix = &a->index;
   const int B = ix->batch;
   const float eps = a->eps_rel > 0.f ? a->eps_rel : 1.0f / 1024.0f;
+  const uint8_t* hkeys = nullptr;
+  const float* hscales = nullptr;
+  uint8_t* skeys = (uint8_t*)(w + l.off_skeys);
+  float* sscales = (float*)(w + l.off_sscales);
+  if (a->keys_on_host) LS_TRY(host_key_ptrs(ix, &hkeys, &hscales));
   // 1. block bounds (+ margin) over the summaries
   LS_TRY(launch_index_tc(ix, 1, nullptr, nullptr, 0, ub, l.ub_stride, a->summaries, a->block_scale, a->max_blocks,
                          a->ub, eps, st));
@@ -609,16 +666,29 @@ ls_status run_c2f(const ls_block_bound_prune_args* a, void* ws, size_t ws_bytes,
   ls::c2f_phase1_kernel<<<(B + 127) / 128, 128, 0, st>>>(B, l.nb0, ix->lens, blk, cnt1, clen1);
   LS_TRY(check_launch("c2f_phase1"));
   // 3. their exact scores; tau0 = the k-th largest
-  LS_TRY(launch_index_tc(ix, 0, blk, cnt1, l.nb0, c1, (long long)l.nb0 * 64, nullptr, nullptr, 0, nullptr, 0.f,
-                         st));
+  if (a->keys_on_host) {
+    LS_TRY(fetch_and_score(ix, hkeys, hscales, blk, cnt1, l.nb0, 0, l.cap, skeys, sscales, c1, (long long)l.nb0 * 64,
+                           st));
+  } else {
+    LS_TRY(launch_index_tc(ix, 0, blk, cnt1, l.nb0, c1, (long long)l.nb0 * 64, nullptr, nullptr, 0, nullptr, 0.f,
+                           st));
+  }
   LS_TRY(launch_topk(B, a->k, c1, l.nb0 * 64, clen1, 1, 1, l.nb0 * 64, nullptr, 0, nullptr, nullptr, tau, st));
   // 4. survivors
   ls::c2f_survivors_kernel<<<B, 1024, 0, st>>>(B, a->max_blocks, l.ub_stride, ix->lens, ub, tau, survivors, n_surv,
                                                clen2);
   LS_TRY(check_launch("c2f_survivors"));
   // 5. exact scores of the survivors, then the top-k over them
-  LS_TRY(launch_index_tc(ix, 0, survivors, n_surv, a->max_blocks, c2, (long long)a->max_blocks * 64, nullptr,
-                         nullptr, 0, nullptr, 0.f, st));
+  if (a->keys_on_host) {
+    // the survivors through the staging, stage-capacity blocks per pass (a pass past a
+    // request's survivor count does nothing for it)
+    for (int base = 0; base < a->max_blocks; base += l.cap)
+      LS_TRY(fetch_and_score(ix, hkeys, hscales, survivors, n_surv, a->max_blocks, base, l.cap, skeys, sscales, c2,
+                             (long long)a->max_blocks * 64, st));
+  } else {
+    LS_TRY(launch_index_tc(ix, 0, survivors, n_surv, a->max_blocks, c2, (long long)a->max_blocks * 64, nullptr,
+                           nullptr, 0, nullptr, 0.f, st));
+  }
   if (ev_topk) cudaEventRecord((cudaEvent_t)ev_topk, st);
   LS_TRY(launch_topk(B, a->k, c2, a->max_blocks * 64, clen2, 1, 1, a->max_blocks * 64, survivors, a->max_blocks,
                      a->idx, a->sel_score, nullptr, st));
@@ -644,6 +714,8 @@ ls_block_bound_prune_args step_c2f_args(const ls_decode_step_args* a, int* idx, 
   c.survivors = a->survivors;
   c.n_survivors = a->n_survivors;
   c.ub = nullptr;
+  c.keys_on_host = a->c2f_keys_on_host;
+  c.stage_blocks = a->c2f_stage_blocks;
   return c;
 }
 

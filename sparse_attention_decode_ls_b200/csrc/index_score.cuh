@@ -112,6 +112,9 @@ struct IdxTcParams {
   long long out_stride;
   float* out_plain;        // mode 1: bound without margin, [B,max_blocks] (may be NULL)
   float eps_rel;           // mode 1: margin relative to the block magnitude bound
+  int staged;              // mode 0 list: entries [unit_base, unit_base + stage_cap) of the list,
+  int unit_base;           //   whose keys were copied to staging units b * stage_cap + (entry -
+  int stage_cap;           //   unit_base) of the pool (key_pool / row_scale point at the staging)
 };
 
 template <int KP, int NCOL>
@@ -140,9 +143,10 @@ __device__ __forceinline__ int idx_unit_row(const IdxTcParams& p, int b, int u, 
     *lp_out = u;
     return b * p.max_blocks + u * 64;
   }
-  int lp = p.unit_list ? p.unit_list[(size_t)b * p.list_stride + u] : u;
+  int lp = p.unit_list ? p.unit_list[(size_t)b * p.list_stride + p.unit_base + u] : u;
   *lp_out = lp;
   if (lp < 0 || lp >= p.max_pages) return -1;
+  if (p.staged) return (b * p.stage_cap + u) * 64;
   const int page = p.page_table[(size_t)b * p.max_pages + lp];
   if (page < 0 || page >= p.num_pages) return -1;
   return page * 64;
@@ -190,6 +194,7 @@ __global__ void __launch_bounds__(192, 1)
       if (cta == 0 && tid == 0) flag(LS_DEV_BOUNDS);
       return;
     }
+    if (p.staged) n_units = min(max(n_units - p.unit_base, 0), p.stage_cap);  // this pass's window
   } else {
     n_units = (L + 63) >> 6;
   }
@@ -402,7 +407,7 @@ __global__ void __launch_bounds__(192, 1)
       } else if (lp >= 0 && lp * 64 + rr < L) {
         valid = true;
         scale = s_scale[st * 128 + r];
-        out_idx = p.unit_list ? (long long)u * 64 + rr : (long long)lp * 64 + rr;
+        out_idx = p.unit_list ? (long long)(p.unit_base + u) * 64 + rr : (long long)lp * 64 + rr;
       }
       if (!mbar_wait(&accf[a], (i / C::kAcc) & 1)) { s_abort = 1; break; }
       tc_fence_after();
@@ -447,6 +452,49 @@ __global__ void __launch_bounds__(192, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
+  }
+}
+
+// Host-resident keys: copy the keys (64 x 128 e4m3 = 8 KB) and token scales (256 B) of
+// list entries [base, base + cap) of each request from pinned host memory (zero-copy
+// reads over the host link) to staging units b * cap + (entry - base).  grid (ctas, B),
+// 128 threads; a warp per block, all of its 16-byte loads in flight before any store.
+struct FetchParams {
+  int B, max_pages, list_stride, base, cap;
+  long long num_pages;
+  const uint8_t* host_keys;   // [num_pages, 64, 128]
+  const float* host_scales;   // [num_pages, 64]
+  const int* page_table;      // [B, max_pages]
+  const int* list;            // [B, list_stride] logical blocks
+  const int* count;           // [B]
+  uint8_t* stage_keys;        // [B * cap, 64, 128]
+  float* stage_scales;        // [B * cap, 64]
+};
+
+__global__ void __launch_bounds__(128) fetch_blocks_kernel(const FetchParams p) {
+  const int b = blockIdx.y;
+  const int cnt = p.count[b];
+  if (cnt < 0 || cnt > p.list_stride) return;  // flagged by the scoring kernel
+  const int n = min(max(cnt - p.base, 0), p.cap);
+  const int lane = lane_id();
+  for (int u = blockIdx.x * 4 + warp_id(); u < n; u += gridDim.x * 4) {
+    const int lp = p.list[(size_t)b * p.list_stride + p.base + u];
+    if (lp < 0 || lp >= p.max_pages) continue;  // flagged by the scoring kernel, which skips it
+    const int page = p.page_table[(size_t)b * p.max_pages + lp];
+    if (page < 0 || page >= p.num_pages) {
+      if (lane == 0) flag(LS_DEV_BOUNDS);
+      continue;
+    }
+    const uint4* src = (const uint4*)(p.host_keys + (size_t)page * 8192);
+    uint4* dst = (uint4*)(p.stage_keys + ((size_t)b * p.cap + u) * 8192);
+    uint4 v[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = src[j * 32 + lane];
+    uint4 sc = make_uint4(0, 0, 0, 0);
+    if (lane < 16) sc = ((const uint4*)(p.host_scales + (size_t)page * 64))[lane];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) dst[j * 32 + lane] = v[j];
+    if (lane < 16) ((uint4*)(p.stage_scales + ((size_t)b * p.cap + u) * 64))[lane] = sc;
   }
 }
 

@@ -291,7 +291,7 @@ def test_block_summaries_exact():
     assert_status_clean()
 
 
-def run_c2f(inp, k, eps_rel=0.0):
+def run_c2f(inp, k, eps_rel=0.0, keys_on_host=False, stage_blocks=0):
     lens = inp.lens.tolist()
     Bn = len(lens)
     d = {kk: v.to(DEV) for kk, v in inp.__dict__.items() if isinstance(v, torch.Tensor)}
@@ -302,15 +302,19 @@ def run_c2f(inp, k, eps_rel=0.0):
     B.ls_build_block_summaries(q=d["q"], w=d["w"], key_pool=d["key_pool"], key_scale=d["key_scale"],
                                q_scale=d["q_scale"], page_table=d["page_table"], lens=d["lens"], max_len=ml,
                                summaries=summ, block_scale=bsc)
-    ix = B.index_args(q=d["q"], w=d["w"], key_pool=d["key_pool"], page_table=d["page_table"], lens=d["lens"],
-                      q_scale=d["q_scale"], key_scale=d["key_scale"], max_len=ml)
+    keys, kscale = d["key_pool"], d["key_scale"]
+    if keys_on_host:  # the summaries came from the device copy; scoring reads the host copy
+        keys, kscale = inp.key_pool.pin_memory(), inp.key_scale.pin_memory()
+        del d["key_pool"], d["key_scale"]
+    ix = B.index_args(q=d["q"], w=d["w"], key_pool=keys, page_table=d["page_table"], lens=d["lens"],
+                      q_scale=d["q_scale"], key_scale=kscale, max_len=ml)
     idx = torch.full((Bn, k), -7, dtype=torch.int32, device=DEV)
     sel = torch.zeros((Bn, k), device=DEV)
     surv = torch.full((Bn, mb), -1, dtype=torch.int32, device=DEV)
     nsurv = torch.zeros((Bn,), dtype=torch.int32, device=DEV)
     ub = torch.full((Bn, mb), float("nan"), device=DEV)
     a = B.c2f_args(index=ix, k=k, summaries=summ, block_scale=bsc, idx=idx, sel_score=sel, survivors=surv,
-                   n_survivors=nsurv, ub=ub, eps_rel=eps_rel)
+                   n_survivors=nsurv, ub=ub, eps_rel=eps_rel, keys_on_host=keys_on_host, stage_blocks=stage_blocks)
     ws = torch.empty(B.ls_block_bound_prune_workspace_size(a), dtype=torch.uint8, device=DEV)
     B.ls_block_bound_prune(a, ws)
     torch.cuda.synchronize()
@@ -344,6 +348,38 @@ def test_c2f_equals_full_scan(clustered, lens, k):
         blockmax = np.array([s[j * 64:(j + 1) * 64].max() for j in range(u.shape[0])])
         assert (u >= blockmax - 1e-4 * np.abs(blockmax).max()).all()
     assert_status_clean()
+
+
+@pytest.mark.parametrize("clustered,lens,stage", [(True, [64 * 4000 + 5, 64 * 2500], 0),
+                                                   (False, [64 * 700 + 33], 64),
+                                                   (True, [1500, 64 * 900 + 9], 40)])
+def test_c2f_host_keys_same_as_device_keys(clustered, lens, stage):
+    """Keys in pinned host memory, fetched block by block into staging (several passes
+    when the survivors outnumber the staging): the same selection, scores, survivors and
+    bounds as with the keys in HBM."""
+    inp = _c2f_inputs(lens, seed=61, clustered=clustered)
+    ref = run_c2f(inp, 2048)
+    got = run_c2f(inp, 2048, keys_on_host=True, stage_blocks=stage)
+    names = ("idx", "sel_score", "survivors", "n_survivors", "ub")
+    for name, r, g in zip(names, ref, got):
+        assert torch.equal(r.nan_to_num(-9.0), g.nan_to_num(-9.0)), name
+    if not clustered:  # every block survives: the survivors took many staging passes
+        assert int(got[3][0]) > 4 * 64
+    assert_status_clean()
+
+
+def test_c2f_host_keys_rejects_device_keys():
+    inp = _c2f_inputs([64 * 200], seed=62)
+    d = {kk: v.to(DEV) for kk, v in inp.__dict__.items() if isinstance(v, torch.Tensor)}
+    ix = B.index_args(q=d["q"], w=d["w"], key_pool=d["key_pool"], page_table=d["page_table"], lens=d["lens"],
+                      q_scale=d["q_scale"], key_scale=d["key_scale"], max_len=64 * 200)
+    summ = torch.zeros((1, 200, 256), dtype=torch.uint8, device=DEV)
+    bsc = torch.ones((1, 200), device=DEV)
+    idx = torch.zeros((1, 2048), dtype=torch.int32, device=DEV)
+    a = B.c2f_args(index=ix, k=2048, summaries=summ, block_scale=bsc, idx=idx, keys_on_host=True)
+    ws = torch.empty(B.ls_block_bound_prune_workspace_size(a), dtype=torch.uint8, device=DEV)
+    with pytest.raises(B.LsError, match="pinned host memory"):
+        B.ls_block_bound_prune(a, ws)
 
 
 def check_topk_band_local(g, s, k):
