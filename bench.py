@@ -445,6 +445,64 @@ def run_hotbuf(args):
     return 0
 
 
+def run_c2f(args):
+    """Optional line (not the headline): the coarse-to-fine decode step at batch 4 x
+    1,048,576 tokens -- block bounds over the summaries, the candidate blocks' exact
+    scores, pruning, the survivors' exact scores, top-k, attention -- with the original
+    indexer keys in HBM or (``--keys host``) in pinned host memory."""
+    import torch
+    from sparse_attention_decode_ls_b200 import binding as B
+    from sparse_attention_decode_ls_b200 import workload as W
+
+    batch, ctx = args.batch or 4, 1048576
+    on_host = args.keys == "host"
+    wl = W.c2f_decode(batch=batch, ctx=ctx, k=TOPK, keys_on_host=on_host, device="cuda")
+    stream = torch.cuda.current_stream()
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush_r = torch.ones(64 << 20, dtype=torch.float32, device="cuda")
+    sink = torch.empty((), dtype=torch.float32, device="cuda")
+
+    def prep():
+        flush_w.zero_()
+        torch.sum(flush_r, dim=0, out=sink)
+
+    for _ in range(args.warmup):
+        prep()
+        wl.step()
+    torch.cuda.synchronize()
+    B.ls_check_device_status()
+    ev = []
+    with ClockSampler(0) as clk:
+        for _ in range(args.steps):
+            prep()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            wl.step()
+            e1.record(stream)
+            ev.append((e0, e1))
+        torch.cuda.synchronize()
+    status = B.ls_check_device_status()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    n_surv = [int(x) for x in wl.tensors["n_survivors"].tolist()]
+    n_blocks = -(-ctx // 64)
+    nb0 = (TOPK + 63) // 64 + 1
+    block_bytes = 64 * 128 + 64 * 4  # e4m3 keys + fp32 token scales
+    out = {"metric": "coarse-to-fine sparse-attn decode tokens/s at 1M ctx", "value": batch / (ms / 1e3),
+           "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3+bf16 (f32 accumulate)",
+           "data": "synthetic",
+           "config": {"workload": wl.name, "batch": batch, "ctx": ctx, "topk": TOPK,
+                      "keys": "pinned host memory (only summaries in HBM)" if on_host else "HBM",
+                      "l2": "evicted before every step (256 MB written, then 256 MB read)"},
+           "survivors": {"per_request": n_surv, "of_blocks": n_blocks},
+           "indexer_key_bytes": {"in_hbm": 0 if on_host else batch * ctx * 132,
+                                 "over_host_link_per_step": (batch * nb0 + sum(n_surv)) * block_bytes if on_host else 0},
+           "gpu_launches": wl.kernels_per_step * args.steps,
+           "clocks": clk.summary(), "device_status": status}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -453,8 +511,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["mla", "hotbuf"], default="mla",
-                    help="mla: the headline step (default); hotbuf: the hot-buffer step, one GPU")
+    ap.add_argument("--workload", choices=["mla", "hotbuf", "c2f"], default="mla",
+                    help="mla: the headline step (default); hotbuf: the hot-buffer step; c2f: the "
+                         "coarse-to-fine step at 1M context (one GPU each)")
+    ap.add_argument("--keys", choices=["hbm", "host"], default="hbm", help="c2f: where the original keys live")
     ap.add_argument("--batch", type=int, default=0, help="hotbuf: requests (default 36)")
     ap.add_argument("--miss", type=float, default=0.2, help="hotbuf: fraction of the selection that misses")
     args = ap.parse_args()
@@ -462,6 +522,8 @@ def main():
         args.warmup = 3
     if args.workload == "hotbuf":
         return run_hotbuf(args)
+    if args.workload == "c2f":
+        return run_c2f(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

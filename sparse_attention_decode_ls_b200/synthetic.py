@@ -134,6 +134,24 @@ def clustered_keys(n_blocks_per_req, B, *, dim=128, within_sigma=0.05, shift_fra
     return torch.cat(out, 0)
 
 
+def coarse_to_fine_indexer(lens, *, seed=1004, sigma=0.05, shift_frac=0.02) -> IndexerInputs:
+    """fp8 indexer inputs with block-clustered keys (see ``clustered_keys``): q ~ N(0,1),
+    w = |N(0, 0.1)|, and the shifted blocks moved toward sum_h w_h q_h of their request."""
+    lens = [int(x) for x in lens]
+    B = len(lens)
+    g = _gen(seed)
+    qf = torch.randn((B, 64, 128), generator=g)
+    table, n_pool = page_layout(lens, seed + 17)
+    w = (torch.randn((B, 64), generator=g) * 0.1).abs()
+    direction = (w[:, :, None] * qf).sum(1)
+    keys = torch.cat([clustered_keys(-(-L // PAGE), 1, within_sigma=sigma, shift_frac=shift_frac,
+                                     direction=direction[b:b + 1], seed=seed + 1 + b)[:L]
+                      for b, L in enumerate(lens)])
+    pool_keys = logical_to_pool(keys, lens, table, n_pool)
+    del keys
+    return indexer_fp8(lens, seed=seed, w_nonneg=True, q=qf, keys=pool_keys)
+
+
 def logical_to_pool(keys_logical: torch.Tensor, lens, page_table: torch.Tensor, n_pool: int):
     """Place per-request logical token rows into pool rows through the page table."""
     dim = keys_logical.shape[-1]

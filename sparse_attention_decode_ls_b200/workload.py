@@ -62,7 +62,8 @@ class DecodeWorkload:
 
 
 def build(name: str, ind: syn.IndexerInputs, *, k: int, attn: dict, device="cuda", hotbuf: dict | None = None,
-          c2f: bool = False, eps_rel: float = 0.0) -> DecodeWorkload:
+          c2f: bool = False, eps_rel: float = 0.0, c2f_keys_on_host: bool = False,
+          c2f_stage_blocks: int = 0) -> DecodeWorkload:
     """ind: indexer inputs (CPU or device tensors).  attn: dict(q, kv) for MLA (kv = latent
     pool [NP,64,576] bf16, on device or CPU) or dict(q, k, v) for the fp32 path, plus
     scale.  hotbuf: dict(pos_of_slot, slot_of_pos, recent, host_kv (pinned)) to read the
@@ -127,8 +128,17 @@ def build(name: str, ind: syn.IndexerInputs, *, k: int, attn: dict, device="cuda
         B.ls_build_block_summaries(q=t["i_q"], w=t["i_w"], key_pool=t["i_key_pool"], key_scale=t["i_key_scale"],
                                    q_scale=t["i_q_scale"], page_table=t["i_page_table"], lens=t["i_lens"],
                                    max_len=ml, summaries=t["summaries"], block_scale=t["block_scale"])
+        if c2f_keys_on_host:
+            # only the summaries stay in HBM: the original keys and scales move to pinned host
+            # memory, where the step fetches the blocks it needs
+            torch.cuda.synchronize()
+            t["i_key_pool"] = ind.key_pool.pin_memory()
+            t["i_key_scale"] = ind.key_scale.pin_memory()
+            ix = B.index_args(q=t["i_q"], w=t["i_w"], key_pool=t["i_key_pool"], page_table=t["i_page_table"],
+                              lens=t["i_lens"], q_scale=t["i_q_scale"], key_scale=t["i_key_scale"], max_len=ml)
         cf = dict(summaries=t["summaries"], block_scale=t["block_scale"], survivors=t["survivors"],
-                  n_survivors=t["n_survivors"], eps_rel=eps_rel)
+                  n_survivors=t["n_survivors"], eps_rel=eps_rel, keys_on_host=c2f_keys_on_host,
+                  stage_blocks=c2f_stage_blocks)
     args = B.decode_step_args(index=ix, k=k, attn=at, c2f=cf, hotbuf=hb, idx=t["idx"], sel_score=t["sel"])
     ws_bytes = B.ls_decode_step_workspace_size(args)
     ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
@@ -136,6 +146,13 @@ def build(name: str, ind: syn.IndexerInputs, *, k: int, attn: dict, device="cuda
     if hotbuf is not None:
         wl.hotbuf_init = {key: t[key].clone() for key in ("pos_of_slot", "slot_of_pos", "recent_score", "hbuf")}
     wl.kernels_per_step = kernels_per_step(wl, c2f=c2f, hotbuf=hotbuf is not None, mla=mla)
+    if c2f and c2f_keys_on_host:
+        # a fetch before the candidate blocks' scoring; the survivors' single scoring launch
+        # becomes fetch + scoring per staging pass
+        mb = t["summaries"].shape[1]
+        nb0 = min(mb, (k + 63) // 64 + 1)
+        cap = min(mb, max(nb0, c2f_stage_blocks if c2f_stage_blocks > 0 else 2048))
+        wl.kernels_per_step += 1 + 2 * (-(-mb // cap)) - 1
     return wl
 
 
@@ -197,6 +214,21 @@ def mla_hotbuf_decode(batch=36, ctx=131072, k=2048, miss_frac=0.2, n_slots=4096,
     return build(f"mla_hotbuf_b{batch}_ctx{ctx}_miss{int(round(miss_frac * 100))}", ind, k=k, device=device,
                  attn=dict(q=q, kv_host=True, scale=syn.softmax_scale(576)),
                  hotbuf=dict(pos_of_slot=pos_of_slot, slot_of_pos=slot_of_pos, recent=recent, host_kv=host))
+
+
+def c2f_decode(batch=4, ctx=1048576, k=2048, keys_on_host=False, stage_blocks=0, seed=1004,
+               device="cuda") -> DecodeWorkload:
+    """The coarse-to-fine configuration: block-clustered fp8 keys (2% of the blocks shifted
+    toward the query) at ``ctx`` tokens per request, per-block summaries in HBM, the
+    original keys in HBM or (``keys_on_host``) in pinned host memory; MLA attention over a
+    paged bf16 pool in HBM."""
+    lens = [ctx] * batch
+    ind = syn.coarse_to_fine_indexer(lens, seed=seed)
+    q, kv = syn.mla_attention(batch, ind.key_pool.shape[0], seed=seed + 1000, device=device)
+    where = "hostkeys" if keys_on_host else "hbmkeys"
+    return build(f"c2f_b{batch}_ctx{ctx}_{where}", ind, k=k, device=device, c2f=True,
+                 attn=dict(q=q, kv=kv, scale=syn.softmax_scale(576)), c2f_keys_on_host=keys_on_host,
+                 c2f_stage_blocks=stage_blocks)
 
 
 def tiny_f32(device="cuda") -> DecodeWorkload:
