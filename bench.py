@@ -503,6 +503,93 @@ def run_c2f(args):
     return 0
 
 
+def run_prefill(args):
+    """Optional line: the two-buffer layer-streaming prefill -- each layer's indexer keys
+    and scales copied from pinned host memory into one of two staging buffers while the
+    previous layer's block summaries are built and its hot buffer is seeded -- at batch 4
+    x 1,048,576 tokens per layer, 4 layers.  Reported against a plain host-to-device copy
+    of the same bytes (the link's rate on this machine)."""
+    import torch
+    from sparse_attention_decode_ls_b200 import binding as B
+    from sparse_attention_decode_ls_b200 import synthetic as syn
+
+    batch, ctx, n_layers, n_slots = args.batch or 4, 1048576, 4, 4096
+    lens = [ctx] * batch
+    table, n_pool = syn.page_layout(lens, 1021)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(1022)
+    keys, scales = [], []
+    for _ in range(n_layers):  # seeded keys per layer, quantised on the device, then pinned
+        k8 = torch.empty((n_pool, 64, 128), dtype=torch.uint8, pin_memory=True)
+        sk = torch.empty((n_pool, 64), dtype=torch.float32, pin_memory=True)
+        for i in range(0, n_pool, 4096):
+            j = min(n_pool, i + 4096)
+            x = torch.randn(((j - i) * 64, 128), generator=gen, device="cuda")
+            amax = x.abs().amax(dim=1, keepdim=True).clamp_min(1e-12)
+            sc = amax / 448.0
+            k8[i:j].copy_((x / sc).to(torch.float8_e4m3fn).view(torch.uint8).view(j - i, 64, 128))
+            sk[i:j].copy_(sc.view(j - i, 64))
+        keys.append(k8)
+        scales.append(sk)
+    kv = torch.empty((n_pool, 64, 576), dtype=torch.bfloat16, pin_memory=True)  # one history, all layers
+    for i in range(0, n_pool, 4096):
+        j = min(n_pool, i + 4096)
+        kv[i:j].copy_(torch.randn((j - i, 64, 576), generator=gen, device="cuda").to(torch.bfloat16))
+    torch.cuda.synchronize()
+    dev = "cuda"
+    mb = -(-ctx // 64)
+    a = B.prefill_args(page_table=table.to(dev), lens=torch.tensor(lens, dtype=torch.int32, device=dev), max_len=ctx,
+                       host_keys=keys, host_key_scales=scales,
+                       summaries=[torch.empty((batch, mb, 256), dtype=torch.uint8, device=dev) for _ in range(n_layers)],
+                       block_scale=[torch.empty((batch, mb), device=dev) for _ in range(n_layers)],
+                       host_kv=[kv] * n_layers,
+                       hbuf=[torch.empty((batch, n_slots, 576), dtype=torch.bfloat16, device=dev)
+                             for _ in range(n_layers)],
+                       pos_of_slot=[torch.empty((batch, n_slots), dtype=torch.int32, device=dev) for _ in range(n_layers)],
+                       slot_of_pos=[torch.empty((batch, ctx), dtype=torch.int32, device=dev) for _ in range(n_layers)],
+                       recent_score=[torch.empty((batch, n_slots), device=dev) for _ in range(n_layers)])
+    ws = torch.empty(B.ls_prefill_stream_workspace_size(a), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, n):
+        ev = []
+        for _ in range(n):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            ev.append((e0, e1))
+        torch.cuda.synchronize()
+        return statistics.mean(x.elapsed_time(y) for x, y in ev)
+
+    for _ in range(args.warmup):
+        B.ls_prefill_stream(a, ws)
+    torch.cuda.synchronize()
+    B.ls_check_device_status()
+    with ClockSampler(0) as clk:
+        ms = timed(lambda: B.ls_prefill_stream(a, ws), args.steps)
+    status = B.ls_check_device_status()
+    # the link's own rate: one layer's keys and scales with two plain copies on this stream
+    dst_k = torch.empty((n_pool, 64, 128), dtype=torch.uint8, device=dev)
+    dst_s = torch.empty((n_pool, 64), dtype=torch.float32, device=dev)
+    copy_ms = timed(lambda: (dst_k.copy_(keys[0], non_blocking=True), dst_s.copy_(scales[0], non_blocking=True)), 5)
+    layer_bytes = n_pool * 64 * (128 + 4)
+    seed_bytes = batch * n_slots * 576 * 2
+    out = {"metric": "layer-streaming prefill: indexer-key GB/s over the host link", "value":
+           n_layers * layer_bytes / (ms / 1e3) / 1e9, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "e4m3 (summaries: exact)", "data": "synthetic",
+           "config": {"workload": f"prefill_stream_b{batch}_ctx{ctx}_layers{n_layers}", "batch": batch, "ctx": ctx,
+                      "layers": n_layers, "hot_slots": n_slots, "step": "one call: every layer streamed, "
+                      "summarised and its hot buffer seeded"},
+           "per_layer_ms": ms / n_layers, "layer_key_bytes": layer_bytes, "seed_bytes_per_layer": seed_bytes,
+           "plain_copy": {"ms_per_layer": copy_ms, "GBps": layer_bytes / (copy_ms / 1e3) / 1e9},
+           "frac_of_plain_copy": (copy_ms * n_layers) / ms,
+           "clocks": clk.summary(), "device_status": status}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -511,9 +598,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["mla", "hotbuf", "c2f"], default="mla",
+    ap.add_argument("--workload", choices=["mla", "hotbuf", "c2f", "prefill"], default="mla",
                     help="mla: the headline step (default); hotbuf: the hot-buffer step; c2f: the "
-                         "coarse-to-fine step at 1M context (one GPU each)")
+                         "coarse-to-fine step at 1M context; prefill: layer-streaming prefill (one GPU each)")
     ap.add_argument("--keys", choices=["hbm", "host"], default="hbm", help="c2f: where the original keys live")
     ap.add_argument("--batch", type=int, default=0, help="hotbuf: requests (default 36)")
     ap.add_argument("--miss", type=float, default=0.2, help="hotbuf: fraction of the selection that misses")
@@ -524,6 +611,8 @@ def main():
         return run_hotbuf(args)
     if args.workload == "c2f":
         return run_c2f(args)
+    if args.workload == "prefill":
+        return run_prefill(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -392,6 +392,56 @@ ls_status ls_decode_step(const ls_decode_step_args* args, void* workspace,
                          size_t workspace_bytes, ls_stream_t stream);
 
 /* ------------------------------------------------------------------------------
+ * Layer-streaming prefill (LeanSparse, abstract: prefill streams each layer's history
+ * through two reusable GPU buffers, so that the full history of every layer never has
+ * to sit in HBM at once).
+ *
+ * For layer l = 0 .. layers-1: the layer's indexer keys and token scales are copied
+ * from pinned host memory into one of two staging buffers in the workspace (layer l
+ * uses buffer l % 2) on a copy stream owned by the library, while `stream` builds the
+ * block summaries of layer l-1 from the other buffer (exactly as
+ * ls_build_block_summaries) and, with n_slots > 0, seeds layer l-1's hot buffer.  A
+ * buffer is refilled only after the summaries built from it are done.
+ *
+ * Hot-buffer seed (the pages give no initial contents; this call uses recency): slot
+ * s of request b holds position p = lens[b] - n_slots + s when p >= 0, else it is empty
+ * (-1); slot_of_pos[b][p] = s for those positions and -1 everywhere else below
+ * max_len; recent_score = 0; the seeded rows are copied from host_kv[l] through the
+ * page table, as ls_gather_misses does.
+ *
+ * All pointer arrays ([layers] entries) are read on the host during the call; the
+ * pointers in them are device pointers, except host_keys, host_key_scales and host_kv
+ * (pinned host memory, device-accessible).  Returns once all work is enqueued; the
+ * last operation is on `stream`.  Needs ls_prefill_stream_workspace_size() bytes of
+ * workspace (256-byte aligned).
+ * --------------------------------------------------------------------------- */
+typedef struct ls_prefill_stream_args {
+  int32_t layers;
+  int32_t batch;
+  int32_t max_pages;          /* row stride of page_table */
+  int32_t max_len;            /* row stride of slot_of_pos; lens[b] <= min(max_len, 64*max_pages) */
+  int32_t max_blocks;         /* row stride of summaries / block_scale; >= ceil(lens[b]/64) */
+  int32_t n_slots;            /* hot-buffer slots per request, 0 = no seeding (<= 4096) */
+  int64_t num_pages;          /* pages in each layer's pool */
+  int64_t row_bytes;          /* seeding: bytes per KV row (multiple of 16) */
+  const int32_t* page_table;  /* [B,max_pages], shared by all layers */
+  const int32_t* lens;        /* [B] */
+  const void* const* host_keys;          /* [layers] -> [num_pages,64,128] e4m3, pinned */
+  const float* const* host_key_scales;   /* [layers] -> [num_pages,64] f32, pinned */
+  uint8_t* const* summaries;             /* [layers] -> [B,max_blocks,256] out */
+  float* const* block_scale;             /* [layers] -> [B,max_blocks] out */
+  const void* const* host_kv;            /* [layers] -> [num_pages,64,row_bytes], pinned (seeding) */
+  void* const* hbuf;                     /* [layers] -> [B,n_slots,row_bytes] out (seeding) */
+  int32_t* const* pos_of_slot;           /* [layers] -> [B,n_slots] out (seeding) */
+  int32_t* const* slot_of_pos;           /* [layers] -> [B,max_len] out (seeding) */
+  float* const* recent_score;            /* [layers] -> [B,n_slots] out (seeding) */
+} ls_prefill_stream_args;
+
+size_t ls_prefill_stream_workspace_size(const ls_prefill_stream_args* args);
+ls_status ls_prefill_stream(const ls_prefill_stream_args* args, void* workspace, size_t workspace_bytes,
+                            ls_stream_t stream);
+
+/* ------------------------------------------------------------------------------
  * Diagnostics.
  * --------------------------------------------------------------------------- */
 /* Message of the calling thread's last error (empty string if none). */

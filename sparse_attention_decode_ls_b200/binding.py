@@ -70,7 +70,15 @@ class DecodeStepArgs(C.Structure):
                 ("events", _p)]
 
 
+class PrefillStreamArgs(C.Structure):
+    _fields_ = [("layers", _i32), ("batch", _i32), ("max_pages", _i32), ("max_len", _i32), ("max_blocks", _i32),
+                ("n_slots", _i32), ("num_pages", _i64), ("row_bytes", _i64), ("page_table", _p), ("lens", _p),
+                ("host_keys", _p), ("host_key_scales", _p), ("summaries", _p), ("block_scale", _p),
+                ("host_kv", _p), ("hbuf", _p), ("pos_of_slot", _p), ("slot_of_pos", _p), ("recent_score", _p)]
+
+
 STRUCTS = {"ls_index_score_args": IndexScoreArgs, "ls_topk_args": TopkArgs,
+           "ls_prefill_stream_args": PrefillStreamArgs,
            "ls_block_bound_prune_args": BlockBoundPruneArgs, "ls_hotbuf_args": HotbufArgs,
            "ls_gather_args": GatherArgs, "ls_sparse_attn_args": SparseAttnArgs,
            "ls_decode_step_args": DecodeStepArgs}
@@ -110,6 +118,10 @@ def lib():
             f = getattr(L, name)
             f.argtypes = [P(st)]
             f.restype = C.c_size_t
+        L.ls_prefill_stream_workspace_size.argtypes = [P(PrefillStreamArgs)]
+        L.ls_prefill_stream_workspace_size.restype = C.c_size_t
+        L.ls_prefill_stream.argtypes = [P(PrefillStreamArgs), _p, C.c_size_t, _p]
+        L.ls_prefill_stream.restype = C.c_int
         L.ls_sparse_attn_decode_noalloc.argtypes = [P(SparseAttnArgs), _p]
         L.ls_sparse_attn_decode_noalloc.restype = C.c_int
         L.ls_build_block_summaries.argtypes = [P(IndexScoreArgs), _p, _p, _i32, _p]
@@ -355,3 +367,47 @@ def event_array(events):
     for i, e in enumerate(events):
         arr[i] = None if e is None else e.cuda_event
     return arr
+
+
+# ------------------------------------------------------------------------------- prefill
+def _ptr_array(ts):
+    arr = (C.c_void_p * len(ts))(*[None if t is None else t.data_ptr() for t in ts])
+    return arr
+
+
+def prefill_args(*, page_table, lens, max_len, host_keys, host_key_scales, summaries, block_scale,
+                 host_kv=None, hbuf=None, pos_of_slot=None, slot_of_pos=None, recent_score=None) -> PrefillStreamArgs:
+    """Per-layer lists: host_keys / host_key_scales / host_kv are pinned CPU tensors, the rest
+    CUDA tensors; the hot-buffer lists are given together or not at all (no seeding)."""
+    a = PrefillStreamArgs()
+    a.layers = len(host_keys)
+    a.batch = page_table.shape[0]
+    a.max_pages = page_table.shape[1]
+    a.max_len = int(max_len)
+    a.max_blocks = summaries[0].shape[1]
+    a.num_pages = host_keys[0].shape[0]
+    seed = hbuf is not None
+    a.n_slots = hbuf[0].shape[1] if seed else 0
+    a.row_bytes = hbuf[0].shape[2] * hbuf[0].element_size() if seed else 0
+    a.page_table, a.lens = _ptr(page_table), _ptr(lens)
+    arrays = {"host_keys": host_keys, "host_key_scales": host_key_scales, "summaries": summaries,
+              "block_scale": block_scale}
+    if seed:
+        arrays.update(host_kv=host_kv, hbuf=hbuf, pos_of_slot=pos_of_slot, slot_of_pos=slot_of_pos,
+                      recent_score=recent_score)
+    held = []
+    for name, ts in arrays.items():
+        arr = _ptr_array(ts)
+        setattr(a, name, C.cast(arr, C.c_void_p).value)
+        held.append(arr)
+        held.extend(ts)
+    return _hold(a, page_table, lens, *held)
+
+
+def ls_prefill_stream_workspace_size(a: PrefillStreamArgs) -> int:
+    return lib().ls_prefill_stream_workspace_size(C.byref(a))
+
+
+def ls_prefill_stream(a: PrefillStreamArgs, workspace, stream=None):
+    _check(lib().ls_prefill_stream(C.byref(a), _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                   _stream(stream)))

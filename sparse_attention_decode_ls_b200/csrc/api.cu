@@ -803,6 +803,90 @@ StepLayout step_layout(const ls_decode_step_args* a) {
   return l;
 }
 
+// ---- layer-streaming prefill --------------------------------------------------------
+struct PrefillLayout {
+  size_t off_keys[2], off_scales[2], off_spos, off_sslot, off_sn, total;
+};
+
+PrefillLayout prefill_layout(const ls_prefill_stream_args* a) {
+  PrefillLayout l{};
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t r = o; o += align256(bytes); return r; };
+  for (int i = 0; i < 2; ++i) {
+    l.off_keys[i] = take((size_t)a->num_pages * 64 * 128);
+    l.off_scales[i] = take((size_t)a->num_pages * 64 * 4);
+  }
+  const size_t ns = a->n_slots > 0 ? (size_t)a->batch * a->n_slots * 4 : 0;
+  l.off_spos = take(ns);
+  l.off_sslot = take(ns);
+  l.off_sn = take(a->n_slots > 0 ? (size_t)a->batch * 4 : 0);
+  l.total = o;
+  return l;
+}
+
+bool pinned_host(const void* p) {
+  cudaPointerAttributes at{};
+  const bool ok = p && cudaPointerGetAttributes(&at, p) == cudaSuccess && at.type == cudaMemoryTypeHost &&
+                  at.devicePointer == p;
+  cudaGetLastError();
+  return ok;
+}
+
+ls_status validate_prefill(const ls_prefill_stream_args* a) {
+  LS_REQUIRE(a, "args is NULL");
+  LS_REQUIRE(a->layers >= 1 && a->batch >= 1, "layers and batch must be >= 1");
+  LS_REQUIRE(a->max_pages >= 1 && a->max_len >= 1 && a->max_blocks >= 1 && a->num_pages >= 1,
+             "max_pages, max_len, max_blocks and num_pages must be >= 1");
+  LS_REQUIRE(a->n_slots >= 0 && a->n_slots <= ls::kHbMaxSlots, "n_slots must be in [0, 4096]");
+  LS_REQUIRE(a->page_table && a->lens && a->host_keys && a->host_key_scales && a->summaries && a->block_scale,
+             "a required pointer is NULL");
+  const bool seed = a->n_slots > 0;
+  if (seed) {
+    LS_REQUIRE(a->host_kv && a->hbuf && a->pos_of_slot && a->slot_of_pos && a->recent_score,
+               "hot-buffer seeding needs host_kv, hbuf, pos_of_slot, slot_of_pos and recent_score");
+    LS_REQUIRE(a->row_bytes >= 16 && a->row_bytes % 16 == 0, "row_bytes must be a positive multiple of 16");
+  }
+  for (int l = 0; l < a->layers; ++l) {
+    LS_REQUIRE(pinned_host(a->host_keys[l]) && pinned_host(a->host_key_scales[l]),
+               "layer %d: host_keys / host_key_scales must be pinned host memory (mapped at the same address)", l);
+    LS_REQUIRE(a->summaries[l] && a->block_scale[l], "layer %d: summaries / block_scale is NULL", l);
+    if (seed) {
+      LS_REQUIRE(pinned_host(a->host_kv[l]) && aligned16(a->host_kv[l]),
+                 "layer %d: host_kv must be 16-byte aligned pinned host memory", l);
+      LS_REQUIRE(a->hbuf[l] && aligned16(a->hbuf[l]) && a->pos_of_slot[l] && a->slot_of_pos[l] &&
+                     a->recent_score[l],
+                 "layer %d: a hot-buffer pointer is NULL or misaligned", l);
+    }
+  }
+  return LS_OK;
+}
+
+// The copy stream of this host thread on the current device and its events (created once).
+struct PrefillStreams {
+  cudaStream_t copy = nullptr;
+  cudaEvent_t start = nullptr, loaded[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
+};
+ls_status prefill_streams(PrefillStreams** out) {
+  thread_local PrefillStreams per_dev[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  PrefillStreams& ps = per_dev[dev & 63];
+  if (!ps.copy) {
+    bool good = cudaEventCreateWithFlags(&ps.start, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; i < 2; ++i) {
+      good = good && cudaEventCreateWithFlags(&ps.loaded[i], cudaEventDisableTiming) == cudaSuccess;
+      good = good && cudaEventCreateWithFlags(&ps.freed[i], cudaEventDisableTiming) == cudaSuccess;
+    }
+    good = good && cudaStreamCreateWithFlags(&ps.copy, cudaStreamNonBlocking) == cudaSuccess;
+    if (!good) {
+      ps.copy = nullptr;
+      return check_launch("prefill streams");
+    }
+  }
+  *out = &ps;
+  return LS_OK;
+}
+
 }  // namespace
 
 // =========================================================================================
@@ -861,6 +945,68 @@ ls_status ls_build_block_summaries(const ls_index_score_args* keys, uint8_t* sum
   const int gx = std::min(max_blocks, std::min(keys->max_pages, (keys->max_len + 63) / 64));
   ls::build_summaries_kernel<<<dim3(gx, keys->batch), 128, 0, (cudaStream_t)stream>>>(p);
   LS_TRY(check_launch("build_summaries"));
+  return ok();
+}
+
+size_t ls_prefill_stream_workspace_size(const ls_prefill_stream_args* args) {
+  if (!args) return 0;
+  return prefill_layout(args).total;
+}
+
+ls_status ls_prefill_stream(const ls_prefill_stream_args* a, void* workspace, size_t workspace_bytes,
+                            ls_stream_t stream) {
+  LS_TRY(validate_prefill(a));
+  const PrefillLayout l = prefill_layout(a);
+  LS_REQUIRE(workspace && workspace_bytes >= l.total, "workspace too small (%zu < %zu bytes)", workspace_bytes,
+             l.total);
+  LS_REQUIRE(((uintptr_t)workspace & 255) == 0, "workspace must be 256-byte aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  char* w = (char*)workspace;
+  PrefillStreams* ps = nullptr;
+  LS_TRY(prefill_streams(&ps));
+  // the staging buffers may still be read by work already queued on `stream`
+  cudaEventRecord(ps->start, st);
+  cudaStreamWaitEvent(ps->copy, ps->start, 0);
+  const size_t key_bytes = (size_t)a->num_pages * 64 * 128, scale_bytes = (size_t)a->num_pages * 64 * 4;
+  for (int layer = 0; layer < a->layers; ++layer) {
+    const int buf = layer & 1;
+    uint8_t* keys = (uint8_t*)(w + l.off_keys[buf]);
+    float* scales = (float*)(w + l.off_scales[buf]);
+    // copy stream: layer `layer` into buffer `buf`, once the summaries of layer - 2 are done
+    if (layer >= 2) cudaStreamWaitEvent(ps->copy, ps->freed[buf], 0);
+    cudaError_t e = cudaMemcpyAsync(keys, a->host_keys[layer], key_bytes, cudaMemcpyHostToDevice, ps->copy);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(scales, a->host_key_scales[layer], scale_bytes, cudaMemcpyHostToDevice,
+                                              ps->copy);
+    if (e != cudaSuccess) return fail(LS_ERR_CUDA, "prefill copy (layer %d): %s", layer, cudaGetErrorString(e));
+    cudaEventRecord(ps->loaded[buf], ps->copy);
+    // `stream`: the layer's summaries from the buffer, then its hot-buffer seed
+    cudaStreamWaitEvent(st, ps->loaded[buf], 0);
+    ls::SummParams sp{};
+    sp.B = a->batch; sp.max_pages = a->max_pages; sp.max_len = a->max_len; sp.max_blocks = a->max_blocks;
+    sp.num_pages = a->num_pages; sp.keys = keys; sp.ks = scales; sp.page_table = a->page_table; sp.lens = a->lens;
+    sp.summ = a->summaries[layer]; sp.bscale = a->block_scale[layer];
+    const int gx = std::min(a->max_blocks, std::min(a->max_pages, (a->max_len + 63) / 64));
+    ls::build_summaries_kernel<<<dim3(gx, a->batch), 128, 0, st>>>(sp);
+    LS_TRY(check_launch("build_summaries"));
+    cudaEventRecord(ps->freed[buf], st);
+    if (a->n_slots > 0) {
+      int* spos = (int*)(w + l.off_spos);
+      int* sslot = (int*)(w + l.off_sslot);
+      int* sn = (int*)(w + l.off_sn);
+      ls::SeedParams q{};
+      q.B = a->batch; q.n_slots = a->n_slots; q.max_len = a->max_len; q.max_pages = a->max_pages; q.lens = a->lens;
+      q.pos_of_slot = a->pos_of_slot[layer]; q.slot_of_pos = a->slot_of_pos[layer]; q.recent = a->recent_score[layer];
+      q.seed_pos = spos; q.seed_slot = sslot; q.seed_n = sn;
+      const int sx = std::max(1, std::min((a->max_len + 255) / 256, (4 * device_sms()) / a->batch));
+      ls::seed_hotbuf_kernel<<<dim3(sx, a->batch), 256, 0, st>>>(q);
+      LS_TRY(check_launch("seed_hotbuf"));
+      ls_gather_args g{};
+      g.batch = a->batch; g.k = a->n_slots; g.n_slots = a->n_slots; g.max_pages = a->max_pages;
+      g.row_bytes = a->row_bytes; g.num_pages = a->num_pages; g.host_kv = a->host_kv[layer];
+      g.page_table = a->page_table; g.miss_pos = spos; g.miss_slot = sslot; g.n_miss = sn; g.hbuf = a->hbuf[layer];
+      LS_TRY(launch_gather(&g, st));
+    }
+  }
   return ok();
 }
 

@@ -301,6 +301,53 @@ __global__ void __launch_bounds__(kGatherThreads, 8) gather_misses_kernel(const 
   }
 }
 
+// Prefill: a hot buffer seeded with each request's most recent n_slots positions (slot
+// s holds p = L - n_slots + s when p >= 0), recent scores 0, and the list of seeded
+// (position, slot) pairs for the row gather.  grid (x, B), 256 threads: the grid strides
+// over slot_of_pos; CTA 0 of each request also writes the slot side and the lists.
+struct SeedParams {
+  int B, n_slots, max_len, max_pages;
+  const int* lens;
+  int* pos_of_slot;  // [B,n_slots]
+  int* slot_of_pos;  // [B,max_len]
+  float* recent;     // [B,n_slots]
+  int* seed_pos;     // [B,n_slots] positions in slot order, -1 after them
+  int* seed_slot;    // [B,n_slots]
+  int* seed_n;       // [B]
+};
+
+__global__ void __launch_bounds__(256) seed_hotbuf_kernel(const SeedParams p) {
+  const int b = blockIdx.y;
+  const int L = p.lens[b], S = p.n_slots;
+  if (L < 0 || L > p.max_len || L > p.max_pages * 64) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      flag(LS_DEV_BOUNDS);
+      p.seed_n[b] = 0;
+    }
+    return;
+  }
+  const int first = L - S;  // position held by slot 0 (may be negative: empty slots)
+  for (int q = blockIdx.x * 256 + threadIdx.x; q < p.max_len; q += gridDim.x * 256)
+    p.slot_of_pos[(size_t)b * p.max_len + q] = (q < L && q >= first) ? q - first : -1;
+  if (blockIdx.x != 0) return;
+  const int s0 = max(0, -first);  // first non-empty slot
+  for (int s = threadIdx.x; s < S; s += 256) {
+    const int pos = first + s;
+    p.pos_of_slot[(size_t)b * S + s] = pos >= 0 ? pos : -1;
+    p.recent[(size_t)b * S + s] = 0.f;
+    const int i = s - s0;  // the gather lists, in slot order
+    if (s >= s0) {
+      p.seed_pos[(size_t)b * S + i] = pos;
+      p.seed_slot[(size_t)b * S + i] = s;
+    }
+    if (s >= S - s0) {  // the tail of the lists past the seeded entries
+      p.seed_pos[(size_t)b * S + s] = -1;
+      p.seed_slot[(size_t)b * S + s] = -1;
+    }
+  }
+  if (threadIdx.x == 0) p.seed_n[b] = S - s0;
+}
+
 struct StageCopyParams {
   int B, k, n_slots;
   long long row_bytes;
