@@ -141,6 +141,8 @@ typedef struct ls_topk_args {
   const int32_t* lens;        /* [B] */
   int32_t* idx;               /* [B,k] out */
   float* sel_score;           /* [B,k] out, may be NULL */
+  const int32_t* pos_offset;  /* optional [B]: added to every emitted position (e.g. the first
+                                 position of this GPU's shard of the request); -1 padding stays */
 } ls_topk_args;
 
 ls_status ls_topk_select(const ls_topk_args* args, ls_stream_t stream);
@@ -310,8 +312,10 @@ typedef struct ls_sparse_attn_args {
   const void* v_rows;
   const int32_t* page_table;  /* PAGED: [B,max_pages] */
   const int32_t* sel;         /* [B,k] positions (PAGED) or slots (SLOTS); -1 skipped */
-  void* o;                    /* [B,heads,dv] out */
+  void* o;                    /* [B,heads,dv] out: bf16 for bf16 inputs, float32 for f32 */
   float* lse;                 /* [B,heads] out */
+  int32_t o_f32;              /* bf16 tensor-core kernel: != 0 writes o as float32 (16-byte
+                                 aligned), e.g. as a partial for ls_attn_merge */
 } ls_sparse_attn_args;
 
 size_t ls_sparse_attn_workspace_size(const ls_sparse_attn_args* args);
@@ -390,6 +394,55 @@ typedef struct ls_decode_step_args {
 size_t ls_decode_step_workspace_size(const ls_decode_step_args* args);
 ls_status ls_decode_step(const ls_decode_step_args* args, void* workspace,
                          size_t workspace_bytes, ls_stream_t stream);
+
+/* ------------------------------------------------------------------------------
+ * Context-parallel split of one request over G GPUs (no counterpart on the pages'
+ * single-GPU path; their 1M-context, batch-4 workload on several GPUs).  GPU g holds
+ * the contiguous positions [shard_begin[b], shard_end[b]) of request b, with its own
+ * page tables and pools, and per step:
+ *   1. ls_index_score + ls_topk_select over its shard, pos_offset = shard_begin, so its
+ *      k candidates carry global positions (ascending, -1 padded) and their scores;
+ *   2. an all-gather (NCCL, by the caller) of every GPU's candidates into
+ *      cand_score / cand_pos [G,B,k], in shard order;
+ *   3. ls_cp_merge_topk: the global top-k of the gathered candidates (the same on every
+ *      GPU, and the same as one GPU scanning the whole context: scores do not depend on
+ *      the shard, ties go to the lower position) and this GPU's part of it as local
+ *      positions (-1 elsewhere);
+ *   4. ls_sparse_attn_decode over the local part with o_f32 set: a normalised partial
+ *      o_g and its lse_g;
+ *   5. an all-gather of (o_g, lse_g) and ls_attn_merge:
+ *      LSE = ln sum_g exp(lse_g), o = sum_g exp(lse_g - LSE) o_g.
+ * --------------------------------------------------------------------------- */
+typedef struct ls_cp_merge_args {
+  int32_t shards;             /* G */
+  int32_t batch;
+  int32_t k;
+  const float* cand_score;    /* [G,B,k] */
+  const int32_t* cand_pos;    /* [G,B,k] global positions, each shard's valid ones first */
+  const int32_t* shard_begin; /* [B] this GPU's shard of each request */
+  const int32_t* shard_end;   /* [B] */
+  int32_t* idx;               /* [B,k] out: global top-k positions, ascending, -1 padded */
+  float* sel_score;           /* [B,k] out, may be NULL */
+  int32_t* local_sel;         /* [B,k] out, may be NULL: idx - shard_begin inside the shard, else -1 */
+} ls_cp_merge_args;
+
+size_t ls_cp_merge_workspace_size(const ls_cp_merge_args* args);
+ls_status ls_cp_merge_topk(const ls_cp_merge_args* args, void* workspace, size_t workspace_bytes,
+                           ls_stream_t stream);
+
+typedef struct ls_attn_merge_args {
+  int32_t parts;              /* G */
+  int32_t batch;
+  int32_t heads;
+  int32_t dv;                 /* multiple of 4 */
+  const float* o_parts;       /* [G,B,heads,dv] normalised partial outputs */
+  const float* lse_parts;     /* [G,B,heads] their lse (natural log; -inf = empty part) */
+  void* o;                    /* [B,heads,dv] out, o_dtype */
+  int32_t o_dtype;            /* LS_BF16 or LS_F32 */
+  float* lse;                 /* [B,heads] out (-inf and o = 0 when every part is empty) */
+} ls_attn_merge_args;
+
+ls_status ls_attn_merge(const ls_attn_merge_args* args, ls_stream_t stream);
 
 /* ------------------------------------------------------------------------------
  * Layer-streaming prefill (LeanSparse, abstract: prefill streams each layer's history

@@ -32,7 +32,7 @@ class IndexScoreArgs(C.Structure):
 
 class TopkArgs(C.Structure):
     _fields_ = [("batch", _i32), ("k", _i32), ("max_len", _i32), ("scores", _p), ("lens", _p), ("idx", _p),
-                ("sel_score", _p)]
+                ("sel_score", _p), ("pos_offset", _p)]
 
 
 class BlockBoundPruneArgs(C.Structure):
@@ -57,7 +57,17 @@ class SparseAttnArgs(C.Structure):
     _fields_ = [("batch", _i32), ("heads", _i32), ("dk", _i32), ("dv", _i32), ("k", _i32), ("dtype", _i32),
                 ("variant", _i32), ("softmax_scale", _f32), ("addressing", _i32), ("max_pages", _i32),
                 ("n_slots", _i32), ("row_stride", _i64), ("num_rows", _i64), ("q", _p), ("k_rows", _p),
-                ("v_rows", _p), ("page_table", _p), ("sel", _p), ("o", _p), ("lse", _p)]
+                ("v_rows", _p), ("page_table", _p), ("sel", _p), ("o", _p), ("lse", _p), ("o_f32", _i32)]
+
+
+class CpMergeArgs(C.Structure):
+    _fields_ = [("shards", _i32), ("batch", _i32), ("k", _i32), ("cand_score", _p), ("cand_pos", _p),
+                ("shard_begin", _p), ("shard_end", _p), ("idx", _p), ("sel_score", _p), ("local_sel", _p)]
+
+
+class AttnMergeArgs(C.Structure):
+    _fields_ = [("parts", _i32), ("batch", _i32), ("heads", _i32), ("dv", _i32), ("o_parts", _p),
+                ("lse_parts", _p), ("o", _p), ("o_dtype", _i32), ("lse", _p)]
 
 
 class DecodeStepArgs(C.Structure):
@@ -78,7 +88,8 @@ class PrefillStreamArgs(C.Structure):
 
 
 STRUCTS = {"ls_index_score_args": IndexScoreArgs, "ls_topk_args": TopkArgs,
-           "ls_prefill_stream_args": PrefillStreamArgs,
+           "ls_prefill_stream_args": PrefillStreamArgs, "ls_cp_merge_args": CpMergeArgs,
+           "ls_attn_merge_args": AttnMergeArgs,
            "ls_block_bound_prune_args": BlockBoundPruneArgs, "ls_hotbuf_args": HotbufArgs,
            "ls_gather_args": GatherArgs, "ls_sparse_attn_args": SparseAttnArgs,
            "ls_decode_step_args": DecodeStepArgs}
@@ -118,6 +129,12 @@ def lib():
             f = getattr(L, name)
             f.argtypes = [P(st)]
             f.restype = C.c_size_t
+        L.ls_cp_merge_workspace_size.argtypes = [P(CpMergeArgs)]
+        L.ls_cp_merge_workspace_size.restype = C.c_size_t
+        L.ls_cp_merge_topk.argtypes = [P(CpMergeArgs), _p, C.c_size_t, _p]
+        L.ls_cp_merge_topk.restype = C.c_int
+        L.ls_attn_merge.argtypes = [P(AttnMergeArgs), _p]
+        L.ls_attn_merge.restype = C.c_int
         L.ls_prefill_stream_workspace_size.argtypes = [P(PrefillStreamArgs)]
         L.ls_prefill_stream_workspace_size.restype = C.c_size_t
         L.ls_prefill_stream.argtypes = [P(PrefillStreamArgs), _p, C.c_size_t, _p]
@@ -205,10 +222,11 @@ def ls_index_score(*, q, w, key_pool, page_table, lens, scores, q_scale=None, ke
 
 
 # ------------------------------------------------------------------------------- a2
-def ls_topk_select(*, scores, lens, idx, sel_score=None, stream=None):
+def ls_topk_select(*, scores, lens, idx, sel_score=None, pos_offset=None, stream=None):
     a = TopkArgs()
     a.batch, a.k, a.max_len = scores.shape[0], idx.shape[1], scores.shape[1]
     a.scores, a.lens, a.idx, a.sel_score = _ptr(scores), _ptr(lens), _ptr(idx), _ptr(sel_score)
+    a.pos_offset = _ptr(pos_offset)
     _check(lib().ls_topk_select(C.byref(a), _stream(stream)))
 
 
@@ -293,6 +311,7 @@ def attn_args(*, q, k_rows, v_rows=None, sel=None, o, lse, scale, page_table=Non
     a.num_rows = k_rows.numel() // k_rows.shape[-1]
     a.q, a.k_rows, a.v_rows = _ptr(q), _ptr(k_rows), _ptr(v_rows)
     a.page_table, a.sel, a.o, a.lse = _ptr(page_table), _ptr(sel), _ptr(o), _ptr(lse)
+    a.o_f32 = 1 if (o.dtype == torch.float32 and q.dtype == torch.bfloat16) else 0
     return _hold(a, q, k_rows, v_rows, page_table, sel, o, lse)
 
 
@@ -411,3 +430,32 @@ def ls_prefill_stream_workspace_size(a: PrefillStreamArgs) -> int:
 def ls_prefill_stream(a: PrefillStreamArgs, workspace, stream=None):
     _check(lib().ls_prefill_stream(C.byref(a), _ptr(workspace), 0 if workspace is None else workspace.numel(),
                                    _stream(stream)))
+
+
+# ------------------------------------------------------------------------------- context parallel
+def cp_merge_args(*, cand_score, cand_pos, shard_begin, shard_end, idx, sel_score=None, local_sel=None):
+    """cand_score / cand_pos: [G, B, k] gathered candidates (CUDA tensors)."""
+    a = CpMergeArgs()
+    a.shards, a.batch, a.k = cand_score.shape
+    a.cand_score, a.cand_pos = _ptr(cand_score), _ptr(cand_pos)
+    a.shard_begin, a.shard_end = _ptr(shard_begin), _ptr(shard_end)
+    a.idx, a.sel_score, a.local_sel = _ptr(idx), _ptr(sel_score), _ptr(local_sel)
+    return _hold(a, cand_score, cand_pos, shard_begin, shard_end, idx, sel_score, local_sel)
+
+
+def ls_cp_merge_workspace_size(a: CpMergeArgs) -> int:
+    return lib().ls_cp_merge_workspace_size(C.byref(a))
+
+
+def ls_cp_merge_topk(a: CpMergeArgs, workspace, stream=None):
+    _check(lib().ls_cp_merge_topk(C.byref(a), _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                                  _stream(stream)))
+
+
+def ls_attn_merge(*, o_parts, lse_parts, o, lse, stream=None):
+    """o_parts [G, B, H, dv] float32, lse_parts [G, B, H]; o [B, H, dv] bf16 or float32."""
+    a = AttnMergeArgs()
+    a.parts, a.batch, a.heads, a.dv = o_parts.shape
+    a.o_parts, a.lse_parts, a.o, a.lse = _ptr(o_parts), _ptr(lse_parts), _ptr(o), _ptr(lse)
+    a.o_dtype = LS_F32 if o.dtype == torch.float32 else LS_BF16
+    _check(lib().ls_attn_merge(C.byref(a), _stream(stream)))

@@ -17,6 +17,7 @@
 #include "c2f.cuh"
 #include "common.cuh"
 #include "hotbuf.cuh"
+#include "cp.cuh"
 #include "index_score.cuh"
 #include "topk.cuh"
 
@@ -58,6 +59,7 @@ ls_status check_launch(const char* what) {
   } while (0)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // ---- per-device cached properties -------------------------------------------------
@@ -312,8 +314,10 @@ ls_status launch_topk_cl(const ls::TopkParams& p0, int B, cudaStream_t st, std::
 
 ls_status launch_topk(int B, int k, const float* scores, int stride, const int* lens, int len_mul, int len_div,
                       int len_limit, const int* unit_list, int list_stride, int* idx, float* sel, float* thr,
-                      cudaStream_t st) {
+                      cudaStream_t st, const int* pos_list = nullptr, int pos_stride = 0,
+                      const int* pos_offset = nullptr) {
   ls::TopkParams p{};
+  p.pos_list = pos_list; p.pos_stride = pos_stride; p.pos_offset = pos_offset;
   p.B = B; p.k = k; p.stride = stride; p.scores = scores; p.lens = lens; p.len_mul = len_mul;
   p.len_div = len_div; p.len_limit = len_limit; p.unit_list = unit_list; p.list_stride = list_stride;
   p.idx = idx; p.sel = sel; p.thr = thr;
@@ -354,6 +358,7 @@ ls_status validate_attn(const ls_sparse_attn_args* a, bool need_sel) {
     if (a->variant == 0 && (a->heads != 128 || a->dk != 576 || a->dv != 512))
       return fail(LS_ERR_UNSUPPORTED, "bf16 tensor-core attention is built for 128 heads, dk 576, dv 512");
     if (a->variant == 0) {
+      LS_REQUIRE(!a->o_f32 || aligned16(a->o), "a float32 o must be 16-byte aligned");
       LS_REQUIRE(a->k_rows == a->v_rows, "MLA attention reads V from the latent rows (v_rows == k_rows)");
       LS_REQUIRE(a->row_stride >= 576 && (a->row_stride % 8) == 0, "row_stride must be >= 576 and % 8 == 0");
       LS_REQUIRE(a->num_rows < 0x7fffffffLL, "num_rows must be below 2^31 - 1");
@@ -362,6 +367,8 @@ ls_status validate_attn(const ls_sparse_attn_args* a, bool need_sel) {
   } else if (a->dtype != LS_F32) {
     return fail(LS_ERR_UNSUPPORTED, "attention dtype must be LS_BF16 or LS_F32");
   }
+  if ((a->variant == 1 && a->dtype == LS_BF16) && a->o_f32)
+    return fail(LS_ERR_UNSUPPORTED, "o_f32 is built for the tensor-core bf16 kernel (variant 0)");
   if (a->variant == 1 || a->dtype == LS_F32) {
     LS_REQUIRE(a->heads >= 1 && a->dk >= 1 && a->dv >= 1 && a->dk <= 1024 && a->dv <= 1024,
                "CUDA-core attention: heads >= 1, 1 <= dk, dv <= 1024");
@@ -409,6 +416,7 @@ ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressi
     p.split_base = pass * ns;
     p.nsplit_total = total;
     p.compacted = compacted ? 1 : 0;
+    p.o_f32 = a->o_f32 ? 1 : 0;
     p.n_valid = n_valid;
     if (total > 1) {
       const size_t need = attn_ws_bytes(a, npasses);
@@ -723,6 +731,7 @@ ls_block_bound_prune_args step_c2f_args(const ls_decode_step_args* a, int* idx, 
 ls_status launch_attn_combine(const ls_sparse_attn_args* a, void* ws, int npasses, cudaStream_t st) {
   ls::AttnParams p{};
   p.B = a->batch; p.H = a->heads; p.dk = a->dk; p.dv = a->dv; p.k = a->k; p.o = a->o; p.lse = a->lse;
+  p.o_f32 = a->o_f32 ? 1 : 0;
   const int ns = attn_nsplit(a), total = ns * npasses;
   p.nsplit = ns;
   p.nsplit_total = total;
@@ -929,7 +938,7 @@ ls_status ls_topk_select(const ls_topk_args* a, ls_stream_t stream) {
   LS_REQUIRE(a->scores && a->lens && a->idx, "scores, lens and idx are required");
   LS_REQUIRE(aligned16(a->scores), "scores must be 16-byte aligned");
   LS_TRY(launch_topk(a->batch, a->k, a->scores, a->max_len, a->lens, 1, 1, a->max_len, nullptr, 0, a->idx,
-                     a->sel_score, nullptr, (cudaStream_t)stream));
+                     a->sel_score, nullptr, (cudaStream_t)stream, nullptr, 0, a->pos_offset));
   return ok();
 }
 
@@ -945,6 +954,59 @@ ls_status ls_build_block_summaries(const ls_index_score_args* keys, uint8_t* sum
   const int gx = std::min(max_blocks, std::min(keys->max_pages, (keys->max_len + 63) / 64));
   ls::build_summaries_kernel<<<dim3(gx, keys->batch), 128, 0, (cudaStream_t)stream>>>(p);
   LS_TRY(check_launch("build_summaries"));
+  return ok();
+}
+
+size_t ls_cp_merge_workspace_size(const ls_cp_merge_args* a) {
+  if (!a || a->shards < 1 || a->batch < 1 || a->k < 1) return 0;
+  const size_t stride = ((size_t)a->shards * a->k + 3) & ~(size_t)3;
+  return align256((size_t)a->batch * stride * 4) * 2 + align256((size_t)a->batch * 4);
+}
+
+ls_status ls_cp_merge_topk(const ls_cp_merge_args* a, void* workspace, size_t workspace_bytes, ls_stream_t stream) {
+  LS_REQUIRE(a, "args is NULL");
+  LS_REQUIRE(a->shards >= 1 && a->batch >= 1 && a->k >= 1 && a->k <= 4096, "shards, batch >= 1, 1 <= k <= 4096");
+  LS_REQUIRE((long long)a->shards * a->k <= (1 << 24), "shards * k too large");
+  LS_REQUIRE(a->cand_score && a->cand_pos && a->shard_begin && a->shard_end && a->idx,
+             "a required pointer is NULL");
+  const size_t need = ls_cp_merge_workspace_size(a);
+  LS_REQUIRE(workspace && workspace_bytes >= need, "workspace too small (%zu < %zu bytes)", workspace_bytes, need);
+  LS_REQUIRE(((uintptr_t)workspace & 255) == 0, "workspace must be 256-byte aligned");
+  cudaStream_t st = (cudaStream_t)stream;
+  const int stride = (a->shards * a->k + 3) & ~3;
+  char* w = (char*)workspace;
+  float* cscore = (float*)w;
+  int* cpos = (int*)(w + align256((size_t)a->batch * stride * 4));
+  int* ccount = (int*)(w + 2 * align256((size_t)a->batch * stride * 4));
+  ls::CpCompactParams c{};
+  c.G = a->shards; c.B = a->batch; c.k = a->k; c.stride = stride; c.cand_score = a->cand_score;
+  c.cand_pos = a->cand_pos; c.score = cscore; c.pos = cpos; c.count = ccount;
+  ls::cp_compact_kernel<<<a->batch, 256, 0, st>>>(c);
+  LS_TRY(check_launch("cp_compact"));
+  LS_TRY(launch_topk(a->batch, a->k, cscore, stride, ccount, 1, 1, stride, nullptr, 0, a->idx, a->sel_score,
+                     nullptr, st, cpos, stride, nullptr));
+  if (a->local_sel) {
+    ls::cp_local_sel_kernel<<<dim3((a->k + 255) / 256, a->batch), 256, 0, st>>>(
+        a->batch, a->k, a->idx, a->shard_begin, a->shard_end, a->local_sel);
+    LS_TRY(check_launch("cp_local_sel"));
+  }
+  return ok();
+}
+
+ls_status ls_attn_merge(const ls_attn_merge_args* a, ls_stream_t stream) {
+  LS_REQUIRE(a, "args is NULL");
+  LS_REQUIRE(a->parts >= 1 && a->batch >= 1 && a->heads >= 1 && a->dv >= 4 && a->dv % 4 == 0,
+             "parts, batch, heads >= 1 and dv a positive multiple of 4 required");
+  LS_REQUIRE(a->o_parts && a->lse_parts && a->o && a->lse, "a required pointer is NULL");
+  LS_REQUIRE(a->o_dtype == LS_BF16 || a->o_dtype == LS_F32, "o_dtype must be LS_BF16 or LS_F32");
+  LS_REQUIRE(aligned16(a->o_parts) && (a->o_dtype == LS_BF16 ? aligned8(a->o) : aligned16(a->o)),
+             "o_parts must be 16-byte aligned, o 8 (bf16) or 16 (f32)");
+  ls::MergeParams p{};
+  p.G = a->parts; p.B = a->batch; p.H = a->heads; p.DV = a->dv; p.o_f32 = a->o_dtype == LS_F32;
+  p.o_parts = a->o_parts; p.lse_parts = a->lse_parts; p.o = a->o; p.lse = a->lse;
+  const long long items = (long long)a->batch * a->heads * (a->dv / 4);
+  ls::attn_merge_kernel<<<(unsigned)((items + 255) / 256), 256, 0, (cudaStream_t)stream>>>(p);
+  LS_TRY(check_launch("attn_merge"));
   return ok();
 }
 

@@ -43,6 +43,7 @@ struct AttnParams {
   int split_base;    // tensor-core kernel: this launch's splits are partial slots
   int nsplit_total;  //   [split_base, split_base + nsplit) of nsplit_total per request
   int compacted;     // the valid entries of every request's selection come first
+  int o_f32;         // tensor-core kernel: o is float32 (else bf16)
   const int* n_valid;  // optional [B]: and there are n_valid[b] of them; the splits share
                        //   those rows instead of all k entries
 };
@@ -602,7 +603,12 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
       for (int c0 = 0; c0 < DVH; c0 += 32) {
         float v[32];
         tmem_ld32(tm_o + lane_off + c0, v);
-        if (single) {
+        if (single && p.o_f32) {
+          float4* o = (float4*)((float*)p.o + ((size_t)b * H + h) * DV + rank * DVH + c0);
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            o[c / 4] = make_float4(v[c] * inv, v[c + 1] * inv, v[c + 2] * inv, v[c + 3] * inv);
+        } else if (single) {
           __nv_bfloat16* o = (__nv_bfloat16*)p.o + ((size_t)b * H + h) * DV + rank * DVH + c0;
 #pragma unroll
           for (int c = 0; c < 32; c += 8) {
@@ -690,14 +696,64 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine(const AttnParams
     }
   }
   const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-  uint32_t w[4];
+  if (p.o_f32) {
+    float4* o = (float4*)((float*)p.o + ((size_t)b * H + h) * DV + d0);
+    o[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    o[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+  } else {
+    uint32_t w[4];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    __nv_bfloat162 two = __floats2bfloat162_rn(acc[2 * q] * inv, acc[2 * q + 1] * inv);
-    w[q] = *(uint32_t*)&two;
+    for (int q = 0; q < 4; ++q) {
+      __nv_bfloat162 two = __floats2bfloat162_rn(acc[2 * q] * inv, acc[2 * q + 1] * inv);
+      w[q] = *(uint32_t*)&two;
+    }
+    *(uint4*)((__nv_bfloat16*)p.o + ((size_t)b * H + h) * DV + d0) = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  *(uint4*)((__nv_bfloat16*)p.o + ((size_t)b * H + h) * DV + d0) = make_uint4(w[0], w[1], w[2], w[3]);
   if (d0 == 0) p.lse[(size_t)b * H + h] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
+}
+
+// Merge of normalised partial attention outputs over disjoint row sets (the shards of a
+// context-parallel request): LSE = ln sum_g exp(lse_g), o = sum_g exp(lse_g - LSE) o_g.
+// One thread per (request, head, 4 dims).
+struct MergeParams {
+  int G, B, H, DV, o_f32;
+  const float* o_parts;    // [G,B,H,DV]
+  const float* lse_parts;  // [G,B,H]
+  void* o;                 // [B,H,DV]
+  float* lse;              // [B,H]
+};
+
+__global__ void __launch_bounds__(256) attn_merge_kernel(const MergeParams p) {
+  const long long item = (long long)blockIdx.x * 256 + threadIdx.x;
+  const int per_head = p.DV / 4;
+  if (item >= (long long)p.B * p.H * per_head) return;
+  const int d0 = (int)(item % per_head) * 4;
+  const long long bh = item / per_head;  // b * H + h
+  const size_t bhs = (size_t)p.B * p.H;
+  float M = -INFINITY;
+  for (int g = 0; g < p.G; ++g) M = fmaxf(M, p.lse_parts[g * bhs + bh]);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float den = 0.f;
+  if (M != -INFINITY) {
+    for (int g = 0; g < p.G; ++g) {
+      const float l = p.lse_parts[g * bhs + bh];
+      if (l == -INFINITY) continue;
+      const float wgt = expf(l - M);
+      den += wgt;
+      const float4 x = *(const float4*)(p.o_parts + (g * bhs + bh) * p.DV + d0);
+      acc.x = fmaf(wgt, x.x, acc.x); acc.y = fmaf(wgt, x.y, acc.y);
+      acc.z = fmaf(wgt, x.z, acc.z); acc.w = fmaf(wgt, x.w, acc.w);
+    }
+  }
+  const float inv = den > 0.f ? 1.f / den : 0.f;
+  if (p.o_f32) {
+    *(float4*)((float*)p.o + bh * p.DV + d0) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  } else {
+    __nv_bfloat162 a2 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    __nv_bfloat162 b2 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    *(uint2*)((__nv_bfloat16*)p.o + bh * p.DV + d0) = make_uint2(*(uint32_t*)&a2, *(uint32_t*)&b2);
+  }
+  if (d0 == 0) p.lse[bh] = den > 0.f ? M + logf(den) : -INFINITY;
 }
 
 }  // namespace ls

@@ -24,6 +24,9 @@ struct TopkParams {
   int len_limit;             // candidate counts above this are out of range
   const int* unit_list;      // optional: position of candidate i = unit_list[b][i/64]*64 + i%64
   int list_stride;
+  const int* pos_list;       // optional: position of candidate i = pos_list[b * pos_stride + i]
+  int pos_stride;
+  const int* pos_offset;     // optional [B]: added to every emitted position
   int* idx;                  // [B,k] (may be NULL: threshold only)
   float* sel;                // [B,k] (may be NULL)
   float* thr;                // [B] optional: k-th largest score, -inf if fewer than k candidates
@@ -34,8 +37,13 @@ constexpr int kTopkThreads = 512;
 constexpr int kTopkCacheKeys = 36864;  // at most 144 KB of cached keys per CTA
 
 __device__ __forceinline__ int topk_pos(const TopkParams& p, int b, int i) {
-  if (!p.unit_list) return i;
-  return p.unit_list[(size_t)b * p.list_stride + (i >> 6)] * 64 + (i & 63);
+  int pos = i;
+  if (p.pos_list) {
+    pos = p.pos_list[(size_t)b * p.pos_stride + i];
+  } else if (p.unit_list) {
+    pos = p.unit_list[(size_t)b * p.list_stride + (i >> 6)] * 64 + (i & 63);
+  }
+  return p.pos_offset ? pos + p.pos_offset[b] : pos;
 }
 
 // Buffers of the fast path (dynamic shared memory after the key cache).
