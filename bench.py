@@ -590,6 +590,98 @@ def run_prefill(args):
     return 0
 
 
+def run_cp(args):
+    """Optional line: one batch of long requests split by context over the ranks
+    (context-parallel, strong scaling): batch 4 x 1,048,576 tokens, full indexer scan of
+    each rank's shard, candidates and partial outputs all-gathered over NCCL."""
+    rank, world, local = rank_env()
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    from sparse_attention_decode_ls_b200 import binding as B
+    from sparse_attention_decode_ls_b200 import cp
+    from sparse_attention_decode_ls_b200 import synthetic as syn
+
+    batch, ctx, k = args.batch or 4, 1048576, TOPK
+    ranges = cp.shard_ranges([ctx] * batch, world)
+    begin = [ranges[b][rank][0] for b in range(batch)]
+    end = [ranges[b][rank][1] for b in range(batch)]
+    llens = [e - s for s, e in zip(begin, end)]
+    table, n_pool = syn.page_layout(llens, 3001 + rank)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(3002 + rank)  # this rank's shard of the history
+    k8 = torch.empty((n_pool, 64, 128), dtype=torch.uint8, device="cuda")
+    sk = torch.empty((n_pool, 64), dtype=torch.float32, device="cuda")
+    kv = torch.empty((n_pool, 64, 576), dtype=torch.bfloat16, device="cuda")
+    for i in range(0, n_pool, 4096):
+        j = min(n_pool, i + 4096)
+        x = torch.randn(((j - i) * 64, 128), generator=gen, device="cuda")
+        sc = x.abs().amax(dim=1, keepdim=True).clamp_min(1e-12) / 448.0
+        k8[i:j] = (x / sc).to(torch.float8_e4m3fn).view(torch.uint8).view(j - i, 64, 128)
+        sk[i:j] = sc.view(j - i, 64)
+        kv[i:j] = torch.randn((j - i, 64, 576), generator=gen, device="cuda").to(torch.bfloat16)
+    g = torch.Generator().manual_seed(3000)  # the queries: the same on every rank
+    q8, qs = syn.quantize_e4m3(torch.randn((batch, 64, 128), generator=g))
+    w = (torch.randn((batch, 64), generator=g) * 0.1).to(torch.bfloat16)
+    qa = torch.randn((batch, 128, 576), generator=g).to(torch.bfloat16)
+    dev = "cuda"
+    tdev = table.to(dev)
+    ml = max(4, (max(llens) + 3) // 4 * 4)
+    ix = B.index_args(q=q8.to(dev), w=w.to(dev), key_pool=k8, page_table=tdev,
+                      lens=torch.tensor(llens, dtype=torch.int32, device=dev), q_scale=qs.view(batch, 64).to(dev),
+                      key_scale=sk, max_len=ml)
+    step = cp.ShardStep(index=ix, k=k, attn=dict(q=qa.to(dev), kv=kv, page_table=tdev, scale=syn.softmax_scale(576)),
+                        begin=torch.tensor(begin, dtype=torch.int32, device=dev),
+                        end=torch.tensor(end, dtype=torch.int32, device=dev), world=world)
+    o = torch.empty((batch, 128, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((batch, 128), device=dev)
+    stream = torch.cuda.current_stream()
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        step.step(o, lse)
+    torch.cuda.synchronize()
+    B.ls_check_device_status()
+    if dist:
+        dist.barrier()
+    ev = []
+    with ClockSampler(local) as clk:
+        for _ in range(args.steps):
+            flush_w.zero_()
+            torch.sum(flush_r, dim=0, out=sink)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            step.step(o, lse)
+            e1.record(stream)
+            ev.append((e0, e1))
+        torch.cuda.synchronize()
+    status = B.ls_check_device_status()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    if dist:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    if rank == 0:
+        out = {"metric": "context-parallel sparse-attn decode tokens/s at 1M ctx", "value": batch / (ms / 1e3),
+               "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+               "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+               "dtype": "e4m3+bf16 (f32 accumulate)", "data": "synthetic",
+               "config": {"workload": f"cp_b{batch}_ctx{ctx}", "batch": batch, "ctx": ctx, "topk": k,
+                          "parallelism": f"context-parallel over {world} GPU(s)",
+                          "exchange_bytes_per_step": world * batch * (k * 8 + 128 * 512 * 4 + 128 * 4),
+                          "l2": "evicted before every step (256 MB written, then 256 MB read)"},
+               "clocks": clk.summary(), "device_status": status}
+        print(json.dumps(out), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -598,9 +690,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["mla", "hotbuf", "c2f", "prefill"], default="mla",
+    ap.add_argument("--workload", choices=["mla", "hotbuf", "c2f", "prefill", "cp"], default="mla",
                     help="mla: the headline step (default); hotbuf: the hot-buffer step; c2f: the "
-                         "coarse-to-fine step at 1M context; prefill: layer-streaming prefill (one GPU each)")
+                         "coarse-to-fine step at 1M context; prefill: layer-streaming prefill (one GPU each); "
+                         "cp: 1M-context requests split by context over the ranks")
     ap.add_argument("--keys", choices=["hbm", "host"], default="hbm", help="c2f: where the original keys live")
     ap.add_argument("--batch", type=int, default=0, help="hotbuf: requests (default 36)")
     ap.add_argument("--miss", type=float, default=0.2, help="hotbuf: fraction of the selection that misses")
@@ -613,6 +706,8 @@ def main():
         return run_c2f(args)
     if args.workload == "prefill":
         return run_prefill(args)
+    if args.workload == "cp":
+        return run_cp(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
