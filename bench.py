@@ -437,10 +437,75 @@ def run_hotbuf(args):
            "config": {"workload": wl.name, "batch": batch, "ctx": CTX, "topk": TOPK, "hot_slots": 4096,
                       "miss_frac": args.miss, "history": "pinned host memory, read over the host link",
                       "l2": "evicted before every step (256 MB written, then 256 MB read)"},
+           "gpu_launches": wl.kernels_per_step * args.steps,
            "host_link": {"bytes_per_step": link_bytes, "GBps": link_bytes / (ms / 1e3) / 1e9,
                          "gather_GBps": link_bytes / (stages["gather"] / 1e3) / 1e9},
            "stages_ms": stages,
            "clocks": clk.summary(), "device_status": status}
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+def run_sweep(args):
+    """Optional line: the ragged mixed-batch sweep -- batch 1, 16, 64, 192 and 256, context
+    lengths ~U[4096, 16384] per request, top-2048, a 4,096-slot hot buffer per request with
+    20% of the selection missing, history in pinned host memory -- per-step latency (the
+    TPOT proxy of one layer) and tokens/s against the batch."""
+    import gc
+    import torch
+    from sparse_attention_decode_ls_b200 import binding as B
+    from sparse_attention_decode_ls_b200 import synthetic as syn
+    from sparse_attention_decode_ls_b200 import workload as W
+
+    batches = [int(x) for x in args.batches.split(",")] if args.batches else [1, 16, 64, 192, 256]
+    stream = torch.cuda.current_stream()
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush_r = torch.ones(64 << 20, dtype=torch.float32, device="cuda")
+    sink = torch.empty((), dtype=torch.float32, device="cuda")
+    rows, statuses = [], []
+    with ClockSampler(0) as clk:
+        for bsz in batches:
+            lens = syn.ragged_lens(bsz, 4096, 16384, seed=1005)
+            wl = W.mla_hotbuf_decode(lens=lens, miss_frac=0.2, seed=1005, device="cuda")
+
+            def prep():
+                wl.restore_hotbuf()
+                flush_w.zero_()
+                torch.sum(flush_r, dim=0, out=sink)
+
+            for _ in range(args.warmup):
+                prep()
+                wl.step()
+            torch.cuda.synchronize()
+            statuses.append(B.ls_check_device_status())
+            ev = []
+            for _ in range(args.steps):
+                prep()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                wl.step()
+                e1.record(stream)
+                ev.append((e0, e1))
+            torch.cuda.synchronize()
+            statuses.append(B.ls_check_device_status())
+            ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+            n_miss = int(wl.tensors["n_miss"].sum().item())
+            rows.append({"batch": bsz, "ms_per_step": ms, "tokens_per_s": bsz / (ms / 1e3),
+                         "mean_ctx": sum(lens) / bsz, "link_bytes_per_step": n_miss * 1152,
+                         "gpu_launches_per_step": wl.kernels_per_step})
+            del wl
+            gc.collect()
+            torch.cuda.empty_cache()
+    out = {"metric": "ragged batch sweep: per-step latency (one layer) and tokens/s vs batch",
+           "value": rows[-1]["tokens_per_s"], "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": rows[-1]["ms_per_step"], "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "e4m3+bf16 (f32 accumulate)", "data": "synthetic",
+           "config": {"workload": "ragged_hotbuf_sweep", "batches": batches, "ctx": "U[4096, 16384] per request",
+                      "topk": TOPK, "hot_slots": 4096, "miss_frac": 0.2,
+                      "history": "pinned host memory, misses read over the host link",
+                      "l2": "evicted before every step (256 MB written, then 256 MB read)",
+                      "statistic": "median over the timed steps"},
+           "sweep": rows, "clocks": clk.summary(), "device_status": max(statuses) if statuses else 0}
     print(json.dumps(out), flush=True)
     return 0
 
@@ -483,6 +548,45 @@ def run_c2f(args):
         torch.cuda.synchronize()
     status = B.ls_check_device_status()
     ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    full = None
+    if not on_host:
+        # the full scan on the same data: every key scored, then the top-k -- the selection
+        # must be the coarse-to-fine one, and its time is what the pruning saves
+        t = wl.tensors
+        scores = torch.empty((batch, ctx), dtype=torch.float32, device="cuda")
+        idx_full = torch.empty((batch, TOPK), dtype=torch.int32, device="cuda")
+
+        def full_scan():
+            B.ls_index_score(q=t["i_q"], w=t["i_w"], key_pool=t["i_key_pool"], page_table=t["i_page_table"],
+                             lens=t["i_lens"], scores=scores, q_scale=t["i_q_scale"], key_scale=t["i_key_scale"])
+            B.ls_topk_select(scores=scores, lens=t["i_lens"], idx=idx_full)
+
+        for _ in range(args.warmup):
+            prep()
+            full_scan()
+        fev = []
+        for _ in range(args.steps):
+            prep()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            full_scan()
+            e1.record(stream)
+            fev.append((e0, e1))
+        # the coarse-to-fine part of the step alone, for the same comparison
+        cev = []
+        for _ in range(args.steps):
+            prep()
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+            for e in evs:
+                e.record(stream)
+            wl.step(events=B.event_array(evs))
+            cev.append(evs)
+        torch.cuda.synchronize()
+        fms = statistics.mean(a.elapsed_time(b) for a, b in fev)
+        cms = statistics.mean(e[0].elapsed_time(e[4]) for e in cev)
+        full = {"indexer_plus_topk_ms": fms, "c2f_indexer_plus_topk_ms": cms, "speedup": fms / cms,
+                "same_selection": bool(torch.equal(idx_full, wl.idx))}
+        status |= B.ls_check_device_status()
     n_surv = [int(x) for x in wl.tensors["n_survivors"].tolist()]
     n_blocks = -(-ctx // 64)
     nb0 = (TOPK + 63) // 64 + 1
@@ -494,7 +598,9 @@ def run_c2f(args):
            "config": {"workload": wl.name, "batch": batch, "ctx": ctx, "topk": TOPK,
                       "keys": "pinned host memory (only summaries in HBM)" if on_host else "HBM",
                       "l2": "evicted before every step (256 MB written, then 256 MB read)"},
-           "survivors": {"per_request": n_surv, "of_blocks": n_blocks},
+           "survivors": {"per_request": n_surv, "of_blocks": n_blocks,
+                         "fraction": sum(n_surv) / (batch * n_blocks)},
+           "full_scan": full,
            "indexer_key_bytes": {"in_hbm": 0 if on_host else batch * ctx * 132,
                                  "over_host_link_per_step": (batch * nb0 + sum(n_surv)) * block_bytes if on_host else 0},
            "gpu_launches": wl.kernels_per_step * args.steps,
@@ -690,10 +796,11 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", choices=["mla", "hotbuf", "c2f", "prefill", "cp"], default="mla",
+    ap.add_argument("--batches", default="", help="sweep: comma-separated batch sizes (default 1,16,64,192,256)")
+    ap.add_argument("--workload", choices=["mla", "hotbuf", "c2f", "prefill", "cp", "sweep"], default="mla",
                     help="mla: the headline step (default); hotbuf: the hot-buffer step; c2f: the "
                          "coarse-to-fine step at 1M context; prefill: layer-streaming prefill (one GPU each); "
-                         "cp: 1M-context requests split by context over the ranks")
+                         "cp: 1M-context requests split by context over the ranks; sweep: ragged batch sweep")
     ap.add_argument("--keys", choices=["hbm", "host"], default="hbm", help="c2f: where the original keys live")
     ap.add_argument("--batch", type=int, default=0, help="hotbuf: requests (default 36)")
     ap.add_argument("--miss", type=float, default=0.2, help="hotbuf: fraction of the selection that misses")
@@ -708,6 +815,8 @@ def main():
         return run_prefill(args)
     if args.workload == "cp":
         return run_cp(args)
+    if args.workload == "sweep":
+        return run_sweep(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

@@ -187,12 +187,14 @@ def mla_decode(batch=8, ctx=131072, k=2048, seed=1002, device="cuda", kv_on_devi
 
 
 def mla_hotbuf_decode(batch=36, ctx=131072, k=2048, miss_frac=0.2, n_slots=4096, seed=1003,
-                      device="cuda") -> DecodeWorkload:
+                      device="cuda", lens=None) -> DecodeWorkload:
     """The hot-buffer configuration: the full KV history in pinned host memory, a
     4,096-slot hot buffer per request in HBM holding all but a seeded ``miss_frac`` of this
     step's selection (the selection of the GPU's own indexer and top-k), filled up with
-    other positions.  Restore the buffer state (``restore_hotbuf``) before every step."""
-    lens = [ctx] * batch
+    other positions.  Restore the buffer state (``restore_hotbuf``) before every step.
+    ``lens`` (one length per request) replaces batch x ctx, e.g. a ragged batch."""
+    lens = [ctx] * batch if lens is None else [int(x) for x in lens]
+    batch, ctx = len(lens), max(lens)
     ind = syn.indexer_fp8(lens, seed=seed)
     n_pool = ind.key_pool.shape[0]
     q, kv_dev = syn.mla_attention(batch, n_pool, seed=seed + 1000, device=device)
@@ -211,7 +213,8 @@ def mla_hotbuf_decode(batch=36, ctx=131072, k=2048, miss_frac=0.2, n_slots=4096,
     del d, scores
     pos_of_slot, slot_of_pos, recent = syn.hot_buffer_state([r[r >= 0] for r in sel], lens, n_slots=n_slots,
                                                             miss_frac=miss_frac, seed=seed + 2000, max_len=ml)
-    return build(f"mla_hotbuf_b{batch}_ctx{ctx}_miss{int(round(miss_frac * 100))}", ind, k=k, device=device,
+    name = f"mla_hotbuf_b{batch}_ctx{ctx}" if len(set(lens)) == 1 else f"mla_hotbuf_ragged_b{batch}"
+    return build(f"{name}_miss{int(round(miss_frac * 100))}", ind, k=k, device=device,
                  attn=dict(q=q, kv_host=True, scale=syn.softmax_scale(576)),
                  hotbuf=dict(pos_of_slot=pos_of_slot, slot_of_pos=slot_of_pos, recent=recent, host_kv=host))
 
