@@ -18,6 +18,7 @@
 #include "common.cuh"
 #include "hotbuf.cuh"
 #include "cp.cuh"
+#include "topk_row.cuh"
 #include "index_score.cuh"
 #include "topk.cuh"
 
@@ -255,7 +256,12 @@ ls_status launch_index_tc(const ls_index_score_args* a, int mode, const int* uni
 // ---- top-k launch -------------------------------------------------------------------
 // One cluster per request: 16 CTAs where the device can co-schedule them (non-portable
 // cluster size), else the portable 8.
-std::atomic<uint64_t> g_smem_topk8{0}, g_smem_topk16{0};
+cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, size_t smem, cudaStream_t st, cudaLaunchAttribute* attr,
+                              bool pdl);
+std::atomic<uint64_t> g_smem_topk8{0}, g_smem_topk16{0}, g_smem_topk_row{0};
+// Requests up to this many candidates go to the one-CTA top-k, longer ones to a cluster
+// (measured: at 131,072 scores per request one CTA takes ~50 us, a 16-CTA cluster ~20 us).
+constexpr int kTopkRowMaxLen = 32768;
 std::atomic<int> g_topk16_ok[64];  // per device: 0 unknown, 1 yes, -1 no
 
 template <int CL>
@@ -321,6 +327,16 @@ ls_status launch_topk(int B, int k, const float* scores, int stride, const int* 
   p.B = B; p.k = k; p.stride = stride; p.scores = scores; p.lens = lens; p.len_mul = len_mul;
   p.len_div = len_div; p.len_limit = len_limit; p.unit_list = unit_list; p.list_stride = list_stride;
   p.idx = idx; p.sel = sel; p.thr = thr;
+  if (len_limit <= kTopkRowMaxLen) {
+    // one CTA per request: few SMs for a small batch and no cluster barriers
+    if (allow_smem(ls::topk_row, ls::kRowSmem, g_smem_topk_row) != cudaSuccess)
+      return check_launch("topk_row attribute");
+    cudaLaunchAttribute attr[2];
+    cudaLaunchConfig_t cfg = pdl_config(dim3(B), dim3(ls::kRowThreads), ls::kRowSmem, st, attr, true);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, ls::topk_row, p);
+    if (e != cudaSuccess) return fail(LS_ERR_CUDA, "topk_row: %s", cudaGetErrorString(e));
+    return check_launch("topk_row");
+  }
   if (topk16_supported(st)) return launch_topk_cl<16>(p, B, st, g_smem_topk16);
   return launch_topk_cl<8>(p, B, st, g_smem_topk8);
 }

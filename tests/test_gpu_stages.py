@@ -65,6 +65,10 @@ def _topk_case(lens, k, seed, kind="normal"):
     elif kind == "zeros":
         s = torch.randint(0, 3, (len(lens), ml), generator=g).float() - 1.0
         s = torch.where(s == 0, torch.where(torch.rand(s.shape, generator=g) < 0.5, -0.0, 0.0), s)
+    elif kind in ("ascending", "descending"):
+        # the largest scores bunched at one end of the request
+        s = torch.arange(ml, dtype=torch.float32)[None].repeat(len(lens), 1)
+        s = s if kind == "ascending" else -s
     else:
         s = torch.randn((len(lens), ml), generator=g)
     lens_t = torch.tensor(lens, dtype=torch.int32)
@@ -91,6 +95,21 @@ def test_topk_exact(lens, k):
 @pytest.mark.parametrize("kind", ["ties", "zeros"])
 def test_topk_ties_lower_position_first(kind):
     _topk_case([3000, 40000, 129], 512, seed=5, kind=kind)
+
+
+@pytest.mark.parametrize("kind", ["ascending", "descending"])
+@pytest.mark.parametrize("lens", [[32768, 20001, 6000], [131072, 70001, 6000]])
+def test_topk_bunched_scores(kind, lens):
+    # the top keys of a request share a few segments: (short requests) the per-segment
+    # lists of the one-CTA kernel overflow and it finishes from the scores; (long ones) the
+    # cluster kernel's candidate buffers overflow into its general path
+    _topk_case(lens, 2048, seed=7, kind=kind)
+
+
+@pytest.mark.parametrize("kind", ["ties", "zeros"])
+def test_topk_ties_short_requests(kind):
+    # the one-CTA kernel (every request at most 32,768 scores)
+    _topk_case([3000, 20000, 129, 32768], 512, seed=6, kind=kind)
 
 
 def test_topk_full_scan_1m_context():
