@@ -504,13 +504,10 @@ ls_status launch_hotbuf(const ls_hotbuf_args* a, cudaStream_t st) {
   p.sel_score = a->sel_score; p.pos_of_slot = a->pos_of_slot; p.recent = a->recent_score;
   p.slot_of_pos = a->slot_of_pos; p.sel_slot = a->sel_slot; p.miss_pos = a->miss_pos; p.miss_slot = a->miss_slot;
   p.n_miss = a->n_miss;
-  int pow2 = 1;
-  while (pow2 < a->n_slots) pow2 <<= 1;
-  const int smem = pow2 * 8;
-  if (allow_smem(ls::hotbuf_resolve_kernel, ls::kHbMaxSlots * 8, g_smem_hb) != cudaSuccess ||
+  if (allow_smem(ls::hotbuf_resolve_kernel, ls::kHbResolveSmem, g_smem_hb) != cudaSuccess ||
       keep_smem_carveout(ls::hotbuf_resolve_kernel, g_carve_hb) != cudaSuccess)
     return check_launch("hotbuf attribute");
-  ls::hotbuf_resolve_kernel<<<a->batch, ls::kHbThreads, smem, st>>>(p);
+  ls::hotbuf_resolve_kernel<<<a->batch, ls::kHbThreads, ls::kHbResolveSmem, st>>>(p);
   return check_launch("hotbuf_resolve");
 }
 

@@ -38,12 +38,18 @@ struct HotbufParams {
 
 constexpr int kHbThreads = 1024;
 constexpr int kHbMaxSlots = 4096;
+// dynamic shared memory of the resolve: keys (8 B), miss list (4 B), then the radix
+// histogram (16 KB) overlaid by up to 4,096 victim keys (8 B)
+constexpr int kHbResolveSmem = kHbMaxSlots * (8 + 4 + 8);
 
 __global__ void __launch_bounds__(kHbThreads, 1) hotbuf_resolve_kernel(const HotbufParams p) {
-  extern __shared__ unsigned long long keys[];       // [next pow2 >= n_slots] sort buffer
+  extern __shared__ unsigned long long keys[];       // [4096] victim keys, then the victim order
+  int* miss_j = (int*)(keys + kHbMaxSlots);          // [4096] selection index of the i-th miss
+  uint32_t* scratch = (uint32_t*)(miss_j + kHbMaxSlots);  // radix histogram, then victim keys
   __shared__ uint8_t pinned[kHbMaxSlots];
-  __shared__ int miss_j[kHbMaxSlots];               // selection index of the i-th miss
   __shared__ unsigned long long scan_tmp[32];
+  __shared__ int s_sel_bin;
+  __shared__ uint32_t s_sel_below, s_nvict;
   const int b = blockIdx.x, tid = threadIdx.x;
   const int k = p.k, S = p.n_slots;
   const int* sel = p.sel + (size_t)b * k;
@@ -97,15 +103,14 @@ __global__ void __launch_bounds__(kHbThreads, 1) hotbuf_resolve_kernel(const Hot
       }
     }
   }
-  // ---- victim order: (class, recent-score key, slot); class 0 empty, 1 occupied, 2 pinned
-  int n_pow2 = 1;
-  while (n_pow2 < S) n_pow2 <<= 1;
+  // ---- victims: the n_miss smallest keys (class, recent-score key, slot), class 0 empty,
+  // 1 occupied, 2 pinned; keys are distinct (the slot is in them).  A radix select (four
+  // 12-bit digits) finds the n_miss-th smallest key; the keys up to it are gathered and each
+  // one's rank among them (a count of the smaller ones) is its victim order.
   __syncthreads();
-  for (int s = tid; s < n_pow2; s += kHbThreads) {
+  for (int s = tid; s < S; s += kHbThreads) {
     unsigned long long key;
-    if (s >= S) {
-      key = ~0ull;
-    } else if (pinned[s]) {
+    if (pinned[s]) {
       key = (2ull << 44) | s;
     } else if (pos_of_slot[s] < 0) {
       key = (unsigned long long)s;
@@ -114,21 +119,55 @@ __global__ void __launch_bounds__(kHbThreads, 1) hotbuf_resolve_kernel(const Hot
     }
     keys[s] = key;
   }
-  __syncthreads();
-  for (int size = 2; size <= n_pow2; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int t = tid; t < (n_pow2 >> 1); t += kHbThreads) {
-        const int lo = 2 * t - (t & (stride - 1));
-        const int hi = lo + stride;
-        const bool up = (lo & size) == 0;
-        const unsigned long long a = keys[lo], c = keys[hi];
-        if ((a > c) == up) {
-          keys[lo] = c;
-          keys[hi] = a;
-        }
+  unsigned long long thr = 0;  // the n_miss-th smallest key
+  if (n_miss > 0) {
+    uint32_t* hist = scratch;  // 4,096 bins
+    unsigned long long prefix = 0;
+    uint32_t m_rem = (uint32_t)n_miss;
+    for (int dg = 3; dg >= 0; --dg) {
+      const int shift = dg * 12;
+      for (int d = tid; d < 4096; d += kHbThreads) hist[d] = 0;
+      __syncthreads();
+      for (int s = tid; s < S; s += kHbThreads) {
+        const unsigned long long key = keys[s];
+        if (dg == 3 || (key >> (shift + 12)) == prefix) atomicAdd(&hist[(key >> shift) & 4095ull], 1u);
       }
       __syncthreads();
+      // bins in ascending order, four per thread
+      uint32_t mine = hist[4 * tid] + hist[4 * tid + 1] + hist[4 * tid + 2] + hist[4 * tid + 3];
+      unsigned long long tot;
+      uint32_t below = (uint32_t)block_excl_scan_u64(mine, scan_tmp, &tot);
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t h = hist[4 * tid + j];
+        if (below < m_rem && below + h >= m_rem) {
+          s_sel_bin = 4 * tid + j;
+          s_sel_below = below;
+        }
+        below += h;
+      }
+      __syncthreads();
+      prefix = (prefix << 12) | (unsigned long long)s_sel_bin;
+      m_rem -= s_sel_below;
+      __syncthreads();
     }
+    thr = prefix;
+    // the keys up to the threshold (exactly n_miss of them), then their ranks
+    if (tid == 0) s_nvict = 0;
+    __syncthreads();
+    unsigned long long* vict = (unsigned long long*)hist;  // reuses the histogram space
+    for (int s = tid; s < S; s += kHbThreads) {
+      const unsigned long long key = keys[s];
+      if (key <= thr) vict[atomicAdd(&s_nvict, 1u)] = key;
+    }
+    __syncthreads();
+    const int nv = (int)s_nvict;  // == n_miss
+    for (int i = tid; i < nv; i += kHbThreads) {
+      const unsigned long long key = vict[i];
+      int rank = 0;
+      for (int j = 0; j < nv; ++j) rank += vict[j] < key ? 1 : 0;
+      keys[rank] = key;  // the victim order, over the start of the key array
+    }
+    __syncthreads();
   }
   // ---- apply: the i-th miss takes the i-th victim
   for (int i = tid; i < n_miss; i += kHbThreads) {
