@@ -681,7 +681,7 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine(const AttnParams
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
   float Lsum = 0.f;
   if (M != -INFINITY) {
-#pragma unroll 4
+#pragma unroll 8
     for (int s = 0; s < p.nsplit_total; ++s) {
       const float l = ml[(size_t)s * H * 2 + 1];
       if (!(l > 0.f)) continue;

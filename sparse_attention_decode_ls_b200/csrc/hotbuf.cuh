@@ -221,20 +221,25 @@ __global__ void __launch_bounds__(kHbThreads, 1) hotbuf_classify_kernel(const Cl
   const int j0 = min(k, tid * per), j1 = min(k, j0 + per);
   int pos[4], slot[4];
   uint32_t n_m = 0, n_h = 0;
-  for (int j = j0; j < j1; ++j) {
-    const int q = j - j0;
-    pos[q] = sel[j];
+  // all of this thread's selections first, then all their map lookups: two round trips
+#pragma unroll
+  for (int q = 0; q < 4; ++q) pos[q] = j0 + q < j1 ? sel[j0 + q] : -1;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
     slot[q] = -2;  // neither (padding or out of range)
     if (pos[q] >= 0) {
       if (pos[q] >= p.max_len) {
         flag(LS_DEV_BOUNDS);
       } else {
         slot[q] = slot_of_pos[pos[q]];
-        if (slot[q] >= S) {
-          flag(LS_DEV_BOUNDS);
-          slot[q] = -2;
-        }
       }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    if (slot[q] >= S) {
+      flag(LS_DEV_BOUNDS);
+      slot[q] = -2;
     }
     n_m += slot[q] == -1;
     n_h += slot[q] >= 0;
