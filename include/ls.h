@@ -497,6 +497,14 @@ ls_status ls_prefill_stream(const ls_prefill_stream_args* args, void* workspace,
 /* ------------------------------------------------------------------------------
  * Diagnostics.
  * --------------------------------------------------------------------------- */
+/* Every wait inside a kernel (on a barrier or a peer) gives up after a time limit,
+ * raises LS_DEV_TIMEOUT in the device status and lets the kernel return; 2 s by
+ * default.  ls_set_wait_limit sets it for the current device, in [1 us, 10 s].
+ * ls_selftest_bounded_wait launches one wait that nothing completes, so a caller can
+ * check that it ends with LS_DEV_TIMEOUT (after the limit) and a usable context. */
+ls_status ls_set_wait_limit(uint64_t ns);
+ls_status ls_selftest_bounded_wait(ls_stream_t stream);
+
 /* Message of the calling thread's last error (empty string if none). */
 const char* ls_get_error_string(void);
 

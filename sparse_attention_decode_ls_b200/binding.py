@@ -143,6 +143,10 @@ def lib():
         L.ls_sparse_attn_decode_noalloc.restype = C.c_int
         L.ls_build_block_summaries.argtypes = [P(IndexScoreArgs), _p, _p, _i32, _p]
         L.ls_build_block_summaries.restype = C.c_int
+        L.ls_set_wait_limit.argtypes = [C.c_uint64]
+        L.ls_set_wait_limit.restype = C.c_int
+        L.ls_selftest_bounded_wait.argtypes = [_p]
+        L.ls_selftest_bounded_wait.restype = C.c_int
         L.ls_get_error_string.restype = C.c_char_p
         L.ls_version.restype = C.c_char_p
         L.ls_check_device_status.argtypes = [_p, P(C.c_uint32)]
@@ -459,3 +463,12 @@ def ls_attn_merge(*, o_parts, lse_parts, o, lse, stream=None):
     a.o_parts, a.lse_parts, a.o, a.lse = _ptr(o_parts), _ptr(lse_parts), _ptr(o), _ptr(lse)
     a.o_dtype = LS_F32 if o.dtype == torch.float32 else LS_BF16
     _check(lib().ls_attn_merge(C.byref(a), _stream(stream)))
+
+
+# ------------------------------------------------------------------------------- diagnostics
+def ls_set_wait_limit(ns: int):
+    _check(lib().ls_set_wait_limit(int(ns)))
+
+
+def ls_selftest_bounded_wait(stream=None):
+    _check(lib().ls_selftest_bounded_wait(_stream(stream)))

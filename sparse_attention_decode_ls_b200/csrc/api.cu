@@ -932,6 +932,20 @@ ls_status ls_check_device_status(ls_stream_t stream, uint32_t* flags) {
   return ok();
 }
 
+ls_status ls_set_wait_limit(uint64_t ns) {
+  LS_REQUIRE(ns >= 1000 && ns <= 10000000000ull, "the wait limit must be in [1 us, 10 s]");
+  const unsigned long long v = ns;
+  cudaError_t e = cudaMemcpyToSymbol(ls::g_wait_limit_ns, &v, sizeof(v));
+  if (e != cudaSuccess) return fail(LS_ERR_CUDA, "set wait limit: %s", cudaGetErrorString(e));
+  return ok();
+}
+
+ls_status ls_selftest_bounded_wait(ls_stream_t stream) {
+  ls::wait_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>();
+  LS_TRY(check_launch("wait_selftest"));
+  return ok();
+}
+
 ls_status ls_index_score(const ls_index_score_args* args, ls_stream_t stream) {
   LS_TRY(validate_index(args, true));
   cudaStream_t st = (cudaStream_t)stream;

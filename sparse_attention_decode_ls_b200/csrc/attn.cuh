@@ -474,7 +474,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
           const uint64_t now = globaltimer();
           if (idle_since == 0) {
             idle_since = now;
-          } else if (now - idle_since > kWaitLimitNs) {
+          } else if (now - idle_since > *(volatile unsigned long long*)&g_wait_limit_ns) {
             flag(LS_DEV_TIMEOUT);
             ok = false;
           }

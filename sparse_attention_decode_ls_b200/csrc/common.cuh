@@ -26,8 +26,10 @@ __device__ unsigned int g_status;
 __device__ __forceinline__ void flag(unsigned int bits) { atomicOr(&g_status, bits); }
 
 // Longest time any single wait inside a kernel may take before it gives up, flags
-// LS_DEV_TIMEOUT and lets the kernel unwind.  No legitimate wait comes close.
+// LS_DEV_TIMEOUT and lets the kernel unwind.  No legitimate wait comes close.  It is read
+// only once a wait has not completed at its first probe; ls_set_wait_limit changes it.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+__device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
 
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
@@ -83,14 +85,14 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete; gives up after kWaitLimitNs,
+// Wait for the phase with the given parity to complete; gives up after g_wait_limit_ns,
 // raising LS_DEV_TIMEOUT.  Returns false on timeout.  The polling loop is out of line;
 // a phase that has already completed costs one inline probe.
 __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer();
+  const uint64_t t0 = globaltimer(), limit = *(volatile unsigned long long*)&g_wait_limit_ns;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit) {
       flag(LS_DEV_TIMEOUT);
       return false;
     }
@@ -150,10 +152,10 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 
 // As mbar_wait, with acquire at cluster scope (the arrivals come from another CTA).
 __device__ __noinline__ bool mbar_wait_cluster_slow(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer();
+  const uint64_t t0 = globaltimer(), limit = *(volatile unsigned long long*)&g_wait_limit_ns;
   while (true) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit) {
       flag(LS_DEV_TIMEOUT);
       return false;
     }
@@ -420,5 +422,16 @@ __device__ __forceinline__ unsigned long long block_excl_scan_u64(unsigned long 
   return res;
 }
 
+
+// Self-test of the bounded wait: one thread waits on a barrier that nothing will ever
+// complete, so the wait must give up, raise LS_DEV_TIMEOUT and let the kernel return.
+__global__ void wait_selftest_kernel() {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait(&bar, 0);  // no arrival: times out
+  }
+}
 
 }  // namespace ls
