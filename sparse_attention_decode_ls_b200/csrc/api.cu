@@ -4,6 +4,7 @@
 // device status word is a single symbol).
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <atomic>
 #include <cmath>
@@ -911,6 +912,13 @@ ls_status prefill_streams(PrefillStreams** out) {
 
 }  // namespace
 
+// An NVTX range around each entry point, so that a profiler's timeline names the calls
+// (without a tool attached a push and a pop cost a few nanoseconds).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+
 // =========================================================================================
 // C ABI
 // =========================================================================================
@@ -947,6 +955,7 @@ ls_status ls_selftest_bounded_wait(ls_stream_t stream) {
 }
 
 ls_status ls_index_score(const ls_index_score_args* args, ls_stream_t stream) {
+  NvtxRange nvtx_range("ls_index_score");
   LS_TRY(validate_index(args, true));
   cudaStream_t st = (cudaStream_t)stream;
   if (args->key_dtype == LS_E4M3 && args->variant == 0) {
@@ -959,6 +968,7 @@ ls_status ls_index_score(const ls_index_score_args* args, ls_stream_t stream) {
 }
 
 ls_status ls_topk_select(const ls_topk_args* a, ls_stream_t stream) {
+  NvtxRange nvtx_range("ls_topk_select");
   LS_REQUIRE(a, "args is NULL");
   LS_REQUIRE(a->batch >= 1 && a->k >= 1 && a->k <= 4096, "batch >= 1 and 1 <= k <= 4096 required");
   LS_REQUIRE(a->max_len >= 1 && (a->max_len % 4) == 0, "max_len must be a positive multiple of 4");
@@ -971,6 +981,7 @@ ls_status ls_topk_select(const ls_topk_args* a, ls_stream_t stream) {
 
 ls_status ls_build_block_summaries(const ls_index_score_args* keys, uint8_t* summaries, float* block_scale,
                                    int32_t max_blocks, ls_stream_t stream) {
+  NvtxRange nvtx_range("ls_build_block_summaries");
   LS_TRY(validate_index(keys, false));
   if (keys->key_dtype != LS_E4M3) return fail(LS_ERR_UNSUPPORTED, "summaries need e4m3 keys");
   LS_REQUIRE(summaries && block_scale && max_blocks >= 1, "summaries, block_scale, max_blocks required");
@@ -991,6 +1002,7 @@ size_t ls_cp_merge_workspace_size(const ls_cp_merge_args* a) {
 }
 
 ls_status ls_cp_merge_topk(const ls_cp_merge_args* a, void* workspace, size_t workspace_bytes, ls_stream_t stream) {
+  NvtxRange nvtx_range("ls_cp_merge_topk");
   LS_REQUIRE(a, "args is NULL");
   LS_REQUIRE(a->shards >= 1 && a->batch >= 1 && a->k >= 1 && a->k <= 4096, "shards, batch >= 1, 1 <= k <= 4096");
   LS_REQUIRE((long long)a->shards * a->k <= (1 << 24), "shards * k too large");
@@ -1021,6 +1033,7 @@ ls_status ls_cp_merge_topk(const ls_cp_merge_args* a, void* workspace, size_t wo
 }
 
 ls_status ls_attn_merge(const ls_attn_merge_args* a, ls_stream_t stream) {
+  NvtxRange nvtx_range("ls_attn_merge");
   LS_REQUIRE(a, "args is NULL");
   LS_REQUIRE(a->parts >= 1 && a->batch >= 1 && a->heads >= 1 && a->dv >= 4 && a->dv % 4 == 0,
              "parts, batch, heads >= 1 and dv a positive multiple of 4 required");
@@ -1044,6 +1057,7 @@ size_t ls_prefill_stream_workspace_size(const ls_prefill_stream_args* args) {
 
 ls_status ls_prefill_stream(const ls_prefill_stream_args* a, void* workspace, size_t workspace_bytes,
                             ls_stream_t stream) {
+  NvtxRange nvtx_range("ls_prefill_stream");
   LS_TRY(validate_prefill(a));
   const PrefillLayout l = prefill_layout(a);
   LS_REQUIRE(workspace && workspace_bytes >= l.total, "workspace too small (%zu < %zu bytes)", workspace_bytes,
@@ -1106,6 +1120,7 @@ size_t ls_block_bound_prune_workspace_size(const ls_block_bound_prune_args* args
 
 ls_status ls_block_bound_prune(const ls_block_bound_prune_args* args, void* workspace, size_t workspace_bytes,
                                ls_stream_t stream) {
+  NvtxRange nvtx_range("ls_block_bound_prune");
   LS_TRY(validate_c2f(args));
   LS_TRY(run_c2f(args, workspace, workspace_bytes, args->survivors, args->n_survivors, nullptr,
                  (cudaStream_t)stream));
@@ -1113,12 +1128,14 @@ ls_status ls_block_bound_prune(const ls_block_bound_prune_args* args, void* work
 }
 
 ls_status ls_hotbuf_resolve(const ls_hotbuf_args* args, ls_stream_t stream) {
+  NvtxRange nvtx_range("ls_hotbuf_resolve");
   LS_TRY(validate_hotbuf(args));
   LS_TRY(launch_hotbuf(args, (cudaStream_t)stream));
   return ok();
 }
 
 ls_status ls_gather_misses(const ls_gather_args* args, ls_stream_t stream) {
+  NvtxRange nvtx_range("ls_gather_misses");
   LS_TRY(validate_gather(args));
   LS_TRY(launch_gather(args, (cudaStream_t)stream));
   return ok();
@@ -1131,6 +1148,7 @@ size_t ls_sparse_attn_workspace_size(const ls_sparse_attn_args* args) {
 
 ls_status ls_sparse_attn_decode(const ls_sparse_attn_args* a, void* workspace, size_t workspace_bytes,
                                 ls_stream_t stream) {
+  NvtxRange nvtx_range("ls_sparse_attn_decode");
   LS_TRY(validate_attn(a, true));
   LS_TRY(launch_attn(a, a->sel, a->addressing, a->page_table, a->max_pages, a->n_slots, nullptr, a->num_rows,
                      workspace, workspace_bytes, (cudaStream_t)stream, false));
@@ -1144,6 +1162,7 @@ size_t ls_decode_step_workspace_size(const ls_decode_step_args* args) {
 
 ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t workspace_bytes,
                          ls_stream_t stream) {
+  NvtxRange nvtx_range("ls_decode_step");
   LS_REQUIRE(a, "args is NULL");
   LS_REQUIRE(a->k >= 1 && a->k <= 4096, "1 <= k <= 4096 required");
   cudaStream_t st = (cudaStream_t)stream;
@@ -1318,6 +1337,7 @@ ls_status static_scratch(void** out) {
 }  // namespace
 
 extern "C" ls_status ls_sparse_attn_decode_noalloc(const ls_sparse_attn_args* a, ls_stream_t stream) {
+  NvtxRange nvtx_range("ls_sparse_attn_decode_noalloc");
   LS_TRY(validate_attn(a, true));
   const size_t need = attn_ws_bytes(a);
   if (need > kStaticAttnScratchBytes)

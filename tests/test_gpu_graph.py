@@ -80,3 +80,23 @@ def test_hot_buffer_step_graph_replay_matches_eager():
         for key, val in ref.items():
             assert torch.equal(wl.tensors[key], val), key
     assert B.ls_check_device_status() == 0
+
+
+def test_full_size_step_is_deterministic():
+    """Race check without a sanitizer: the full-size step (batch 8 at 131,072 tokens), run
+    three times on the same inputs with L2 evicted in between, gives bit-identical selection,
+    output and log-sum-exp."""
+    wl = W.mla_decode(batch=8, ctx=131072, k=2048, seed=1002, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(3):
+        flush.zero_()
+        wl.o.zero_()
+        wl.idx.fill_(-5)
+        wl.step()
+        torch.cuda.synchronize()
+        outs.append((wl.idx.clone(), wl.o.clone(), wl.lse.clone()))
+    for other in outs[1:]:
+        for a, b in zip(outs[0], other):
+            assert torch.equal(a, b)
+    assert B.ls_check_device_status() == 0
