@@ -168,3 +168,13 @@ def test_decode_step_coarse_to_fine():
     n = wl.tensors["n_survivors"].cpu().numpy()
     assert (n < np.array([-(-L // 64) for L in lens]) * 0.5).all()
     _check_mla_step(full, inp, q, kv, 2048, heads_sample=slice(0, 128, 16))
+    # the same step with the original keys in pinned host memory (small staging: several
+    # passes over the survivors): the same selection and output
+    host = W.build("c2f_host", inp, k=2048, attn=dict(q=q, kv=kv, scale=syn.softmax_scale(576)), c2f=True,
+                   c2f_keys_on_host=True, c2f_stage_blocks=64)
+    host.step()
+    torch.cuda.synchronize()
+    assert_status_clean()
+    assert torch.equal(host.idx, full.idx)
+    assert torch.equal(host.o, full.o)
+    assert torch.equal(host.tensors["n_survivors"], wl.tensors["n_survivors"])
