@@ -92,16 +92,36 @@ __global__ void __launch_bounds__(256) attn_simt(const AttnParams p) {
   __syncthreads();
   const T* K = (const T*)p.krows;
   const T* V = (const T*)p.vrows;
-  for (int j = warp; j < p.k; j += 8) {
+  // four-element vector loads when every row starts on a 4-element boundary
+  const bool vec = (p.row_stride % 4) == 0 && (((uintptr_t)K | (uintptr_t)V) % (4 * sizeof(T))) == 0;
+  // scores: a thread per selected row computes its whole dot product (all of the row's
+  // loads in flight at once)
+  for (int j = tid; j < p.k; j += 256) {
     const long long r = rows[j];
-    float acc = 0.f;
+    float sc = -INFINITY;
     if (r >= 0) {
       const T* kr = K + r * p.row_stride;
-      for (int d = lane; d < p.dk; d += 32) acc = fmaf(qs[d], (float)kr[d], acc);
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+      int d = 0;
+      if (vec) {
+        for (; d + 3 < p.dk; d += 4) {
+          float x0, x1, x2, x3;
+          if (BF16) {
+            const uint2 u = *(const uint2*)(kr + d);
+            x0 = __uint_as_float(u.x << 16); x1 = __uint_as_float(u.x & 0xFFFF0000u);
+            x2 = __uint_as_float(u.y << 16); x3 = __uint_as_float(u.y & 0xFFFF0000u);
+          } else {
+            const float4 v = *(const float4*)(kr + d);
+            x0 = v.x; x1 = v.y; x2 = v.z; x3 = v.w;
+          }
+          a0 = fmaf(qs[d], x0, a0); a1 = fmaf(qs[d + 1], x1, a1);
+          a2 = fmaf(qs[d + 2], x2, a2); a3 = fmaf(qs[d + 3], x3, a3);
+        }
+      }
+      for (; d < p.dk; ++d) a0 = fmaf(qs[d], (float)kr[d], a0);
+      sc = ((a0 + a1) + (a2 + a3)) * p.scale;
     }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) s[j] = r >= 0 ? acc * p.scale : -INFINITY;
+    s[j] = sc;
   }
   __syncthreads();
   float mx = -INFINITY;
@@ -126,13 +146,53 @@ __global__ void __launch_bounds__(256) attn_simt(const AttnParams p) {
   float l = 0.f;
   for (int w = 0; w < 8; ++w) l += red[w];
   T* o = (T*)p.o + ((size_t)b * p.H + h) * p.dv;
-  for (int d = tid; d < p.dv; d += 256) {
-    float acc = 0.f;
-    for (int j = 0; j < p.k; ++j) {
-      const long long r = rows[j];
-      if (r >= 0) acc = fmaf(s[j], (float)V[r * p.row_stride + d], acc);
+  // output: warp w sums rows j = w (mod 8), lane c a group of four dims (one 512-byte
+  // piece of a row per warp instruction); the eight warps' sums meet in shared memory
+  __shared__ float4 part[8][32];
+  const int ng = (p.dv + 3) / 4;
+  for (int g0 = 0; g0 < ng; g0 += 32) {
+    const int g = g0 + lane, d0 = 4 * g;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (g < ng) {
+#pragma unroll 4
+      for (int j = warp; j < p.k; j += 8) {
+        const long long r = rows[j];
+        const float w = r >= 0 ? s[j] : 0.f;
+        const T* vr = V + (r >= 0 ? r : 0) * p.row_stride + d0;  // a skipped row reads row 0
+        float x0 = 0.f, x1 = 0.f, x2 = 0.f, x3 = 0.f;
+        if (vec && d0 + 3 < p.dv) {
+          if (BF16) {
+            const uint2 u = *(const uint2*)vr;
+            x0 = __uint_as_float(u.x << 16); x1 = __uint_as_float(u.x & 0xFFFF0000u);
+            x2 = __uint_as_float(u.y << 16); x3 = __uint_as_float(u.y & 0xFFFF0000u);
+          } else {
+            const float4 v = *(const float4*)vr;
+            x0 = v.x; x1 = v.y; x2 = v.z; x3 = v.w;
+          }
+        } else {
+          x0 = (float)vr[0];
+          if (d0 + 1 < p.dv) x1 = (float)vr[1];
+          if (d0 + 2 < p.dv) x2 = (float)vr[2];
+          if (d0 + 3 < p.dv) x3 = (float)vr[3];
+        }
+        if (r < 0) x0 = x1 = x2 = x3 = 0.f;  // a skipped row adds nothing, whatever row 0 holds
+        acc.x = fmaf(w, x0, acc.x); acc.y = fmaf(w, x1, acc.y);
+        acc.z = fmaf(w, x2, acc.z); acc.w = fmaf(w, x3, acc.w);
+      }
     }
-    o[d] = (T)(l > 0.f ? acc / l : 0.f);
+    part[warp][lane] = acc;
+    __syncthreads();
+    if (warp == 0 && g < ng) {
+      float4 t = part[0][lane];
+      for (int w = 1; w < 8; ++w) {
+        const float4 u = part[w][lane];
+        t.x += u.x; t.y += u.y; t.z += u.z; t.w += u.w;
+      }
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float vals[4] = {t.x * inv, t.y * inv, t.z * inv, t.w * inv};
+      for (int e = 0; e < 4 && d0 + e < p.dv; ++e) o[d0 + e] = (T)vals[e];
+    }
+    __syncthreads();
   }
   if (tid == 0) p.lse[(size_t)b * p.H + h] = l > 0.f ? mx + logf(l) : -INFINITY;
 }
