@@ -389,6 +389,10 @@ typedef struct ls_decode_step_args {
   int32_t* idx;               /* [B,k] out, may be NULL (workspace) */
   float* sel_score;           /* [B,k] out, may be NULL (workspace) */
   ls_event_t* events;         /* NULL or 6 events */
+  ls_event_t attn_q_ready;    /* optional: an event the step waits for just before the
+                                 attention reads attn.q -- e.g. the end of its host-to-device
+                                 copy on another stream, so that copy overlaps the indexer
+                                 and top-k; NULL: attn.q is ready when the call is made */
 } ls_decode_step_args;
 
 size_t ls_decode_step_workspace_size(const ls_decode_step_args* args);

@@ -77,7 +77,7 @@ class DecodeStepArgs(C.Structure):
                 ("attn", SparseAttnArgs), ("use_hotbuf", _i32), ("n_slots", _i32),
                 ("pos_of_slot", _p), ("recent_score", _p), ("slot_of_pos", _p), ("host_kv", _p),
                 ("host_num_pages", _i64), ("hbuf", _p), ("n_miss", _p), ("idx", _p), ("sel_score", _p),
-                ("events", _p)]
+                ("events", _p), ("attn_q_ready", _p)]
 
 
 class PrefillStreamArgs(C.Structure):

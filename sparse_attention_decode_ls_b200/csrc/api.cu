@@ -1191,6 +1191,9 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
   auto rec = [&](int i) {
     if (ev && ev[i]) cudaEventRecord((cudaEvent_t)ev[i], st);
   };
+  auto wait_q = [&](cudaStream_t s) {
+    if (a->attn_q_ready) cudaStreamWaitEvent(s, (cudaEvent_t)a->attn_q_ready, 0);
+  };
   // a1 (+a2) or a3
   rec(0);
   if (a->use_c2f) {
@@ -1248,6 +1251,7 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
       cudaStreamWaitEvent(ss->s[0], ss->fork, 0);
       cudaStreamWaitEvent(ss->s[1], ss->fork, 0);
       LS_TRY(launch_hotbuf(&h, ss->s[0]));
+      wait_q(ss->s[1]);
       LS_TRY(launch_attn(&at, hit_slot, LS_ROWS_SLOTS, nullptr, 0, a->n_slots, a->hbuf, n_rows, attn_ws, attn_ws_b,
                          ss->s[1], false, true, 0, 2, false, chit));
       cudaEventRecord(ss->join[1], ss->s[1]);
@@ -1258,6 +1262,7 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
       rec(4);
       // the staging area as rows: request b's i-th miss at row b*k + i (launched straight
       // after the gather, so that its prologue overlaps the gather's end)
+      wait_q(st);
       LS_TRY(launch_attn(&at, crow, LS_ROWS_SLOTS, nullptr, 0, a->k, stage, (long long)ix->batch * a->k, attn_ws,
                          attn_ws_b, st, true, true, 1, 2, false, cn));
       cudaEventRecord(ss->gathered, st);
@@ -1272,6 +1277,7 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
       rec(3);
       LS_TRY(launch_gather(&g, st));
       rec(4);
+      wait_q(st);
       LS_TRY(launch_attn(&at, sel_slot, LS_ROWS_SLOTS, nullptr, 0, a->n_slots, a->hbuf, n_rows, attn_ws, attn_ws_b,
                          st, true));
     }
@@ -1282,6 +1288,7 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
     rec(4);
     const int* pt = at.page_table ? at.page_table : ix->page_table;
     const int mp = at.page_table ? at.max_pages : ix->max_pages;
+    wait_q(st);
     LS_TRY(launch_attn(&at, idx, LS_ROWS_PAGED, pt, mp, 0, nullptr, at.num_rows, attn_ws, attn_ws_b, st, true,
                        true));
   }

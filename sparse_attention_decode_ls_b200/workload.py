@@ -61,6 +61,31 @@ class DecodeWorkload:
         return self.tensors["idx"]
 
 
+# the per-step inputs (the queries, head weights, scales, lengths, page tables) and
+# outputs of a step: each set lives in one device buffer, so that a step's traffic with the
+# host is one copy each way
+STEP_INPUTS = ("i_q", "i_q_scale", "i_w", "i_lens", "i_page_table")  # the indexer's
+STEP_INPUTS_ATTN = ("a_q",)  # the attention's queries: needed only after the top-k
+STEP_OUTPUTS = ("o", "lse")
+
+
+def _pack(t: dict, names, dev):
+    """Rebind t[name] for each name to a view of one shared device buffer (256-byte aligned
+    pieces, contents copied); returns the buffer."""
+    names = [n for n in names if t.get(n) is not None]
+    offs, o = [], 0
+    for n in names:
+        offs.append(o)
+        o += (t[n].numel() * t[n].element_size() + 255) // 256 * 256
+    buf = torch.empty(max(o, 256), dtype=torch.uint8, device=dev)
+    for n, off in zip(names, offs):
+        nbytes = t[n].numel() * t[n].element_size()
+        view = buf[off: off + nbytes].view(t[n].dtype).view(t[n].shape)
+        view.copy_(t[n])
+        t[n] = view
+    return buf
+
+
 def build(name: str, ind: syn.IndexerInputs, *, k: int, attn: dict, device="cuda", hotbuf: dict | None = None,
           c2f: bool = False, eps_rel: float = 0.0, c2f_keys_on_host: bool = False,
           c2f_stage_blocks: int = 0) -> DecodeWorkload:
@@ -76,14 +101,17 @@ def build(name: str, ind: syn.IndexerInputs, *, k: int, attn: dict, device="cuda
     for key in ("q", "q_scale", "w", "key_pool", "key_scale", "page_table", "lens"):
         v = getattr(ind, key)
         t["i_" + key] = None if v is None else v.to(dev)
-    ix = B.index_args(q=t["i_q"], w=t["i_w"], key_pool=t["i_key_pool"], page_table=t["i_page_table"],
-                      lens=t["i_lens"], q_scale=t["i_q_scale"], key_scale=t["i_key_scale"], max_len=ml)
     mla = "kv" in attn or "kv_host" in attn
     t["a_q"] = attn["q"].to(dev)
     heads = t["a_q"].shape[1]
     dv = 512 if mla else attn["v"].shape[-1]
     t["o"] = torch.zeros((Bn, heads, dv), dtype=torch.bfloat16 if mla else torch.float32, device=dev)
     t["lse"] = torch.zeros((Bn, heads), dtype=torch.float32, device=dev)
+    t["step_in"] = _pack(t, STEP_INPUTS, dev)
+    t["step_in_attn"] = _pack(t, STEP_INPUTS_ATTN, dev)
+    t["step_out"] = _pack(t, STEP_OUTPUTS, dev)
+    ix = B.index_args(q=t["i_q"], w=t["i_w"], key_pool=t["i_key_pool"], page_table=t["i_page_table"],
+                      lens=t["i_lens"], q_scale=t["i_q_scale"], key_scale=t["i_key_scale"], max_len=ml)
     t["idx"] = torch.full((Bn, k), -1, dtype=torch.int32, device=dev)
     t["sel"] = torch.zeros((Bn, k), dtype=torch.float32, device=dev)
     hb = None
