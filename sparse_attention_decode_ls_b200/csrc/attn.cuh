@@ -680,13 +680,30 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
             }
             *(uint4*)(o + c) = make_uint4(w[0], w[1], w[2], w[3]);
           }
-        } else {
-          // layout [b][split][dim / 4][head][4]: a warp's store is 512 contiguous bytes
+        } else if (p.o_f32) {
+          // float32 partials, layout [b][split][dim / 4][head][4]: a warp's store is 512
+          // contiguous bytes
           float4* o = (float4*)p.part_o + (pslot * (DV / 4) + (rank * DVH + c0) / 4) * H + h;
           const bool any = l_run > 0.f;
 #pragma unroll
           for (int c = 0; c < 32; c += 4)
             o[(size_t)(c / 4) * H] = any ? make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+          // for a bf16 output the partials are bf16 too (one more rounding of what is rounded
+          // to bf16 at the end), layout [b][split][dim / 8][head][8]: a warp's store is 512
+          // contiguous bytes
+          uint4* o = (uint4*)p.part_o + (pslot * (DV / 8) + (rank * DVH + c0) / 8) * H + h;
+          const float any = l_run > 0.f ? 1.f : 0.f;
+#pragma unroll
+          for (int c = 0; c < 32; c += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              __nv_bfloat162 two = __floats2bfloat162_rn(v[c + 2 * e] * any, v[c + 2 * e + 1] * any);
+              w[e] = *(uint32_t*)&two;
+            }
+            o[(size_t)(c / 8) * H] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
         }
       }
       if (rank == 0) {  // both ranks hold the same running max and sum
@@ -699,8 +716,13 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
         }
       }
     } else if (my_tiles == 0 && p.nsplit_total > 1) {
-      float4* o = (float4*)p.part_o + (pslot * (DV / 4) + rank * DVH / 4) * H + h;
-      for (int c = 0; c < DVH / 4; ++c) o[(size_t)c * H] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (p.o_f32) {
+        float4* o = (float4*)p.part_o + (pslot * (DV / 4) + rank * DVH / 4) * H + h;
+        for (int c = 0; c < DVH / 4; ++c) o[(size_t)c * H] = make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+        uint4* o = (uint4*)p.part_o + (pslot * (DV / 8) + rank * DVH / 8) * H + h;
+        for (int c = 0; c < DVH / 8; ++c) o[(size_t)c * H] = make_uint4(0u, 0u, 0u, 0u);
+      }
       if (rank == 0) {
         float* ml = p.part_ml + (pslot * H + h) * 2;
         ml[0] = -INFINITY;
@@ -724,8 +746,8 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
 // Merge split-KV partials: o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
 // One thread per (request, head, 8 consecutive dims); grid (H * DV / 8 / 256, B), 256
 // threads.  A warp covers 32 consecutive heads at the same dims, so each of its partial
-// reads is a 512-byte run of the [dim / 4][head][4] layout; the 2 x nsplit 16-byte loads
-// of a thread are independent of one another.
+// reads is a 512-byte run of the [dim / 4][head][4] (float32) or [dim / 8][head][8] (bf16)
+// layout; the 16-byte loads of a thread (2 or 1 per split) are independent of one another.
 constexpr int kCombineThreads = 256;
 __global__ void __launch_bounds__(kCombineThreads) attn_combine(const AttnParams p) {
   using namespace mla;
@@ -747,12 +769,24 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine(const AttnParams
       if (!(l > 0.f)) continue;
       const float wgt = exp2f(ml[(size_t)s * H * 2] - M);
       Lsum += wgt * l;
-      const float4* po = (const float4*)p.part_o + (((size_t)b * p.nsplit_total + s) * (DV / 4) + d0 / 4) * H + h;
-      const float4 x = po[0], y = po[H];
-      acc[0] = fmaf(wgt, x.x, acc[0]); acc[1] = fmaf(wgt, x.y, acc[1]);
-      acc[2] = fmaf(wgt, x.z, acc[2]); acc[3] = fmaf(wgt, x.w, acc[3]);
-      acc[4] = fmaf(wgt, y.x, acc[4]); acc[5] = fmaf(wgt, y.y, acc[5]);
-      acc[6] = fmaf(wgt, y.z, acc[6]); acc[7] = fmaf(wgt, y.w, acc[7]);
+      float x[8];
+      if (p.o_f32) {
+        const float4* po = (const float4*)p.part_o + (((size_t)b * p.nsplit_total + s) * (DV / 4) + d0 / 4) * H + h;
+        const float4 u = po[0], w = po[H];
+        x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+        x[4] = w.x; x[5] = w.y; x[6] = w.z; x[7] = w.w;
+      } else {
+        const uint4 u = *((const uint4*)p.part_o + (((size_t)b * p.nsplit_total + s) * (DV / 8) + d0 / 8) * H + h);
+        const uint32_t q4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(*(const __nv_bfloat162*)&q4[e]);
+          x[2 * e] = f.x;
+          x[2 * e + 1] = f.y;
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = fmaf(wgt, x[e], acc[e]);
     }
   }
   const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
