@@ -749,6 +749,56 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
 // reads is a 512-byte run of the [dim / 4][head][4] (float32) or [dim / 8][head][8] (bf16)
 // layout; the 16-byte loads of a thread (2 or 1 per split) are independent of one another.
 constexpr int kCombineThreads = 256;
+constexpr int kCombineBatch = 8;  // splits whose loads are in flight together
+
+// One split's 8 dims of the partial, as float.
+template <bool F32>
+__device__ __forceinline__ void load_part8(const AttnParams& p, int b, int s, int h, int d0, float* x) {
+  using namespace mla;
+  if constexpr (F32) {
+    const float4* po = (const float4*)p.part_o + (((size_t)b * p.nsplit_total + s) * (DV / 4) + d0 / 4) * H + h;
+    const float4 u = po[0], w = po[H];
+    x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+    x[4] = w.x; x[5] = w.y; x[6] = w.z; x[7] = w.w;
+  } else {
+    const uint4 u = *((const uint4*)p.part_o + (((size_t)b * p.nsplit_total + s) * (DV / 8) + d0 / 8) * H + h);
+    const uint32_t q4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(*(const __nv_bfloat162*)&q4[e]);
+      x[2 * e] = f.x;
+      x[2 * e + 1] = f.y;
+    }
+  }
+}
+
+// The weighted sum over the splits, kCombineBatch splits at a time.  Every load of a batch
+// (max, sum and partial of each split) is issued unconditionally -- slots past the last
+// split re-read the last one and get weight 0 -- so that they are all in flight at once.
+template <bool F32>
+__device__ __forceinline__ void combine_splits(const AttnParams& p, int b, int h, int d0, const float* ml, float M,
+                                               float* acc, float& Lsum) {
+  const int ns = p.nsplit_total;
+  for (int s0 = 0; s0 < ns; s0 += kCombineBatch) {
+    float mv[kCombineBatch], lv[kCombineBatch], x[kCombineBatch][8];
+#pragma unroll
+    for (int j = 0; j < kCombineBatch; ++j) {
+      const int s = min(s0 + j, ns - 1);
+      mv[j] = ml[(size_t)s * mla::H * 2];
+      lv[j] = ml[(size_t)s * mla::H * 2 + 1];
+      load_part8<F32>(p, b, s, h, d0, x[j]);
+    }
+#pragma unroll
+    for (int j = 0; j < kCombineBatch; ++j) {
+      // an empty split, or a slot past the last split, adds nothing
+      const float wgt = (s0 + j < ns && lv[j] > 0.f) ? exp2f(mv[j] - M) : 0.f;
+      Lsum += wgt * lv[j];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = fmaf(wgt, x[j][e], acc[e]);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kCombineThreads) attn_combine(const AttnParams p) {
   using namespace mla;
   griddep_wait();  // the partials come from the kernel before
@@ -757,36 +807,22 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine(const AttnParams
   const int g = item / H, h = item - g * H, d0 = g * 8;
   const float* ml = p.part_ml + (size_t)b * p.nsplit_total * H * 2 + (size_t)h * 2;
   float M = -INFINITY;
-  for (int s = 0; s < p.nsplit_total; ++s) M = fmaxf(M, ml[(size_t)s * H * 2]);
+  for (int s0 = 0; s0 < p.nsplit_total; s0 += kCombineBatch) {
+    float mv[kCombineBatch];
+#pragma unroll
+    for (int j = 0; j < kCombineBatch; ++j) mv[j] = ml[(size_t)min(s0 + j, p.nsplit_total - 1) * H * 2];
+#pragma unroll
+    for (int j = 0; j < kCombineBatch; ++j) M = fmaxf(M, mv[j]);
+  }
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
   float Lsum = 0.f;
   if (M != -INFINITY) {
-#pragma unroll 8
-    for (int s = 0; s < p.nsplit_total; ++s) {
-      const float l = ml[(size_t)s * H * 2 + 1];
-      if (!(l > 0.f)) continue;
-      const float wgt = exp2f(ml[(size_t)s * H * 2] - M);
-      Lsum += wgt * l;
-      float x[8];
-      if (p.o_f32) {
-        const float4* po = (const float4*)p.part_o + (((size_t)b * p.nsplit_total + s) * (DV / 4) + d0 / 4) * H + h;
-        const float4 u = po[0], w = po[H];
-        x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
-        x[4] = w.x; x[5] = w.y; x[6] = w.z; x[7] = w.w;
-      } else {
-        const uint4 u = *((const uint4*)p.part_o + (((size_t)b * p.nsplit_total + s) * (DV / 8) + d0 / 8) * H + h);
-        const uint32_t q4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(*(const __nv_bfloat162*)&q4[e]);
-          x[2 * e] = f.x;
-          x[2 * e + 1] = f.y;
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] = fmaf(wgt, x[e], acc[e]);
+    if (p.o_f32) {
+      combine_splits<true>(p, b, h, d0, ml, M, acc, Lsum);
+    } else {
+      combine_splits<false>(p, b, h, d0, ml, M, acc, Lsum);
     }
   }
   const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
