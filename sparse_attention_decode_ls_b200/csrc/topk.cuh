@@ -77,7 +77,8 @@ constexpr int kTopkExtraBytes = kCandCap * 4 + kCandTotal * 4 + (kTopkThreads / 
   } while (0)
 
 template <int CL>
-__global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams p) {
+// At most 64 registers: two CTAs per SM, so that all clusters of a batch are resident at once.
+__global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster(const TopkParams p) {
   cg::cluster_group cluster = cg::this_cluster();
   extern __shared__ __align__(16) uint32_t sm_keys[];  // [cache_keys] then candidate buffers
   __shared__ uint32_t hist[2048];
@@ -156,13 +157,19 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
   }
 
   if (cached) {
+    // four 16-byte loads in flight per thread (indices clamped into the slice, so every
+    // load is issued), then their keys into shared memory
+    constexpr int kU = 4, kStep = kTopkThreads * 4;
     const int m4 = m & ~3;
-    for (int i = tid * 4; i < m4; i += kTopkThreads * 4) {
-      const float4 v = *(const float4*)(row + c0 + i);
-      sm_keys[i] = float_key(v.x);
-      sm_keys[i + 1] = float_key(v.y);
-      sm_keys[i + 2] = float_key(v.z);
-      sm_keys[i + 3] = float_key(v.w);
+    for (int i0 = tid * 4; i0 < m4; i0 += kStep * kU) {
+      float4 v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) v[u] = *(const float4*)(row + c0 + min(i0 + u * kStep, m4 - 4));
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int i = i0 + u * kStep;
+        if (i < m4) *(uint4*)(sm_keys + i) = make_uint4(float_key(v[u].x), float_key(v[u].y), float_key(v[u].z), float_key(v[u].w));
+      }
     }
     for (int i = m4 + tid; i < m; i += kTopkThreads) sm_keys[i] = float_key(row[c0 + i]);
   }
@@ -213,7 +220,18 @@ __global__ void __launch_bounds__(kTopkThreads, 1) topk_cluster(const TopkParams
         red[d] = s;
       }
       cluster.sync();
-      for (int d = tid; d < nbins; d += kTopkThreads) ghist[d] = cluster.map_shared_rank(red, d / slice)[d % slice];
+      // all of this thread's remote reads first (nbins <= 2048 = 4 per thread), then the stores
+      uint32_t gv[2048 / kTopkThreads];
+#pragma unroll
+      for (int u = 0; u < 2048 / kTopkThreads; ++u) {
+        const int d = tid + u * kTopkThreads;
+        gv[u] = d < nbins ? cluster.map_shared_rank(red, d / slice)[d % slice] : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < 2048 / kTopkThreads; ++u) {
+        const int d = tid + u * kTopkThreads;
+        if (d < nbins) ghist[d] = gv[u];
+      }
       __syncthreads();
       h_all = ghist;
     }
