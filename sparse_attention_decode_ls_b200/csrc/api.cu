@@ -348,7 +348,10 @@ int attn_nsplit(const ls_sparse_attn_args* a) {
   const int tiles = (a->k + ls::mla::N - 1) / ls::mla::N;
   int ns = device_sms() / (2 * a->batch);
   ns = std::max(1, std::min(ns, (tiles + 1) / 2));
-  return ns;
+  // the fewest splits with the same longest share (e.g. 32 tiles: 8 splits of 4, not 9 of
+  // 3-4): the same critical path, fewer partials to store and merge, SMs left free
+  const int per = (tiles + ns - 1) / ns;
+  return (tiles + per - 1) / per;
 }
 
 // Split-KV partials of `npasses` launches over the same requests (each with
