@@ -156,6 +156,8 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster(const TopkParams
     return;  // no distributed shared memory was touched
   }
 
+  // the histogram starts zeroed here; every radix pass leaves it zeroed again
+  for (int d = tid; d < 2048; d += kTopkThreads) hist[d] = 0;
   if (cached) {
     // four 16-byte loads in flight per thread (indices clamped into the slice, so every
     // load is issued), then their keys into shared memory
@@ -176,15 +178,16 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster(const TopkParams
 
   // Find the bin (of `width` bits at `shift`) holding the k_rem-th largest key among the
   // keys whose bits above the digit equal `prefix`; bins scanned high to low.  With
-  // `local`, only this CTA's `vals` are counted; otherwise the cluster's slices.
+  // `local`, only this CTA's `vals` are counted; otherwise the cluster's slices.  `hist` is
+  // zero on entry and on exit: each thread clears the bins it read once no other CTA reads
+  // them any more.
   uint32_t prefix = 0;
   uint32_t k_rem = (uint32_t)k;
   auto radix_pass = [&](int shift, int width, bool local, const uint32_t* vals, int nvals) {
     const int nbins = 1 << width;
     const uint32_t dmask = (uint32_t)nbins - 1u;
     const int hi_shift = shift + width;
-    for (int d = tid; d < 2048; d += kTopkThreads) hist[d] = 0;
-    __syncthreads();
+    __syncthreads();  // the keys (and, in the first pass, the zeroed histogram) are in place
     // scores crowd into few bins, so lanes of a warp that hit the same bin add once
     auto count = [&](bool ok, uint32_t key) {
       if (ok) atomicAdd(&hist[(key >> shift) & dmask], 1u);
@@ -220,6 +223,8 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster(const TopkParams
         red[d] = s;
       }
       cluster.sync();
+      // no CTA reads this one's histogram any more: clear it for the next pass
+      for (int d = tid; d < 2048; d += kTopkThreads) hist[d] = 0;
       // all of this thread's remote reads first (nbins <= 2048 = 4 per thread), then the stores
       uint32_t gv[2048 / kTopkThreads];
 #pragma unroll
@@ -236,23 +241,36 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster(const TopkParams
       h_all = ghist;
     }
     const int per = nbins / kTopkThreads;  // 4 or 2 bins per thread
+    uint32_t hv[2048 / kTopkThreads];
     uint32_t mine = 0;
-    for (int j = 0; j < per; ++j) mine += h_all[nbins - 1 - (tid * per + j)];
+#pragma unroll
+    for (int j = 0; j < 2048 / kTopkThreads; ++j) {
+      hv[j] = j < per ? h_all[nbins - 1 - (tid * per + j)] : 0u;
+      mine += hv[j];
+    }
+    if (local) {  // this thread's bins are read: clear them for the next pass
+#pragma unroll
+      for (int j = 0; j < 2048 / kTopkThreads; ++j)
+        if (j < per) hist[nbins - 1 - (tid * per + j)] = 0;
+    }
     unsigned long long tot;
     uint32_t above = (uint32_t)block_excl_scan_u64(mine, scan_tmp, &tot);
-    for (int j = 0; j < per; ++j) {
-      const int d = nbins - 1 - (tid * per + j);
-      const uint32_t h = h_all[d];
-      if (above < k_rem && above + h >= k_rem) {
-        s_found_bin = d;
-        s_found_above = above;
+#pragma unroll
+    for (int j = 0; j < 2048 / kTopkThreads; ++j) {
+      if (j < per) {
+        const int d = nbins - 1 - (tid * per + j);
+        if (above < k_rem && above + hv[j] >= k_rem) {
+          s_found_bin = d;
+          s_found_above = above;
+        }
+        above += hv[j];
       }
-      above += h;
     }
     __syncthreads();
+    // no barrier after these reads: the next write of s_found_* comes after the next pass's
+    // counting barrier, which every thread reaches only after reading them
     prefix = (prefix << width) | (uint32_t)s_found_bin;
     k_rem -= s_found_above;
-    __syncthreads();
   };
 
   // ---- pass 0 over the whole request: the top 11 bits
