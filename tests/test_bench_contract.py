@@ -1,0 +1,37 @@
+"""bench.py's output contract, checked on its CPU arm: `--impl reference` times the oracle
+on this machine's cores and prints one JSON line with the keys every bench line carries,
+plus the CPU-baseline and end-to-end objects that describe this run.  CPU only."""
+import json
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+COMMON_KEYS = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+               "scaling", "vs_baseline", "dtype", "data", "config"}
+
+
+def run_reference_arm(*extra):
+    out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", *extra], cwd=ROOT,
+                         capture_output=True, text=True, timeout=600, check=True).stdout
+    lines = [ln for ln in out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out  # exactly one JSON line
+    return json.loads(lines[0])
+
+
+def test_reference_arm_line():
+    d = run_reference_arm("--steps", "1", "--warmup", "0")
+    assert COMMON_KEYS <= set(d)
+    assert d["impl"] == "reference"
+    assert d["n_gpus"] == 1 and d["steps"] == 1
+    assert d["warmup"] >= 3  # the timing rules' minimum, whatever was asked for
+    assert d["higher_is_better"] is True and d["unit"] == "tokens/s"
+    assert d["value"] > 0 and d["ms_per_step"] > 0
+    assert d["config"]["workload"] == "mla_decode_b8_ctx131072_top2048"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"]
+    assert cb["value"] == d["value"] and cb["unit"] == d["unit"]
+    e2e = d["e2e"]
+    assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
