@@ -171,6 +171,29 @@ def test_mla_attention_paged(variant, scale):
     assert_status_clean()
 
 
+@pytest.mark.parametrize("lens,k,n_valid", [
+    ([3000, 700], 100, [100, 37]),        # two tiles: one KV split, the output written by the attention itself
+    ([70000, 5000], 4096, [4096, 3000]),  # the largest k: 64 tiles
+])
+def test_mla_attention_split_extremes(lens, k, n_valid):
+    Bn = len(lens)
+    table, n_pool = syn.page_layout(lens, seed=21)
+    q, kv = syn.mla_attention(Bn, n_pool, seed=22)
+    sel = _random_selection(Bn, k, lens, seed=23, n_valid=n_valid)
+    scale = 1 / math.sqrt(576)
+    o = torch.zeros((Bn, 128, 512), dtype=torch.bfloat16, device=DEV)
+    lse = torch.zeros((Bn, 128), device=DEV)
+    a = B.attn_args(q=q.to(DEV), k_rows=kv.to(DEV), sel=sel.to(DEV), o=o, lse=lse, scale=scale,
+                    page_table=table.to(DEV))
+    ws = torch.empty(max(1, B.ls_sparse_attn_workspace_size(a)), dtype=torch.uint8, device=DEV)
+    B.ls_sparse_attn_decode(a, ws)
+    torch.cuda.synchronize()
+    ref_o, ref_l = _oracle_attn(bits16(q), bits16(kv), table.numpy(), sel.numpy(), scale, 512)
+    assert np.abs(o.float().cpu().numpy() - ref_o).max() <= 2e-2
+    assert np.abs(lse.cpu().numpy() - ref_l).max() <= 2e-2
+    assert_status_clean()
+
+
 def test_mla_attention_slots_and_empty_selection():
     Bn, S, k = 2, 4096, 64
     g = torch.Generator().manual_seed(21)
