@@ -273,13 +273,13 @@ __device__ __forceinline__ void load_q_tmem(const uint8_t* q_smem, int rank, int
 }
 
 // One cluster of two CTAs = (request b, KV split); rank r of the pair produces output
-// dims [256r, 256r + 256).  Per 32-row tile, each CTA gathers its five 64-dim panels of
-// the selected rows (TMA gather4, eight stages), forms its part of S = Q K^T over its latent
-// dims in TMEM (Q, the A operand, also lives in TMEM), sends that 128 x 32 partial to the other CTA through distributed shared
-// memory and adds the one it receives, so both hold the same S (fp32 addition commutes,
-// so the two sums are bit-identical) and run the same online softmax (one thread per
-// head).  P goes to shared memory as bf16 and O_half += P V_half accumulates in TMEM
-// (256 columns).
+// dims [256r, 256r + 256).  Per 64-row tile, each CTA gathers its five 64-dim panels of the
+// selected rows (TMA gather4 into a three-stage ring), forms its part of S = Q K^T over its
+// latent dims in TMEM (Q, the A operand, also lives in TMEM), sends that 128 x 64 partial to
+// the other CTA through distributed shared memory and adds the one it receives, so both hold
+// the same S (fp32 addition commutes, so the two sums are bit-identical) and run the same
+// online softmax (one thread per head).  P goes to TMEM as bf16 pairs (the A operand of PV)
+// and O_half += P V_half accumulates in TMEM (256 columns).
 __global__ void __launch_bounds__(mla::kThreads, 1)
     attn_mla_tc(const AttnParams p, const __grid_constant__ CUtensorMap kv_map,
                 const __grid_constant__ CUtensorMap q_map) {
