@@ -3,10 +3,10 @@
 // selected KV that misses it is fetched from the full history).
 //
 // hotbuf_resolve: one CTA per request.  Classifies each selection as hit (resident)
-// or miss, compacts the misses in selection order, orders the unpinned slots by
-// (empty first, recent score, slot) with a shared-memory bitonic sort of 64-bit
-// composite keys, hands the i-th victim to the i-th miss, and updates both maps
-// and the recent scores in place.
+// or miss, compacts the misses in selection order, finds the n_miss first victims in
+// the order (empty first, recent score, slot) by a radix select over 64-bit composite
+// keys and ranks them by counting, hands the i-th victim to the i-th miss, and updates
+// both maps and the recent scores in place.
 //
 // gather_misses: copies each missed 1,152-byte row from pinned host memory into its
 // slot (or, in the decode step, into a staging row in miss order); every thread moves

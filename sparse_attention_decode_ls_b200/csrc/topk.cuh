@@ -3,11 +3,12 @@
 //
 // One thread-block cluster per request.  Each CTA owns a contiguous slice of the
 // request's scores, converts them once to order-preserving 32-bit keys and keeps them
-// in shared memory.  Three radix passes (11, 11, 10 bits) build shared-memory
-// histograms of the candidates, merged across the cluster through distributed
-// shared memory, until the exact k-th key T is known.  The emit pass then writes, in
-// ascending position order, every position with key > T plus the lowest-positioned
-// ones with key == T -- the tie rule "lower position first".
+// in shared memory.  The first radix pass (the top 11 bits) is merged across the
+// cluster through distributed shared memory; every CTA then gathers the keys of the bin
+// holding the k-th largest key and finishes the exact k-th key T with two local passes
+// (11, 10 bits), or, when that bin is too crowded, two more cluster-wide passes.  The
+// emit pass then writes, in ascending position order, every position with key > T plus
+// the lowest-positioned ones with key == T -- the tie rule "lower position first".
 #pragma once
 #include <cooperative_groups.h>
 
