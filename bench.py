@@ -150,26 +150,52 @@ def oracle_request_runner(ctx, k, seed=1002):
     return run
 
 
+def _oracle_runs(run, budget_s, min_runs=1):
+    """Call `run` until the next call would pass `budget_s` seconds (at least `min_runs`
+    calls); returns the per-call times in seconds."""
+    times, t_all = [], time.perf_counter()
+    while True:
+        t0 = time.perf_counter()
+        run()
+        times.append(time.perf_counter() - t0)
+        el = time.perf_counter() - t_all
+        if len(times) >= min_runs and el * (len(times) + 1) / len(times) > budget_s:
+            return times
+
+
+def oracle_single_thread(budget_s=6.0, frac=0.125):
+    """The CPU oracle restricted to one thread, on one request at `frac` of the workload's
+    context and top-k (a bounded sample): tokens/s, counting a run as `frac` tokens."""
+    from threadpoolctl import threadpool_limits
+    ctx_f = max(64 * 64, int(round(frac * CTX / 64)) * 64)
+    f = ctx_f / CTX
+    k_f = max(1, int(round(TOPK * f)))
+    run = oracle_request_runner(ctx_f, k_f)
+    with threadpool_limits(limits=1):
+        times = _oracle_runs(run, budget_s)
+    return {"value": len(times) * f / sum(times), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{len(times)} request(s) at context {ctx_f} with top-{k_f} ({f:.4f} of a {WORKLOAD} "
+                      f"request each), one thread, float64 numpy, {sum(times):.1f} s"}
+
+
 def cpu_oracle_sample(seconds_budget=15.0):
     """The CPU oracle on whole requests of the workload (indexer over 131,072 tokens,
-    top-2048, MLA attention), as many as fit the budget (at least one)."""
+    top-2048, MLA attention), as many as fit the budget (at least one), on all the host's
+    cores; beside it the same oracle on one thread over a smaller sample."""
     run = oracle_request_runner(CTX, TOPK)
-    done, t0 = 0, time.perf_counter()
-    while True:
-        run()
-        done += 1
-        el = time.perf_counter() - t0
-        if el * (done + 1) / done > seconds_budget:
-            break
-    return {"value": done / el, "unit": UNIT, "cores": _oracle_cores(), "kind": "oracle",
-            "sample": f"{done} whole request(s) of {WORKLOAD} (one decode token each), float64 numpy, "
-                      f"{el:.1f} s"}
+    times = _oracle_runs(run, seconds_budget)
+    el = sum(times)
+    return {"value": len(times) / el, "unit": UNIT, "cores": _oracle_cores(), "kind": "oracle",
+            "sample": f"{len(times)} whole request(s) of {WORKLOAD} (one decode token each), float64 numpy, "
+                      f"{el:.1f} s",
+            "single_thread": oracle_single_thread()}
 
 
 def run_reference(args):
-    """Reference arm: the CPU oracle as it stands.  Each step runs it on one request whose
+    """Reference arm: the CPU oracle as it stands.  Each step runs it on ONE request whose
     context (and selection) is a fixed fraction f of the workload's, sized so the whole
-    run stays within LS_REF_BUDGET_S seconds; a step counts as f decode tokens."""
+    run stays within LS_REF_BUDGET_S seconds; a step counts as f decode tokens, and
+    ms_per_step is the measured time of those steps."""
     rank, world, _ = rank_env()
     if rank != 0:
         return 0
@@ -179,7 +205,7 @@ def run_reference(args):
     full()
     t_full = time.perf_counter() - t0
     n = args.warmup + args.steps
-    f = min(1.0, budget / max(n * t_full, 1e-9))
+    f = min(1.0, 0.85 * budget / max(n * t_full, 1e-9))
     ctx_f = max(64 * 64, int(round(f * CTX / 64)) * 64)
     f = ctx_f / CTX
     k_f = max(1, int(round(TOPK * f)))
@@ -191,14 +217,18 @@ def run_reference(args):
         if i >= args.warmup:
             times.append(time.perf_counter() - t0)
     value = len(times) * f / sum(times)
-    sample = (f"each step: 1 request at context {ctx_f} with top-{k_f} ({f:.4f} of a {WORKLOAD} request) on the "
-              f"CPU oracle (float64 numpy); one full request took {t_full:.2f} s")
+    sample = (f"each step: 1 request at context {ctx_f} with top-{k_f} ({f:.4f} of a {WORKLOAD} request, so "
+              f"{f:.4f} tokens per step) on the CPU oracle (float64 numpy, all cores); one full request took "
+              f"{t_full:.2f} s")
+    config = dict(CONFIG, batch=1, reference_step=f"one request at context {ctx_f}, top-{k_f}",
+                  tokens_per_step=f)
     out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
-           "warmup": args.warmup, "ms_per_step": 1e3 * BATCH / value, "higher_is_better": True,
-           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": CONFIG,
+           "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
            "impl": "reference",
            "cpu_baseline": {"value": value, "unit": UNIT, "cores": _oracle_cores(), "kind": "oracle",
-                            "sample": sample},
+                            "sample": sample,
+                            "single_thread": oracle_single_thread(budget_s=min(10.0, 0.1 * budget))},
            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
     return 0

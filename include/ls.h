@@ -338,8 +338,12 @@ ls_status ls_sparse_attn_decode(const ls_sparse_attn_args* args, void* workspace
  *     process exits.  A configuration whose partials need more returns
  *     LS_ERR_INVALID_ARG with a message (ls_sparse_attn_workspace_size() gives the
  *     need); one that needs none does not touch the scratch.
- *   - The first call on a device looks up the scratch's device address, with that
- *     device current; make that first call before any stream capture.
+ *   - The first call in each CUDA context looks up the scratch's device address in
+ *     that context (the device's primary context for runtime users, or a context the
+ *     caller created and made current); make that first call before any stream capture.
+ *     The address is cached under the context's process-unique id, so a context made
+ *     after cudaDeviceReset, or a second context on the same device, gets its own
+ *     lookup and never a stale address.
  *   - All calls on a device share the one array, which keeps the last call's
  *     contents.  Nothing in it has to start at zero: each call writes every partial
  *     before it reads it.  Calls whose kernels overlap on the GPU (for example on two
@@ -363,6 +367,12 @@ ls_status ls_sparse_attn_decode_noalloc(const ls_sparse_attn_args* args, ls_stre
  * events: optional; when non-NULL, events[i] is recorded on `stream` before stage
  *   i (0 indexer, 1 top-k, 2 resolve, 3 gather, 4 attention) and events[5] after
  *   the last stage, so a caller can time each stage.
+ * sel_slot / miss_pos / miss_slot: optional outputs of the hot-buffer resolve (as in a4).
+ * Streams: the hot-buffer step forks onto two streams of its own and joins back into
+ *   `stream`.  Each (host thread, device, caller stream) gets its own pair, created on
+ *   first use, so steps issued on independent streams stay independent; steps issued
+ *   on one stream reuse it in order.  Device ordinals from 64 up are refused
+ *   (LS_ERR_UNSUPPORTED).
  * --------------------------------------------------------------------------- */
 typedef struct ls_decode_step_args {
   ls_index_score_args index;
@@ -393,6 +403,9 @@ typedef struct ls_decode_step_args {
                                  attention reads attn.q -- e.g. the end of its host-to-device
                                  copy on another stream, so that copy overlaps the indexer
                                  and top-k; NULL: attn.q is ready when the call is made */
+  int32_t* sel_slot;          /* hot buffer: [B,k] out, may be NULL (workspace); as in a4 */
+  int32_t* miss_pos;          /* hot buffer: [B,k] out, may be NULL (workspace); as in a4 */
+  int32_t* miss_slot;         /* hot buffer: [B,k] out, may be NULL (workspace); as in a4 */
 } ls_decode_step_args;
 
 size_t ls_decode_step_workspace_size(const ls_decode_step_args* args);

@@ -77,7 +77,7 @@ class DecodeStepArgs(C.Structure):
                 ("attn", SparseAttnArgs), ("use_hotbuf", _i32), ("n_slots", _i32),
                 ("pos_of_slot", _p), ("recent_score", _p), ("slot_of_pos", _p), ("host_kv", _p),
                 ("host_num_pages", _i64), ("hbuf", _p), ("n_miss", _p), ("idx", _p), ("sel_score", _p),
-                ("events", _p), ("attn_q_ready", _p)]
+                ("events", _p), ("attn_q_ready", _p), ("sel_slot", _p), ("miss_pos", _p), ("miss_slot", _p)]
 
 
 class PrefillStreamArgs(C.Structure):
@@ -339,7 +339,8 @@ def decode_step_args(*, index: IndexScoreArgs, k, attn: SparseAttnArgs, c2f=None
                      sel_score=None, events=None) -> DecodeStepArgs:
     """c2f: dict(summaries, block_scale, survivors=None, n_survivors=None, eps_rel=0.0,
     keys_on_host=False, stage_blocks=0);
-    hotbuf: dict(pos_of_slot, recent_score, slot_of_pos, host_kv, hbuf, n_miss=None).
+    hotbuf: dict(pos_of_slot, recent_score, slot_of_pos, host_kv, hbuf, n_miss=None,
+    sel_slot=None, miss_pos=None, miss_slot=None).
     events: optional ctypes array of 6 cudaEvent_t handles."""
     a = DecodeStepArgs()
     a.index = index
@@ -360,6 +361,8 @@ def decode_step_args(*, index: IndexScoreArgs, k, attn: SparseAttnArgs, c2f=None
         a.slot_of_pos, a.host_kv = _ptr(hotbuf["slot_of_pos"]), _ptr(hotbuf["host_kv"])
         a.host_num_pages = hotbuf["host_kv"].shape[0]
         a.hbuf, a.n_miss = _ptr(hotbuf["hbuf"]), _ptr(hotbuf.get("n_miss"))
+        a.sel_slot, a.miss_pos = _ptr(hotbuf.get("sel_slot")), _ptr(hotbuf.get("miss_pos"))
+        a.miss_slot = _ptr(hotbuf.get("miss_slot"))
     a.idx, a.sel_score = _ptr(idx), _ptr(sel_score)
     a.events = None if events is None else C.cast(events, C.c_void_p).value
     return _hold(a, index, attn, c2f, hotbuf, idx, sel_score, events)

@@ -11,6 +11,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <string>
 
@@ -65,15 +66,19 @@ bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // ---- per-device cached properties -------------------------------------------------
+// Per-device caches below hold this many devices; a higher ordinal is refused
+// (LS_ERR_UNSUPPORTED or cudaErrorInvalidDevice), never folded onto a lower one.
+constexpr int kMaxDevices = 64;
+
 int device_sms() {
-  static std::atomic<int> cache[64];
+  static std::atomic<int> cache[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
-  int v = cache[dev].load();
+  const bool cached = dev >= 0 && dev < kMaxDevices;
+  int v = cached ? cache[dev].load() : 0;
   if (v <= 0) {
     if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
-    cache[dev].store(v);
+    if (cached) cache[dev].store(v);
   }
   return v;
 }
@@ -83,7 +88,8 @@ template <typename K>
 cudaError_t allow_smem(K kernel, int bytes, std::atomic<uint64_t>& done) {
   int dev = 0;
   cudaGetDevice(&dev);
-  const uint64_t bit = 1ull << (dev & 63);
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  const uint64_t bit = 1ull << dev;
   if (done.load() & bit) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e == cudaSuccess) done.fetch_or(bit);
@@ -98,7 +104,8 @@ template <typename K>
 cudaError_t keep_smem_carveout(K kernel, std::atomic<uint64_t>& done) {
   int dev = 0;
   cudaGetDevice(&dev);
-  const uint64_t bit = 1ull << (dev & 63);
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  const uint64_t bit = 1ull << dev;
   if (done.load() & bit) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                                        (int)cudaSharedmemCarveoutMaxShared);
@@ -263,7 +270,7 @@ std::atomic<uint64_t> g_smem_topk8{0}, g_smem_topk16{0}, g_smem_topk_row{0};
 // Requests up to this many candidates go to the one-CTA top-k, longer ones to a cluster
 // (measured: at 131,072 scores per request one CTA takes ~50 us, a 16-CTA cluster ~20 us).
 constexpr int kTopkRowMaxLen = 32768;
-std::atomic<int> g_topk16_ok[64];  // per device: 0 unknown, 1 yes, -1 no
+std::atomic<int> g_topk16_ok[kMaxDevices];  // per device: 0 unknown, 1 yes, -1 no
 
 template <int CL>
 cudaLaunchConfig_t topk_config(int B, int smem, cudaStream_t st, cudaLaunchAttribute* attr) {
@@ -288,7 +295,8 @@ cudaLaunchConfig_t topk_config(int B, int smem, cudaStream_t st, cudaLaunchAttri
 bool topk16_supported(cudaStream_t st) {
   int dev = 0;
   cudaGetDevice(&dev);
-  std::atomic<int>& flag16 = g_topk16_ok[dev & 63];
+  if (dev < 0 || dev >= kMaxDevices) return false;  // the 8-CTA launch then reports the ordinal
+  std::atomic<int>& flag16 = g_topk16_ok[dev];
   int v = flag16.load();
   if (v != 0) return v > 0;
   bool ok = cudaFuncSetAttribute(ls::topk_cluster<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
@@ -763,17 +771,21 @@ ls_status launch_attn_combine(const ls_sparse_attn_args* a, void* ws, int npasse
 // gathered (tensor-core attention), or strictly after the gather.
 bool overlap_misses(const ls_sparse_attn_args* at) { return at->dtype == LS_BF16 && at->variant == 0; }
 
-// Two more streams of this host thread on the current device, and the events for the
-// fork and joins of the overlapped hot-buffer step (created once, reused).
+// Two more streams of this host thread for one (device, caller stream), and the events for
+// the fork and joins of the overlapped hot-buffer step (created once, reused).  Keyed by the
+// caller's stream, so that steps issued from one thread on independent streams neither
+// share side streams (a false serialisation) nor re-record each other's events (a join on
+// the wrong step); calls on one stream are ordered, so their reuse is safe.
 struct SideStream {
   cudaStream_t s[2] = {nullptr, nullptr};
   cudaEvent_t fork = nullptr, gathered = nullptr, join[2] = {nullptr, nullptr};
 };
-ls_status side_stream(SideStream** out) {
-  thread_local SideStream per_dev[64];
+ls_status side_stream(cudaStream_t caller, SideStream** out) {
+  thread_local std::map<std::pair<int, cudaStream_t>, SideStream> per_stream;
   int dev = 0;
   cudaGetDevice(&dev);
-  SideStream& ss = per_dev[dev & 63];
+  if (dev < 0 || dev >= kMaxDevices) return fail(LS_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  SideStream& ss = per_stream[std::make_pair(dev, caller)];
   if (!ss.s[1]) {
     bool good = true;
     for (int i = 0; i < 2; ++i) {
@@ -893,10 +905,11 @@ struct PrefillStreams {
   cudaEvent_t start = nullptr, loaded[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr};
 };
 ls_status prefill_streams(PrefillStreams** out) {
-  thread_local PrefillStreams per_dev[64];
+  thread_local PrefillStreams per_dev[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
-  PrefillStreams& ps = per_dev[dev & 63];
+  if (dev < 0 || dev >= kMaxDevices) return fail(LS_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  PrefillStreams& ps = per_dev[dev];
   if (!ps.copy) {
     bool good = cudaEventCreateWithFlags(&ps.start, cudaEventDisableTiming) == cudaSuccess;
     for (int i = 0; i < 2; ++i) {
@@ -1218,9 +1231,9 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
   }
   void* attn_ws = w + l.off_attn;
   if (a->use_hotbuf) {
-    int* sel_slot = (int*)(w + l.off_selslot);
-    int* mpos = (int*)(w + l.off_mpos);
-    int* mslot = (int*)(w + l.off_mslot);
+    int* sel_slot = a->sel_slot ? a->sel_slot : (int*)(w + l.off_selslot);
+    int* mpos = a->miss_pos ? a->miss_pos : (int*)(w + l.off_mpos);
+    int* mslot = a->miss_slot ? a->miss_slot : (int*)(w + l.off_mslot);
     int* nmiss = a->n_miss ? a->n_miss : (int*)(w + l.off_nmiss);
     const bool two_pass = overlap_misses(&at);
     const size_t attn_ws_b = attn_ws_bytes(&at, two_pass ? 2 : 1);
@@ -1249,7 +1262,7 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
       LS_TRY(launch_classify(&h, hit_slot, chit, cpos, crow, cn, st));
       rec(3);
       SideStream* ss = nullptr;
-      LS_TRY(side_stream(&ss));
+      LS_TRY(side_stream(st, &ss));
       cudaEventRecord(ss->fork, st);
       cudaStreamWaitEvent(ss->s[0], ss->fork, 0);
       cudaStreamWaitEvent(ss->s[1], ss->fork, 0);
@@ -1319,26 +1332,63 @@ static __device__ __align__(256) unsigned char g_attn_scratch[kStaticAttnScratch
 
 namespace {
 
-// Device address of g_attn_scratch on the current device.  In host code the symbol is
-// only a host-side stand-in, so the address is asked for once per device (with that
-// device current) and cached.
+// Id of the calling thread's current CUDA context, unique for the life of the process (a
+// context made after another was destroyed -- e.g. after cudaDeviceReset, or one a C
+// caller creates itself -- gets a new id, even at the same handle address).  False when no
+// context is current or the driver lacks the calls.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+bool current_ctx_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+    cudaGetLastError();
+  });
+  CUcontext c = nullptr;
+  return get_cur && get_id && get_cur(&c) == CUDA_SUCCESS && c && get_id(c, id) == CUDA_SUCCESS;
+}
+
+// Device address of g_attn_scratch in the current context.  In host code the symbol is
+// only a host-side stand-in, so the address is asked for once per context (with that
+// context current) and cached under the context's id: an address never outlives the
+// context it belongs to.  Without a context id the address is looked up on every call.
 ls_status static_scratch(void** out) {
-  static std::atomic<void*> cache[64];
+  struct Entry {
+    unsigned long long ctx;
+    void* ptr;
+  };
+  static Entry cache[64];
+  static int n_cached = 0, next_slot = 0;
   static std::mutex mu;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return fail(LS_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-  if (dev < 0 || dev >= 64) return fail(LS_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
-  void* p = cache[dev].load();
-  if (!p) {
+  unsigned long long id = 0;
+  if (current_ctx_id(&id)) {
     std::lock_guard<std::mutex> lock(mu);
-    p = cache[dev].load();
-    if (!p) {
-      e = cudaGetSymbolAddress(&p, g_attn_scratch);
-      if (e != cudaSuccess || !p)
-        return fail(LS_ERR_CUDA, "cudaGetSymbolAddress(attention scratch): %s", cudaGetErrorString(e));
-      cache[dev].store(p);
-    }
+    for (int i = 0; i < n_cached; ++i)
+      if (cache[i].ctx == id) {
+        *out = cache[i].ptr;
+        return LS_OK;
+      }
+  }
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_attn_scratch);
+  if (e != cudaSuccess || !p)
+    return fail(LS_ERR_CUDA, "cudaGetSymbolAddress(attention scratch): %s", cudaGetErrorString(e));
+  // the lookup makes the device's primary context current if none was: ask for the id again
+  if (current_ctx_id(&id)) {
+    std::lock_guard<std::mutex> lock(mu);
+    Entry& slot = n_cached < 64 ? cache[n_cached++] : cache[(next_slot++) & 63];
+    slot.ctx = id;
+    slot.ptr = p;
   }
   *out = p;
   return LS_OK;

@@ -123,6 +123,8 @@ def build(name: str, ind: syn.IndexerInputs, *, k: int, attn: dict, device="cuda
         t["slot_of_pos"] = hotbuf["slot_of_pos"].to(dev)
         t["recent_score"] = hotbuf["recent"].to(dev)
         t["n_miss"] = torch.zeros((Bn,), dtype=torch.int32, device=dev)
+        for key in ("sel_slot", "miss_pos", "miss_slot"):  # the resolve's lists, kept for inspection
+            t[key] = torch.full((Bn, k), -1, dtype=torch.int32, device=dev)
         # hot buffer rows: the resident positions' KV, copied from the host history
         hbuf = torch.zeros((Bn, n_slots, 576), dtype=torch.bfloat16)
         pt = ind.page_table.cpu()
@@ -133,7 +135,8 @@ def build(name: str, ind: syn.IndexerInputs, *, k: int, attn: dict, device="cuda
             hbuf[b, slots] = host[pt[b, pos // 64].long(), pos % 64]
         t["hbuf"] = hbuf.to(dev)
         hb = dict(pos_of_slot=t["pos_of_slot"], recent_score=t["recent_score"], slot_of_pos=t["slot_of_pos"],
-                  host_kv=host, hbuf=t["hbuf"], n_miss=t["n_miss"])
+                  host_kv=host, hbuf=t["hbuf"], n_miss=t["n_miss"], sel_slot=t["sel_slot"],
+                  miss_pos=t["miss_pos"], miss_slot=t["miss_slot"])
         at = B.attn_args(q=t["a_q"], k_rows=t["hbuf"], o=t["o"], lse=t["lse"], scale=attn["scale"],
                          n_slots=n_slots, k=k)
     else:

@@ -6,6 +6,7 @@ import os
 import socket
 import subprocess
 import sys
+import time
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -14,11 +15,15 @@ COMMON_KEYS = {"metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_s
 
 
 def run_reference_arm(*extra):
+    t0 = time.perf_counter()
     out = subprocess.run([sys.executable, "bench.py", "--impl", "reference", *extra], cwd=ROOT,
                          capture_output=True, text=True, timeout=600, check=True).stdout
+    wall = time.perf_counter() - t0
     lines = [ln for ln in out.splitlines() if ln.startswith("{")]
     assert len(lines) == 1, out  # exactly one JSON line
-    return json.loads(lines[0])
+    d = json.loads(lines[0])
+    d["_wall_s"] = wall
+    return d
 
 
 def test_reference_arm_line():
@@ -30,9 +35,18 @@ def test_reference_arm_line():
     assert d["higher_is_better"] is True and d["unit"] == "tokens/s"
     assert d["value"] > 0 and d["ms_per_step"] > 0
     assert d["config"]["workload"] == "mla_decode_b8_ctx131072_top2048"
+    # the line reports the steps it ran: one request each (a fraction of a token), and
+    # steps x ms_per_step fits inside the process's own wall time
+    assert d["config"]["batch"] == 1
+    f = d["config"]["tokens_per_step"]
+    assert 0 < f <= 1
+    assert abs(d["value"] - f / (d["ms_per_step"] / 1e3)) <= 1e-6 * d["value"]
+    assert (d["steps"] + d["warmup"]) * d["ms_per_step"] / 1e3 <= d["_wall_s"]
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"]
     assert cb["value"] == d["value"] and cb["unit"] == d["unit"]
+    st = cb["single_thread"]
+    assert st["cores"] == 1 and st["value"] > 0 and st["kind"] == "oracle" and st["sample"]
     e2e = d["e2e"]
     assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0

@@ -295,7 +295,9 @@ def test_hotbuf_resolve_and_gather_exact(miss_frac, partial):
 
 
 # ----------------------------------------------------------------------------- a3 coarse-to-fine
-def _c2f_inputs(lens, seed, clustered=True, sigma=0.05):
+def _c2f_inputs(lens, seed, clustered=True, sigma=0.05, w_mixed=False):
+    """Coarse-to-fine indexer inputs: block-clustered keys (2% of the blocks shifted toward
+    the query) or i.i.d. keys; head weights >= 0, or of both signs with ``w_mixed``."""
     Bn = len(lens)
     g = torch.Generator().manual_seed(seed)
     qf = torch.randn((Bn, 64, 128), generator=g)
@@ -308,7 +310,7 @@ def _c2f_inputs(lens, seed, clustered=True, sigma=0.05):
     else:
         keys = torch.randn((sum(lens), 128), generator=g)
     pool_keys = syn.logical_to_pool(keys, lens, table, n_pool)
-    inp = syn.indexer_fp8(lens, seed=seed, w_nonneg=True, q=qf, keys=pool_keys)
+    inp = syn.indexer_fp8(lens, seed=seed, w_nonneg=not w_mixed, q=qf, keys=pool_keys)
     return inp
 
 
@@ -422,6 +424,59 @@ def test_c2f_host_keys_rejects_device_keys():
     ws = torch.empty(B.ls_block_bound_prune_workspace_size(a), dtype=torch.uint8, device=DEV)
     with pytest.raises(B.LsError, match="pinned host memory"):
         B.ls_block_bound_prune(a, ws)
+
+
+@pytest.mark.parametrize("clustered,w_mixed", [(True, False), (False, False), (True, True)])
+def test_block_bound_matches_oracle(clustered, w_mixed):
+    """The bound the GPU prunes with (without its margin) against the oracle's block bound
+    from the same stored summaries: equal to within fp32 rounding, which is held to 2^-12 of
+    the block's magnitude bound M_j = 448 bs_j sum_h |w_h sq_h| sum_d |q_hd| -- a quarter of
+    the 2^-10 M_j margin the pruning adds, so the margin covers the rounding; a dropped head
+    or dim, a sign or a scale slip moves the bound by far more.  With head weights of both
+    signs the bound uses the lower box end for w_h < 0."""
+    lens = [64 * 900 + 21, 64 * 300]
+    inp = _c2f_inputs(lens, seed=71, clustered=clustered, w_mixed=w_mixed)
+    if w_mixed:
+        assert (inp.w.float() < 0).any() and (inp.w.float() > 0).any()
+    idx, sel, surv, nsurv, ub = run_c2f(inp, 2048)
+    wb = inp.w.view(torch.int16).numpy().view(np.uint16)
+    for b, L in enumerate(lens):
+        kmax8, kmin8, bs = O.block_summaries(inp.key_pool.numpy(), inp.key_scale.numpy(),
+                                             inp.page_table.numpy()[b], L)
+        ref = O.block_bound(inp.q[b].numpy(), inp.q_scale[b].numpy(), wb[b], kmax8, kmin8, bs)
+        qabs = np.abs(O.e4m3_decode(inp.q[b].numpy())).sum(axis=1)          # [H]
+        wsq = np.abs(O.bf16_decode(wb[b]) * inp.q_scale[b].numpy().astype(np.float64))
+        mag = 448.0 * bs.astype(np.float64) * float((wsq * qabs).sum())     # [NB]
+        got = ub[b, :ref.shape[0]].cpu().numpy().astype(np.float64)
+        err = np.abs(got - ref)
+        assert (err <= 2.0 ** -12 * mag).all(), float((err / mag).max())
+        assert (ref > 0).any()
+    assert_status_clean()
+
+
+def test_c2f_million_token_context_against_oracle():
+    """The coarse-to-fine indexer at the 1,048,576-token context of its workload (one
+    request): the selection lies within the tie band of the oracle's full-scan top-k,
+    equals the GPU's own full scan, comes only from surviving blocks, and pruning
+    happened."""
+    lens = [1048576]
+    k = 2048
+    inp = _c2f_inputs(lens, seed=81, clustered=True)
+    idx, sel, surv, nsurv, ub = run_c2f(inp, k)
+    ref = O.index_score(**oracle_index_inputs(inp))[0]
+    g = idx[0].cpu().numpy()
+    check_topk_band_local(g, ref, k)
+    s = sel[0].cpu().numpy()
+    assert np.abs(s - ref[g]).max() <= 1e-3 * np.abs(ref).max()
+    scores = gpu_index_scores(inp)
+    full = torch.empty((1, k), dtype=torch.int32, device=DEV)
+    B.ls_topk_select(scores=scores, lens=inp.lens.to(DEV), idx=full)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, full)
+    n = int(nsurv[0])
+    assert n < 0.25 * (lens[0] // 64), f"clustered keys should prune (kept {n} of {lens[0] // 64})"
+    assert set((g // 64).tolist()) <= set(surv[0, :n].cpu().numpy().tolist())
+    assert_status_clean()
 
 
 def check_topk_band_local(g, s, k):
