@@ -5,19 +5,24 @@
 //
 // * attn_mla_tc: MLA-absorbed decode, 128 query heads against one 576-wide latent KV
 //   head whose first 512 dims are V, bf16, on tcgen05 tensor cores.
-//     - Heads are the MMA M dimension (128); a tile of 32 selected rows is N.
+//     - Heads are the MMA M dimension (128); a tile of 64 selected rows is N.
 //     - S = Q K^T (K = 576) and O += P V are tcgen05.mma kind::f16 with f32 TMEM
-//       accumulators.  O for all 512 V dims would fill the whole 512-column TMEM,
-//       so each CTA owns one 256-wide half of V (the pair recomputes S) and keeps
-//       O_half (256 columns) + a double-buffered S (2 x 32 columns) in TMEM.
-//     - Rows are gathered through the page table or the hot-buffer slots by TMA: one
-//       128-byte box per (row, 64-dim panel), landing swizzled in the row's line of
-//       the panel; the same panels serve as the K-major B operand of S and the
+//       accumulators.  O for all 512 V dims would fill the whole 512-column TMEM, so a
+//       pair of CTAs (a 2-CTA cluster) shares each (request, KV split): rank r keeps the
+//       256-wide half O_r in TMEM and contracts S only over its own latent dims (its four
+//       V panels and half of the K-only panel 8); the two 128 x 64 partials are swapped
+//       through distributed shared memory and added, identically, on both sides.
+//     - TMEM: O half (256 columns), two S tiles (2 x 64; P, as bf16 pairs, is written
+//       over the first half of its own S tile), four Q panels (128).  Q panel 8 stays in
+//       shared memory as the A operand of its K steps.
+//     - Rows are gathered through the page table or the hot-buffer slots by TMA
+//       tile::gather4 (four rows x one 128-byte panel per load, 128-byte swizzle) into a
+//       three-stage ring; the same panels serve as the K-major B operand of S and the
 //       MN-major B operand of PV.
 //     - Online softmax in the exp2 domain with lazy rescaling (O is only rescaled
 //       when the running max grows by more than 2^8).
-//     - Split-KV across CTAs (enough CTAs to fill the GPU at small batch), merged
-//       by attn_combine with the log-sum-exp rule.
+//     - Split-KV across CTA pairs (enough to fill the GPU at small batch), merged by
+//       attn_combine with the log-sum-exp rule.
 // * attn_simt: CUDA-core kernel for fp32 (and a bf16 cross-check variant).
 #pragma once
 #include "common.cuh"
@@ -203,33 +208,36 @@ __global__ void __launch_bounds__(256) attn_simt(const AttnParams p) {
 namespace mla {
 constexpr int H = 128, DK = 576, DV = 512, DVH = 256, N = 64;  // N: selected rows per tile
 constexpr int kPanels = DK / 64;                       // 9 panels of 64 bf16 (128 bytes)
-// The two CTAs of a pair split the latent dims of S = Q K^T: rank 0 takes panels 0-4,
-// rank 1 panels 5-8.  Each loads panels 4r .. 4r+4 of every row (its S panels plus its
-// half of V: panels 0-3 or 4-7).
+// Rank r of a pair owns V dims [256r, 256r + 256) = panels 4r .. 4r+3 and contracts S = Q K^T
+// over those four panels plus half of panel 8 (dims 512-575, a K-only panel): K steps 2r,
+// 2r+1 of its four.  Both ranks issue 18 MMAs per tile.  Each loads five panels of every
+// row: its four V panels (local panels 0-3) and panel 8 (local panel 4).
 constexpr int kLocalPanels = 5;
-__host__ __device__ constexpr int s_panels(int rank) { return rank == 0 ? 5 : 4; }  // S panels per rank
 constexpr int kKvPanel = N * 128;                      // 8192
 constexpr int kStageBytes = kLocalPanels * kKvPanel;   // 40960
 constexpr int kStages = 3;
 constexpr int kOffKv = 0;
 constexpr int kOffX = kOffKv + kStages * kStageBytes;  // the peer's S partials
 constexpr int kXBytes = H * N * 4;                     // 32768 per buffer, two buffers
+constexpr int kQPanelBytes = H * 128;                  // one 128-head x 64-dim Q panel
+constexpr int kOffQ8 = kOffX + 2 * kXBytes;            // Q panel 8, the A operand from shared memory
 constexpr int kMaxRows = 4096;                         // k <= 4096: a CTA's rows, resolved once
-constexpr int kOffRows = kOffX + 2 * kXBytes;
+constexpr int kOffRows = kOffQ8 + kQPanelBytes;
 constexpr int kOffBar = kOffRows + kMaxRows * 4;
-// One S tile in TMEM: every MMA instruction costs about the same whatever its N, so the
-// tile is as wide as the TMEM budget allows.  TMEM columns: O half [0, 256), S [256, 320),
-// P as bf16 pairs [320, 352), this rank's Q [352, 512).
-constexpr int kSBufs = 1;
-constexpr int kTmemS = DVH, kTmemP = kTmemS + kSBufs * N, kTmemQ = kTmemP + N / 2;
-static_assert(kTmemQ + 5 * 32 <= 512, "TMEM budget");
-// kv_full[kStages] kv_empty[kStages] s_full[kSBufs] s_read[kSBufs] x_full[2] x_free[2]
-// x_read[2] p_full p_free o_done q_full q_tma
-constexpr int kNumBars = 2 * kStages + 2 * kSBufs + 2 + 2 + 2 + 5;
-// Q arrives by TMA (one 128-head x 64-dim box per panel, 128-byte swizzle) in the KV
-// stage buffers, which the row gathers use only once Q has moved on into TMEM
-constexpr int kQPanelBytes = H * 128;
-static_assert(5 * kQPanelBytes <= kStages * kStageBytes, "Q staging fits the KV stages");
+static_assert(kOffQ8 % 1024 == 0, "128-byte swizzled operand needs 1024-byte alignment");
+// TMEM columns: O half [0, 256), two S tiles [256, 384) (P of a tile, bf16 pairs, is written
+// over the first 32 columns of its own S tile once S has been read), this rank's Q panels
+// 4r .. 4r+3 [384, 512).  Two S tiles let S(i+1) run while the softmax works on tile i.
+constexpr int kSBufs = 2;
+constexpr int kTmemS = DVH, kTmemQ = kTmemS + kSBufs * N;
+static_assert(kTmemQ + 4 * 32 == 512, "TMEM budget");
+// kv_full[kStages] kv_empty[kStages] s_full[2] s_read[2] s_sent[2] x_full[2] x_free[2]
+// x_read[2] p_full[2] p_free o_done q_full q_tma
+constexpr int kNumBars = 2 * kStages + 3 * kSBufs + 2 + 2 + 2 + kSBufs + 4;
+// Q arrives by TMA (one 128-head x 64-dim box per panel, 128-byte swizzle): panels 4r .. 4r+3
+// in the KV stage buffers, which the row gathers use only once Q has moved on into TMEM, and
+// panel 8 straight into its own buffer
+static_assert(4 * kQPanelBytes <= kStages * kStageBytes, "Q staging fits the KV stages");
 constexpr int kOffTmem = kOffBar + kNumBars * 8;
 constexpr int kSmem = 1024 + kOffTmem + 16;
 // warps 0-3 softmax and 4-7 S senders (warp w reads TMEM lanes 32(w%4) .. +31),
@@ -247,16 +255,18 @@ constexpr uint32_t kIdescS = make_idesc(1 /*bf16*/, 128, N, false, false);
 constexpr uint32_t kIdescO = make_idesc(1 /*bf16*/, 128, DVH, false, true);
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
+// Global panel of local panel lp of rank r.
+__host__ __device__ constexpr int global_panel(int rank, int lp) { return lp < 4 ? 4 * rank + lp : 8; }
 }  // namespace mla
 
-// This rank's Q panels (head h's row), staged in shared memory by TMA (128-byte swizzle:
-// 16-byte chunk j of row h sits at chunk j ^ (h & 7)), into TMEM lane h as the MMA's A
-// operand: 64 dims = 32 columns per panel, two bf16 per column.  Every thread of warps
+// This rank's four TMEM Q panels (head h's row), staged in shared memory by TMA (128-byte
+// swizzle: 16-byte chunk j of row h sits at chunk j ^ (h & 7)), into TMEM lane h as the MMA's
+// A operand: 64 dims = 32 columns per panel, two bf16 per column.  Every thread of warps
 // 0-3, converged.
-__device__ __forceinline__ void load_q_tmem(const uint8_t* q_smem, int rank, int h, uint32_t t_row) {
+__device__ __forceinline__ void load_q_tmem(const uint8_t* q_smem, int h, uint32_t t_row) {
   using namespace mla;
 #pragma unroll 1
-  for (int c = 0; c < s_panels(rank); ++c) {
+  for (int c = 0; c < 4; ++c) {
     const uint4* row = (const uint4*)(q_smem + c * kQPanelBytes + h * 128);
     float f[32];
 #pragma unroll
@@ -275,11 +285,13 @@ __device__ __forceinline__ void load_q_tmem(const uint8_t* q_smem, int rank, int
 // One cluster of two CTAs = (request b, KV split); rank r of the pair produces output
 // dims [256r, 256r + 256).  Per 64-row tile, each CTA gathers its five 64-dim panels of the
 // selected rows (TMA gather4 into a three-stage ring), forms its part of S = Q K^T over its
-// latent dims in TMEM (Q, the A operand, also lives in TMEM), sends that 128 x 64 partial to
-// the other CTA through distributed shared memory and adds the one it receives, so both hold
-// the same S (fp32 addition commutes, so the two sums are bit-identical) and run the same
-// online softmax (one thread per head).  P goes to TMEM as bf16 pairs (the A operand of PV)
-// and O_half += P V_half accumulates in TMEM (256 columns).
+// latent dims in TMEM (four Q panels in TMEM and Q panel 8 in shared memory are the A
+// operands), sends that 128 x 64 partial to the other CTA through distributed shared memory
+// and adds the one it receives, so both hold the same S (fp32 addition commutes, so the two
+// sums are bit-identical) and run the same online softmax (one thread per head).  S tiles
+// alternate between two TMEM buffers, so the MMAs of S(i+1) overlap the exchange and softmax
+// of tile i.  P goes back over its own S tile as bf16 pairs (the A operand of PV) and
+// O_half += P V_half accumulates in TMEM (256 columns).
 __global__ void __launch_bounds__(mla::kThreads, 1)
     attn_mla_tc(const AttnParams p, const __grid_constant__ CUtensorMap kv_map,
                 const __grid_constant__ CUtensorMap q_map) {
@@ -289,16 +301,17 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   uint64_t* bars = (uint64_t*)(sm + kOffBar);
   uint64_t* kv_full = bars;
   uint64_t* kv_empty = bars + kStages;
-  uint64_t* s_full = bars + 2 * kStages;   // S partial of the tile in TMEM buffer i % kSBufs
-  uint64_t* s_read = s_full + kSBufs;      // ... and the senders and the softmax have read it
-  uint64_t* x_full = s_read + kSBufs;      // the other rank's partial has arrived here
+  uint64_t* s_full = bars + 2 * kStages;   // S partial of the tile in TMEM buffer i % 2
+  uint64_t* s_read = s_full + kSBufs;      // ... read by the senders and the softmax
+  uint64_t* s_sent = s_read + kSBufs;      // ... read by the senders (P may overwrite it)
+  uint64_t* x_full = s_sent + kSBufs;      // the other rank's partial has arrived here
   uint64_t* x_free = x_full + 2;           // the other rank has read our partial (credit)
   uint64_t* x_read = x_free + 2;           // our softmax has read receive buffer b
-  uint64_t* p_full = x_read + 2;
-  uint64_t* p_free = p_full + 1;
-  uint64_t* o_done = p_full + 2;
-  uint64_t* q_full = p_full + 3;
-  uint64_t* q_tma = p_full + 4;
+  uint64_t* p_full = x_read + 2;           // P of the tile in buffer i % 2 is in TMEM
+  uint64_t* p_free = p_full + kSBufs;      // PV of the latest tile has finished
+  uint64_t* o_done = p_free + 1;
+  uint64_t* q_full = p_free + 2;
+  uint64_t* q_tma = p_free + 3;
   uint32_t* tmem_slot = (uint32_t*)(sm + kOffTmem);
   __shared__ int s_abort;
   __shared__ uint64_t s_mask[kStages];  // valid rows of the tile in each stage
@@ -324,13 +337,14 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     for (int s = 0; s < kSBufs; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&s_read[s], 256);  // this CTA's sender and softmax threads
+      mbar_init(&s_sent[s], 128);  // this CTA's sender threads
+      mbar_init(&p_full[s], 128);  // this CTA's softmax threads
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&x_full[s], 1);  // armed with the partial's bytes; the other CTA's stores land on it
       mbar_init(&x_free[s], 1);    // the other CTA's forwarding thread, remotely
       mbar_init(&x_read[s], 128);  // this CTA's softmax threads
     }
-    mbar_init(p_full, 128);
     mbar_init(p_free, 1);
     mbar_init(o_done, 1);
     mbar_init(q_full, 128);  // the softmax threads, once Q is in TMEM (and out of the stages)
@@ -339,9 +353,10 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     fence_mbar_init();
     // Q is an input of the step, never written by the kernel before: fetch it at once
     if (my_tiles_max > 0) {
-      mbar_arrive_expect_tx(q_tma, s_panels(rank) * kQPanelBytes);
-      for (int c = 0; c < s_panels(rank); ++c)
-        tma_load_2d(sbase + kOffKv + c * kQPanelBytes, &q_map, q_tma, (rank * s_panels(0) + c) * 64, b * H);
+      mbar_arrive_expect_tx(q_tma, 5 * kQPanelBytes);
+      for (int c = 0; c < 4; ++c)
+        tma_load_2d(sbase + kOffKv + c * kQPanelBytes, &q_map, q_tma, global_panel(rank, c) * 64, b * H);
+      tma_load_2d(sbase + kOffQ8, &q_map, q_tma, 8 * 64, b * H);
     }
     // arm the receive buffers for tiles 0 and 1 before the other CTA can send (an armed
     // buffer that no tile uses is never waited on)
@@ -358,13 +373,12 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tm_o = tmem;          // columns [0, 256): O half
-  const uint32_t tm_s = tmem + kTmemS;  // kSBufs S tiles
-  const uint32_t tm_p = tmem + kTmemP;  // P of the current tile, bf16 pairs (PV's A operand)
-  const uint32_t tm_q = tmem + kTmemQ;  // this rank's Q panels
+  const uint32_t tm_s = tmem + kTmemS;  // two S tiles (P over the first half of each)
+  const uint32_t tm_q = tmem + kTmemQ;  // this rank's Q panels 4r .. 4r+3
   if (warp < 4 && my_tiles_max > 0) {
     // a wait that gives up (recorded in the device status) aborts the whole CTA
     if (mbar_wait(q_tma, 0)) {
-      load_q_tmem(sm + kOffKv, rank, threadIdx.x, tm_q + ((uint32_t)(warp * 32) << 16));
+      load_q_tmem(sm + kOffKv, threadIdx.x, tm_q + ((uint32_t)(warp * 32) << 16));
       tc_fence_before();
     } else if (threadIdx.x == 0) {
       s_abort = 1;
@@ -409,11 +423,11 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     // ================= row gathers: tile i goes to stage i % kStages =================
     // The gather warps first resolve all of this CTA's rows (selection -> page table) into
     // shared memory.  A tile's 16 groups of 4 rows x 5 panels are then 80 TMA gather4
-    // loads; gather e (group e % 16, panel e / 16) is issued by lane e % 20 of gather warp
-    // e / 20, each landing as four 128-byte-swizzled lines of its panel.  Padding rows point one past the pool, which the TMA unit fills
-    // with zeros; the softmax masks them.
+    // loads; gather e (group e % 16, local panel e / 16) is issued by lane e % 20 of gather
+    // warp e / 20, each landing as four 128-byte-swizzled lines of its panel.  Padding rows
+    // point one past the pool, which the TMA unit fills with zeros; the softmax masks them.
     const int lw = warp - kLoadWarp0;
-    const int e = lw * kGathersPerWarp + lane;  // this lane's gather (if lane < 10)
+    const int e = lw * kGathersPerWarp + lane;  // this lane's gather (if lane < 20)
     const int lx = e % (N / 4), lp = e / (N / 4);
     // resolve all of this CTA's rows once (out-of-range marker: one past the pool)
     int* s_rows = (int*)(sm + kOffRows);
@@ -457,7 +471,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
       if (lane < kGathersPerWarp) {
         const int* rr = s_rows + i * N + 4 * lx;
         tma_gather4(sbase + kOffKv + st * kStageBytes + lp * kKvPanel + lx * 512, &kv_map, &kv_full[st],
-                    (rank * 4 + lp) * 64, rr[0], rr[1], rr[2], rr[3]);
+                    global_panel(rank, lp) * 64, rr[0], rr[1], rr[2], rr[3]);
       }
     }
     // never leave with copies in flight (the tiles of the last kStages loads)
@@ -482,47 +496,55 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ================= MMA issuer: event driven =================
-    // S(i) (this rank's panels) goes out whole once tile i has landed and S(i-kSBufs) has
-    // been read out of its TMEM buffer; PV(i) as soon as P(i) is ready.  Neither blocks
-    // the other.
+    // S(i) goes out whole once tile i has landed and S buffer i % 2 is free again: tile
+    // i-2's S has been read (by the senders and the softmax) and PV(i-2), which reads P(i-2)
+    // from the same columns, has been issued (the tensor pipe runs one thread's MMAs in
+    // order).  PV(i) goes out as soon as P(i) is ready.  Neither blocks the other.
     if (lane == 0 && my_tiles > 0) {
-      const int nsp = s_panels(rank);
-      const int lp0 = rank;  // first local panel used by S: rank 1 skips panel 4 (V only)
+      const uint32_t q8 = sbase + kOffQ8;
       bool ok = mbar_wait(q_full, 0);
       tc_fence_after();
       int ns = 0, npv = 0;
       uint64_t idle_since = 0;
       while (ok && npv < my_tiles) {
         bool progressed = false;
-        if (npv < ns && mbar_test_wait(p_full, npv & 1)) {
+        if (npv < ns && mbar_test_wait(&p_full[npv % kSBufs], (npv / kSBufs) & 1)) {
           tc_fence_after();
-          // this rank's V half is local panels 0-3 of the stage
+          // this rank's V half is local panels 0-3 of the stage; P(npv) sits over its S tile
           const uint32_t v = sbase + kOffKv + (npv % kStages) * kStageBytes;
+          const uint32_t pa = tm_s + (npv % kSBufs) * N;
 #pragma unroll
           for (int kk = 0; kk < N / 16; ++kk) {
             const uint64_t bd = make_sdesc(v + kk * 16 * 128, kKvPanel, 1024, kSwizzle128);
-            mma_bf16_ta(tm_o, tm_p + kk * 8, bd, kIdescO, (npv > 0 || kk > 0));
+            mma_bf16_ta(tm_o, pa + kk * 8, bd, kIdescO, (npv > 0 || kk > 0));
           }
           tc_commit(&kv_empty[npv % kStages]);
           tc_commit(p_free);
           ++npv;
           progressed = true;
         }
-        // S(i): this rank's 20 (or 16) K steps into TMEM buffer i % kSBufs.  Each MMA
-        // waits on the previous one (same accumulator), so S costs about as many MMA
-        // latencies as it has K steps, whatever N is.
-        if (ns < my_tiles && (ns < kSBufs || mbar_test_wait(&s_read[ns % kSBufs], ((ns / kSBufs) - 1) & 1)) &&
+        // S(i): 16 K steps over the TMEM Q panels, then this rank's two steps of panel 8
+        // with Q from shared memory.  Each MMA waits on the previous one (same
+        // accumulator), so S costs about as many MMA latencies as it has K steps.
+        if (ns < my_tiles &&
+            (ns < kSBufs || (npv >= ns - 1 && mbar_test_wait(&s_read[ns % kSBufs], ((ns / kSBufs) - 1) & 1))) &&
             mbar_test_wait(&kv_full[ns % kStages], (ns / kStages) & 1)) {
           tc_fence_after();
-          const uint32_t kv = sbase + kOffKv + (ns % kStages) * kStageBytes + lp0 * kKvPanel;
+          const uint32_t kv = sbase + kOffKv + (ns % kStages) * kStageBytes;
           const uint32_t sb = tm_s + (ns % kSBufs) * N;
 #pragma unroll 1
-          for (int pn = 0; pn < nsp; ++pn) {
+          for (int pn = 0; pn < 4; ++pn) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t bd = make_sdesc(kv + pn * kKvPanel + kk * 32, 16, 1024, kSwizzle128);
               mma_bf16_ta(sb, tm_q + pn * 32 + kk * 8, bd, kIdescS, (pn | kk) != 0);
             }
+          }
+#pragma unroll
+          for (int kk = 2 * rank; kk < 2 * rank + 2; ++kk) {
+            const uint64_t ad = make_sdesc(q8 + kk * 32, 16, 1024, kSwizzle128);
+            const uint64_t bd = make_sdesc(kv + 4 * kKvPanel + kk * 32, 16, 1024, kSwizzle128);
+            mma_bf16(sb, ad, bd, kIdescS, 1);
           }
           tc_commit(&s_full[ns % kSBufs]);
           ++ns;
@@ -531,6 +553,9 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
         if (progressed) {
           idle_since = 0;
         } else {
+          // nothing to issue yet: step aside briefly, so that this polling loop does not take
+          // issue slots from the softmax warp that shares its scheduler
+          __nanosleep(64);
           const uint64_t now = globaltimer();
           if (idle_since == 0) {
             idle_since = now;
@@ -562,14 +587,15 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     cluster_waited = true;
     for (int i = 0; i < my_tiles; ++i) {
       const int sb = i % kSBufs, xb = i & 1;
-      if (!mbar_wait(&s_full[sb], (i / kSBufs) & 1)) break;
+      // every wait in front of a warp-collective TMEM access is decided for the whole warp
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], (i / kSBufs) & 1))) break;
       tc_fence_after();
       float cur[N];
-#pragma unroll
-      for (int c = 0; c < N; c += 32) tmem_ld32(tm_s + lane_off + sb * N + c, cur + c);
+      tmem_ld64(tm_s + lane_off + sb * N, cur);
       tc_fence_before();
       mbar_arrive(&s_read[sb]);
-      if (i >= 2 && !mbar_wait_cluster(&x_free[xb], ((i >> 1) - 1) & 1)) break;
+      mbar_arrive(&s_sent[sb]);  // the softmax may now write P over this S tile
+      if (i >= 2 && !__all_sync(0xffffffffu, mbar_wait_cluster(&x_free[xb], ((i >> 1) - 1) & 1))) break;
 #pragma unroll
       for (int c = 0; c < N / 4; ++c)
         st_async_v4(x_peer + xb * kXBytes + c * 2048 + h * 16, cur[4 * c], cur[4 * c + 1], cur[4 * c + 2],
@@ -585,17 +611,17 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     for (int i = 0; i < my_tiles; ++i) {
       const int st = i % kStages, sb = i % kSBufs, xb = i & 1;
       // the loaders published the tile's valid rows with their kv_full arrivals
-      if (!mbar_wait(&kv_full[st], (i / kStages) & 1)) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&kv_full[st], (i / kStages) & 1))) { ok = false; break; }
       const uint64_t vmask = s_mask[st];
       // S = this rank's partial (TMEM) + the other rank's (receive buffer xb)
-      if (!mbar_wait(&s_full[sb], (i / kSBufs) & 1)) { ok = false; break; }
+      // every wait in front of a warp-collective TMEM access is decided for the whole warp
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], (i / kSBufs) & 1))) { ok = false; break; }
       tc_fence_after();
       float s[N];
-#pragma unroll
-      for (int c = 0; c < N; c += 32) tmem_ld32(tm_s + lane_off + sb * N + c, s + c);
+      tmem_ld64(tm_s + lane_off + sb * N, s);
       tc_fence_before();
       mbar_arrive(&s_read[sb]);  // with the senders' reads, this frees the S buffer
-      if (!mbar_wait_cluster(&x_full[xb], (i >> 1) & 1)) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait_cluster(&x_full[xb], (i >> 1) & 1))) { ok = false; break; }
 #pragma unroll
       for (int c = 0; c < N / 4; ++c) {
         const float4 o = *(const float4*)(sm + kOffX + xb * kXBytes + c * 2048 + h * 16);
@@ -605,10 +631,19 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
         s[4 * c + 3] += o.w;
       }
       mbar_arrive(&x_read[xb]);  // the forwarding thread re-arms buffer xb and passes the credit
-      float tmax = -INFINITY;
+      // a tile whose rows are all valid (every tile but a ragged last one) skips the masking;
+      // max and sum run as four independent chains
+      const bool full = vmask == ~0ull;
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (full) {
 #pragma unroll
-      for (int r = 0; r < N; ++r)
-        if ((vmask >> r) & 1u) tmax = fmaxf(tmax, s[r]);
+        for (int r = 0; r < N; ++r) m4[r & 3] = fmaxf(m4[r & 3], s[r]);
+      } else {
+#pragma unroll
+        for (int r = 0; r < N; ++r)
+          if ((vmask >> r) & 1u) m4[r & 3] = fmaxf(m4[r & 3], s[r]);
+      }
+      const float tmax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       const float mt = tmax * sl2;
       float factor = 1.f;
       bool rescale = false;
@@ -619,16 +654,26 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
         }
         m_run = mt;
       }
-      float psum = 0.f;  // s becomes P in place
+      float p4[4] = {0.f, 0.f, 0.f, 0.f};  // s becomes P in place
+      if (full) {
 #pragma unroll
-      for (int r = 0; r < N; ++r) {
-        s[r] = ((vmask >> r) & 1u) ? ex2_ftz(fmaf(s[r], sl2, -m_run)) : 0.f;
-        psum += s[r];
+        for (int r = 0; r < N; ++r) {
+          s[r] = ex2_ftz(fmaf(s[r], sl2, -m_run));
+          p4[r & 3] += s[r];
+        }
+      } else {
+#pragma unroll
+        for (int r = 0; r < N; ++r) {
+          s[r] = ((vmask >> r) & 1u) ? ex2_ftz(fmaf(s[r], sl2, -m_run)) : 0.f;
+          p4[r & 3] += s[r];
+        }
       }
-      if (i >= 1 && !mbar_wait(p_free, (i - 1) & 1)) { ok = false; break; }
+      const float psum = (p4[0] + p4[1]) + (p4[2] + p4[3]);
       // tcgen05.ld/st are warp-collective: the whole warp rescales when any lane must
-      // (lanes that need not have factor 1)
+      // (lanes that need not have factor 1).  O may be rescaled only once PV(i-1) has
+      // finished adding into it (a rescale never happens at the first tile).
       if (__any_sync(0xffffffffu, rescale)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(p_free, (i - 1) & 1))) { ok = false; break; }
         tc_fence_after();
 #pragma unroll 1
         for (int c0 = 0; c0 < DVH; c0 += 32) {
@@ -641,17 +686,20 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
         tmem_wait_st();
       }
       l_run = l_run * factor + psum;
-      // P(i) into TMEM lane h: column c holds rows 2c, 2c+1 as bf16 (PV(i-1) has read P(i-1))
+      // P(i) into TMEM lane h over the first 32 columns of its own S tile: column c holds
+      // rows 2c, 2c+1 as bf16 -- once the senders have read that S tile
       float pw[N / 2];
 #pragma unroll
       for (int c = 0; c < N / 2; ++c) {
         __nv_bfloat162 two = __floats2bfloat162_rn(s[2 * c], s[2 * c + 1]);
         pw[c] = __uint_as_float(*(uint32_t*)&two);
       }
-      tmem_st32(tm_p + lane_off, pw);
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_sent[sb], (i / kSBufs) & 1))) { ok = false; break; }
+      tc_fence_after();
+      tmem_st32(tm_s + lane_off + sb * N, pw);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[sb]);
     }
     // ---- epilogue
     bool fin = ok && my_tiles > 0 && mbar_wait(o_done, 0);
