@@ -422,6 +422,44 @@ def run_ours(args):
     return 0
 
 
+def host_link_peaks(batch, n_slots=4096, reps=5):
+    """The host link's read rate measured in this process, two ways over the same bytes (a
+    whole hot buffer's worth of 1,152-byte rows, contiguous in pinned host memory): a plain
+    copy-engine host-to-device copy, and the library's miss-gather kernel reading every row
+    over the link (SM zero-copy loads, its own launch shape).  Best of `reps`, GB/s."""
+    import torch
+    from sparse_attention_decode_ls_b200 import binding as B
+    stream = torch.cuda.current_stream()
+    rows = batch * n_slots
+    host = torch.empty((rows // 64, 64, 576), dtype=torch.bfloat16, pin_memory=True)
+    host.view(torch.int16).random_(generator=torch.Generator().manual_seed(5))
+    dev = torch.empty(host.shape, dtype=torch.bfloat16, device="cuda")
+    nbytes = host.numel() * 2
+
+    def best(fn):
+        t = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            t.append(e0.elapsed_time(e1))
+        return nbytes / (min(t) / 1e3) / 1e9
+
+    ce = best(lambda: dev.copy_(host, non_blocking=True))
+    pages = n_slots // 64
+    table = torch.arange(rows // 64, dtype=torch.int32, device="cuda").view(batch, pages)
+    pos = torch.arange(n_slots, dtype=torch.int32, device="cuda").repeat(batch, 1)
+    n = torch.full((batch,), n_slots, dtype=torch.int32, device="cuda")
+    hbuf = dev.view(batch, n_slots, 576)
+    sm = best(lambda: B.ls_gather_misses(host_kv=host, page_table=table, miss_pos=pos, miss_slot=pos, n_miss=n,
+                                         hbuf=hbuf))
+    assert torch.equal(hbuf.view(-1).view(torch.int16).cpu(), host.view(-1).view(torch.int16))
+    del host, dev
+    return {"copy_engine_GBps": ce, "sm_gather_contiguous_GBps": sm, "bytes": nbytes}
+
+
 def run_hotbuf(args):
     """Optional line (not the headline): the hot-buffer decode step -- indexer, top-k,
     hot-buffer resolve, gather of the misses from pinned host memory over the host link,
@@ -474,6 +512,10 @@ def run_hotbuf(args):
     stages = {n: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in stage_ev) for i, n in enumerate(names)}
     n_miss = int(wl.tensors["n_miss"].sum().item())
     link_bytes = n_miss * 576 * 2
+    peaks = host_link_peaks(batch)
+    link_peak = max(peaks["copy_engine_GBps"], peaks["sm_gather_contiguous_GBps"])
+    fetch_GBps = link_bytes / (stages["gather"] / 1e3) / 1e9
+    step_GBps = link_bytes / (ms / 1e3) / 1e9
     out = {"metric": "hot-buffer sparse-attn decode tokens/s at 128K ctx", "value": batch / (ms / 1e3),
            "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3+bf16 (f32 accumulate)",
@@ -482,8 +524,13 @@ def run_hotbuf(args):
                       "miss_frac": args.miss, "history": "pinned host memory, read over the host link",
                       "l2": "evicted before every step (256 MB written, then 256 MB read)"},
            "gpu_launches": wl.kernels_per_step * args.steps,
-           "host_link": {"bytes_per_step": link_bytes, "GBps": link_bytes / (ms / 1e3) / 1e9,
-                         "gather_GBps": link_bytes / (stages["gather"] / 1e3) / 1e9},
+           "host_link": {"bytes_per_step": link_bytes, "GBps": step_GBps, "gather_GBps": fetch_GBps,
+                         "peak_GBps": link_peak, "peaks_measured": peaks,
+                         "fetch_frac": fetch_GBps / link_peak, "step_frac": step_GBps / link_peak,
+                         "note": "peak = the faster of a plain pinned host-to-device copy and the miss-gather "
+                                 "kernel over contiguous rows, measured in this run; fetch_frac: the step's miss "
+                                 "fetch (scattered 1,152-byte rows) over its stage time; step_frac: the misses' "
+                                 "bytes over the whole step"},
            "stages_ms": stages,
            "clocks": clk.summary(), "device_status": status}
     print(json.dumps(out), flush=True)
@@ -566,6 +613,8 @@ def run_sweep(args):
     flush_r = torch.ones(64 << 20, dtype=torch.float32, device="cuda")
     sink = torch.empty((), dtype=torch.float32, device="cuda")
     rows, statuses = [], []
+    peaks = host_link_peaks(64)
+    link_peak = max(peaks["copy_engine_GBps"], peaks["sm_gather_contiguous_GBps"])
     with ClockSampler(0) as clk:
         for bsz in batches:
             lens = syn.ragged_lens(bsz, 4096, 16384, seed=1005)
@@ -592,9 +641,23 @@ def run_sweep(args):
             torch.cuda.synchronize()
             statuses.append(B.ls_check_device_status())
             ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+            # the miss fetch's own time from a pass with the stage boundaries recorded
+            stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(5)]
+            for evs in stage_ev:
+                for e in evs:
+                    e.record(stream)
+            for evs in stage_ev:
+                prep()
+                wl.step(events=B.event_array(evs))
+            torch.cuda.synchronize()
+            gather_ms = statistics.median(e[3].elapsed_time(e[4]) for e in stage_ev)
             n_miss = int(wl.tensors["n_miss"].sum().item())
+            link = n_miss * 1152
             rows.append({"batch": bsz, "ms_per_step": ms, "tokens_per_s": bsz / (ms / 1e3),
-                         "mean_ctx": sum(lens) / bsz, "link_bytes_per_step": n_miss * 1152,
+                         "mean_ctx": sum(lens) / bsz, "link_bytes_per_step": link,
+                         "fetch_GBps": link / (gather_ms / 1e3) / 1e9, "step_link_GBps": link / (ms / 1e3) / 1e9,
+                         "fetch_frac": link / (gather_ms / 1e3) / 1e9 / link_peak,
+                         "step_frac": link / (ms / 1e3) / 1e9 / link_peak,
                          "gpu_launches_per_step": wl.kernels_per_step})
             del wl
             gc.collect()
@@ -608,7 +671,8 @@ def run_sweep(args):
                       "history": "pinned host memory, misses read over the host link",
                       "l2": "evicted before every step (256 MB written, then 256 MB read)",
                       "statistic": "median over the timed steps"},
-           "sweep": rows, "clocks": clk.summary(), "device_status": max(statuses) if statuses else 0}
+           "sweep": rows, "host_link_peak_GBps": link_peak, "host_link_peaks_measured": peaks,
+           "clocks": clk.summary(), "device_status": max(statuses) if statuses else 0}
     print(json.dumps(out), flush=True)
     return 0
 

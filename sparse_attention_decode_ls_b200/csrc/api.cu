@@ -330,8 +330,9 @@ ls_status launch_topk_cl(const ls::TopkParams& p0, int B, cudaStream_t st, std::
 ls_status launch_topk(int B, int k, const float* scores, int stride, const int* lens, int len_mul, int len_div,
                       int len_limit, const int* unit_list, int list_stride, int* idx, float* sel, float* thr,
                       cudaStream_t st, const int* pos_list = nullptr, int pos_stride = 0,
-                      const int* pos_offset = nullptr) {
+                      const int* pos_offset = nullptr, int* clear = nullptr) {
   ls::TopkParams p{};
+  p.clear = clear;
   p.pos_list = pos_list; p.pos_stride = pos_stride; p.pos_offset = pos_offset;
   p.B = B; p.k = k; p.stride = stride; p.scores = scores; p.lens = lens; p.len_mul = len_mul;
   p.len_div = len_div; p.len_limit = len_limit; p.unit_list = unit_list; p.list_stride = list_stride;
@@ -362,11 +363,56 @@ int attn_nsplit(const ls_sparse_attn_args* a) {
   return (tiles + per - 1) / per;
 }
 
+std::atomic<uint64_t> g_smem_attn_tc{0}, g_smem_attn_simt_f{0}, g_smem_attn_simt_b{0};
+
+// Most clusters of 2 * ns tensor-core attention CTAs the device runs at once (asked once
+// per device and split count); 0 when such a cluster cannot be launched.
+int attn_max_clusters(int ns) {
+  static std::atomic<int> cache[kMaxDevices][ls::mla::kMergeBatch + 1];  // 0 unknown, -1 none
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= kMaxDevices || ns < 1 || ns > ls::mla::kMergeBatch) return 0;
+  const int known = cache[dev][ns].load();
+  if (known != 0) return known > 0 ? known : 0;
+  int n = 0;
+  bool ok = allow_smem(ls::attn_mla_tc, ls::mla::kSmem, g_smem_attn_tc) == cudaSuccess;
+  if (ok && 2 * ns > 8)
+    ok = cudaFuncSetAttribute(ls::attn_mla_tc, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess;
+  if (ok) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3(2 * ns, 1);
+    cfg.blockDim = dim3(ls::mla::kThreads);
+    cfg.dynamicSmemBytes = ls::mla::kSmem;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2 * ns;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    ok = cudaOccupancyMaxActiveClusters(&n, ls::attn_mla_tc, &cfg) == cudaSuccess && n > 0;
+  }
+  cudaGetLastError();  // a refused query leaves no sticky error
+  cache[dev][ns].store(ok ? n : -1);
+  return ok ? n : 0;
+}
+
+// Whether the splits of a tensor-core attention launch are merged inside one cluster per
+// request instead of by attn_combine: one pass, a bf16 output, a split count that divides
+// the heads (2, 4 or 8 -- at most a 16-CTA cluster), and every request's cluster resident
+// at once (otherwise the clusters would run in waves).
+bool attn_merge(const ls_sparse_attn_args* a, int npasses) {
+  if (a->dtype != LS_BF16 || a->variant != 0 || npasses != 1 || a->o_f32) return false;
+  const int ns = attn_nsplit(a);
+  if (ns != 2 && ns != 4 && ns != 8) return false;
+  return attn_max_clusters(ns) >= a->batch;
+}
+
 // Split-KV partials of `npasses` launches over the same requests (each with
-// attn_nsplit splits), merged by one combine.
+// attn_nsplit splits), merged by one combine; none when the splits merge in the cluster.
 size_t attn_ws_bytes(const ls_sparse_attn_args* a, int npasses = 1) {
   const int ns = attn_nsplit(a) * npasses;
-  if (ns <= 1) return 0;
+  if (ns <= 1 || attn_merge(a, npasses)) return 0;
   return align256((size_t)a->batch * ns * a->heads * a->dv * 4) + align256((size_t)a->batch * ns * a->heads * 8);
 }
 
@@ -405,8 +451,6 @@ ls_status validate_attn(const ls_sparse_attn_args* a, bool need_sel) {
   return LS_OK;
 }
 
-std::atomic<uint64_t> g_smem_attn_tc{0}, g_smem_attn_simt_f{0}, g_smem_attn_simt_b{0};
-
 // Programmatic dependent launch: the kernel may start while the one before it finishes
 // (it waits for it with griddepcontrol.wait before touching its output).
 cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, size_t smem, cudaStream_t st, cudaLaunchAttribute* attr,
@@ -431,7 +475,7 @@ cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, size_t smem, cudaStream_t s
 ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressing, const int* page_table,
                       int max_pages, int n_slots, const void* rows, long long num_rows, void* ws, size_t ws_bytes,
                       cudaStream_t st, bool pdl, bool compacted = false, int pass = 0, int npasses = 1,
-                      bool combine = true, const int* n_valid = nullptr) {
+                      bool combine = true, const int* n_valid = nullptr, int* done = nullptr) {
   ls::AttnParams p{};
   p.B = a->batch; p.H = a->heads; p.dk = a->dk; p.dv = a->dv; p.k = a->k; p.scale = a->softmax_scale;
   p.addressing = addressing; p.max_pages = max_pages; p.n_slots = n_slots; p.row_stride = a->row_stride;
@@ -446,7 +490,12 @@ ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressi
     p.compacted = compacted ? 1 : 0;
     p.o_f32 = a->o_f32 ? 1 : 0;
     p.n_valid = n_valid;
-    if (total > 1) {
+    const bool merge = attn_merge(a, npasses);
+    p.merge = merge ? 1 : 0;
+    // a per-request completion count lets the combine start request by request; only for a
+    // single pass whose count the kernel before (the top-k) has just zeroed
+    p.done = (total > 1 && !merge && combine && npasses == 1) ? done : nullptr;
+    if (total > 1 && !merge) {
       const size_t need = attn_ws_bytes(a, npasses);
       LS_REQUIRE(ws && ws_bytes >= need, "attention workspace too small (%zu < %zu bytes)", ws_bytes, need);
       LS_REQUIRE(((uintptr_t)ws & 255) == 0, "workspace must be 256-byte aligned");
@@ -457,9 +506,10 @@ ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressi
       return check_launch("attn_mla_tc attribute");
     cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = pdl_config(dim3(2 * ns, a->batch), dim3(ls::mla::kThreads), ls::mla::kSmem, st, attr, pdl);
-    // the two CTAs of an (request, split) pair form a cluster
+    // the two CTAs of an (request, split) pair form a cluster; with the in-cluster merge,
+    // all splits of a request do
     attr[cfg.numAttrs].id = cudaLaunchAttributeClusterDimension;
-    attr[cfg.numAttrs].val.clusterDim.x = 2;
+    attr[cfg.numAttrs].val.clusterDim.x = merge ? 2 * ns : 2;
     attr[cfg.numAttrs].val.clusterDim.y = 1;
     attr[cfg.numAttrs].val.clusterDim.z = 1;
     cfg.numAttrs += 1;
@@ -471,7 +521,7 @@ ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressi
     cudaError_t e = cudaLaunchKernelEx(&cfg, ls::attn_mla_tc, p, kv_map, q_map);
     if (e != cudaSuccess) return fail(LS_ERR_CUDA, "attn_mla_tc: %s", cudaGetErrorString(e));
     LS_TRY(check_launch("attn_mla_tc"));
-    if (total > 1 && combine) {
+    if (total > 1 && combine && !merge) {
       cudaLaunchConfig_t cc = pdl_config(dim3(ls::mla::H * ls::mla::DV / 8 / ls::kCombineThreads, a->batch),
                                          dim3(ls::kCombineThreads), 0, st, attr, true);
       e = cudaLaunchKernelEx(&cc, ls::attn_combine, p);
@@ -731,7 +781,7 @@ ls_status run_c2f(const ls_block_bound_prune_args* a, void* ws, size_t ws_bytes,
 // ---- decode step workspace ------------------------------------------------------------
 struct StepLayout {
   size_t off_scores, off_idx, off_sel, off_selslot, off_mpos, off_mslot, off_nmiss, off_hitslot, off_cpos, off_crow,
-      off_cnmiss, off_cnhit, off_stage, off_attn, off_c2f, total;
+      off_cnmiss, off_cnhit, off_stage, off_attn, off_done, off_c2f, total;
 };
 
 ls_block_bound_prune_args step_c2f_args(const ls_decode_step_args* a, int* idx, float* sel) {
@@ -831,6 +881,7 @@ StepLayout step_layout(const ls_decode_step_args* a) {
   l.off_cnhit = take(two_pass ? (size_t)B * 4 : 0);
   l.off_stage = take(two_pass ? (size_t)B * k * t.row_stride * 2 : 0);
   l.off_attn = take(attn_ws_bytes(&t, two_pass ? 2 : 1));
+  l.off_done = take((size_t)B * 4);  // per-request attention completion counts
   if (a->use_c2f) {
     ls_block_bound_prune_args c = step_c2f_args(a, nullptr, nullptr);
     l.off_c2f = take(c2f_layout(&c).total);
@@ -1226,8 +1277,10 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
       LS_TRY(launch_index_simt(&tmp, st));
     }
     rec(1);
+    // the top-k also zeroes the attention's per-request completion counts (paged path)
+    int* done = !a->use_hotbuf ? (int*)(w + l.off_done) : nullptr;
     LS_TRY(launch_topk(ix->batch, a->k, scores, ix->max_len, ix->lens, 1, 1, ix->max_len, nullptr, 0, idx, sel,
-                       nullptr, st));
+                       nullptr, st, nullptr, 0, nullptr, done));
   }
   void* attn_ws = w + l.off_attn;
   if (a->use_hotbuf) {
@@ -1305,8 +1358,9 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
     const int* pt = at.page_table ? at.page_table : ix->page_table;
     const int mp = at.page_table ? at.max_pages : ix->max_pages;
     wait_q(st);
+    int* done = !a->use_c2f ? (int*)(w + l.off_done) : nullptr;
     LS_TRY(launch_attn(&at, idx, LS_ROWS_PAGED, pt, mp, 0, nullptr, at.num_rows, attn_ws, attn_ws_b, st, true,
-                       true));
+                       true, 0, 1, true, nullptr, done));
   }
   rec(5);
   return ok();

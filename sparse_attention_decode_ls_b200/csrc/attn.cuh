@@ -51,6 +51,12 @@ struct AttnParams {
   int o_f32;         // tensor-core kernel: o is float32 (else bf16)
   const int* n_valid;  // optional [B]: and there are n_valid[b] of them; the splits share
                        //   those rows instead of all k entries
+  int* done;           // optional [B], zero at launch: every CTA adds 1 once its split partial
+                       //   is stored, and attn_combine starts on a request as soon as all
+                       //   2 * nsplit of its CTAs have, instead of after the whole grid
+  int merge;           // tensor-core kernel: the CTAs of all splits of a request form one
+                       //   cluster and merge the splits in distributed shared memory (no
+                       //   partials in global memory, no combine kernel); nsplit in {2, 4, 8}
 };
 
 // 2^x with the hardware approximation (relative error about 2^-22; results below the
@@ -215,12 +221,14 @@ constexpr int kPanels = DK / 64;                       // 9 panels of 64 bf16 (1
 constexpr int kLocalPanels = 5;
 constexpr int kKvPanel = N * 128;                      // 8192
 constexpr int kStageBytes = kLocalPanels * kKvPanel;   // 40960
-constexpr int kStages = 3;
+// Four stages: at the headline batch a CTA's whole share (four tiles) is in flight at once
+constexpr int kStages = 4;
 constexpr int kOffKv = 0;
-constexpr int kOffX = kOffKv + kStages * kStageBytes;  // the peer's S partials
-constexpr int kXBytes = H * N * 4;                     // 32768 per buffer, two buffers
+constexpr int kOffX = kOffKv + kStages * kStageBytes;  // the peer's S partial
+constexpr int kXBytes = H * N * 4;                     // 32768
+constexpr int kXBufs = 1;  // one receive buffer: the sender of tile i waits for the read of i-1
 constexpr int kQPanelBytes = H * 128;                  // one 128-head x 64-dim Q panel
-constexpr int kOffQ8 = kOffX + 2 * kXBytes;            // Q panel 8, the A operand from shared memory
+constexpr int kOffQ8 = kOffX + kXBufs * kXBytes;       // Q panel 8, the A operand from shared memory
 constexpr int kMaxRows = 4096;                         // k <= 4096: a CTA's rows, resolved once
 constexpr int kOffRows = kOffQ8 + kQPanelBytes;
 constexpr int kOffBar = kOffRows + kMaxRows * 4;
@@ -231,9 +239,16 @@ static_assert(kOffQ8 % 1024 == 0, "128-byte swizzled operand needs 1024-byte ali
 constexpr int kSBufs = 2;
 constexpr int kTmemS = DVH, kTmemQ = kTmemS + kSBufs * N;
 static_assert(kTmemQ + 4 * 32 == 512, "TMEM budget");
-// kv_full[kStages] kv_empty[kStages] s_full[2] s_read[2] s_sent[2] x_full[2] x_free[2]
-// x_read[2] p_full[2] p_free o_done q_full q_tma
-constexpr int kNumBars = 2 * kStages + 3 * kSBufs + 2 + 2 + 2 + kSBufs + 4;
+// kv_full[kStages] kv_empty[kStages] s_full[2] s_read[2] s_sent[2] x_full[kXBufs]
+// x_free[kXBufs] x_read[kXBufs] p_full[2] p_free o_done q_full q_tma merge_full
+constexpr int kNumBars = 2 * kStages + 3 * kSBufs + 3 * kXBufs + kSBufs + 5;
+// Split merge inside the cluster (after the tiles, in the free stage ring): the CTA owning
+// heads [split * hp, + hp) of its V half receives, from every split s, those heads' rows of
+// O (bf16, unnormalised, 512 bytes each) at [s][head][512 B] and their (max, sum) at
+// [s][head][16 B]; hp = 128 / nsplit, so both areas are the same size for every split count.
+constexpr int kOffMerge = kOffKv;
+constexpr int kOffMergeMl = kOffMerge + H * 512;
+static_assert(kOffMergeMl + H * 16 <= kStages * kStageBytes, "merge buffers fit the stage ring");
 // Q arrives by TMA (one 128-head x 64-dim box per panel, 128-byte swizzle): panels 4r .. 4r+3
 // in the KV stage buffers, which the row gathers use only once Q has moved on into TMEM, and
 // panel 8 straight into its own buffer
@@ -253,6 +268,7 @@ static_assert(kGathers % kLoadWarps == 0 && kGathersPerWarp <= 32, "gathers per 
 static_assert(kSmem <= 227 * 1024, "shared memory budget");
 constexpr uint32_t kIdescS = make_idesc(1 /*bf16*/, 128, N, false, false);
 constexpr uint32_t kIdescO = make_idesc(1 /*bf16*/, 128, DVH, false, true);
+constexpr int kMergeBatch = 8;  // the most splits the in-cluster merge takes (the cluster's 16 CTAs)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 // Global panel of local panel lp of rank r.
@@ -305,19 +321,22 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   uint64_t* s_read = s_full + kSBufs;      // ... read by the senders and the softmax
   uint64_t* s_sent = s_read + kSBufs;      // ... read by the senders (P may overwrite it)
   uint64_t* x_full = s_sent + kSBufs;      // the other rank's partial has arrived here
-  uint64_t* x_free = x_full + 2;           // the other rank has read our partial (credit)
-  uint64_t* x_read = x_free + 2;           // our softmax has read receive buffer b
-  uint64_t* p_full = x_read + 2;           // P of the tile in buffer i % 2 is in TMEM
+  uint64_t* x_free = x_full + kXBufs;      // the other rank has read our partial (credit)
+  uint64_t* x_read = x_free + kXBufs;      // our softmax has read receive buffer b
+  uint64_t* p_full = x_read + kXBufs;      // P of the tile in buffer i % 2 is in TMEM
   uint64_t* p_free = p_full + kSBufs;      // PV of the latest tile has finished
   uint64_t* o_done = p_free + 1;
   uint64_t* q_full = p_free + 2;
   uint64_t* q_tma = p_free + 3;
+  uint64_t* merge_full = p_free + 4;       // every split's rows for this CTA's heads have landed
   uint32_t* tmem_slot = (uint32_t*)(sm + kOffTmem);
   __shared__ int s_abort;
   __shared__ uint64_t s_mask[kStages];  // valid rows of the tile in each stage
 
   const int b = blockIdx.y;
-  const int rank = (int)cluster_rank();  // == blockIdx.x & 1
+  const uint32_t crank = cluster_rank();  // == blockIdx.x (the cluster spans the splits)
+  const int rank = (int)(crank & 1u);      // which half of V
+  const uint32_t peer_crank = crank ^ 1u;  // the other CTA of the pair
   const int split = blockIdx.x >> 1;
   const int warp = warp_id(), lane = lane_id();
   const int T_all = (p.k + N - 1) / N;
@@ -340,7 +359,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
       mbar_init(&s_sent[s], 128);  // this CTA's sender threads
       mbar_init(&p_full[s], 128);  // this CTA's softmax threads
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kXBufs; ++s) {
       mbar_init(&x_full[s], 1);  // armed with the partial's bytes; the other CTA's stores land on it
       mbar_init(&x_free[s], 1);    // the other CTA's forwarding thread, remotely
       mbar_init(&x_read[s], 128);  // this CTA's softmax threads
@@ -349,6 +368,9 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     mbar_init(o_done, 1);
     mbar_init(q_full, 128);  // the softmax threads, once Q is in TMEM (and out of the stages)
     mbar_init(q_tma, 1);
+    mbar_init(merge_full, 1);
+    // armed now; the rows arrive only after the cluster-wide barrier that follows the tiles
+    if (p.merge) mbar_arrive_expect_tx(merge_full, (uint32_t)(H * (512 + 16)));
     s_abort = 0;
     fence_mbar_init();
     // Q is an input of the step, never written by the kernel before: fetch it at once
@@ -358,9 +380,9 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
         tma_load_2d(sbase + kOffKv + c * kQPanelBytes, &q_map, q_tma, global_panel(rank, c) * 64, b * H);
       tma_load_2d(sbase + kOffQ8, &q_map, q_tma, 8 * 64, b * H);
     }
-    // arm the receive buffers for tiles 0 and 1 before the other CTA can send (an armed
+    // arm the receive buffers for the first tiles before the other CTA can send (an armed
     // buffer that no tile uses is never waited on)
-    for (int s = 0; s < 2 && s < my_tiles_max; ++s) mbar_arrive_expect_tx(&x_full[s], kXBytes);
+    for (int s = 0; s < kXBufs && s < my_tiles_max; ++s) mbar_arrive_expect_tx(&x_full[s], kXBytes);
   }
   if (warp == kMmaWarp) tmem_alloc(tmem_slot, 512);
   tc_fence_before();
@@ -418,6 +440,10 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     my_tiles = 0;
   }
   const size_t pslot = (size_t)b * p.nsplit_total + p.split_base + split;  // partial slot
+  // the softmax threads' final running max and sum, and whether O in TMEM is complete
+  // (for the split merge after the cluster-wide barrier)
+  float m_out = -INFINITY, l_out = 0.f;
+  bool o_ready = false;
 
   if (warp >= kLoadWarp0) {
     // ================= row gathers: tile i goes to stage i % kStages =================
@@ -481,15 +507,15 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   } else if (warp == kFwdWarp) {
     // ================= credit forwarding =================
     // Once this CTA's softmax has read receive buffer b (tile j), re-arm its barrier for
-    // tile j + 2 and tell the other CTA's senders they may write it.  The remote arrival
-    // (a cluster-scope release) is slow, so it is kept off the softmax warps.
+    // tile j + kXBufs and tell the other CTA's senders they may write it.  The remote
+    // arrival (a cluster-scope release) is slow, so it is kept off the softmax warps.
     cluster_wait();
     cluster_waited = true;
     if (lane == 0) {
-      const uint32_t xfree_peer = dsmem_map(smem_u32(x_free), (uint32_t)(rank ^ 1));
-      for (int j = 0; j + 2 < my_tiles; ++j) {
-        const int xb = j & 1;
-        if (!mbar_wait(&x_read[xb], (j >> 1) & 1)) break;
+      const uint32_t xfree_peer = dsmem_map(smem_u32(x_free), peer_crank);
+      for (int j = 0; j + kXBufs < my_tiles; ++j) {
+        const int xb = j % kXBufs;
+        if (!mbar_wait(&x_read[xb], (j / kXBufs) & 1)) break;
         mbar_arrive_expect_tx(&x_full[xb], kXBytes);
         mbar_arrive_remote(xfree_peer + xb * 8);
       }
@@ -572,13 +598,13 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     // ================= S senders: warps 4..7, thread = head =================
     // This rank's partial S of each tile goes from TMEM to the other CTA as asynchronous
     // stores that count their bytes on the receiver's barrier (armed by the receiver for
-    // each tile).  Receive buffer i % 2 of the other CTA is written only after that CTA's
-    // softmax has read tile i-2 from it and its forwarding thread has re-armed the barrier
-    // (x_free credit), so the senders run ahead of both softmaxes by up to two tiles.
+    // each tile).  The other CTA's receive buffer is written for tile i only after that CTA's
+    // softmax has read tile i - kXBufs from it and its forwarding thread has re-armed the
+    // barrier (x_free credit), so the senders run ahead of both softmaxes by kXBufs tiles.
     const int q = warp & 3;
     const int h = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const uint32_t peer = (uint32_t)(rank ^ 1);
+    const uint32_t peer = peer_crank;
     // partials are stored chunk-major (chunk c of head h at c * 2048 + h * 16), so a
     // warp's 16-byte accesses are consecutive
     const uint32_t x_peer = dsmem_map(sbase + kOffX, peer);
@@ -586,7 +612,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     cluster_wait();
     cluster_waited = true;
     for (int i = 0; i < my_tiles; ++i) {
-      const int sb = i % kSBufs, xb = i & 1;
+      const int sb = i % kSBufs, xb = i % kXBufs;
       // every wait in front of a warp-collective TMEM access is decided for the whole warp
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], (i / kSBufs) & 1))) break;
       tc_fence_after();
@@ -595,7 +621,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
       tc_fence_before();
       mbar_arrive(&s_read[sb]);
       mbar_arrive(&s_sent[sb]);  // the softmax may now write P over this S tile
-      if (i >= 2 && !__all_sync(0xffffffffu, mbar_wait_cluster(&x_free[xb], ((i >> 1) - 1) & 1))) break;
+      if (i >= kXBufs && !__all_sync(0xffffffffu, mbar_wait_cluster(&x_free[xb], ((i / kXBufs) - 1) & 1))) break;
 #pragma unroll
       for (int c = 0; c < N / 4; ++c)
         st_async_v4(x_peer + xb * kXBytes + c * 2048 + h * 16, cur[4 * c], cur[4 * c + 1], cur[4 * c + 2],
@@ -609,7 +635,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int i = 0; i < my_tiles; ++i) {
-      const int st = i % kStages, sb = i % kSBufs, xb = i & 1;
+      const int st = i % kStages, sb = i % kSBufs, xb = i % kXBufs;
       // the loaders published the tile's valid rows with their kv_full arrivals
       if (!__all_sync(0xffffffffu, mbar_wait(&kv_full[st], (i / kStages) & 1))) { ok = false; break; }
       const uint64_t vmask = s_mask[st];
@@ -621,7 +647,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
       tmem_ld64(tm_s + lane_off + sb * N, s);
       tc_fence_before();
       mbar_arrive(&s_read[sb]);  // with the senders' reads, this frees the S buffer
-      if (!__all_sync(0xffffffffu, mbar_wait_cluster(&x_full[xb], (i >> 1) & 1))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait_cluster(&x_full[xb], (i / kXBufs) & 1))) { ok = false; break; }
 #pragma unroll
       for (int c = 0; c < N / 4; ++c) {
         const float4 o = *(const float4*)(sm + kOffX + xb * kXBytes + c * 2048 + h * 16);
@@ -704,7 +730,12 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     // ---- epilogue
     bool fin = ok && my_tiles > 0 && mbar_wait(o_done, 0);
     fin = __all_sync(0xffffffffu, fin);  // the TMEM reads below are warp-collective
-    if (fin) {
+    m_out = m_run;
+    l_out = l_run;
+    o_ready = fin;
+    if (p.merge) {
+      // the splits are merged after the cluster-wide barrier below
+    } else if (fin) {
       tc_fence_after();
       const bool single = p.nsplit_total == 1;
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
@@ -777,12 +808,113 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
         ml[1] = 0.f;
       }
     }
+    if (p.done && !p.merge) {
+      // this CTA's part of the split partial is stored (every path above ends here):
+      // count it for the combine
+      asm volatile("bar.sync 2, 128;" ::: "memory");  // the four softmax warps
+      if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(p.done + b, 1);
+      }
+    }
   }
   // every warp must reach the barrier converged (the MMA warp's lane 0 arrives last).
   // The cluster-wide barrier also keeps this CTA's shared memory alive until the other
-  // CTA has made its last remote write and arrival; only then may TMEM be released.
+  // CTAs have made their last remote writes and arrivals; only then may TMEM be released.
   __syncwarp();
   if (!cluster_waited) cluster_wait();
+  if (p.merge) {
+    // ================= split merge inside the cluster =================
+    // Past this barrier every CTA of the request has finished its tiles: its stage ring is
+    // free and every remote store into it has landed.
+    tc_fence_before();
+    cluster_sync_all();
+    const int hp = H / p.nsplit;
+    if (warp < 4) {
+      // thread = head h: its unnormalised O row over this CTA's V half (bf16, like a split
+      // partial) and its (max, sum) go to the CTA of this rank that owns head h
+      tc_fence_after();
+      const int h = threadIdx.x;
+      const int owner = h / hp, hl = h - owner * hp;
+      const uint32_t dst = (uint32_t)(2 * owner + rank);
+      const uint32_t bar_dst = dsmem_map(smem_u32(merge_full), dst);
+      const uint32_t row_dst = dsmem_map(sbase + kOffMerge + (uint32_t)((split * hp + hl) * 512), dst);
+      const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+      const float any = (o_ready && l_out > 0.f) ? 1.f : 0.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < DVH; c0 += 32) {
+        float v[32];
+        if (o_ready) {
+          tmem_ld32(tm_o + lane_off + c0, v);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) v[c] = 0.f;
+        }
+#pragma unroll
+        for (int c = 0; c < 32; c += 8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            __nv_bfloat162 two = __floats2bfloat162_rn(v[c + 2 * e] * any, v[c + 2 * e + 1] * any);
+            w[e] = *(uint32_t*)&two;
+          }
+          st_async_v4_b32(row_dst + (uint32_t)(c0 + c) * 2, w[0], w[1], w[2], w[3], bar_dst);
+        }
+      }
+      const float m_send = any > 0.f ? m_out : -INFINITY, l_send = any > 0.f ? l_out : 0.f;
+      st_async_v4(dsmem_map(sbase + kOffMergeMl + (uint32_t)((split * hp + hl) * 16), dst), m_send, l_send, 0.f,
+                  0.f, bar_dst);
+    }
+    if (warp < 8) {
+      // heads [split * hp, + hp) x this rank's 256 dims, 8 dims per item: the same weights and
+      // summation order as attn_combine, so both ways give the same bits
+      const bool got = __all_sync(0xffffffffu, mbar_wait(merge_full, 0));
+      const int ns = p.nsplit;
+      for (int item = threadIdx.x; got && item < hp * 32; item += 256) {
+        const int hl = item >> 5, j = item & 31, h = split * hp + hl;
+        float mv[kMergeBatch], lv[kMergeBatch], x[kMergeBatch][8];
+#pragma unroll
+        for (int s2 = 0; s2 < kMergeBatch; ++s2) {
+          const int sc = min(s2, ns - 1);
+          const float4 ml4 = *(const float4*)(sm + kOffMergeMl + (sc * hp + hl) * 16);
+          mv[s2] = ml4.x;
+          lv[s2] = ml4.y;
+          const uint4 u = *(const uint4*)(sm + kOffMerge + (sc * hp + hl) * 512 + j * 16);
+          const uint32_t q4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*(const __nv_bfloat162*)&q4[e]);
+            x[s2][2 * e] = f.x;
+            x[s2][2 * e + 1] = f.y;
+          }
+        }
+        float M = -INFINITY, Lsum = 0.f, acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int s2 = 0; s2 < kMergeBatch; ++s2) M = fmaxf(M, mv[s2]);
+        if (M != -INFINITY) {
+#pragma unroll
+          for (int s2 = 0; s2 < kMergeBatch; ++s2) {
+            const float wgt = (s2 < ns && lv[s2] > 0.f) ? exp2f(mv[s2] - M) : 0.f;
+            Lsum += wgt * lv[s2];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = fmaf(wgt, x[s2][e], acc[e]);
+          }
+        }
+        const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+        uint32_t wo[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          __nv_bfloat162 two = __floats2bfloat162_rn(acc[2 * q] * inv, acc[2 * q + 1] * inv);
+          wo[q] = *(uint32_t*)&two;
+        }
+        *(uint4*)((__nv_bfloat16*)p.o + ((size_t)b * H + h) * DV + rank * DVH + j * 8) =
+            make_uint4(wo[0], wo[1], wo[2], wo[3]);
+        if (rank == 0 && j == 0) p.lse[(size_t)b * H + h] = Lsum > 0.f ? (M + log2f(Lsum)) * kLn2 : -INFINITY;
+      }
+    }
+  }
   tc_fence_before();
   cluster_sync_all();
   if (warp == kMmaWarp) {
@@ -847,14 +979,10 @@ __device__ __forceinline__ void combine_splits(const AttnParams& p, int b, int h
   }
 }
 
-__global__ void __launch_bounds__(kCombineThreads) attn_combine(const AttnParams p) {
+// More splits than one batch holds: the maximum first, then the weighted sum batch by batch.
+__device__ __forceinline__ void combine_general(const AttnParams& p, int b, int h, int d0, const float* ml, float& M,
+                                                float* acc, float& Lsum) {
   using namespace mla;
-  griddep_wait();  // the partials come from the kernel before
-  const int b = blockIdx.y;
-  const int item = blockIdx.x * kCombineThreads + threadIdx.x;
-  const int g = item / H, h = item - g * H, d0 = g * 8;
-  const float* ml = p.part_ml + (size_t)b * p.nsplit_total * H * 2 + (size_t)h * 2;
-  float M = -INFINITY;
   for (int s0 = 0; s0 < p.nsplit_total; s0 += kCombineBatch) {
     float mv[kCombineBatch];
 #pragma unroll
@@ -862,16 +990,76 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine(const AttnParams
 #pragma unroll
     for (int j = 0; j < kCombineBatch; ++j) M = fmaxf(M, mv[j]);
   }
-  float acc[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  float Lsum = 0.f;
   if (M != -INFINITY) {
     if (p.o_f32) {
       combine_splits<true>(p, b, h, d0, ml, M, acc, Lsum);
     } else {
       combine_splits<false>(p, b, h, d0, ml, M, acc, Lsum);
     }
+  }
+}
+
+__global__ void __launch_bounds__(kCombineThreads) attn_combine(const AttnParams p) {
+  using namespace mla;
+  const int b = blockIdx.y;
+  if (p.done) {
+    // the partials of request b are complete once all 2 * nsplit of its attention CTAs have
+    // counted themselves (this kernel runs only after every one of them has started, so the
+    // wait cannot hold a slot one of them needs); one thread polls, the rest wait at the barrier
+    if (threadIdx.x == 0) {
+      const int want = 2 * p.nsplit_total;
+      const uint64_t t0 = globaltimer();
+      while (true) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p.done + b) : "memory");
+        if (v >= want) break;
+        if (globaltimer() - t0 > *(volatile unsigned long long*)&g_wait_limit_ns) {
+          flag(LS_DEV_TIMEOUT);
+          break;
+        }
+        __nanosleep(128);
+      }
+    }
+    __syncthreads();
+  } else {
+    griddep_wait();  // the partials come from the kernel before
+  }
+  const int item = blockIdx.x * kCombineThreads + threadIdx.x;
+  const int g = item / H, h = item - g * H, d0 = g * 8;
+  const float* ml = p.part_ml + (size_t)b * p.nsplit_total * H * 2 + (size_t)h * 2;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  float Lsum = 0.f, M = -INFINITY;
+  if (p.nsplit_total <= kCombineBatch) {
+    // every split in one batch: the maxima, sums and partials of all splits are loaded
+    // together (one round trip), then weighted and summed in split order
+    const int ns = p.nsplit_total;
+    float mv[kCombineBatch], lv[kCombineBatch], x[kCombineBatch][8];
+#pragma unroll
+    for (int j = 0; j < kCombineBatch; ++j) {
+      const int s = min(j, ns - 1);
+      mv[j] = ml[(size_t)s * H * 2];
+      lv[j] = ml[(size_t)s * H * 2 + 1];
+      if (p.o_f32) {
+        load_part8<true>(p, b, s, h, d0, x[j]);
+      } else {
+        load_part8<false>(p, b, s, h, d0, x[j]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kCombineBatch; ++j) M = fmaxf(M, mv[j]);
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int j = 0; j < kCombineBatch; ++j) {
+        const float wgt = (j < ns && lv[j] > 0.f) ? exp2f(mv[j] - M) : 0.f;
+        Lsum += wgt * lv[j];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = fmaf(wgt, x[j][e], acc[e]);
+      }
+    }
+  } else {
+    combine_general(p, b, h, d0, ml, M, acc, Lsum);
   }
   const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
   if (p.o_f32) {

@@ -133,6 +133,15 @@ __device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, float a, floa
                : "memory");
 }
 
+// As st_async_v4, for raw 32-bit words (packed bf16 pairs).
+__device__ __forceinline__ void st_async_v4_b32(uint32_t cluster_addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                                uint32_t cluster_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   cluster_addr),
+               "r"(a), "r"(b), "r"(c), "r"(d), "r"(cluster_bar)
+               : "memory");
+}
+
 // Arrive on an mbarrier of another CTA of the cluster; this thread's earlier writes
 // (remote ones included) are released to whoever waits on it with cluster scope.
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {

@@ -32,6 +32,8 @@ struct TopkParams {
   float* sel;                // [B,k] (may be NULL)
   float* thr;                // [B] optional: k-th largest score, -inf if fewer than k candidates
   int cache_keys;            // keys of dynamic shared memory available per CTA
+  int* clear;                // optional [B]: set to 0 (a per-request count the next kernel of
+                             //   the step adds up; see AttnParams::done)
 };
 
 constexpr int kTopkThreads = 512;
@@ -103,6 +105,7 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster(const TopkParams
   const int k = p.k;
   griddep_wait();  // the scores come from the kernel before
   griddep_launch_dependents();
+  if (p.clear && rank == 0 && tid == 0) p.clear[b] = 0;
 
   long long nll = ((long long)p.lens[b] * p.len_mul + p.len_div - 1) / p.len_div;
   bool bad = nll < 0 || nll > p.len_limit;

@@ -63,6 +63,7 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row(const TopkParams p) {
   const uint32_t lt = (1u << lane) - 1u;
   const int k = p.k;
   griddep_wait();  // the scores come from the kernel before
+  if (p.clear && threadIdx.x == 0) p.clear[blockIdx.x] = 0;
   griddep_launch_dependents();
 
   const long long nll = ((long long)p.lens[b] * p.len_mul + p.len_div - 1) / p.len_div;

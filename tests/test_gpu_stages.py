@@ -194,6 +194,43 @@ def test_mla_attention_split_extremes(lens, k, n_valid):
     assert_status_clean()
 
 
+@pytest.mark.parametrize("Bn,heads_step", [
+    (8, 4),    # 8 KV splits: the splits of a request merge in one 16-CTA cluster
+    (15, 8),   # 4 splits: an 8-CTA cluster
+    (30, 16),  # 2 splits: a 4-CTA cluster
+    (10, 8),   # 7 splits: partials through the workspace and the combine kernel
+])
+def test_mla_attention_batch_sizes_and_split_merges(Bn, heads_step):
+    """Batch sizes whose KV split counts take each way of merging the splits: inside the
+    cluster (2, 4, 8 splits) or through the workspace (7); ragged and empty selections
+    included.  Heads sampled every `heads_step` for the oracle."""
+    L, k = 8192, 2048
+    lens = [L] * Bn
+    table, n_pool = syn.page_layout(lens, seed=31 + Bn)
+    q, kv = syn.mla_attention(Bn, n_pool, seed=32 + Bn)
+    n_valid = [k] * Bn
+    n_valid[1] = 1111
+    n_valid[Bn - 1] = 0  # an empty selection: o = 0, lse = -inf
+    sel = _random_selection(Bn, k, lens, seed=33 + Bn, n_valid=n_valid)
+    scale = 1 / math.sqrt(576)
+    o = torch.full((Bn, 128, 512), float("nan"), dtype=torch.bfloat16, device=DEV)
+    lse = torch.full((Bn, 128), float("nan"), device=DEV)
+    a = B.attn_args(q=q.to(DEV), k_rows=kv.to(DEV), sel=sel.to(DEV), o=o, lse=lse, scale=scale,
+                    page_table=table.to(DEV))
+    ws = torch.empty(max(1, B.ls_sparse_attn_workspace_size(a)), dtype=torch.uint8, device=DEV)
+    B.ls_sparse_attn_decode(a, ws)
+    torch.cuda.synchronize()
+    hs = slice(0, 128, heads_step)
+    qb, kvb = bits16(q), bits16(kv)
+    for b in range(Bn - 1):
+        rows = O.bf16_decode(O.selected_rows(kvb, table.numpy()[b], sel.numpy()[b]))
+        ref_o, ref_l = O.sparse_attn_decode(O.bf16_decode(qb[b][hs]), rows, rows[:, :512], scale)
+        assert np.abs(o[b][hs].float().cpu().numpy() - ref_o).max() <= 2e-2, b
+        assert np.abs(lse[b][hs].cpu().numpy() - ref_l).max() <= 2e-2, b
+    assert (o[Bn - 1].float() == 0).all() and torch.isneginf(lse[Bn - 1]).all()
+    assert_status_clean()
+
+
 def test_mla_attention_slots_and_empty_selection():
     Bn, S, k = 2, 4096, 64
     g = torch.Generator().manual_seed(21)

@@ -21,8 +21,11 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
+BATCH = 10  # seven KV splits per request: their partials go through the split scratch
+
+
 def _inputs(seed):
-    lens = [131072] * 8  # batch 8: the partials need the scratch (several KV splits)
+    lens = [131072] * BATCH
     table, n_pool = syn.page_layout(lens, seed=seed)
     q, kv = syn.mla_attention(len(lens), n_pool, seed=seed + 1, device=DEV)
     g = torch.Generator().manual_seed(seed + 2)
@@ -32,8 +35,8 @@ def _inputs(seed):
 
 
 def _run(table, q, kv, sel, noalloc):
-    o = torch.full((8, 128, 512), float("nan"), dtype=torch.bfloat16, device=DEV)
-    lse = torch.full((8, 128), float("nan"), device=DEV)
+    o = torch.full((BATCH, 128, 512), float("nan"), dtype=torch.bfloat16, device=DEV)
+    lse = torch.full((BATCH, 128), float("nan"), device=DEV)
     a = B.attn_args(q=q, k_rows=kv, sel=sel, o=o, lse=lse, scale=syn.softmax_scale(576), page_table=table)
     need = B.ls_sparse_attn_workspace_size(a)
     assert need > 0, "this configuration should use split-KV scratch"
