@@ -218,8 +218,9 @@ ls_status launch_index_simt(const ls_index_score_args* a, cudaStream_t st) {
 ls_status launch_index_tc(const ls_index_score_args* a, int mode, const int* unit_list, const int* unit_count,
                           int list_stride, float* out, long long out_stride, const uint8_t* summ,
                           const float* bscale, int max_blocks, float* out_plain, float eps_rel, cudaStream_t st,
-                          int staged_base = -1, int stage_cap = 0) {
+                          int staged_base = -1, int stage_cap = 0, int* clear = nullptr) {
   ls::IdxTcParams p{};
+  p.clear = clear;
   p.staged = staged_base >= 0 ? 1 : 0;  // list entries [staged_base, + stage_cap) from staging units
   p.unit_base = staged_base >= 0 ? staged_base : 0;
   p.stage_cap = stage_cap;
@@ -330,9 +331,10 @@ ls_status launch_topk_cl(const ls::TopkParams& p0, int B, cudaStream_t st, std::
 ls_status launch_topk(int B, int k, const float* scores, int stride, const int* lens, int len_mul, int len_div,
                       int len_limit, const int* unit_list, int list_stride, int* idx, float* sel, float* thr,
                       cudaStream_t st, const int* pos_list = nullptr, int pos_stride = 0,
-                      const int* pos_offset = nullptr, int* clear = nullptr) {
+                      const int* pos_offset = nullptr, int* clear = nullptr, int* done = nullptr) {
   ls::TopkParams p{};
   p.clear = clear;
+  p.done = done;
   p.pos_list = pos_list; p.pos_stride = pos_stride; p.pos_offset = pos_offset;
   p.B = B; p.k = k; p.stride = stride; p.scores = scores; p.lens = lens; p.len_mul = len_mul;
   p.len_div = len_div; p.len_limit = len_limit; p.unit_list = unit_list; p.list_stride = list_stride;
@@ -475,7 +477,8 @@ cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, size_t smem, cudaStream_t s
 ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressing, const int* page_table,
                       int max_pages, int n_slots, const void* rows, long long num_rows, void* ws, size_t ws_bytes,
                       cudaStream_t st, bool pdl, bool compacted = false, int pass = 0, int npasses = 1,
-                      bool combine = true, const int* n_valid = nullptr, int* done = nullptr) {
+                      bool combine = true, const int* n_valid = nullptr, int* done = nullptr,
+                      const int* ready = nullptr, int ready_want = 0) {
   ls::AttnParams p{};
   p.B = a->batch; p.H = a->heads; p.dk = a->dk; p.dv = a->dv; p.k = a->k; p.scale = a->softmax_scale;
   p.addressing = addressing; p.max_pages = max_pages; p.n_slots = n_slots; p.row_stride = a->row_stride;
@@ -495,6 +498,8 @@ ls_status launch_attn(const ls_sparse_attn_args* a, const int* sel, int addressi
     // a per-request completion count lets the combine start request by request; only for a
     // single pass whose count the kernel before (the top-k) has just zeroed
     p.done = (total > 1 && !merge && combine && npasses == 1) ? done : nullptr;
+    p.ready = ready;
+    p.ready_want = ready_want;
     if (total > 1 && !merge) {
       const size_t need = attn_ws_bytes(a, npasses);
       LS_REQUIRE(ws && ws_bytes >= need, "attention workspace too small (%zu < %zu bytes)", ws_bytes, need);
@@ -781,7 +786,7 @@ ls_status run_c2f(const ls_block_bound_prune_args* a, void* ws, size_t ws_bytes,
 // ---- decode step workspace ------------------------------------------------------------
 struct StepLayout {
   size_t off_scores, off_idx, off_sel, off_selslot, off_mpos, off_mslot, off_nmiss, off_hitslot, off_cpos, off_crow,
-      off_cnmiss, off_cnhit, off_stage, off_attn, off_done, off_c2f, total;
+      off_cnmiss, off_cnhit, off_stage, off_attn, off_done, off_ready, off_c2f, total;
 };
 
 ls_block_bound_prune_args step_c2f_args(const ls_decode_step_args* a, int* idx, float* sel) {
@@ -881,7 +886,8 @@ StepLayout step_layout(const ls_decode_step_args* a) {
   l.off_cnhit = take(two_pass ? (size_t)B * 4 : 0);
   l.off_stage = take(two_pass ? (size_t)B * k * t.row_stride * 2 : 0);
   l.off_attn = take(attn_ws_bytes(&t, two_pass ? 2 : 1));
-  l.off_done = take((size_t)B * 4);  // per-request attention completion counts
+  l.off_done = take((size_t)B * 4);   // per-request attention completion counts
+  l.off_ready = take((size_t)B * 4);  // per-request top-k completion counts
   if (a->use_c2f) {
     ls_block_bound_prune_args c = step_c2f_args(a, nullptr, nullptr);
     l.off_c2f = take(c2f_layout(&c).total);
@@ -1262,6 +1268,8 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
     if (a->attn_q_ready) cudaStreamWaitEvent(s, (cudaEvent_t)a->attn_q_ready, 0);
   };
   // a1 (+a2) or a3
+  int* ready = nullptr;
+  int ready_want = 0;
   rec(0);
   if (a->use_c2f) {
     ls_block_bound_prune_args c = step_c2f_args(a, idx, sel);
@@ -1269,18 +1277,23 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
     LS_TRY(run_c2f(&c, w + l.off_c2f, l.total - l.off_c2f, a->survivors, a->n_survivors, ev ? ev[1] : nullptr, st));
   } else {
     float* scores = ix->scores ? ix->scores : (float*)(w + l.off_scores);
+    // paged path with the tensor-core indexer: per-request completion counts hand each
+    // request from the top-k to the attention, and from the attention to the combine; each
+    // count is zeroed by the kernel before the one that adds it up
+    ready = (!a->use_hotbuf && ix->key_dtype == LS_E4M3 && ix->variant == 0) ? (int*)(w + l.off_ready) : nullptr;
     if (ix->key_dtype == LS_E4M3 && ix->variant == 0) {
-      LS_TRY(launch_index_tc(ix, 0, nullptr, nullptr, 0, scores, ix->max_len, nullptr, nullptr, 0, nullptr, 0.f, st));
+      LS_TRY(launch_index_tc(ix, 0, nullptr, nullptr, 0, scores, ix->max_len, nullptr, nullptr, 0, nullptr, 0.f, st,
+                             -1, 0, ready));
     } else {
       ls_index_score_args tmp = *ix;
       tmp.scores = scores;
       LS_TRY(launch_index_simt(&tmp, st));
     }
     rec(1);
-    // the top-k also zeroes the attention's per-request completion counts (paged path)
     int* done = !a->use_hotbuf ? (int*)(w + l.off_done) : nullptr;
+    ready_want = ix->max_len <= kTopkRowMaxLen ? 1 : (topk16_supported(st) ? 16 : 8);
     LS_TRY(launch_topk(ix->batch, a->k, scores, ix->max_len, ix->lens, 1, 1, ix->max_len, nullptr, 0, idx, sel,
-                       nullptr, st, nullptr, 0, nullptr, done));
+                       nullptr, st, nullptr, 0, nullptr, done, ready));
   }
   void* attn_ws = w + l.off_attn;
   if (a->use_hotbuf) {
@@ -1360,7 +1373,7 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
     wait_q(st);
     int* done = !a->use_c2f ? (int*)(w + l.off_done) : nullptr;
     LS_TRY(launch_attn(&at, idx, LS_ROWS_PAGED, pt, mp, 0, nullptr, at.num_rows, attn_ws, attn_ws_b, st, true,
-                       true, 0, 1, true, nullptr, done));
+                       true, 0, 1, true, nullptr, done, ready, ready_want));
   }
   rec(5);
   return ok();

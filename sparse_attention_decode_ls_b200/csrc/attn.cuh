@@ -51,6 +51,9 @@ struct AttnParams {
   int o_f32;         // tensor-core kernel: o is float32 (else bf16)
   const int* n_valid;  // optional [B]: and there are n_valid[b] of them; the splits share
                        //   those rows instead of all k entries
+  const int* ready;    // optional [B]: the selection of request b is complete once ready[b]
+  int ready_want;      //   reaches ready_want (the top-k's CTAs per request count themselves);
+                       //   waited for per request instead of the whole kernel before
   int* done;           // optional [B], zero at launch: every CTA adds 1 once its split partial
                        //   is stored, and attn_combine starts on a request as soon as all
                        //   2 * nsplit of its CTAs have, instead of after the whole grid
@@ -252,7 +255,10 @@ static_assert(kOffMergeMl + H * 16 <= kStages * kStageBytes, "merge buffers fit 
 // Q arrives by TMA (one 128-head x 64-dim box per panel, 128-byte swizzle): panels 4r .. 4r+3
 // in the KV stage buffers, which the row gathers use only once Q has moved on into TMEM, and
 // panel 8 straight into its own buffer
-static_assert(4 * kQPanelBytes <= kStages * kStageBytes, "Q staging fits the KV stages");
+// Q is staged in stages 2-3, so that the gathers of tiles 0 and 1 need not wait for it
+constexpr int kOffQStage = 2 * kStageBytes;
+static_assert(kOffQStage % 1024 == 0 && kOffQStage + 4 * kQPanelBytes <= kStages * kStageBytes,
+              "Q staging fits the KV stages");
 constexpr int kOffTmem = kOffBar + kNumBars * 8;
 constexpr int kSmem = 1024 + kOffTmem + 16;
 // warps 0-3 softmax and 4-7 S senders (warp w reads TMEM lanes 32(w%4) .. +31),
@@ -348,6 +354,44 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   const int my_tiles_max = p.n_valid ? (T_all + p.nsplit - 1) / p.nsplit : my_tiles0;
   const uint32_t sbase = smem_u32(sm);
 
+  // With a ready count the gather warps resolve this CTA's rows (selection -> page table ->
+  // shared memory) as soon as this request's selection is complete, before they join the
+  // set-up barrier: a CTA that started late (on an SM the kernel before had held) resolves
+  // its rows while its other warps set up, instead of after them.
+  constexpr int kRStep = kLoadWarps * 32;
+  int* s_rows = (int*)(sm + kOffRows);
+  auto resolve_rows = [&](int tb_, int ntiles, const int* spec_sv, bool spec_ok) {
+    const int lw = warp - kLoadWarp0;
+    const int nrows = ntiles * N;
+    for (int r0 = lw * 32 + lane; r0 < nrows; r0 += 4 * kRStep) {
+      int sv[4];  // four rows' selections, then their page-table lookups, in flight together
+      const bool spec = spec_ok && r0 < kRStep;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int r = r0 + u * kRStep, j = tb_ * N + r;
+        sv[u] = (r < nrows && j < p.k) ? (spec ? spec_sv[u] : p.sel[(size_t)b * p.k + j]) : -1;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int r = r0 + u * kRStep;
+        const long long row = attn_row(p, b, sv[u]);
+        if (r < nrows) s_rows[r] = row >= 0 ? (int)row : (int)p.num_rows;
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kLoadWarps * 32) : "memory");  // the gather warps only
+  };
+  const bool early_rows = p.ready != nullptr;  // (then the share is the split's: t0 .. t1)
+  if (early_rows && warp >= kLoadWarp0) {
+    if (p.addressing == LS_ROWS_PAGED) {
+      const int* pt = p.page_table + (size_t)b * p.max_pages;
+      for (int i = ((warp - kLoadWarp0) * 32 + lane) * 32; i < p.max_pages; i += kLoadWarps * 32 * 32)
+        prefetch_l2(pt + i);
+    }
+    if (lane == 0) wait_count(p.ready + b, p.ready_want);
+    __syncwarp();
+    resolve_rows(t0, my_tiles0, nullptr, false);
+  }
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&kv_full[s], kLoadWarps);  // each gather warp arrives with its bytes
@@ -377,7 +421,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     if (my_tiles_max > 0) {
       mbar_arrive_expect_tx(q_tma, 5 * kQPanelBytes);
       for (int c = 0; c < 4; ++c)
-        tma_load_2d(sbase + kOffKv + c * kQPanelBytes, &q_map, q_tma, global_panel(rank, c) * 64, b * H);
+        tma_load_2d(sbase + kOffQStage + c * kQPanelBytes, &q_map, q_tma, global_panel(rank, c) * 64, b * H);
       tma_load_2d(sbase + kOffQ8, &q_map, q_tma, 8 * 64, b * H);
     }
     // arm the receive buffers for the first tiles before the other CTA can send (an armed
@@ -400,28 +444,30 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
   if (warp < 4 && my_tiles_max > 0) {
     // a wait that gives up (recorded in the device status) aborts the whole CTA
     if (mbar_wait(q_tma, 0)) {
-      load_q_tmem(sm + kOffKv, threadIdx.x, tm_q + ((uint32_t)(warp * 32) << 16));
+      load_q_tmem(sm + kOffQStage, threadIdx.x, tm_q + ((uint32_t)(warp * 32) << 16));
       tc_fence_before();
     } else if (threadIdx.x == 0) {
       s_abort = 1;
     }
     mbar_arrive(q_full);
   }
-  if (warp >= kLoadWarp0 && p.addressing == LS_ROWS_PAGED) {
+  if (warp >= kLoadWarp0 && p.addressing == LS_ROWS_PAGED && !early_rows) {
     // the page table is an input of the step: warm its rows for this request in L2
     const int* pt = p.page_table + (size_t)b * p.max_pages;
     for (int i = ((warp - kLoadWarp0) * 32 + lane) * 32; i < p.max_pages; i += kLoadWarps * 32 * 32)
       prefetch_l2(pt + i);
   }
   // under programmatic dependent launch everything above overlaps the kernel before;
-  // the selection, the rows and the outputs are touched only after it has finished
-  griddep_wait();
+  // the selection, the rows and the outputs are touched only after it has finished.  With a
+  // ready count only the gather warps read what the kernel before wrote (the selection), so
+  // only they wait, for this request's part of it: the other warps go on (a CTA that started
+  // late finishes its prologue meanwhile) and size their work from the split alone
+  if (!p.ready) griddep_wait();
   griddep_launch_dependents();
   // the gather warps load the selections of their first rows (for the usual tile range)
   // while the tile range is settled below, so that the two loads overlap
-  constexpr int kRStep = kLoadWarps * 32;
   int spec_sv[4];
-  if (warp >= kLoadWarp0) {
+  if (warp >= kLoadWarp0 && !early_rows) {
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int r = (warp - kLoadWarp0) * 32 + lane + u * kRStep, j = t0 * N + r;
@@ -436,8 +482,8 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     const int tv = (nv + N - 1) / N;
     tb = (int)(((long long)tv * split) / p.nsplit);
     my_tiles = min((int)(((long long)tv * (split + 1)) / p.nsplit) - tb, my_tiles_max);
-  } else if (p.compacted && my_tiles0 > 0 && p.sel[(size_t)b * p.k + (size_t)t0 * N] < 0) {
-    my_tiles = 0;
+  } else if (p.compacted && !p.ready && my_tiles0 > 0 && p.sel[(size_t)b * p.k + (size_t)t0 * N] < 0) {
+    my_tiles = 0;  // (with a ready count a share of padding is gathered as zero rows and masked)
   }
   const size_t pslot = (size_t)b * p.nsplit_total + p.split_base + split;  // partial slot
   // the softmax threads' final running max and sum, and whether O in TMEM is complete
@@ -455,31 +501,15 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
     const int lw = warp - kLoadWarp0;
     const int e = lw * kGathersPerWarp + lane;  // this lane's gather (if lane < 20)
     const int lx = e % (N / 4), lp = e / (N / 4);
-    // resolve all of this CTA's rows once (out-of-range marker: one past the pool)
-    int* s_rows = (int*)(sm + kOffRows);
-    const int nrows = my_tiles * N;
-    for (int r0 = lw * 32 + lane; r0 < nrows; r0 += 4 * kRStep) {
-      int sv[4];  // four rows' selections, then their page-table lookups, in flight together
-      const bool spec = r0 < kRStep && tb == t0 && my_tiles <= my_tiles0;
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int r = r0 + u * kRStep, j = tb * N + r;
-        sv[u] = (r < nrows && j < p.k) ? (spec ? spec_sv[u] : p.sel[(size_t)b * p.k + j]) : -1;
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int r = r0 + u * kRStep;
-        const long long row = attn_row(p, b, sv[u]);
-        if (r < nrows) s_rows[r] = row >= 0 ? (int)row : (int)p.num_rows;
-      }
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(kLoadWarps * 32) : "memory");  // the gather warps only
+    // resolve all of this CTA's rows once (out-of-range marker: one past the pool), unless
+    // that was done ahead of the set-up
+    if (!early_rows) resolve_rows(tb, my_tiles, spec_sv, tb == t0 && my_tiles <= my_tiles0);
     for (int i = 0; i < my_tiles; ++i) {
       const int st = i % kStages;
       int go = 1;
       if (lane == 0) {  // one lane decides, so the warp stays converged
-        // the first tiles land where Q was staged: only once Q is in TMEM
-        go = i >= kStages ? mbar_wait(&kv_empty[st], ((i / kStages) - 1) & 1) : (i > 0 || mbar_wait(q_full, 0));
+        // the first tiles of stages 2 and 3 land where Q was staged: only once Q is in TMEM
+        go = i >= kStages ? mbar_wait(&kv_empty[st], ((i / kStages) - 1) & 1) : (i < 2 || mbar_wait(q_full, 0));
         if (*(volatile int*)&s_abort) go = 0;
         if (!go) s_abort = 1;
       }
@@ -739,49 +769,55 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
       tc_fence_after();
       const bool single = p.nsplit_total == 1;
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      for (int c0 = 0; c0 < DVH; c0 += 32) {
-        float v[32];
-        tmem_ld32(tm_o + lane_off + c0, v);
-        if (single && p.o_f32) {
-          float4* o = (float4*)((float*)p.o + ((size_t)b * H + h) * DV + rank * DVH + c0);
+      // 64 columns per TMEM load (half the round trips), stored 32 at a time
+      for (int c64 = 0; c64 < DVH; c64 += 64) {
+        float v64[64];
+        tmem_ld64(tm_o + lane_off + c64, v64);
 #pragma unroll
-          for (int c = 0; c < 32; c += 4)
-            o[c / 4] = make_float4(v[c] * inv, v[c + 1] * inv, v[c + 2] * inv, v[c + 3] * inv);
-        } else if (single) {
-          __nv_bfloat16* o = (__nv_bfloat16*)p.o + ((size_t)b * H + h) * DV + rank * DVH + c0;
+        for (int hh = 0; hh < 2; ++hh) {
+          const int c0 = c64 + 32 * hh;
+          const float* v = v64 + 32 * hh;
+          if (single && p.o_f32) {
+            float4* o = (float4*)((float*)p.o + ((size_t)b * H + h) * DV + rank * DVH + c0);
 #pragma unroll
-          for (int c = 0; c < 32; c += 8) {
-            uint32_t w[4];
+            for (int c = 0; c < 32; c += 4)
+              o[c / 4] = make_float4(v[c] * inv, v[c + 1] * inv, v[c + 2] * inv, v[c + 3] * inv);
+          } else if (single) {
+            __nv_bfloat16* o = (__nv_bfloat16*)p.o + ((size_t)b * H + h) * DV + rank * DVH + c0;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 two = __floats2bfloat162_rn(v[c + 2 * e] * inv, v[c + 2 * e + 1] * inv);
-              w[e] = *(uint32_t*)&two;
+            for (int c = 0; c < 32; c += 8) {
+              uint32_t w[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                __nv_bfloat162 two = __floats2bfloat162_rn(v[c + 2 * e] * inv, v[c + 2 * e + 1] * inv);
+                w[e] = *(uint32_t*)&two;
+              }
+              *(uint4*)(o + c) = make_uint4(w[0], w[1], w[2], w[3]);
             }
-            *(uint4*)(o + c) = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        } else if (p.o_f32) {
-          // float32 partials, layout [b][split][dim / 4][head][4]: a warp's store is 512
-          // contiguous bytes
-          float4* o = (float4*)p.part_o + (pslot * (DV / 4) + (rank * DVH + c0) / 4) * H + h;
-          const bool any = l_run > 0.f;
+          } else if (p.o_f32) {
+            // float32 partials, layout [b][split][dim / 4][head][4]: a warp's store is 512
+            // contiguous bytes
+            float4* o = (float4*)p.part_o + (pslot * (DV / 4) + (rank * DVH + c0) / 4) * H + h;
+            const bool any = l_run > 0.f;
 #pragma unroll
-          for (int c = 0; c < 32; c += 4)
-            o[(size_t)(c / 4) * H] = any ? make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
-        } else {
-          // for a bf16 output the partials are bf16 too (one more rounding of what is rounded
-          // to bf16 at the end), layout [b][split][dim / 8][head][8]: a warp's store is 512
-          // contiguous bytes
-          uint4* o = (uint4*)p.part_o + (pslot * (DV / 8) + (rank * DVH + c0) / 8) * H + h;
-          const float any = l_run > 0.f ? 1.f : 0.f;
+            for (int c = 0; c < 32; c += 4)
+              o[(size_t)(c / 4) * H] = any ? make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]) : make_float4(0.f, 0.f, 0.f, 0.f);
+          } else {
+            // for a bf16 output the partials are bf16 too (one more rounding of what is rounded
+            // to bf16 at the end), layout [b][split][dim / 8][head][8]: a warp's store is 512
+            // contiguous bytes
+            uint4* o = (uint4*)p.part_o + (pslot * (DV / 8) + (rank * DVH + c0) / 8) * H + h;
+            const float any = l_run > 0.f ? 1.f : 0.f;
 #pragma unroll
-          for (int c = 0; c < 32; c += 8) {
-            uint32_t w[4];
+            for (int c = 0; c < 32; c += 8) {
+              uint32_t w[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 two = __floats2bfloat162_rn(v[c + 2 * e] * any, v[c + 2 * e + 1] * any);
-              w[e] = *(uint32_t*)&two;
+              for (int e = 0; e < 4; ++e) {
+                __nv_bfloat162 two = __floats2bfloat162_rn(v[c + 2 * e] * any, v[c + 2 * e + 1] * any);
+                w[e] = *(uint32_t*)&two;
+              }
+              o[(size_t)(c / 8) * H] = make_uint4(w[0], w[1], w[2], w[3]);
             }
-            o[(size_t)(c / 8) * H] = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
@@ -812,10 +848,7 @@ __global__ void __launch_bounds__(mla::kThreads, 1)
       // this CTA's part of the split partial is stored (every path above ends here):
       // count it for the combine
       asm volatile("bar.sync 2, 128;" ::: "memory");  // the four softmax warps
-      if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(p.done + b, 1);
-      }
+      count_done(p.done + b);
     }
   }
   // every warp must reach the barrier converged (the MMA warp's lane 0 arrives last).
@@ -1006,20 +1039,7 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine(const AttnParams
     // the partials of request b are complete once all 2 * nsplit of its attention CTAs have
     // counted themselves (this kernel runs only after every one of them has started, so the
     // wait cannot hold a slot one of them needs); one thread polls, the rest wait at the barrier
-    if (threadIdx.x == 0) {
-      const int want = 2 * p.nsplit_total;
-      const uint64_t t0 = globaltimer();
-      while (true) {
-        int v;
-        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p.done + b) : "memory");
-        if (v >= want) break;
-        if (globaltimer() - t0 > *(volatile unsigned long long*)&g_wait_limit_ns) {
-          flag(LS_DEV_TIMEOUT);
-          break;
-        }
-        __nanosleep(128);
-      }
-    }
+    if (threadIdx.x == 0) wait_count(p.done + b, 2 * p.nsplit_total);
     __syncthreads();
   } else {
     griddep_wait();  // the partials come from the kernel before

@@ -191,6 +191,36 @@ __device__ __forceinline__ void prefetch_l2(const void* ptr) {
 }
 
 // ---------------------------------------------------------------------------------
+// Per-request completion counts between the kernels of a decode step.  A producer CTA,
+// once every one of its threads has passed a CTA barrier after its last store, publishes
+// those stores at GPU scope and adds itself to its request's count; a consumer CTA that was
+// launched behind the producer (so that every producer CTA is already resident and the wait
+// cannot hold a slot one of them needs) has one thread wait for the full count, then a CTA
+// barrier.  The count is zeroed by a kernel that runs before the producer.
+// ---------------------------------------------------------------------------------
+__device__ __forceinline__ void count_done(int* counter) {
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(counter, 1);
+  }
+}
+// One thread: wait until *counter >= want (acquire at GPU scope); gives up after
+// g_wait_limit_ns, raising LS_DEV_TIMEOUT.
+__device__ __noinline__ void wait_count(const int* counter, int want) {
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+    if (v >= want) return;
+    if (globaltimer() - t0 > *(volatile unsigned long long*)&g_wait_limit_ns) {
+      flag(LS_DEV_TIMEOUT);
+      return;
+    }
+    __nanosleep(64);
+  }
+}
+
+// ---------------------------------------------------------------------------------
 // Programmatic dependent launch.  A kernel launched with programmatic stream
 // serialization may start while the kernel before it is still running; it must call
 // griddep_wait() (every thread that touches that kernel's output, or that writes memory

@@ -115,6 +115,8 @@ struct IdxTcParams {
   int staged;              // mode 0 list: entries [unit_base, unit_base + stage_cap) of the list,
   int unit_base;           //   whose keys were copied to staging units b * stage_cap + (entry -
   int stage_cap;           //   unit_base) of the pool (key_pool / row_scale point at the staging)
+  int* clear;              // optional [B]: set to 0 (the top-k's per-request count, which the
+                           //   top-k adds up after this kernel has finished)
 };
 
 template <int KP, int NCOL>
@@ -175,6 +177,7 @@ __global__ void __launch_bounds__(192, 1)
 
   const int b = blockIdx.y, cta = blockIdx.x, tid = threadIdx.x, warp = warp_id(), lane = lane_id();
   griddep_launch_dependents();  // the next kernel may be scheduled now; it waits for this one
+  if (p.clear && cta == 0 && tid == 0) p.clear[b] = 0;
   const int L = p.lens[b];
   const bool len_ok = L >= 0 && L <= p.max_len && L <= p.max_pages * 64;
   if (!len_ok) {

@@ -34,6 +34,8 @@ struct TopkParams {
   int cache_keys;            // keys of dynamic shared memory available per CTA
   int* clear;                // optional [B]: set to 0 (a per-request count the next kernel of
                              //   the step adds up; see AttnParams::done)
+  int* done;                 // optional [B], zero at launch: every CTA adds 1 once its outputs
+                             //   are stored (see AttnParams::ready)
 };
 
 constexpr int kTopkThreads = 512;
@@ -156,6 +158,10 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster(const TopkParams
         if (p.sel) p.sel[(size_t)b * k + i] = 0.f;
       }
       if (p.thr && tid == 0) p.thr[b] = -INFINITY;
+    }
+    if (p.done) {
+      __syncthreads();
+      count_done(p.done + b);
     }
     return;  // no distributed shared memory was touched
   }
@@ -525,6 +531,10 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster(const TopkParams
     }
   }
   if (p.thr && rank == 0 && tid == 0) p.thr[b] = key_float(T);
+  if (p.done) {
+    __syncthreads();
+    count_done(p.done + b);
+  }
   cluster.sync();  // keep this CTA's shared memory alive until the cluster is done with it
 }
 

@@ -78,6 +78,10 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row(const TopkParams p) {
       if (p.sel) p.sel[(size_t)b * k + i] = i < n ? row[i] : 0.f;
     }
     if (p.thr && tid == 0) p.thr[b] = -INFINITY;
+    if (p.done) {
+      __syncthreads();
+      count_done(p.done + b);
+    }
     return;
   }
   const int seg = ((n + kRowWarps * 4 - 1) / (kRowWarps * 4)) * 4;  // keys per warp, multiple of 4
@@ -265,6 +269,10 @@ __global__ void __launch_bounds__(kRowThreads, 1) topk_row(const TopkParams p) {
     }
   }
   if (p.thr && tid == 0) p.thr[b] = key_float(T);
+  if (p.done) {
+    __syncthreads();
+    count_done(p.done + b);
+  }
 }
 
 }  // namespace ls
