@@ -312,10 +312,13 @@ typedef struct ls_sparse_attn_args {
   const void* v_rows;
   const int32_t* page_table;  /* PAGED: [B,max_pages] */
   const int32_t* sel;         /* [B,k] positions (PAGED) or slots (SLOTS); -1 skipped */
-  void* o;                    /* [B,heads,dv] out: bf16 for bf16 inputs, float32 for f32 */
-  float* lse;                 /* [B,heads] out */
-  int32_t o_f32;              /* bf16 tensor-core kernel: != 0 writes o as float32 (16-byte
-                                 aligned), e.g. as a partial for ls_attn_merge */
+  void* o;                    /* [B,heads,dv] out: bf16 for bf16 inputs, float32 for f32;
+                                 16-byte aligned for the tensor-core kernel.  Device memory,
+                                 or pinned host memory the GPU can address (the last kernel
+                                 then writes it over the host link) */
+  float* lse;                 /* [B,heads] out; device or pinned host memory like o */
+  int32_t o_f32;              /* bf16 tensor-core kernel: != 0 writes o as float32, e.g. as a
+                                 partial for ls_attn_merge */
 } ls_sparse_attn_args;
 
 size_t ls_sparse_attn_workspace_size(const ls_sparse_attn_args* args);

@@ -434,7 +434,7 @@ ls_status validate_attn(const ls_sparse_attn_args* a, bool need_sel) {
     if (a->variant == 0 && (a->heads != 128 || a->dk != 576 || a->dv != 512))
       return fail(LS_ERR_UNSUPPORTED, "bf16 tensor-core attention is built for 128 heads, dk 576, dv 512");
     if (a->variant == 0) {
-      LS_REQUIRE(!a->o_f32 || aligned16(a->o), "a float32 o must be 16-byte aligned");
+      LS_REQUIRE(aligned16(a->o), "o must be 16-byte aligned");
       LS_REQUIRE(a->k_rows == a->v_rows, "MLA attention reads V from the latent rows (v_rows == k_rows)");
       LS_REQUIRE(a->row_stride >= 576 && (a->row_stride % 8) == 0, "row_stride must be >= 576 and % 8 == 0");
       LS_REQUIRE(a->num_rows < 0x7fffffffLL, "num_rows must be below 2^31 - 1");

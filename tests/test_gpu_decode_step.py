@@ -180,3 +180,26 @@ def test_decode_step_coarse_to_fine():
     assert torch.equal(host.idx, full.idx)
     assert torch.equal(host.o, full.o)
     assert torch.equal(host.tensors["n_survivors"], wl.tensors["n_survivors"])
+
+
+@pytest.mark.parametrize("lens", [[20000, 9000], [16384] * 8])
+def test_decode_step_writes_outputs_to_host_memory(lens):
+    """o and lse are plain addresses: with pinned host buffers the step's last kernel writes
+    them over the host link, and the bits equal those of the step with device outputs (two
+    requests: 16 KV splits; eight: the per-request completion counts)."""
+    inp = syn.indexer_fp8(lens, seed=701)
+    q, kv = syn.mla_attention(len(lens), inp.key_pool.shape[0], seed=702)
+    wl = W.build("host_out", inp, k=2048, attn=dict(q=q, kv=kv, scale=syn.softmax_scale(576)))
+    wl.step()
+    torch.cuda.synchronize()
+    ref_o, ref_lse = wl.o.cpu(), wl.lse.cpu()
+    host_o = torch.full(ref_o.shape, float("nan"), dtype=ref_o.dtype).pin_memory()
+    host_lse = torch.full(ref_lse.shape, float("nan")).pin_memory()
+    dev_o, dev_lse = wl.args.attn.o, wl.args.attn.lse
+    wl.args.attn.o, wl.args.attn.lse = host_o.data_ptr(), host_lse.data_ptr()
+    for _ in range(2):  # twice: the per-request counts start from zero again every step
+        wl.step()
+        torch.cuda.synchronize()
+        assert torch.equal(host_o, ref_o) and torch.equal(host_lse, ref_lse)
+    wl.args.attn.o, wl.args.attn.lse = dev_o, dev_lse
+    assert_status_clean()
