@@ -215,12 +215,32 @@ ls_status launch_index_simt(const ls_index_score_args* a, cudaStream_t st) {
 }
 
 // tcgen05 tile engine over keys (mode 0) or block summaries (mode 1).
+cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, size_t smem, cudaStream_t st, cudaLaunchAttribute* attr,
+                              bool pdl);
+
+// CTAs per request of the tensor-core indexer: two (key scoring) or one (block bound) per SM
+// over the batch, at most one per tile of two 64-row units.
+int idx_ctas_per_req(int mode, int batch, long long max_units, int sms) {
+  const long long max_tiles = (max_units + 1) / 2;
+  const int per_sm = (mode == 0) ? 2 : 1;
+  long long c = std::max<long long>(1, (long long)per_sm * sms / std::max(1, batch));
+  return (int)std::min<long long>(c, std::max<long long>(1, max_tiles));
+}
+
 ls_status launch_index_tc(const ls_index_score_args* a, int mode, const int* unit_list, const int* unit_count,
                           int list_stride, float* out, long long out_stride, const uint8_t* summ,
                           const float* bscale, int max_blocks, float* out_plain, float eps_rel, cudaStream_t st,
-                          int staged_base = -1, int stage_cap = 0, int* clear = nullptr) {
+                          int staged_base = -1, int stage_cap = 0, int* clear = nullptr,
+                          const ls::IdxTcParams* filt = nullptr) {
   ls::IdxTcParams p{};
   p.clear = clear;
+  if (filt) {  // the candidate filter's buffers
+    p.filt = filt->filt;
+    p.cand_cnt = filt->cand_cnt;
+    p.cand_pos = filt->cand_pos;
+    p.cand_score = filt->cand_score;
+    p.filt_k = filt->filt_k;
+  }
   p.staged = staged_base >= 0 ? 1 : 0;  // list entries [staged_base, + stage_cap) from staging units
   p.unit_base = staged_base >= 0 ? staged_base : 0;
   p.stage_cap = stage_cap;
@@ -242,11 +262,8 @@ ls_status launch_index_tc(const ls_index_score_args* a, int mode, const int* uni
     LS_TRY(make_tmap_u8(&tmap, summ, 256, (uint64_t)a->batch * max_blocks, 256));
     max_units = (max_blocks + 63) / 64;
   }
-  const long long max_tiles = (max_units + 1) / 2;
-  const int per_sm = (mode == 0) ? 2 : 1;
-  long long c = std::max<long long>(1, (long long)per_sm * sms / a->batch);
-  c = std::min<long long>(c, std::max<long long>(1, max_tiles));
-  p.ctas_per_req = (int)c;
+  const int c = idx_ctas_per_req(mode, a->batch, max_units, sms);
+  p.ctas_per_req = c;
   dim3 grid((unsigned)c, a->batch);
   if (mode == 0) {
     using C = ls::IdxTc<1, 64>;
@@ -322,7 +339,8 @@ ls_status launch_topk_cl(const ls::TopkParams& p0, int B, cudaStream_t st, std::
   if (allow_smem(ls::topk_cluster<CL>, ls::kTopkCacheKeys * 4 + ls::kTopkExtraBytes, smem_done) != cudaSuccess)
     return check_launch("topk attribute");
   cudaLaunchAttribute attr[2];
-  cudaLaunchConfig_t cfg = topk_config<CL>(B, p.cache_keys * 4 + ls::kTopkExtraBytes, st, attr);
+  p.smem_bytes = p.cache_keys * 4 + ls::kTopkExtraBytes;
+  cudaLaunchConfig_t cfg = topk_config<CL>(B, p.smem_bytes, st, attr);
   cudaError_t e = cudaLaunchKernelEx(&cfg, ls::topk_cluster<CL>, p);
   if (e != cudaSuccess) return fail(LS_ERR_CUDA, "topk_cluster: %s", cudaGetErrorString(e));
   return check_launch("topk_cluster");
@@ -331,10 +349,18 @@ ls_status launch_topk_cl(const ls::TopkParams& p0, int B, cudaStream_t st, std::
 ls_status launch_topk(int B, int k, const float* scores, int stride, const int* lens, int len_mul, int len_div,
                       int len_limit, const int* unit_list, int list_stride, int* idx, float* sel, float* thr,
                       cudaStream_t st, const int* pos_list = nullptr, int pos_stride = 0,
-                      const int* pos_offset = nullptr, int* clear = nullptr, int* done = nullptr) {
+                      const int* pos_offset = nullptr, int* clear = nullptr, int* done = nullptr,
+                      const ls::IdxTcParams* filt = nullptr, int filt_lists = 0) {
   ls::TopkParams p{};
   p.clear = clear;
   p.done = done;
+  if (filt) {  // the indexer's candidate lists
+    p.filt = filt->filt;
+    p.cand_cnt = filt->cand_cnt;
+    p.cand_pos = filt->cand_pos;
+    p.cand_score = filt->cand_score;
+    p.cand_lists = filt_lists;
+  }
   p.pos_list = pos_list; p.pos_stride = pos_stride; p.pos_offset = pos_offset;
   p.B = B; p.k = k; p.stride = stride; p.scores = scores; p.lens = lens; p.len_mul = len_mul;
   p.len_div = len_div; p.len_limit = len_limit; p.unit_list = unit_list; p.list_stride = list_stride;
@@ -786,7 +812,8 @@ ls_status run_c2f(const ls_block_bound_prune_args* a, void* ws, size_t ws_bytes,
 // ---- decode step workspace ------------------------------------------------------------
 struct StepLayout {
   size_t off_scores, off_idx, off_sel, off_selslot, off_mpos, off_mslot, off_nmiss, off_hitslot, off_cpos, off_crow,
-      off_cnmiss, off_cnhit, off_stage, off_attn, off_done, off_ready, off_c2f, total;
+      off_cnmiss, off_cnhit, off_stage, off_attn, off_done, off_ready, off_filt, off_candcnt, off_candpos,
+      off_candscore, off_c2f, total;
 };
 
 ls_block_bound_prune_args step_c2f_args(const ls_decode_step_args* a, int* idx, float* sel) {
@@ -865,6 +892,28 @@ ls_sparse_attn_args step_attn_args(const ls_decode_step_args* a) {
   return t;
 }
 
+// The indexer's CTAs per request in the decode step (the layout of the candidate lists).
+int step_idx_ctas(const ls_decode_step_args* a);
+
+// Whether the step's indexer keeps candidate lists for the cluster top-k: the tensor-core
+// indexer over whole requests (not the coarse-to-fine pass), requests long enough for the
+// cluster top-k and short enough for its key cache (the candidate path's position bitmap
+// shares that room), k within the candidates the path holds, and enough tiles per indexer CTA
+// (at least 12) for the threshold to arrive while a CTA still has tiles to score.
+bool step_uses_candidates(const ls_decode_step_args* a) {
+  const ls_index_score_args* ix = &a->index;
+  if (a->use_c2f || ix->key_dtype != LS_E4M3 || ix->variant != 0 || ix->max_len <= kTopkRowMaxLen ||
+      ix->max_len > 16 * ls::kTopkCacheKeys || a->k < 1 || a->k > ls::kFastMaxCand)
+    return false;
+  const long long tiles = (((long long)ix->max_len + 63) / 64 + 1) / 2;
+  return tiles >= 12LL * step_idx_ctas(a);
+}
+
+// The indexer's CTAs per request in the decode step (the layout of the candidate lists).
+int step_idx_ctas(const ls_decode_step_args* a) {
+  return idx_ctas_per_req(0, a->index.batch, ((long long)a->index.max_len + 63) / 64, device_sms());
+}
+
 StepLayout step_layout(const ls_decode_step_args* a) {
   StepLayout l{};
   const int B = a->index.batch, k = a->k;
@@ -888,6 +937,14 @@ StepLayout step_layout(const ls_decode_step_args* a) {
   l.off_attn = take(attn_ws_bytes(&t, two_pass ? 2 : 1));
   l.off_done = take((size_t)B * 4);   // per-request attention completion counts
   l.off_ready = take((size_t)B * 4);  // per-request top-k completion counts
+  // the indexer's candidate filter and the candidate top-k (whole requests of the paged or
+  // hot-buffer step whose top-k is the cluster kernel)
+  const bool cand = step_uses_candidates(a);
+  const size_t cpr = cand ? (size_t)step_idx_ctas(a) : 0;
+  l.off_filt = take(cand ? (size_t)B * ls::kFiltInts * 4 : 0);
+  l.off_candcnt = take((size_t)B * cpr * 4 * 4);
+  l.off_candpos = take((size_t)B * cpr * ls::kCandPerCta * 4);
+  l.off_candscore = take((size_t)B * cpr * ls::kCandPerCta * 4);
   if (a->use_c2f) {
     ls_block_bound_prune_args c = step_c2f_args(a, nullptr, nullptr);
     l.off_c2f = take(c2f_layout(&c).total);
@@ -1281,9 +1338,18 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
     // request from the top-k to the attention, and from the attention to the combine; each
     // count is zeroed by the kernel before the one that adds it up
     ready = (!a->use_hotbuf && ix->key_dtype == LS_E4M3 && ix->variant == 0) ? (int*)(w + l.off_ready) : nullptr;
+    const bool cand = step_uses_candidates(a);
+    ls::IdxTcParams fp{};
+    if (cand) {
+      fp.filt = (int*)(w + l.off_filt);
+      fp.cand_cnt = (int*)(w + l.off_candcnt);
+      fp.cand_pos = (int*)(w + l.off_candpos);
+      fp.cand_score = (float*)(w + l.off_candscore);
+      fp.filt_k = a->k;  // the filter's words: zeroed by the top-k that reads them
+    }
     if (ix->key_dtype == LS_E4M3 && ix->variant == 0) {
       LS_TRY(launch_index_tc(ix, 0, nullptr, nullptr, 0, scores, ix->max_len, nullptr, nullptr, 0, nullptr, 0.f, st,
-                             -1, 0, ready));
+                             -1, 0, ready, cand ? &fp : nullptr));
     } else {
       ls_index_score_args tmp = *ix;
       tmp.scores = scores;
@@ -1293,7 +1359,8 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
     int* done = !a->use_hotbuf ? (int*)(w + l.off_done) : nullptr;
     ready_want = ix->max_len <= kTopkRowMaxLen ? 1 : (topk16_supported(st) ? 16 : 8);
     LS_TRY(launch_topk(ix->batch, a->k, scores, ix->max_len, ix->lens, 1, 1, ix->max_len, nullptr, 0, idx, sel,
-                       nullptr, st, nullptr, 0, nullptr, done, ready));
+                       nullptr, st, nullptr, 0, nullptr, done, ready, cand ? &fp : nullptr,
+                       cand ? 4 * step_idx_ctas(a) : 0));
   }
   void* attn_ws = w + l.off_attn;
   if (a->use_hotbuf) {

@@ -198,19 +198,44 @@ __device__ __forceinline__ void prefetch_l2(const void* ptr) {
 // cannot hold a slot one of them needs) has one thread wait for the full count, then a CTA
 // barrier.  The count is zeroed by a kernel that runs before the producer.
 // ---------------------------------------------------------------------------------
-__device__ __forceinline__ void count_done(int* counter) {
+__device__ __forceinline__ void count_done(int* counter, int n = 1) {
   if (threadIdx.x == 0) {
     __threadfence();
-    atomicAdd(counter, 1);
+    atomicAdd(counter, n);
   }
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// ---------------------------------------------------------------------------------
+// Candidate filter between the indexer and the top-k (decode step, whole requests).  Per
+// request, kFiltInts ints, zeroed before the indexer runs: a 64-bit word adding up the
+// indexer CTAs' statistics (count from bit 40, the sum of their keys below), a 64-bit word
+// holding the threshold-ready flag (low half) and the threshold (high half, float bits),
+// written once, and an "incomplete" mark.  Each indexer epilogue warp keeps its candidates in
+// a list of its own, with its count beside it.
+// ---------------------------------------------------------------------------------
+constexpr int kFiltInts = 8;
+constexpr int kFiltStat = 0, kFiltReady = 2, kFiltTau = 3, kFiltIncomplete = 4;
+constexpr int kCandPerWarp = 128;               // candidates an indexer warp keeps (~28 expected)
+constexpr int kCandPerCta = 4 * kCandPerWarp;   // and its CTA (four epilogue warps)
+__device__ __forceinline__ unsigned long long ld_relaxed_gpu_u64(const void* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
 }
 // One thread: wait until *counter >= want (acquire at GPU scope); gives up after
 // g_wait_limit_ns, raising LS_DEV_TIMEOUT.
 __device__ __noinline__ void wait_count(const int* counter, int want) {
   const uint64_t t0 = globaltimer();
   while (true) {
-    int v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+    const int v = ld_acquire_gpu(counter);
     if (v >= want) return;
     if (globaltimer() - t0 > *(volatile unsigned long long*)&g_wait_limit_ns) {
       flag(LS_DEV_TIMEOUT);
@@ -245,6 +270,11 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void* src) 
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// The mbarrier's pending arrival completes once this thread's earlier cp.async copies have
+// landed (the barrier counts it as one of its expected arrivals).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
@@ -430,6 +460,30 @@ __device__ __forceinline__ float key_float(uint32_t k) {
 
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }
 __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
+
+// Exclusive scan of a 32-bit value across the block; returns the exclusive prefix and writes
+// the block total to *total.  tmp: 32 words of shared scratch.  One barrier: every warp scans
+// the warp totals itself.  The caller takes a barrier before tmp is written again.
+__device__ __forceinline__ uint32_t block_excl_scan_u32(uint32_t v, uint32_t* tmp, uint32_t* total) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) tmp[w] = x;
+  __syncthreads();
+  uint32_t t = lane < nw ? tmp[lane] : 0u;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, t, o);
+    if (lane >= o) t += y;
+  }
+  const uint32_t before = __shfl_sync(0xffffffffu, t, (w + 31) & 31);  // warps 0 .. w-1
+  *total = __shfl_sync(0xffffffffu, t, nw - 1);
+  return (w ? before : 0u) + x - v;
+}
 
 // Exclusive scan of a 64-bit value across the block; returns the exclusive prefix and
 // writes the block total to *total.  tmp: 32 entries of shared scratch.

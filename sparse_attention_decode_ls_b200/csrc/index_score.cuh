@@ -117,6 +117,13 @@ struct IdxTcParams {
   int stage_cap;           //   unit_base) of the pool (key_pool / row_scale point at the staging)
   int* clear;              // optional [B]: set to 0 (the top-k's per-request count, which the
                            //   top-k adds up after this kernel has finished)
+  // optional candidate filter (mode 0 over whole requests): see the epilogue
+  int* filt;               // [B][kFiltInts]: zeroed by the top-k that reads them (any contents
+                           //   give exact results; stale ones can only cost the fast path)
+  int* cand_cnt;           // [B][ctas_per_req * 4] candidates each epilogue warp found
+  int* cand_pos;           // [B][ctas_per_req * 4][kCandPerWarp] their positions
+  float* cand_score;       // [B][ctas_per_req * 4][kCandPerWarp] and scores
+  int filt_k;              // the k of the selection the candidates serve
 };
 
 template <int KP, int NCOL>
@@ -124,7 +131,7 @@ struct IdxTc {
   static constexpr int kThreads = 192;                 // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
   static constexpr int kPanel = 128 * 128;             // one 128-row x 128-byte K panel
   static constexpr int kStageBytes = KP * kPanel;
-  static constexpr int kStages = (KP == 1) ? 6 : 3;
+  static constexpr int kStages = (KP == 1) ? 5 : 3;
   static constexpr int kAcc = 256 / NCOL;              // accumulators in 256 TMEM columns
   static constexpr int kBBytes = KP * NCOL * 128;
   static constexpr int kOffB = kStages * kStageBytes;
@@ -134,7 +141,14 @@ struct IdxTc {
   static constexpr int kOffBar = kOffCoef + NCOL * 4 + 16;
   static constexpr int kNumBars = 2 * kStages + 2 * kAcc + 1;  // + b_ready
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
-  static constexpr int kSmem = 1024 + kOffTmem + 16;   // +1024: runtime alignment slack
+  // candidate filter (key scoring only): the scores of the tiles scored before the threshold
+  // is known, and each row's scores that passed it with their tile numbers
+  static constexpr int kFiltBacklog = (KP == 1) ? 16 : 0;   // tiles
+  static constexpr int kRowCand = (KP == 1) ? 8 : 0;        // passing scores kept per row
+  static constexpr int kOffBl = (kOffTmem + 16 + 15) & ~15;
+  static constexpr int kOffLcs = kOffBl + kFiltBacklog * 128 * 4;
+  static constexpr int kOffLct = kOffLcs + 128 * kRowCand * 4;
+  static constexpr int kSmem = 1024 + kOffLct + 128 * kRowCand * 2;  // +1024: runtime alignment slack
   static constexpr uint32_t kIdesc = make_idesc(0 /*e4m3*/, 128, NCOL, false, false);
 };
 
@@ -154,8 +168,9 @@ __device__ __forceinline__ int idx_unit_row(const IdxTcParams& p, int b, int u, 
   return page * 64;
 }
 
+// The key-scoring instance (KP = 1) runs two CTAs per SM, so it must stay within 168 registers.
 template <int KP, int NCOL>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, KP == 1 ? 2 : 1)
     index_score_tc(const IdxTcParams p, const __grid_constant__ CUtensorMap tmap) {
   using C = IdxTc<KP, NCOL>;
   extern __shared__ uint8_t sm_raw[];
@@ -173,7 +188,12 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* acce = accf + C::kAcc;
   uint64_t* b_ready = acce + C::kAcc;
   uint32_t* tmem_slot = (uint32_t*)(sm + C::kOffTmem);
+  float* s_bl = (float*)(sm + C::kOffBl);        // [kFiltBacklog][128]
+  float* s_lcs = (float*)(sm + C::kOffLcs);      // [128][kRowCand]
+  uint16_t* s_lct = (uint16_t*)(sm + C::kOffLct);
   __shared__ int s_abort;
+  __shared__ __align__(16) int s_fpoll[4][4];  // each epilogue warp's copy of the filter's words
+  __shared__ __align__(8) uint64_t s_pbar[4];  // each epilogue warp's copy of the request's words
 
   const int b = blockIdx.y, cta = blockIdx.x, tid = threadIdx.x, warp = warp_id(), lane = lane_id();
   griddep_launch_dependents();  // the next kernel may be scheduled now; it waits for this one
@@ -205,7 +225,11 @@ __global__ void __launch_bounds__(192, 1)
   const int t_begin = (int)(((long long)n_tiles * cta) / p.ctas_per_req);
   const int t_end = (int)(((long long)n_tiles * (cta + 1)) / p.ctas_per_req);
   const int my_tiles = t_end - t_begin;
-  if (my_tiles <= 0) return;
+  if (my_tiles <= 0) {
+    // a CTA without tiles has no candidates (the top-k reads every CTA's count)
+    if (p.filt && p.mode == 0 && !p.unit_list && tid < 4) p.cand_cnt[((size_t)b * p.ctas_per_req + cta) * 4 + tid] = 0;
+    return;
+  }
 
   // ---- query side: B operand in 128-byte-swizzled K-major layout, coefficients and, for
   // the bound, the magnitude used by the margin.  The epilogue warps build it while the
@@ -280,6 +304,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     mbar_init(b_ready, 128);
     s_abort = 0;
+    for (int w = 0; w < 4; ++w) mbar_init(&s_pbar[w], 1);
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(tmem_slot, 256);
@@ -390,6 +415,50 @@ __global__ void __launch_bounds__(192, 1)
     const int rr = r & 63;
     const float mag = (p.mode == 1) ? gmag[0] : 0.f;
     const int nb = (L + 63) >> 6;
+    // ---- candidate filter.  Besides every score, the scores at or above a per-request
+    // threshold tau go to candidate lists, so that the top-k can select among a few thousand
+    // entries instead of the whole request.  tau comes from the request's own scores: each
+    // epilogue warp takes the j-th largest score of its 32 rows of its first tile (j ~ 64 k / L,
+    // so that about 2k scores of the request lie above such a statistic) and adds it, as an
+    // order-preserving key, with a count into one 64-bit word of the request; the first warp of
+    // CTA 0, once it sees the word hold 32 of them (fewer for a short request), sets tau to the
+    // mean of the keys it saw.  The tile loop never waits on memory for this: the additions
+    // return nothing, and each warp learns of tau from an asynchronous copy of the request's
+    // words whose barrier it tests without blocking; a load issued then is checked at the end
+    // against the tau it used.  Until tau is known, every
+    // score also goes to shared memory; then those tiles are checked from there.  A row keeps
+    // the scores that passed (with their tile numbers) in shared memory, and each epilogue warp
+    // writes its rows' candidates to a list of its own after its last tile.  Any tau gives an
+    // exact result: the top-k uses the lists only when at least k scores passed (then the k-th
+    // largest is among them) and every list is complete; a warp that did not see tau within
+    // kFiltBacklog tiles (or saw another tau than the one set), a row or list that ran full or
+    // an aborted CTA marks the request incomplete.
+    const bool filt = p.filt != nullptr && p.mode == 0 && !p.unit_list;
+    int* fctl = filt ? p.filt + (size_t)b * kFiltInts : nullptr;
+    const int n_need = 4 * min(min(p.ctas_per_req, n_tiles), 8);  // statistics that set tau
+    const int fj = filt ? min(8, max(1, (int)((64LL * p.filt_k + L - 1) / max(L, 1)))) : 1;
+    const bool publisher = filt && cta == 0 && wq == 0;
+    bool tau_known = false, gave_up = false;
+    float tau = 0.f;
+    int nk = 0;                            // this row's passing scores
+    unsigned long long tau_check = 0;      // lane 0: the request's tau word, loaded when seen
+    uint32_t poll_ph = 0;
+    bool poll_inflight = false;            // lane 0: a copy of the request's words in flight
+    float* my_lcs = s_lcs + r * C::kRowCand;
+    uint16_t* my_lct = s_lct + r * C::kRowCand;
+    auto keep = [&](int t, float v) {
+      if (nk < C::kRowCand) {
+        my_lcs[nk] = v;
+        my_lct[nk] = (uint16_t)t;
+      }
+      ++nk;
+    };
+    auto look = [&]() {  // lane 0: copy the request's first 16 bytes in (through the load path)
+      cp_async_16(smem_u32(&s_fpoll[wq][0]), fctl);
+      cp_async_mbar_arrive(&s_pbar[wq]);
+      poll_inflight = true;
+    };
+    if (filt && lane == 0) look();
     for (int i = 0; i < my_tiles; ++i) {
       const int st = i % C::kStages, a = i % C::kAcc;
       const int tile = t_begin + i;
@@ -412,6 +481,10 @@ __global__ void __launch_bounds__(192, 1)
         scale = s_scale[st * 128 + r];
         out_idx = p.unit_list ? (long long)(p.unit_base + u) * 64 + rr : (long long)lp * 64 + rr;
       }
+      // the stage's metadata is read: the producer may refill it once the MMA has read its keys
+      // too (the MMA's commit is the stage's other arrival), so the loads need not wait for
+      // this tile's epilogue
+      mbar_arrive(&empty[st]);
       if (!mbar_wait(&accf[a], (i / C::kAcc) & 1)) { s_abort = 1; break; }
       tc_fence_after();
       // four independent partial sums (fixed order: the result is the same for a token
@@ -434,7 +507,6 @@ __global__ void __launch_bounds__(192, 1)
       const float sum = (acc0 + acc1) + (acc2 + acc3);
       tc_fence_before();
       mbar_arrive(&acce[a]);
-      mbar_arrive(&empty[st]);
       if (valid) {
         float* o = p.out + (size_t)b * p.out_stride;
         if (p.mode == 1) {
@@ -444,6 +516,92 @@ __global__ void __launch_bounds__(192, 1)
         } else {
           o[out_idx] = sum * scale;
         }
+      }
+      if (filt) {
+        const float sc = valid ? sum * scale : -INFINITY;
+        if (!tau_known && !gave_up) {
+          s_bl[i * 128 + r] = sc;
+          if (i == 0) {
+            // this warp's statistic: the fj-th largest score of its rows of the first tile; its
+            // key goes into the request's word with a count from bit 48 (the sum of the keys
+            // below; at most 2^16 additions)
+            float v = sc, kth = -INFINITY;
+            for (int q = 0; q < fj; ++q) {
+              float mx = v;
+#pragma unroll
+              for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+              kth = mx;
+              const uint32_t own = __ballot_sync(0xffffffffu, v == mx);
+              if (lane == __ffs(own) - 1) v = -INFINITY;  // take one copy of the maximum out
+            }
+            if (lane == 0) atomicAdd((unsigned long long*)(fctl + kFiltStat), (1ull << 48) | float_key(kth));
+          }
+          int f = 0;
+          float t = 0.f;
+          if (lane == 0 && poll_inflight && mbar_test_wait(&s_pbar[wq], poll_ph)) {
+            poll_ph ^= 1u;
+            poll_inflight = false;
+            f = *(volatile int*)&s_fpoll[wq][kFiltReady];
+            t = *(volatile float*)&s_fpoll[wq][kFiltTau];
+            const unsigned long long sw = *(volatile unsigned long long*)&s_fpoll[wq][kFiltStat];
+            if (f) {
+              tau_check = ld_relaxed_gpu_u64(fctl + kFiltReady);  // looked at after the last tile
+            } else if (publisher && (int)(sw >> 48) >= n_need) {
+              // enough statistics: tau = the mean of their keys, published once
+              const unsigned long long cnt = sw >> 48;
+              t = key_float((uint32_t)((sw & ((1ull << 48) - 1)) / cnt));
+              tau_check = ((unsigned long long)__float_as_uint(t) << 32) | 1ull;
+              atomicExch((unsigned long long*)(fctl + kFiltReady), tau_check);
+              f = 1;
+            } else {
+              look();
+            }
+          }
+          f = __shfl_sync(0xffffffffu, f, 0);
+          if (f) {
+            tau = __shfl_sync(0xffffffffu, t, 0);
+            tau_known = true;
+            // the tiles scored before (this one included), from shared memory
+            for (int t2 = 0; t2 <= i; ++t2) {
+              const float v = s_bl[t2 * 128 + r];
+              if (v >= tau && v != -INFINITY) keep(t2, v);
+            }
+          } else if (i + 1 >= C::kFiltBacklog) {
+            gave_up = true;  // too many tiles to keep: this request's lists stay incomplete
+          }
+        } else if (tau_known && sc >= tau && valid) {
+          keep(i, sc);
+        }
+      }
+    }
+    if (filt) {
+      // the statistic if not yet looked at, then the rows' candidates into this warp's list
+      const bool aborted = *(volatile int*)&s_abort != 0;
+      bool bad = __any_sync(0xffffffffu, nk > C::kRowCand) || !tau_known || aborted;
+      if (lane == 0) {
+        if (poll_inflight) mbar_wait(&s_pbar[wq], poll_ph);  // the copy lands before the CTA ends
+        if (tau_known && (!(uint32_t)tau_check || (tau_check >> 32) != __float_as_uint(tau))) bad = true;
+      }
+      bad = __shfl_sync(0xffffffffu, (int)bad, 0) != 0;
+      const size_t wlist = (((size_t)b * p.ctas_per_req + cta) * 4 + wq) * kCandPerWarp;
+      int wcnt = 0;
+      if (!bad) {
+        const int mine = min(nk, C::kRowCand);
+        const int rounds = __reduce_max_sync(0xffffffffu, (uint32_t)mine);
+        for (int q = 0; q < rounds; ++q) {
+          const bool take = q < mine;
+          const uint32_t m = __ballot_sync(0xffffffffu, take);
+          const int o = wcnt + __popc(m & ((1u << lane) - 1u));
+          if (take && o < kCandPerWarp) {
+            p.cand_pos[wlist + o] = (2 * (t_begin + (int)my_lct[q]) + (r >> 6)) * 64 + rr;
+            p.cand_score[wlist + o] = my_lcs[q];
+          }
+          wcnt += __popc(m);
+        }
+      }
+      if (lane == 0) {
+        if (bad || wcnt > kCandPerWarp) fctl[kFiltIncomplete] = 1;
+        p.cand_cnt[((size_t)b * p.ctas_per_req + cta) * 4 + wq] = min(wcnt, kCandPerWarp);
       }
     }
   }

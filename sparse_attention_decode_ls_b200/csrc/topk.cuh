@@ -32,10 +32,17 @@ struct TopkParams {
   float* sel;                // [B,k] (may be NULL)
   float* thr;                // [B] optional: k-th largest score, -inf if fewer than k candidates
   int cache_keys;            // keys of dynamic shared memory available per CTA
+  int smem_bytes;            // dynamic shared memory of the launch
   int* clear;                // optional [B]: set to 0 (a per-request count the next kernel of
                              //   the step adds up; see AttnParams::done)
   int* done;                 // optional [B], zero at launch: every CTA adds 1 once its outputs
                              //   are stored (see AttnParams::ready)
+  // optional: the indexer's candidate lists (see the candidate filter in index_score.cuh)
+  int* filt;                 // [B][kFiltInts]: read, then zeroed for the next step
+  const int* cand_cnt;       // [B][cand_lists] candidates per list (one per indexer epilogue warp)
+  const int* cand_pos;       // [B][cand_lists][kCandPerWarp]
+  const float* cand_score;
+  int cand_lists;            // the indexer's lists per request
 };
 
 constexpr int kTopkThreads = 512;
@@ -81,6 +88,258 @@ constexpr int kTopkExtraBytes = kCandCap * 4 + kCandTotal * 4 + (kTopkThreads / 
     }                                                                                   \
   } while (0)
 
+
+constexpr int kFastMaxCand = 6144;  // candidates the candidate path holds
+constexpr int kFastBins = 4096;     // histogram bins (12 bits of a key at a time)
+constexpr int kFastShift = 12;      // first pass: bins of 2^12 keys above key(tau), the last open
+constexpr int kFastList = 64;       // keys in the k-th key's bin that the list rank takes
+
+__host__ __device__ constexpr int fast_round(int x, int m) { return (x + m - 1) / m * m; }
+// Shared memory (bytes) the candidate path needs for a request of L positions and n
+// candidates: their keys and positions, a bitmap of the chosen positions and a room that
+// holds the histogram, then the bitmap words' prefix counts (or, on the general route, the
+// bitmap of the keys equal to the k-th).
+__host__ __device__ constexpr int fast_smem_bytes(int L, int n) {
+  return (fast_round(2 * n, 4) + fast_round((L + 31) / 32, 8) +
+          (fast_round((L + 31) / 32, 8) > kFastBins ? fast_round((L + 31) / 32, 8) : kFastBins)) * 4;
+}
+
+// The top-k of one request from the indexer's candidate lists (every key of the top k is
+// among them, see TopkParams::filt), by one CTA of kTopkThreads threads.  coff[c] is where
+// list c starts (coff[lists] = n); list: 2 * kFastList words of shared scratch.
+//  1. Each candidate is loaded (eight per thread in flight) and counted in the bin of
+//     (key - key(tau)) >> 12 (the candidates crowd just above tau: bins measured from there
+//     spread them; the last bin is open-ended).
+//  2. One scan of the bins from the top finds the bin tb of the k-th largest key.
+//  3. Every key in a higher bin is chosen; bin tb's keys go to a list, where each is ranked
+//     exactly (larger key first, then lower position) and the first k - (keys above tb) are
+//     chosen.  A bin too crowded for the list (many equal keys) takes the general route: the
+//     k-th largest key T by a radix pass over the low 12 bits of bin tb's keys (over whole keys,
+//     12 bits at a time, for the open last bin), then the keys equal to T in a bitmap, of which
+//     the lowest-positioned are taken.
+//  4. A bitmap holds the chosen positions; from its words' prefix counts each chosen candidate
+//     writes its own slot, so the positions leave in ascending order.  Its score is its key
+//     read back as a float: the same bits the indexer stored in the score row.
+__device__ __forceinline__ void topk_from_candidates(const TopkParams& p, int b, int L, int n, uint32_t* smem,
+                                                     const int* coff, uint32_t* list, uint32_t* scan32,
+                                                     uint32_t* s_misc) {
+  const int tid = threadIdx.x;
+  const int k = p.k, nl = p.cand_lists, nw8 = fast_round((L + 31) >> 5, 8);
+  uint32_t* keys = smem;
+  int* cpos = (int*)(keys + n);
+  uint32_t* bits = smem + fast_round(2 * n, 4);  // 16-byte aligned
+  uint32_t* room = bits + nw8;
+  uint32_t* lkey = list;
+  int* lpos = (int*)(list + kFastList);
+  const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+  for (int w = tid * 4; w < nw8; w += kTopkThreads * 4) *(uint4*)(bits + w) = z4;
+  for (int w = tid * 4; w < kFastBins; w += kTopkThreads * 4) *(uint4*)(room + w) = z4;
+  if (tid == 0) {
+    s_misc[1] = 0u;         // keys in the list
+    s_misc[2] = kFastBins;  // the k-th key's bin (none yet)
+  }
+  const uint32_t tk = float_key(__int_as_float(p.filt[(size_t)b * kFiltInts + kFiltTau]));
+  __syncthreads();
+  // ---- 1. load and count
+  const size_t base = (size_t)b * nl * kCandPerWarp;
+  for (int i0 = 0; i0 < n; i0 += 8 * kTopkThreads) {
+    float sq[8];
+    int pq[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = i0 + e * kTopkThreads + tid;
+      sq[e] = -INFINITY;
+      pq[e] = -1;
+      if (i < n) {
+        int lo = 0, hi = nl - 1;  // the list holding entry i: coff[lo] <= i < coff[lo + 1]
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (coff[mid] <= i) lo = mid; else hi = mid - 1;
+        }
+        const int j = i - coff[lo];
+        if (j < kCandPerWarp) {  // always: a longer list marks the request incomplete
+          const size_t src = base + (size_t)lo * kCandPerWarp + j;
+          sq[e] = p.cand_score[src];
+          pq[e] = p.cand_pos[src];
+        }
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i = i0 + e * kTopkThreads + tid;
+      if (i < n) {
+        const uint32_t key = float_key(sq[e]);
+        keys[i] = key;
+        cpos[i] = pq[e];
+        if (key >= tk) atomicAdd(&room[min((key - tk) >> kFastShift, (uint32_t)(kFastBins - 1))], 1u);
+      }
+    }
+  }
+  __syncthreads();
+  // ---- 2. the k-th key's bin: thread t reads bins [4088 - 8t, 4095 - 8t] from the top
+  {
+    constexpr int per = kFastBins / kTopkThreads;
+    static_assert(per == 8, "eight bins per thread");
+    const int top = kFastBins - per * (tid + 1);
+    const uint4 a = *(const uint4*)(room + top), c = *(const uint4*)(room + top + 4);
+    const uint32_t h[per] = {c.w, c.z, c.y, c.x, a.w, a.z, a.y, a.x};
+    uint32_t mine = 0;
+#pragma unroll
+    for (int j = 0; j < per; ++j) mine += h[j];
+    uint32_t tot;
+    uint32_t above = block_excl_scan_u32(mine, scan32, &tot);
+#pragma unroll
+    for (int j = 0; j < per; ++j) {
+      if (above < (uint32_t)k && above + h[j] >= (uint32_t)k) {
+        s_misc[2] = (uint32_t)(top + per - 1 - j);
+        s_misc[3] = above;
+      }
+      above += h[j];
+    }
+  }
+  __syncthreads();
+  const uint32_t tb = s_misc[2], r0 = (uint32_t)k - s_misc[3];  // r0 of bin tb's keys are chosen
+  // ---- 3. keys above bin tb chosen, bin tb's keys listed
+  for (int i = tid; i < n; i += kTopkThreads) {
+    const uint32_t key = keys[i];
+    const int ps = cpos[i];
+    if (key < tk || ps < 0 || ps >= L) continue;
+    const uint32_t bin = min((key - tk) >> kFastShift, (uint32_t)(kFastBins - 1));
+    if (bin > tb) {
+      atomicOr(&bits[ps >> 5], 1u << (ps & 31));
+    } else if (bin == tb) {
+      const uint32_t o = atomicAdd(&s_misc[1], 1u);
+      if (o < (uint32_t)kFastList) {
+        lkey[o] = key;
+        lpos[o] = ps;
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t m = s_misc[1];
+  if (tb < (uint32_t)kFastBins && m <= (uint32_t)kFastList) {
+    for (int e = tid; e < (int)m; e += kTopkThreads) {
+      const uint32_t ke = lkey[e];
+      const int pe = lpos[e];
+      uint32_t r = 0;
+      for (int j = 0; j < (int)m; ++j) {
+        const uint32_t kj = lkey[j];
+        r += (kj > ke || (kj == ke && lpos[j] < pe)) ? 1u : 0u;
+      }
+      if (r < r0) atomicOr(&bits[pe >> 5], 1u << (pe & 31));
+    }
+  } else {
+    // the general route: T and R by radix passes over d = key - base from bit hi down, among
+    // the keys whose bits above hi equal prefix: the low 12 bits of bin tb, or whole keys
+    constexpr int per = kFastBins / kTopkThreads;
+    const bool open = tb >= (uint32_t)(kFastBins - 1);
+    const uint32_t base = open ? 0u : tk;
+    uint32_t prefix = open ? 0u : tb, k_rem = open ? (uint32_t)k : r0;
+    for (int hi = open ? 32 : kFastShift; hi > 0;) {
+      const int width = min(12, hi), shift = hi - width;
+      const uint32_t nb = 1u << width;
+      for (int d = tid; d < kFastBins; d += kTopkThreads) room[d] = 0u;
+      __syncthreads();
+      for (int i = tid; i < n; i += kTopkThreads) {
+        const uint32_t key = keys[i], d = key - base;
+        if (key >= base && (hi >= 32 || (d >> hi) == prefix)) atomicAdd(&room[(d >> shift) & (nb - 1u)], 1u);
+      }
+      __syncthreads();
+      uint32_t h[per], mine = 0;
+#pragma unroll
+      for (int j = 0; j < per; ++j) {
+        const int bin = (int)nb - 1 - (tid * per + j);
+        h[j] = bin >= 0 ? room[bin] : 0u;
+        mine += h[j];
+      }
+      uint32_t tot;
+      uint32_t above = block_excl_scan_u32(mine, scan32, &tot);
+#pragma unroll
+      for (int j = 0; j < per; ++j) {
+        if (above < k_rem && above + h[j] >= k_rem) {
+          s_misc[2] = (uint32_t)((int)nb - 1 - (tid * per + j));
+          s_misc[3] = above;
+        }
+        above += h[j];
+      }
+      __syncthreads();
+      prefix = (prefix << width) | s_misc[2];
+      k_rem -= s_misc[3];
+      hi = shift;
+      __syncthreads();
+    }
+    const uint32_t T = base + prefix, R = k_rem;  // every key > T, and the R lowest-positioned == T
+    uint32_t* tbits = room;
+    for (int w = tid; w < nw8; w += kTopkThreads) tbits[w] = 0u;
+    __syncthreads();
+    for (int i = tid; i < n; i += kTopkThreads) {
+      const int ps = cpos[i];
+      if (ps < 0 || ps >= L) continue;
+      if (keys[i] > T) {
+        atomicOr(&bits[ps >> 5], 1u << (ps & 31));
+      } else if (keys[i] == T) {
+        atomicOr(&tbits[ps >> 5], 1u << (ps & 31));
+      }
+    }
+    __syncthreads();
+    const int wpt = (nw8 + kTopkThreads - 1) / kTopkThreads;
+    const int w0 = min(nw8, tid * wpt), w1 = min(nw8, w0 + wpt);
+    uint32_t c = 0;
+    for (int w = w0; w < w1; ++w) c += __popc(tbits[w]);
+    uint32_t tot;
+    uint32_t seen = block_excl_scan_u32(c, scan32, &tot);
+    for (int w = w0; w < w1 && seen < R; ++w) {
+      uint32_t mm = tbits[w], take = 0u;
+      while (mm && seen < R) {
+        take |= mm & (~mm + 1u);  // lowest set bit
+        mm &= mm - 1u;
+        ++seen;
+      }
+      if (take) atomicOr(&bits[w], take);
+    }
+  }
+  __syncthreads();
+  // ---- 4. the words' prefix counts (in the room), then every chosen candidate's slot
+  {
+    const int wpt = fast_round((nw8 + kTopkThreads - 1) / kTopkThreads, 4);
+    const int w0 = min(nw8, tid * wpt), w1 = min(nw8, w0 + wpt);
+    uint32_t c = 0;
+    for (int w = w0; w < w1; w += 4) {
+      const uint4 v = *(const uint4*)(bits + w);
+      c += __popc(v.x) + __popc(v.y) + __popc(v.z) + __popc(v.w);
+    }
+    uint32_t tot;
+    uint32_t o = block_excl_scan_u32(c, scan32, &tot);
+    for (int w = w0; w < w1; w += 4) {
+      const uint4 v = *(const uint4*)(bits + w);
+      uint4 q;
+      q.x = o;
+      o += __popc(v.x);
+      q.y = o;
+      o += __popc(v.y);
+      q.z = o;
+      o += __popc(v.z);
+      q.w = o;
+      o += __popc(v.w);
+      *(uint4*)(room + w) = q;
+    }
+    if (tid == 0 && tot != (uint32_t)k) flag(LS_DEV_BOUNDS);  // cannot happen: exactly k chosen
+  }
+  __syncthreads();
+  const int off = p.pos_offset ? p.pos_offset[b] : 0;
+  for (int i = tid; i < n; i += kTopkThreads) {
+    const int ps = cpos[i];
+    if (ps < 0 || ps >= L) continue;
+    const uint32_t word = bits[ps >> 5], bit = 1u << (ps & 31);
+    if (!(word & bit)) continue;
+    const uint32_t o = room[ps >> 5] + __popc(word & (bit - 1u));
+    if (o < (uint32_t)k) {
+      if (p.idx) p.idx[(size_t)b * k + o] = ps + off;
+      if (p.sel) p.sel[(size_t)b * k + o] = key_float(keys[i]);
+    }
+  }
+}
+
 template <int CL>
 // At most 64 registers: two CTAs per SM, so that all clusters of a batch are resident at once.
 __global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster(const TopkParams p) {
@@ -108,6 +367,60 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster(const TopkParams
   griddep_wait();  // the scores come from the kernel before
   griddep_launch_dependents();
   if (p.clear && rank == 0 && tid == 0) p.clear[b] = 0;
+
+  if (p.filt) {
+    // The candidate path: when the indexer's lists for this request are complete, hold at
+    // least k candidates and fit this CTA's shared memory, CTA 0 selects from them alone and
+    // the other CTAs leave at once.  Every CTA reads the same words, so the choice is the same
+    // in the whole cluster (and no distributed shared memory has been touched).  Warp 0 adds
+    // up the lists' lengths into their offsets (in ghist), warp 1 reads the filter's state.
+    const int* f = p.filt + (size_t)b * kFiltInts;
+    int* coff = (int*)ghist;
+    if (warp == 0) {
+      uint32_t run = 0;
+      for (int c0 = 0; c0 < p.cand_lists; c0 += 32) {
+        const uint32_t v = c0 + lane < p.cand_lists ? (uint32_t)p.cand_cnt[(size_t)b * p.cand_lists + c0 + lane] : 0u;
+        uint32_t incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        if (c0 + lane < p.cand_lists) coff[c0 + lane] = (int)(run + incl - v);
+        run += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      if (lane == 0) {
+        coff[p.cand_lists] = (int)run;
+        s_total = run;
+      }
+    } else if (warp == 1 && lane == 0) {
+      s_fast = (f[kFiltReady] != 0 && f[kFiltIncomplete] == 0) ? 1u : 0u;
+    }
+    const long long L0 = ((long long)p.lens[b] * p.len_mul + p.len_div - 1) / p.len_div;
+    __syncthreads();
+    const int nc = (int)s_total;
+    const int Lq = (L0 < 0 || L0 > p.len_limit) ? 0 : (int)L0;
+    const bool use = s_fast != 0 && nc >= k && nc <= kFastMaxCand && Lq > 0 && p.cand_lists < 2048 &&
+                     fast_smem_bytes(Lq, nc) <= p.smem_bytes && !p.unit_list && !p.pos_list && !p.thr;
+    // once every CTA of the cluster has read the request's words, CTA 0 zeroes them for the
+    // next step (arrive now, wait when done: the candidate path does not wait for the others)
+    cluster_arrive();
+    if (use) {
+      if (rank == 0) {
+        topk_from_candidates(p, b, Lq, nc, sm_keys, coff, hist, (uint32_t*)scan_tmp, s_off);
+        if (p.done) {
+          __syncthreads();
+          count_done(p.done + b, CL);  // counts for the whole cluster
+        }
+      }
+      cluster_wait();
+      if (rank == 0 && tid < kFiltInts) p.filt[(size_t)b * kFiltInts + tid] = 0;
+      return;  // no distributed shared memory was touched
+    }
+    cluster_wait();
+    if (rank == 0 && tid < kFiltInts) p.filt[(size_t)b * kFiltInts + tid] = 0;
+    __syncthreads();  // the fallback reuses ghist
+  }
 
   long long nll = ((long long)p.lens[b] * p.len_mul + p.len_div - 1) / p.len_div;
   bool bad = nll < 0 || nll > p.len_limit;

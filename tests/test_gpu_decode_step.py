@@ -13,7 +13,7 @@ from sparse_attention_decode_ls_b200 import binding as B
 from sparse_attention_decode_ls_b200 import synthetic as syn
 from sparse_attention_decode_ls_b200 import workload as W
 
-from gpu_helpers import DEV, assert_status_clean, bits16, check_topk_band, oracle_index_inputs
+from gpu_helpers import DEV, assert_status_clean, bits16, check_topk_band, gpu_index_scores, oracle_index_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -203,3 +203,57 @@ def test_decode_step_writes_outputs_to_host_memory(lens):
         assert torch.equal(host_o, ref_o) and torch.equal(host_lse, ref_lse)
     wl.args.attn.o, wl.args.attn.lse = dev_o, dev_lse
     assert_status_clean()
+
+
+@pytest.mark.parametrize("kind", ["iid", "ties_at_k", "all_equal", "clustered", "ragged"])
+def test_decode_step_selection_equals_full_topk(kind):
+    """The step's selection (indexer candidates + candidate top-k, or the cluster top-k where
+    the candidates do not serve) equals ls_topk_select over the same scores bit for bit --
+    positions and selection scores -- for scores drawn i.i.d., for 600 tokens given the key of
+    the token ranked ~2000th (exact ties across the k-th score: the lower positions must win),
+    for scores that all tie (too many equal keys: the cluster top-k decides), for
+    block-clustered keys (a skewed request), and for a ragged batch whose short requests give
+    fewer candidates than k or leave indexer CTAs without tiles (those go to the cluster
+    top-k, the long one to the candidates)."""
+    lens = [131072, 3000, 40000, 1] if kind == "ragged" else [131072, 131072, 100000, 70001]
+    if kind == "clustered":
+        from test_gpu_stages import _c2f_inputs
+        inp = _c2f_inputs(lens, seed=801, clustered=True)
+    else:
+        inp = syn.indexer_fp8(lens, seed=801)
+        if kind == "all_equal":
+            inp.key_pool[:] = inp.key_pool[0, 0]
+            inp.key_scale[:] = inp.key_scale[0, 0]
+        elif kind == "ties_at_k":
+            sc = gpu_index_scores(inp).cpu()
+            g = torch.Generator().manual_seed(803)
+            pt = inp.page_table
+            for b, L in enumerate(lens):
+                src = int(torch.argsort(sc[b, :L], descending=True)[2000])
+                dst = torch.randperm(L, generator=g)[:600]
+                sp, so = int(pt[b, src // 64]), src % 64
+                for d in dst.tolist():
+                    inp.key_pool[int(pt[b, d // 64]), d % 64] = inp.key_pool[sp, so]
+                    inp.key_scale[int(pt[b, d // 64]), d % 64] = inp.key_scale[sp, so]
+    q, kv = syn.mla_attention(len(lens), inp.key_pool.shape[0], seed=802)
+    wl = W.build("cand", inp, k=2048, attn=dict(q=q, kv=kv, scale=syn.softmax_scale(576)))
+    for _ in range(2):  # the filter's counts restart every step
+        wl.step()
+        torch.cuda.synchronize()
+        assert_status_clean()
+        scores = gpu_index_scores_from(wl)
+        full = torch.full_like(wl.idx, -7)
+        full_sel = torch.zeros_like(wl.tensors["sel"])
+        B.ls_topk_select(scores=scores, lens=wl.tensors["i_lens"], idx=full, sel_score=full_sel)
+        torch.cuda.synchronize()
+        assert torch.equal(wl.idx, full)
+        assert torch.equal(wl.tensors["sel"], full_sel)
+
+
+def gpu_index_scores_from(wl):
+    """The indexer's scores for the workload's own device inputs."""
+    t = wl.tensors
+    scores = torch.full((wl.batch, wl.args.index.max_len), float("nan"), device=DEV)
+    B.ls_index_score(q=t["i_q"], w=t["i_w"], key_pool=t["i_key_pool"], page_table=t["i_page_table"],
+                     lens=t["i_lens"], scores=scores, q_scale=t["i_q_scale"], key_scale=t["i_key_scale"])
+    return scores
