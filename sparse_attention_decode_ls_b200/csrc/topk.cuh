@@ -123,7 +123,7 @@ __host__ __device__ constexpr int fast_smem_bytes(int L, int n) {
 __device__ __forceinline__ void topk_from_candidates(const TopkParams& p, int b, int L, int n, uint32_t* smem,
                                                      const int* coff, uint32_t* list, uint32_t* scan32,
                                                      uint32_t* s_misc) {
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int k = p.k, nl = p.cand_lists, nw8 = fast_round((L + 31) >> 5, 8);
   uint32_t* keys = smem;
   int* cpos = (int*)(keys + n);
@@ -140,38 +140,43 @@ __device__ __forceinline__ void topk_from_candidates(const TopkParams& p, int b,
   }
   const uint32_t tk = float_key(__int_as_float(p.filt[(size_t)b * kFiltInts + kFiltTau]));
   __syncthreads();
-  // ---- 1. load and count
+  // ---- 1. load and count: warp w takes lists w, w + 16, ..., eight at a time (lane j entry
+  // j; a list longer than 32 entries takes more turns), all their loads in flight at once
   const size_t base = (size_t)b * nl * kCandPerWarp;
-  for (int i0 = 0; i0 < n; i0 += 8 * kTopkThreads) {
+  constexpr int kW = kTopkThreads / 32;
+  auto take = [&](float sc, int ps, int at) {
+    const uint32_t key = float_key(sc);
+    keys[at] = key;
+    cpos[at] = ps;
+    if (key >= tk) atomicAdd(&room[min((key - tk) >> kFastShift, (uint32_t)(kFastBins - 1))], 1u);
+  };
+  for (int l0 = warp; l0 < nl; l0 += 8 * kW) {
     float sq[8];
-    int pq[8];
+    int pq[8], at[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int i = i0 + e * kTopkThreads + tid;
-      sq[e] = -INFINITY;
-      pq[e] = -1;
-      if (i < n) {
-        int lo = 0, hi = nl - 1;  // the list holding entry i: coff[lo] <= i < coff[lo + 1]
-        while (lo < hi) {
-          const int mid = (lo + hi + 1) >> 1;
-          if (coff[mid] <= i) lo = mid; else hi = mid - 1;
-        }
-        const int j = i - coff[lo];
-        if (j < kCandPerWarp) {  // always: a longer list marks the request incomplete
-          const size_t src = base + (size_t)lo * kCandPerWarp + j;
-          sq[e] = p.cand_score[src];
-          pq[e] = p.cand_pos[src];
+    for (int u = 0; u < 8; ++u) {
+      const int l = l0 + u * kW;
+      at[u] = -1;
+      if (l < nl) {
+        const int o = coff[l], c = min(coff[l + 1] - o, kCandPerWarp);
+        if (lane < c) {
+          const size_t src = base + (size_t)l * kCandPerWarp + lane;
+          sq[u] = p.cand_score[src];
+          pq[u] = p.cand_pos[src];
+          at[u] = o + lane;
         }
       }
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int i = i0 + e * kTopkThreads + tid;
-      if (i < n) {
-        const uint32_t key = float_key(sq[e]);
-        keys[i] = key;
-        cpos[i] = pq[e];
-        if (key >= tk) atomicAdd(&room[min((key - tk) >> kFastShift, (uint32_t)(kFastBins - 1))], 1u);
+    for (int u = 0; u < 8; ++u)
+      if (at[u] >= 0) take(sq[u], pq[u], at[u]);
+    for (int u = 0; u < 8; ++u) {  // entries 32 and up (a rare long list)
+      const int l = l0 + u * kW;
+      if (l >= nl) break;
+      const int o = coff[l], c = min(coff[l + 1] - o, kCandPerWarp);
+      for (int j = 32 + lane; j < c; j += 32) {
+        const size_t src = base + (size_t)l * kCandPerWarp + j;
+        take(p.cand_score[src], p.cand_pos[src], o + j);
       }
     }
   }
@@ -377,20 +382,36 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster(const TopkParams
     const int* f = p.filt + (size_t)b * kFiltInts;
     int* coff = (int*)ghist;
     if (warp == 0) {
+      // lane j adds up lists [8j, 8j + 8) of each 256, their counts loaded together
+      const int nl = p.cand_lists;
+      const int* cnt = p.cand_cnt + (size_t)b * nl;
       uint32_t run = 0;
-      for (int c0 = 0; c0 < p.cand_lists; c0 += 32) {
-        const uint32_t v = c0 + lane < p.cand_lists ? (uint32_t)p.cand_cnt[(size_t)b * p.cand_lists + c0 + lane] : 0u;
-        uint32_t incl = v;
+      for (int c0 = 0; c0 < nl; c0 += 256) {
+        uint32_t v[8], mine = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int l = c0 + lane * 8 + e;
+          v[e] = l < nl ? (uint32_t)max(cnt[l], 0) : 0u;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mine += v[e];
+        uint32_t incl = mine;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
           if (lane >= o) incl += y;
         }
-        if (c0 + lane < p.cand_lists) coff[c0 + lane] = (int)(run + incl - v);
+        uint32_t at = run + incl - mine;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int l = c0 + lane * 8 + e;
+          if (l < nl) coff[l] = (int)at;
+          at += v[e];
+        }
         run += __shfl_sync(0xffffffffu, incl, 31);
       }
       if (lane == 0) {
-        coff[p.cand_lists] = (int)run;
+        coff[nl] = (int)run;
         s_total = run;
       }
     } else if (warp == 1 && lane == 0) {
