@@ -191,7 +191,7 @@ ls_status validate_index(const ls_index_score_args* a, bool need_scores) {
   return LS_OK;
 }
 
-std::atomic<uint64_t> g_smem_idx_simt_f32{0}, g_smem_idx_simt_e4m3{0}, g_smem_idx_tc{0}, g_smem_bound_tc{0};
+std::atomic<uint64_t> g_smem_idx_simt_f32{0}, g_smem_idx_simt_e4m3{0}, g_smem_idx_tc{0}, g_smem_idx_tc_f{0}, g_smem_bound_tc{0};
 
 ls_status launch_index_simt(const ls_index_score_args* a, cudaStream_t st) {
   ls::IdxSimtParams p{};
@@ -266,10 +266,17 @@ ls_status launch_index_tc(const ls_index_score_args* a, int mode, const int* uni
   p.ctas_per_req = c;
   dim3 grid((unsigned)c, a->batch);
   if (mode == 0) {
-    using C = ls::IdxTc<1, 64>;
-    if (allow_smem(ls::index_score_tc<1, 64>, C::kSmem, g_smem_idx_tc) != cudaSuccess)
-      return check_launch("index_score_tc attribute");
-    ls::index_score_tc<1, 64><<<grid, C::kThreads, C::kSmem, st>>>(p, tmap);
+    if (p.filt) {  // the instance that keeps candidate lists
+      using C = ls::IdxTc<1, 64, true>;
+      if (allow_smem(ls::index_score_tc<1, 64, true>, C::kSmem, g_smem_idx_tc_f) != cudaSuccess)
+        return check_launch("index_score_tc attribute");
+      ls::index_score_tc<1, 64, true><<<grid, C::kThreads, C::kSmem, st>>>(p, tmap);
+    } else {
+      using C = ls::IdxTc<1, 64>;
+      if (allow_smem(ls::index_score_tc<1, 64>, C::kSmem, g_smem_idx_tc) != cudaSuccess)
+        return check_launch("index_score_tc attribute");
+      ls::index_score_tc<1, 64><<<grid, C::kThreads, C::kSmem, st>>>(p, tmap);
+    }
   } else {
     using C = ls::IdxTc<2, 128>;
     if (allow_smem(ls::index_score_tc<2, 128>, C::kSmem, g_smem_bound_tc) != cudaSuccess)

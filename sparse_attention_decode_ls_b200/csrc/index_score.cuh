@@ -126,12 +126,14 @@ struct IdxTcParams {
   int filt_k;              // the k of the selection the candidates serve
 };
 
-template <int KP, int NCOL>
+// FILT: the instance that also keeps candidate lists (key scoring in the decode step); its
+// filter state takes the room of one pipeline stage.
+template <int KP, int NCOL, bool FILT = false>
 struct IdxTc {
   static constexpr int kThreads = 192;                 // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
   static constexpr int kPanel = 128 * 128;             // one 128-row x 128-byte K panel
   static constexpr int kStageBytes = KP * kPanel;
-  static constexpr int kStages = (KP == 1) ? 5 : 3;
+  static constexpr int kStages = (KP == 1) ? (FILT ? 5 : 6) : 3;
   static constexpr int kAcc = 256 / NCOL;              // accumulators in 256 TMEM columns
   static constexpr int kBBytes = KP * NCOL * 128;
   static constexpr int kOffB = kStages * kStageBytes;
@@ -143,8 +145,8 @@ struct IdxTc {
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   // candidate filter (key scoring only): the scores of the tiles scored before the threshold
   // is known, and each row's scores that passed it with their tile numbers
-  static constexpr int kFiltBacklog = (KP == 1) ? 16 : 0;   // tiles
-  static constexpr int kRowCand = (KP == 1) ? 8 : 0;        // passing scores kept per row
+  static constexpr int kFiltBacklog = FILT ? 16 : 0;   // tiles
+  static constexpr int kRowCand = FILT ? 8 : 0;        // passing scores kept per row
   static constexpr int kOffBl = (kOffTmem + 16 + 15) & ~15;
   static constexpr int kOffLcs = kOffBl + kFiltBacklog * 128 * 4;
   static constexpr int kOffLct = kOffLcs + 128 * kRowCand * 4;
@@ -169,10 +171,10 @@ __device__ __forceinline__ int idx_unit_row(const IdxTcParams& p, int b, int u, 
 }
 
 // The key-scoring instance (KP = 1) runs two CTAs per SM, so it must stay within 168 registers.
-template <int KP, int NCOL>
+template <int KP, int NCOL, bool FILT = false>
 __global__ void __launch_bounds__(192, KP == 1 ? 2 : 1)
     index_score_tc(const IdxTcParams p, const __grid_constant__ CUtensorMap tmap) {
-  using C = IdxTc<KP, NCOL>;
+  using C = IdxTc<KP, NCOL, FILT>;
   extern __shared__ uint8_t sm_raw[];
   uint8_t* sm = (uint8_t*)(((uintptr_t)sm_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sA = sm;
@@ -227,7 +229,7 @@ __global__ void __launch_bounds__(192, KP == 1 ? 2 : 1)
   const int my_tiles = t_end - t_begin;
   if (my_tiles <= 0) {
     // a CTA without tiles has no candidates (the top-k reads every CTA's count)
-    if (p.filt && p.mode == 0 && !p.unit_list && tid < 4) p.cand_cnt[((size_t)b * p.ctas_per_req + cta) * 4 + tid] = 0;
+    if (FILT && p.filt && p.mode == 0 && !p.unit_list && tid < 4) p.cand_cnt[((size_t)b * p.ctas_per_req + cta) * 4 + tid] = 0;
     return;
   }
 
@@ -433,7 +435,7 @@ __global__ void __launch_bounds__(192, KP == 1 ? 2 : 1)
     // largest is among them) and every list is complete; a warp that did not see tau within
     // kFiltBacklog tiles (or saw another tau than the one set), a row or list that ran full or
     // an aborted CTA marks the request incomplete.
-    const bool filt = p.filt != nullptr && p.mode == 0 && !p.unit_list;
+    const bool filt = FILT && p.filt != nullptr && p.mode == 0 && !p.unit_list;
     int* fctl = filt ? p.filt + (size_t)b * kFiltInts : nullptr;
     const int n_need = 4 * min(min(p.ctas_per_req, n_tiles), 8);  // statistics that set tau
     const int fj = filt ? min(8, max(1, (int)((64LL * p.filt_k + L - 1) / max(L, 1)))) : 1;
