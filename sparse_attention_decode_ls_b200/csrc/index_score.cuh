@@ -317,6 +317,7 @@ __global__ void __launch_bounds__(192, KP == 1 ? 2 : 1)
 
   if (warp == 0) {
     // ================= TMA producer =================
+    const uint64_t stream_pol = l2_evict_first_policy();  // keys and scales are read once
     // Per tile: the keys of its two 64-row units (TMA, 128-byte swizzle) and, for keys,
     // their 64 token scales (bulk copy) into the stage, plus each unit's logical id.
     // A stage is released only when the MMA has consumed it and the epilogue has read
@@ -362,9 +363,11 @@ __global__ void __launch_bounds__(192, KP == 1 ? 2 : 1)
             for (int uu = 0; uu < 2; ++uu) {
               if (rows[uu] < 0) continue;
               for (int pk = 0; pk < KP; ++pk)
-                tma_load_2d(dst + pk * C::kPanel + uu * 64 * 128, &tmap, &full[st], pk * 128, rows[uu]);
+                tma_load_2d_hint(dst + pk * C::kPanel + uu * 64 * 128, &tmap, &full[st], pk * 128, rows[uu],
+                                 stream_pol);
               if (p.mode == 0)
-                bulk_load(smem_u32(s_scale + st * 128 + uu * 64), p.row_scale + rows[uu], 256, &full[st]);
+                bulk_load_hint(smem_u32(s_scale + st * 128 + uu * 64), p.row_scale + rows[uu], 256, &full[st],
+                               stream_pol);
             }
           }
         }

@@ -122,7 +122,7 @@ __host__ __device__ constexpr int fast_smem_bytes(int L, int n) {
 //     read back as a float: the same bits the indexer stored in the score row.
 __device__ __forceinline__ void topk_from_candidates(const TopkParams& p, int b, int L, int n, uint32_t* smem,
                                                      const int* coff, uint32_t* list, uint32_t* scan32,
-                                                     uint32_t* s_misc) {
+                                                     uint32_t* s_misc, uint32_t tau_bits) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int k = p.k, nl = p.cand_lists, nw8 = fast_round((L + 31) >> 5, 8);
   uint32_t* keys = smem;
@@ -138,7 +138,7 @@ __device__ __forceinline__ void topk_from_candidates(const TopkParams& p, int b,
     s_misc[1] = 0u;         // keys in the list
     s_misc[2] = kFastBins;  // the k-th key's bin (none yet)
   }
-  const uint32_t tk = float_key(__int_as_float(p.filt[(size_t)b * kFiltInts + kFiltTau]));
+  const uint32_t tk = float_key(__uint_as_float(tau_bits));
   __syncthreads();
   // ---- 1. load and count: warp w takes lists w, w + 16, ..., eight at a time (lane j entry
   // j; a list longer than 32 entries takes more turns), all their loads in flight at once
@@ -416,6 +416,7 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster(const TopkParams
       }
     } else if (warp == 1 && lane == 0) {
       s_fast = (f[kFiltReady] != 0 && f[kFiltIncomplete] == 0) ? 1u : 0u;
+      s_Tb = (uint32_t)f[kFiltTau];  // the threshold's bits (s_Tb is the cluster path's, later)
     }
     const long long L0 = ((long long)p.lens[b] * p.len_mul + p.len_div - 1) / p.len_div;
     __syncthreads();
@@ -428,7 +429,7 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster(const TopkParams
     cluster_arrive();
     if (use) {
       if (rank == 0) {
-        topk_from_candidates(p, b, Lq, nc, sm_keys, coff, hist, (uint32_t*)scan_tmp, s_off);
+        topk_from_candidates(p, b, Lq, nc, sm_keys, coff, hist, (uint32_t*)scan_tmp, s_off, s_Tb);
         if (p.done) {
           __syncthreads();
           count_done(p.done + b, CL);  // counts for the whole cluster
