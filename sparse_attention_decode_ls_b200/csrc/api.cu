@@ -357,7 +357,8 @@ ls_status launch_topk(int B, int k, const float* scores, int stride, const int* 
                       int len_limit, const int* unit_list, int list_stride, int* idx, float* sel, float* thr,
                       cudaStream_t st, const int* pos_list = nullptr, int pos_stride = 0,
                       const int* pos_offset = nullptr, int* clear = nullptr, int* done = nullptr,
-                      const ls::IdxTcParams* filt = nullptr, int filt_lists = 0) {
+                      const ls::IdxTcParams* filt = nullptr, int filt_lists = 0,
+                      const ls_sparse_attn_args* pf = nullptr) {
   ls::TopkParams p{};
   p.clear = clear;
   p.done = done;
@@ -367,6 +368,18 @@ ls_status launch_topk(int B, int k, const float* scores, int stride, const int* 
     p.cand_pos = filt->cand_pos;
     p.cand_score = filt->cand_score;
     p.cand_lists = filt_lists;
+    // the attention's bf16 paged rows, prefetched by the CTAs the candidate path leaves idle
+    const bool pf_ok = pf && pf->addressing == LS_ROWS_PAGED && pf->dtype == LS_BF16 && pf->k_rows &&
+                       pf->page_table && pf->row_stride >= pf->dk && pf->row_stride % 8 == 0 && pf->dk % 8 == 0 &&
+                       ((uintptr_t)pf->k_rows & 15) == 0 && pf->num_rows > 0 && pf->max_pages > 0;
+    if (pf_ok) {
+      p.pf_rows = (const uint8_t*)pf->k_rows;
+      p.pf_pt = pf->page_table;
+      p.pf_max_pages = pf->max_pages;
+      p.pf_num_rows = pf->num_rows;
+      p.pf_row_bytes = pf->row_stride * 2;
+      p.pf_bytes = pf->dk * 2;
+    }
   }
   p.pos_list = pos_list; p.pos_stride = pos_stride; p.pos_offset = pos_offset;
   p.B = B; p.k = k; p.stride = stride; p.scores = scores; p.lens = lens; p.len_mul = len_mul;
@@ -1367,7 +1380,7 @@ ls_status ls_decode_step(const ls_decode_step_args* a, void* workspace, size_t w
     ready_want = ix->max_len <= kTopkRowMaxLen ? 1 : (topk16_supported(st) ? 16 : 8);
     LS_TRY(launch_topk(ix->batch, a->k, scores, ix->max_len, ix->lens, 1, 1, ix->max_len, nullptr, 0, idx, sel,
                        nullptr, st, nullptr, 0, nullptr, done, ready, cand ? &fp : nullptr,
-                       cand ? 4 * step_idx_ctas(a) : 0));
+                       cand ? 4 * step_idx_ctas(a) : 0, cand && !a->use_hotbuf ? &a->attn : nullptr));
   }
   void* attn_ws = w + l.off_attn;
   if (a->use_hotbuf) {

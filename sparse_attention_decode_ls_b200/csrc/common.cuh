@@ -189,6 +189,10 @@ __device__ __forceinline__ void cluster_wait() {
 __device__ __forceinline__ void prefetch_l2(const void* ptr) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
 }
+// Bulk prefetch of [ptr, ptr + bytes) into L2 (16-byte aligned address, bytes % 16 == 0).
+__device__ __forceinline__ void prefetch_l2_bulk(const void* ptr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(ptr), "r"(bytes) : "memory");
+}
 
 // ---------------------------------------------------------------------------------
 // Per-request completion counts between the kernels of a decode step.  A producer CTA,

@@ -43,6 +43,14 @@ struct TopkParams {
   const int* cand_pos;       // [B][cand_lists][kCandPerWarp]
   const float* cand_score;
   int cand_lists;            // the indexer's lists per request
+  // optional, with the candidate lists: the attention's paged rows, which the CTAs other than
+  // CTA 0 bring into L2 (bulk prefetch) while CTA 0 selects
+  const uint8_t* pf_rows;    // row r at pf_rows + r * pf_row_bytes, pf_bytes of it fetched
+  const int* pf_pt;          // [B][pf_max_pages] page table (row = page * 64 + position % 64)
+  int pf_max_pages;
+  long long pf_num_rows;
+  long long pf_row_bytes;
+  int pf_bytes;
 };
 
 constexpr int kTopkThreads = 512;
@@ -132,7 +140,6 @@ __device__ __forceinline__ void topk_from_candidates(const TopkParams& p, int b,
   uint32_t* lkey = list;
   int* lpos = (int*)(list + kFastList);
   const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-  for (int w = tid * 4; w < nw8; w += kTopkThreads * 4) *(uint4*)(bits + w) = z4;
   for (int w = tid * 4; w < kFastBins; w += kTopkThreads * 4) *(uint4*)(room + w) = z4;
   if (tid == 0) {
     s_misc[1] = 0u;         // keys in the list
@@ -140,7 +147,7 @@ __device__ __forceinline__ void topk_from_candidates(const TopkParams& p, int b,
   }
   const uint32_t tk = float_key(__uint_as_float(tau_bits));
   __syncthreads();
-  // ---- 1. load and count: warp w takes lists w, w + 16, ..., eight at a time (lane j entry
+  // ---- 1. load and count: warp w takes lists w, w + 16, ..., ten at a time (lane j entry
   // j; a list longer than 32 entries takes more turns), all their loads in flight at once
   const size_t base = (size_t)b * nl * kCandPerWarp;
   constexpr int kW = kTopkThreads / 32;
@@ -150,11 +157,12 @@ __device__ __forceinline__ void topk_from_candidates(const TopkParams& p, int b,
     cpos[at] = ps;
     if (key >= tk) atomicAdd(&room[min((key - tk) >> kFastShift, (uint32_t)(kFastBins - 1))], 1u);
   };
-  for (int l0 = warp; l0 < nl; l0 += 8 * kW) {
-    float sq[8];
-    int pq[8], at[8];
+  constexpr int kPer = 10;  // 16 warps x 10: the 148 lists of a 37-CTA indexer in one round
+  for (int l0 = warp; l0 < nl; l0 += kPer * kW) {
+    float sq[kPer];
+    int pq[kPer], at[kPer];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < kPer; ++u) {
       const int l = l0 + u * kW;
       at[u] = -1;
       if (l < nl) {
@@ -168,9 +176,9 @@ __device__ __forceinline__ void topk_from_candidates(const TopkParams& p, int b,
       }
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u)
+    for (int u = 0; u < kPer; ++u)
       if (at[u] >= 0) take(sq[u], pq[u], at[u]);
-    for (int u = 0; u < 8; ++u) {  // entries 32 and up (a rare long list)
+    for (int u = 0; u < kPer; ++u) {  // entries 32 and up (a rare long list)
       const int l = l0 + u * kW;
       if (l >= nl) break;
       const int o = coff[l], c = min(coff[l + 1] - o, kCandPerWarp);
@@ -204,6 +212,8 @@ __device__ __forceinline__ void topk_from_candidates(const TopkParams& p, int b,
   }
   __syncthreads();
   const uint32_t tb = s_misc[2], r0 = (uint32_t)k - s_misc[3];  // r0 of bin tb's keys are chosen
+  for (int w = tid * 4; w < nw8; w += kTopkThreads * 4) *(uint4*)(bits + w) = z4;
+  __syncthreads();
   // ---- 3. keys above bin tb chosen, bin tb's keys listed
   for (int i = tid; i < n; i += kTopkThreads) {
     const uint32_t key = keys[i];
@@ -433,6 +443,21 @@ __global__ void __launch_bounds__(kTopkThreads, 2) topk_cluster(const TopkParams
         if (p.done) {
           __syncthreads();
           count_done(p.done + b, CL);  // counts for the whole cluster
+        }
+      } else if (p.pf_rows) {
+        // the candidates' attention rows into L2 while CTA 0 selects (the HBM is idle then):
+        // each warp of CTAs 1 .. CL-1 one list, one lane per entry
+        const size_t lbase = (size_t)b * p.cand_lists * kCandPerWarp;
+        for (int l = (rank - 1) * kWarps + warp; l < p.cand_lists; l += (CL - 1) * kWarps) {
+          const int o = coff[l], c = min(coff[l + 1] - o, kCandPerWarp);
+          for (int j = lane; j < c; j += 32) {
+            const int ps = p.cand_pos[lbase + (size_t)l * kCandPerWarp + j];
+            if (ps < 0 || ps >= Lq || (ps >> 6) >= p.pf_max_pages) continue;
+            const int pg = p.pf_pt[(size_t)b * p.pf_max_pages + (ps >> 6)];
+            const long long row = (long long)pg * 64 + (ps & 63);
+            if (pg < 0 || row >= p.pf_num_rows) continue;
+            prefetch_l2_bulk(p.pf_rows + row * p.pf_row_bytes, (uint32_t)p.pf_bytes);
+          }
         }
       }
       cluster_wait();
