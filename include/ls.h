@@ -371,6 +371,14 @@ ls_status ls_sparse_attn_decode_noalloc(const ls_sparse_attn_args* args, ls_stre
  *   i (0 indexer, 1 top-k, 2 resolve, 3 gather, 4 attention) and events[5] after
  *   the last stage, so a caller can time each stage.
  * sel_slot / miss_pos / miss_slot: optional outputs of the hot-buffer resolve (as in a4).
+ * Selection: with the fp8 tensor-core indexer over whole requests longer than 32,768
+ *   tokens (and k <= 6144), the indexer also keeps lists of the scores above a threshold
+ *   it derives from the request's own scores, and the top-k selects among them; where a
+ *   request's lists are incomplete it selects over all scores.  Either way the selection
+ *   equals a2's over the same scores bit for bit.
+ * Workspace: needs no initialisation; every count and flag the step keeps there is
+ *   reset by the step's own kernels (contents left by a failed step can only send the
+ *   next step's selection to the full path).
  * Streams: the hot-buffer step forks onto two streams of its own and joins back into
  *   `stream`.  Each (host thread, device, caller stream) gets its own pair, created on
  *   first use, so steps issued on independent streams stay independent; steps issued
