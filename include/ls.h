@@ -377,8 +377,8 @@ ls_status ls_sparse_attn_decode_noalloc(const ls_sparse_attn_args* args, ls_stre
  *   request's lists are incomplete it selects over all scores.  Either way the selection
  *   equals a2's over the same scores bit for bit.
  * Workspace: needs no initialisation; every count and flag the step keeps there is
- *   reset by the step's own kernels (contents left by a failed step can only send the
- *   next step's selection to the full path).
+ *   reset by the step's own kernels, and whatever an earlier (or failed) call left there
+ *   never changes a result (at most it sends a selection to the full path).
  * Streams: the hot-buffer step forks onto two streams of its own and joins back into
  *   `stream`.  Each (host thread, device, caller stream) gets its own pair, created on
  *   first use, so steps issued on independent streams stay independent; steps issued
