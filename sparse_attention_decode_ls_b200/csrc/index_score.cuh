@@ -524,7 +524,7 @@ __global__ void __launch_bounds__(192, KP == 1 ? 2 : 1)
       }
       if (filt) {
         const float sc = valid ? sum * scale : -INFINITY;
-        if (!tau_known && !gave_up) {
+        if (!tau_known) {  // (giving up sets tau_known with tau = +inf: one test per tile after)
           s_bl[i * 128 + r] = sc;
           if (i == 0) {
             // this warp's statistic: the fj-th largest score of its rows of the first tile; its
@@ -573,8 +573,10 @@ __global__ void __launch_bounds__(192, KP == 1 ? 2 : 1)
             }
           } else if (i + 1 >= C::kFiltBacklog) {
             gave_up = true;  // too many tiles to keep: this request's lists stay incomplete
+            tau_known = true;
+            tau = INFINITY;
           }
-        } else if (tau_known && sc >= tau && valid) {
+        } else if (sc >= tau && valid) {
           keep(i, sc);
         }
       }
@@ -582,10 +584,11 @@ __global__ void __launch_bounds__(192, KP == 1 ? 2 : 1)
     if (filt) {
       // the statistic if not yet looked at, then the rows' candidates into this warp's list
       const bool aborted = *(volatile int*)&s_abort != 0;
-      bool bad = __any_sync(0xffffffffu, nk > C::kRowCand) || !tau_known || aborted;
+      bool bad = __any_sync(0xffffffffu, nk > C::kRowCand) || !tau_known || gave_up || aborted;
       if (lane == 0) {
         if (poll_inflight) mbar_wait(&s_pbar[wq], poll_ph);  // the copy lands before the CTA ends
-        if (tau_known && (!(uint32_t)tau_check || (tau_check >> 32) != __float_as_uint(tau))) bad = true;
+        if (tau_known && !gave_up && (!(uint32_t)tau_check || (tau_check >> 32) != __float_as_uint(tau)))
+          bad = true;
       }
       bad = __shfl_sync(0xffffffffu, (int)bad, 0) != 0;
       const size_t wlist = (((size_t)b * p.ctas_per_req + cta) * 4 + wq) * kCandPerWarp;
