@@ -92,6 +92,23 @@ def test_topk_hand_example():
     assert idx.tolist() == [0, 1, 2, -1]
 
 
+def test_decode_step_hand_example():
+    """The composed step on the hand example (tests/golden/hand_examples.md, decode step):
+    the indexer's top 2 are positions 1 and 2, and one head over their rows gives closed forms."""
+    q8, sq, w, pool, ks, pt = _hand_indexer()
+    kv = np.zeros((1, 64, 2), dtype=np.uint16)
+    kv[0, :3] = [[0x4040, 0x4110], [0x3F80, 0x4000], [0x0000, 0x4080]]
+    q_attn = np.array([[[0x3F80, 0x0000]]], dtype=np.uint16)
+    scores, idx, o, lse = O.decode_step(q8=q8, q_scale=sq, w_bits=w, key_pool=pool, key_scale_pool=ks,
+                                        page_table=pt, lens=[3], k=2, q_attn_bits=q_attn, kv_pool_bits=kv,
+                                        scale=1.0, dv=1)
+    assert np.array_equal(np.asarray(scores[0])[:3], [-2.5, 0.25, 0.0])
+    assert idx.tolist() == [[1, 2]]
+    e = math.e
+    assert o.shape == (1, 1, 1) and abs(o[0, 0, 0] - e / (1 + e)) < 1e-15
+    assert abs(lse[0, 0] - math.log1p(e)) < 1e-15
+
+
 def test_index_score_page_shuffle_invariance():
     inp = syn.indexer_fp8([700, 300], heads=8, dim=32, seed=5)
     a = O.index_score(inp.q.numpy(), inp.w.view(torch.int16).numpy().view(np.uint16),
